@@ -1,0 +1,392 @@
+"""Pins for the CPU oracle: invariants, closed forms and exact rational brute force.
+
+These run without a GPU.  Each test pins the oracle to something other than
+itself, chosen so that a dropped term, a wrong sign or index, or a transposed
+operand in ``oracle/gdn_oracle.py`` fails at least one of them.
+"""
+from fractions import Fraction
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------- #
+# helpers independent of the oracle
+# --------------------------------------------------------------------------- #
+def random_chunks(nc, k, d, seed, gate_scale=1.0):
+    """Chunks drawn like the workloads (unit-norm keys, sigmoid beta, -softplus gates)."""
+    rng = np.random.default_rng(seed)
+    K = rng.standard_normal((nc, k, d))
+    K /= np.linalg.norm(K, axis=-1, keepdims=True)
+    V = rng.standard_normal((nc, k, d))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((nc, k))))
+    lg = -np.log1p(np.exp(rng.standard_normal((nc, k)))) * gate_scale
+    g = np.cumsum(lg, axis=-1)
+    return K, V, beta, g, lg
+
+
+def frac_matrix(a):
+    return [[Fraction(float(x)) for x in row] for row in a]
+
+
+def frac_matmul(X, Y):
+    n, m, p = len(X), len(Y), len(Y[0])
+    return [[sum((X[i][l] * Y[l][j] for l in range(m)), Fraction(0)) for j in range(p)]
+            for i in range(n)]
+
+
+def frac_eye(n):
+    return [[Fraction(int(i == j)) for j in range(n)] for i in range(n)]
+
+
+def frac_sub(X, Y):
+    return [[a - b for a, b in zip(r, s)] for r, s in zip(X, Y)]
+
+
+def frac_add(X, Y):
+    return [[a + b for a, b in zip(r, s)] for r, s in zip(X, Y)]
+
+
+def frac_gauss_jordan_inverse(M):
+    """Inverse by Gauss-Jordan elimination with exact rationals (no triangular shortcut)."""
+    n = len(M)
+    aug = [list(r) + [Fraction(int(i == j)) for j in range(n)] for i, r in enumerate(M)]
+    for c in range(n):
+        p = next(r for r in range(c, n) if aug[r][c] != 0)
+        aug[c], aug[p] = aug[p], aug[c]
+        piv = aug[c][c]
+        aug[c] = [x / piv for x in aug[c]]
+        for r in range(n):
+            if r != c and aug[r][c] != 0:
+                f = aug[r][c]
+                aug[r] = [x - f * y for x, y in zip(aug[r], aug[c])]
+    return [r[n:] for r in aug]
+
+
+def frac_to_np(X):
+    return np.array([[float(x) for x in r] for r in X])
+
+
+def load_golden():
+    out, name, rows = {}, None, []
+    with open(os.path.join(GOLDEN, "unit_lower_4x4.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            if len(parts) == 1 and not parts[0].lstrip("-").isdigit():
+                name, rows = parts[0], []
+                out[name] = rows
+            else:
+                rows.append([float(x) for x in parts])
+    return {k: np.array(v) for k, v in out.items()}
+
+
+# --------------------------------------------------------------------------- #
+# golden hand-derived example
+# --------------------------------------------------------------------------- #
+def test_golden_4x4_closed_forms():
+    G = load_golden()
+    A = G["A"][None]
+    np.testing.assert_array_equal(O.invert_fwdsub(A)[0], G["T_exact"])
+    np.testing.assert_array_equal(O.neumann_powers_sum(A, 3)[0], G["T_exact"])
+    np.testing.assert_array_equal((A @ A)[0], G["A2"])
+    np.testing.assert_array_equal(O.invert_neumann(A, 1, False, 0)[0], G["T0_N1_nomask"])
+    np.testing.assert_array_equal(O.invert_neumann(A, 1, True, 0)[0], G["T0_N1_mask"])
+    np.testing.assert_array_equal(O.invert_neumann(A, 2, False, 0)[0], G["T0_N2_nomask"])
+    np.testing.assert_array_equal(O.invert_neumann(A, 2, True, 0)[0], G["T0_N2_mask"])
+    T0 = O.invert_neumann(A, 1, True, 0)
+    np.testing.assert_array_equal(O.residual_matrix(A, T0)[0], G["E_N1_mask"])
+    np.testing.assert_array_equal(O.invert_neumann(A, 1, True, 1)[0], G["T_N1_mask_S1"])
+
+
+def test_closed_form_2x2_3x3():
+    a21, a31, a32 = 0.3, -0.7, 1.9
+    A2 = np.array([[[0, 0], [a21, 0]]], float)
+    np.testing.assert_allclose(O.invert_fwdsub(A2)[0], [[1, 0], [a21, 1]], rtol=0, atol=1e-15)
+    A3 = np.array([[[0, 0, 0], [a21, 0, 0], [a31, a32, 0]]], float)
+    T3 = O.invert_fwdsub(A3)[0]
+    np.testing.assert_allclose(T3[2, 0], a31 + a32 * a21, rtol=1e-15)
+    np.testing.assert_allclose(T3[2, 1], a32, rtol=1e-15)
+    # Neumann N=1 is I + A: it misses only the a32*a21 path
+    T0 = O.invert_neumann(A3, 1, False, 0)[0]
+    np.testing.assert_allclose(T3 - T0, [[0, 0, 0], [0, 0, 0], [a32 * a21, 0, 0]], atol=1e-15)
+
+
+def test_band_mask_definition():
+    M = O.band_mask(6, 2)
+    for i in range(6):
+        for j in range(6):
+            assert M[i, j] == (1.0 if i - j <= 2 else 0.0)
+
+
+# --------------------------------------------------------------------------- #
+# A
+# --------------------------------------------------------------------------- #
+def test_build_A_structure_and_no_overflow():
+    K, _, beta, g, _ = random_chunks(3, 16, 8, seed=1)
+    A = O.build_A(K, beta, g)
+    assert np.all(np.triu(A) == 0.0)                       # strictly lower
+    assert np.all(A[np.tril(np.ones((16, 16), bool), -1)[None].repeat(3, 0)] != 0.0)
+    # a huge positive g_i - g_j above the diagonal must not reach exp
+    g2 = np.tile(-1000.0 * np.arange(16.0), (3, 1))
+    A2 = O.build_A(K, beta, g2)
+    assert np.all(np.isfinite(A2))
+
+
+def test_build_A_entry_by_entry_small():
+    """Entry (i,j) against an explicit scalar loop with math.exp (3 tokens)."""
+    K, _, beta, g, _ = random_chunks(1, 3, 4, seed=2)
+    A = O.build_A(K, beta, g)[0]
+    for i in range(3):
+        for j in range(3):
+            if i > j:
+                dot = math.fsum(K[0, i, t] * K[0, j, t] for t in range(4))
+                want = -beta[0, i] * dot * math.exp(g[0, i] - g[0, j])
+                assert A[i, j] == pytest.approx(want, rel=1e-14)
+            else:
+                assert A[i, j] == 0.0
+
+
+# --------------------------------------------------------------------------- #
+# exact inverse and Lemma 3.1
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("k", [8, 64, 256])
+def test_I1_fwdsub_is_inverse(k):
+    K, _, beta, g, _ = random_chunks(4, k, 32, seed=k)
+    A = O.build_A(K, beta, g)
+    T = O.invert_fwdsub(A)
+    R = (np.eye(k) - A) @ T
+    assert np.abs(R - np.eye(k)).max() <= 1e-13 * max(1.0, np.abs(T).max())
+
+
+@pytest.mark.parametrize("k", [4, 8])
+def test_I6_bruteforce_rational(k):
+    """fwdsub, the full series, T0 and the residual against exact rationals."""
+    K, _, beta, g, _ = random_chunks(1, k, 5, seed=10 + k, gate_scale=0.1)
+    A = O.build_A(K, beta, g)
+    Af = frac_matrix(A[0])
+    I = frac_eye(k)
+    Tf = frac_gauss_jordan_inverse(frac_sub(I, Af))
+    T = frac_to_np(Tf)
+    np.testing.assert_allclose(O.invert_fwdsub(A)[0], T, rtol=1e-15, atol=1e-15)
+    # truncated series with mask, then the residual correction (exact rationals)
+    N, S = 1, 2
+    P, T0f = I, I
+    for _ in range(N):
+        P = frac_matmul(P, Af)
+        T0f = frac_add(T0f, P)
+    T0f = [[x if i - j <= N else Fraction(0) for j, x in enumerate(r)] for i, r in enumerate(T0f)]
+    Ef = frac_sub(I, frac_matmul(frac_sub(I, Af), T0f))
+    acc, Ep = I, I
+    for _ in range(S):
+        Ep = frac_matmul(Ep, Ef)
+        acc = frac_add(acc, Ep)
+    Tres = frac_to_np(frac_matmul(T0f, acc))
+    np.testing.assert_allclose(O.invert_neumann(A, N, True, 0)[0], frac_to_np(T0f),
+                               rtol=1e-15, atol=1e-15)
+    np.testing.assert_allclose(O.residual_matrix(A, O.invert_neumann(A, N, True, 0))[0],
+                               frac_to_np(Ef), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(O.invert_neumann(A, N, True, S)[0], Tres, rtol=1e-14, atol=1e-15)
+
+
+@pytest.mark.parametrize("k", [16, 64])
+def test_I2_lemma_3_1_powers_vanish(k):
+    K, _, beta, g, _ = random_chunks(2, k, 16, seed=3)
+    A = O.build_A(K, beta, g)
+    i = np.arange(k)[:, None]
+    j = np.arange(k)[None, :]
+    P = np.broadcast_to(np.eye(k), A.shape).copy()
+    for n in range(1, k + 1):
+        P = P @ A
+        assert np.all(P[:, (i - j) < n] == 0.0), n          # exact zeros
+    assert np.all(P == 0.0)                                  # A^k = 0
+
+
+@pytest.mark.parametrize("k", [16, 64])
+def test_I3_full_series_is_exact(k):
+    K, _, beta, g, _ = random_chunks(2, k, 32, seed=4, gate_scale=0.2)
+    A = O.build_A(K, beta, g)
+    T = O.invert_fwdsub(A)
+    T_full = O.invert_neumann(A, k - 1, False, 0)
+    assert O.rel_fro(T_full, T) <= 1e-12
+
+
+@pytest.mark.parametrize("N", [1, 2, 3, 4])
+def test_I4_band_equality(N):
+    k = 64
+    K, _, beta, g, _ = random_chunks(3, k, 64, seed=5, gate_scale=0.2)
+    A = O.build_A(K, beta, g)
+    T = O.invert_fwdsub(A)
+    dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+    band = dist <= N
+    for mask in (False, True):
+        T0 = O.invert_neumann(A, N, mask, 0)
+        err = np.abs(T0 - T)[:, band].max()
+        assert err <= 1e-13 * np.abs(T).max()
+        if mask:
+            assert np.all(T0[:, ~band] == 0.0)
+        else:
+            # outside the band, the unmasked truncation differs from T
+            assert np.abs(T0 - T)[:, dist == N + 1].max() > 0
+
+
+@pytest.mark.parametrize("N,S", [(1, 1), (3, 1), (3, 8), (2, 3)])
+def test_I5_residual_band_law(N, S):
+    k = 64
+    K, _, beta, g, _ = random_chunks(2, k, 64, seed=6, gate_scale=0.2)
+    A = O.build_A(K, beta, g)
+    T = O.invert_fwdsub(A)
+    L = (S + 1) * (N + 1)
+    dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+    scale = np.abs(T).max()
+    for mask in (False, True):
+        Tr = O.invert_neumann(A, N, mask, S)
+        assert np.abs(Tr - T)[:, dist <= L - 1].max() <= 1e-12 * scale
+        if L >= k:
+            assert O.rel_fro(Tr, T) <= 1e-12
+        else:
+            assert np.abs(Tr - T)[:, dist == L].max() > 0
+    # without the mask E = A^{N+1}, so the result is the Neumann series of order L-1
+    Tr = O.invert_neumann(A, N, False, S)
+    assert O.rel_fro(Tr, O.invert_neumann(A, L - 1, False, 0)) <= 1e-12
+    E = O.residual_matrix(A, O.invert_neumann(A, N, False, 0))
+    Ap = np.linalg.matrix_power(A, N + 1)
+    assert np.abs(E - Ap).max() <= 1e-13
+
+
+# --------------------------------------------------------------------------- #
+# WY
+# --------------------------------------------------------------------------- #
+def test_I7_wy_triangular_solve_identity():
+    k, d = 64, 32
+    K, V, beta, g, _ = random_chunks(3, k, d, seed=7)
+    A = O.build_A(K, beta, g)
+    T = O.invert_fwdsub(A)
+    W, U = O.wy(T, K, V, beta)
+    I_A = np.eye(k) - A
+    np.testing.assert_allclose(I_A @ W, beta[..., None] * K, atol=1e-12)
+    np.testing.assert_allclose(I_A @ U, beta[..., None] * V, atol=1e-12)
+    Wg, U2 = O.wy(T, K, V, beta, g)
+    np.testing.assert_allclose(I_A @ Wg, (beta * np.exp(g))[..., None] * K, atol=1e-12)
+    np.testing.assert_array_equal(U, U2)
+
+
+def test_wy_rows_small_explicit():
+    """W row i = sum_j T_ij beta_j k_j, explicit loop on a 3x3 chunk."""
+    K, V, beta, g, _ = random_chunks(1, 3, 2, seed=8)
+    T = np.array([[[1.0, 0, 0], [0.5, 1.0, 0], [-0.25, 2.0, 1.0]]])
+    W, U = O.wy(T, K, V, beta)
+    for i in range(3):
+        for t in range(2):
+            w = math.fsum(T[0, i, j] * beta[0, j] * K[0, j, t] for j in range(3))
+            u = math.fsum(T[0, i, j] * beta[0, j] * V[0, j, t] for j in range(3))
+            assert W[0, i, t] == pytest.approx(w, rel=1e-14)
+            assert U[0, i, t] == pytest.approx(u, rel=1e-14)
+
+
+# --------------------------------------------------------------------------- #
+# full chunk-wise forward vs the token recurrence
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("T_len,d", [(256, 32), (1024, 128)])
+def test_I8_chunk_form_equals_token_recurrence(T_len, d):
+    k, BH = 64, 2
+    rng = np.random.default_rng(9)
+    K, V, beta, _, lg = random_chunks(BH * T_len // k, k, d, seed=9)
+    K = K.reshape(BH, T_len, d)
+    V = V.reshape(BH, T_len, d)
+    beta = beta.reshape(BH, T_len)
+    lg = lg.reshape(BH, T_len)
+    Q = rng.standard_normal((BH, T_len, d))
+    Q /= np.linalg.norm(Q, axis=-1, keepdims=True)
+    S0 = 0.1 * rng.standard_normal((BH, d, d))
+    n = T_len // k
+    g = np.cumsum(lg.reshape(BH, n, k), axis=-1)
+    Kc, Vc, Qc, bc = (x.reshape(BH, n, k, -1) for x in (K, V, Q, beta[..., None]))
+    bc = bc[..., 0]
+    A = O.build_A(Kc, bc, g)
+    T = O.invert_fwdsub(A)
+    Oc, Sc = O.chunk_forward(Qc, Kc, Vc, bc, g, T, S0)
+    Ot, St = O.token_recurrence(Q, K, V, beta, lg, S0)
+    assert O.rel_fro(Oc.reshape(BH, T_len, d), Ot) <= 1e-10
+    assert O.rel_fro(Sc, St) <= 1e-10
+
+
+# --------------------------------------------------------------------------- #
+# INT8 scheme
+# --------------------------------------------------------------------------- #
+def test_I9_int8_codes_and_accumulators():
+    k, N = 16, 3
+    K, _, beta, g, _ = random_chunks(4, k, 16, seed=11, gate_scale=0.2)
+    A32 = O.build_A(K, beta, g).astype(np.float32)
+    dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+    for mask in (False, True):
+        r = O.int8_neumann(A32, N, mask)
+        q, acc = r["q"], r["acc"]
+        assert q.min() >= -127 and q.max() <= 127
+        assert np.any(np.abs(q[:, 0]) == 127)               # amax maps to +-127
+        for n in range(1, N):
+            for c in range(4):
+                for i in range(k):
+                    for j in range(k):
+                        want = sum(int(q[c, n - 1, i, l]) * int(q[c, 0, l, j]) for l in range(k))
+                        if mask and dist[i, j] > N:
+                            want = 0
+                        assert int(acc[c, n, i, j]) == want
+        if mask:
+            assert np.all(q[:, :, dist > N] == 0)
+            assert np.all(r["T"][:, dist > N] == 0)
+
+
+def test_int8_rounding_half_even_and_scale():
+    # amax = 127 gives r = 1 exactly, so the codes are rint of the entries
+    A = np.zeros((1, 4, 4), np.float32)
+    A[0, 1, 0] = 127.0
+    A[0, 2, 0] = 2.5
+    A[0, 2, 1] = -1.5
+    A[0, 3, 0] = 0.5
+    A[0, 3, 2] = 3.5
+    r = O.int8_neumann(A, 1, False)
+    assert r["q"][0, 0, 1, 0] == 127
+    assert r["q"][0, 0, 2, 0] == 2      # half to even
+    assert r["q"][0, 0, 2, 1] == -2
+    assert r["q"][0, 0, 3, 0] == 0
+    assert r["q"][0, 0, 3, 2] == 4
+    assert r["scale"][0, 0] == np.float32(1.0)
+
+
+def test_int8_scale_recursion_exact_integers():
+    """Integer A with max 127: q_1 = A, s_1 = 1, and s_2 q_2 approximates A^2."""
+    rng = np.random.default_rng(12)
+    k = 8
+    A = np.tril(rng.integers(-127, 128, (1, k, k)), -1).astype(np.float32)
+    A[0, 1, 0] = 127.0
+    r = O.int8_neumann(A, 2, False)
+    np.testing.assert_array_equal(r["q"][0, 0], A[0].astype(np.int8))
+    A2 = (A[0].astype(np.int64) @ A[0].astype(np.int64))
+    m = np.abs(A2).max()
+    assert r["scale"][0, 1] == np.float32(np.float32(m) / np.float32(127.0))
+    # dequantised power within half a code step of the exact A^2
+    deq = r["scale"][0, 1] * r["q"][0, 1].astype(np.float64)
+    assert np.abs(deq - A2).max() <= 0.5 * m / 127 * (1 + 1e-6)
+    # and the dequantised T is I + A + (that)
+    np.testing.assert_allclose(r["T"][0], np.eye(k) + A[0] + deq, rtol=1e-6, atol=1e-3)
+
+
+def test_int8_dequantised_close_to_float64():
+    k, N = 64, 3
+    K, _, beta, g, _ = random_chunks(8, k, 128, seed=13)
+    A = O.build_A(K, beta, g)
+    A32 = A.astype(np.float32)
+    for mask in (False, True):
+        r = O.int8_neumann(A32, N, mask)
+        ref = O.invert_neumann(A32.astype(np.float64), N, mask, 0)
+        # each power carries at most half a code step (1/254 of its max) of error
+        assert O.rel_fro(r["T"], ref) <= 1e-2
