@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of the fused per-chunk inverse + WY hot path on B200.
+
+Workload (one "step"): the fused chunk pipeline (A from K K^T, Neumann order
+N=3 with the band mask and S=8 residual steps, then W = T diag(beta) K and
+U = T diag(beta) V) over B=4, H=16, T=4096, k=64, d=128, bf16 — 4096 chunks.
+Inputs are seeded synthetic tensors with the recipe of
+``gated_deltanet_chunk_02_b200.inputs``; three input/output copies rotate so
+each step's 270 MB working set is cold in the 126 MB L2.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
+a bounded sample of the same workload instead.
+
+Multi-GPU (torchrun): every rank runs its own independent batch (weak scaling,
+no collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(B=4, H=16, T=4096, k=64, d=128, dtype="bf16", N=3, mask=1, S=8, gated=0)
+METRIC = "GDN chunk inverse+WY: chunks/s and % of roofline (k=64, d=128, bf16)"
+ROTATE = 3
+
+
+def algorithmic_bytes_per_chunk(k: int, d: int, elem: int) -> int:
+    """K, V in + beta, g in + W, U out (the fused kernel reads and writes nothing else)."""
+    return 2 * k * d * elem + 2 * k * 4 + 2 * k * d * elem
+
+
+def algorithmic_flops_per_chunk(k: int, d: int, N: int, S: int) -> int:
+    """Dense product flops the method issues per chunk: K K^T, (N-1) chain
+    products, the residual (A T0, S-1 Horner products, T0 Q) and the two WY
+    products."""
+    kk = 2 * k * k * d
+    chain = (N - 1) * 2 * k ** 3
+    resid = (S + 1) * 2 * k ** 3 if S > 0 else 0
+    wy = 2 * 2 * k * k * d
+    return kk + chain + resid + wy
+
+
+def load_peaks() -> tuple[dict, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_deltanet_chunk_02_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str) -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    summary is missing or was taken on different kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                key, v = line.split(":", 1)
+                vals[key.strip()] = v.strip()
+    if vals.get("source_hash") != kernel_source_hash():
+        return None
+    v = vals.get(f"{kernel}.dram_bytes_per_launch")
+    return float(v) if v else None
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_sample(w: dict, n_sample: int, seed: int = 0) -> tuple[float, int, dict]:
+    """Time the oracle (as it stands) on the first n_sample chunks of the
+    workload; returns (seconds, threads used, info)."""
+    import numpy as np
+    import oracle as O
+    from threadpoolctl import threadpool_info
+    from gated_deltanet_chunk_02_b200.inputs import Workload, make_inputs, as_f64_numpy
+    wl = Workload(B=w["B"], H=w["H"], T=w["T"], k=w["k"], d=w["d"], dtype=w["dtype"])
+    inp = make_inputs(wl, seed=seed)
+    k = w["k"]
+    K = O.to_chunks(as_f64_numpy(inp["K"]), k)[:n_sample]
+    V = O.to_chunks(as_f64_numpy(inp["V"]), k)[:n_sample]
+    b = O.to_chunks(as_f64_numpy(inp["beta"]), k)[:n_sample]
+    g = O.to_chunks(as_f64_numpy(inp["g"]), k)[:n_sample]
+    t0 = time.perf_counter()
+    A = O.build_A(K, b, g)
+    T = O.invert_neumann(A, w["N"], bool(w["mask"]), w["S"])
+    W, U = O.wy(T, K, V, b, g if w["gated"] else None)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()
+                   if i.get("user_api") == "blas"] or [1])
+    return dt, threads, {"W_norm": float(np.linalg.norm(W))}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle on a bounded sample per step (rank 0 only)."""
+    if rank != 0:
+        return 0
+    w = dict(WORKLOAD)
+    n_sample = args.sample_chunks
+    nc = w["B"] * w["H"] * (w["T"] // w["k"])
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, n_sample)
+    total, threads = 0.0, 1
+    for _ in range(args.steps):
+        dt, threads, _ = cpu_oracle_sample(w, n_sample)
+        total += dt
+    value = n_sample * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "chunks/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps * nc / n_sample, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, nc),
+        "cpu_baseline": {"value": value, "unit": "chunks/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {n_sample} of {nc} chunks per step"},
+        "e2e": {"value": value, "unit": "chunks/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: dict, nc: int) -> dict:
+    return {"workload": "fused chunk inverse+WY (A=KK^T gated, Neumann N=3 + band mask, "
+                        "S=8 residual, W/U), B=4 H=16 T=4096 k=64 d=128 bf16",
+            "B": w["B"], "H": w["H"], "T": w["T"], "k": w["k"], "d": w["d"], "N": w["N"],
+            "mask": w["mask"], "S": w["S"], "chunks": nc,
+            "l2": f"inputs larger than L2: {ROTATE} rotating input/output sets of 270 MB"}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--sample-chunks", type=int, default=512,
+                    help="chunks per step for the CPU oracle timings")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+
+    import torch
+    from gated_deltanet_chunk_02_b200 import gdn
+    from gated_deltanet_chunk_02_b200.inputs import Workload, make_inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = dict(WORKLOAD)
+    wl = Workload(B=w["B"], H=w["H"], T=w["T"], k=w["k"], d=w["d"], dtype=w["dtype"])
+    nc = wl.n_chunks
+    k, d = w["k"], w["d"]
+    elem = 2
+    sets = []
+    for r in range(ROTATE):
+        inp = make_inputs(wl, seed=1000 * rank + r)
+        s = {key: inp[key].to(dev) for key in ("K", "V", "beta", "g")}
+        s["W"] = torch.empty_like(s["K"])
+        s["U"] = torch.empty_like(s["V"])
+        sets.append(s)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        s = sets[i % ROTATE]
+        gdn.gdn_chunk_wy_fused(s["K"], s["V"], s["beta"], s["g"], w["N"], w["mask"], w["S"],
+                               w["gated"], s["W"], s["U"], None, k=k, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert gdn.gdn_get_status(stream) == gdn.GDN_OK
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launches0 = gdn.gdn_launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = gdn.gdn_launch_count() - launches0
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world, dev)
+    status = gdn.gdn_get_status(stream)
+    assert status == gdn.GDN_OK, status
+
+    # end to end through the public API: pinned host inputs in, host outputs back
+    host = {key: sets[0][key].cpu().pin_memory() for key in ("K", "V", "beta", "g")}
+    hostW = torch.empty(sets[0]["W"].shape, dtype=sets[0]["W"].dtype).pin_memory()
+    hostU = torch.empty_like(hostW).pin_memory()
+    dbuf = {key: torch.empty_like(sets[0][key]) for key in ("K", "V", "beta", "g", "W", "U")}
+
+    def e2e_step():
+        for key in ("K", "V", "beta", "g"):
+            dbuf[key].copy_(host[key], non_blocking=True)
+        gdn.gdn_chunk_wy_fused(dbuf["K"], dbuf["V"], dbuf["beta"], dbuf["g"], w["N"], w["mask"],
+                               w["S"], w["gated"], dbuf["W"], dbuf["U"], None, k=k, stream=stream)
+        hostW.copy_(dbuf["W"], non_blocking=True)
+        hostU.copy_(dbuf["U"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+    h2d = sum(host[key].numel() * host[key].element_size() for key in host)
+    d2h = 2 * hostW.numel() * hostW.element_size()
+
+    peaks, peak_kind = load_peaks()
+    ms_step = ms / args.steps
+    bytes_per_launch = algorithmic_bytes_per_chunk(k, d, elem) * nc
+    flops_per_launch = algorithmic_flops_per_chunk(k, d, w["N"], w["S"]) * nc
+    achieved_gbs = bytes_per_launch / (ms_step * 1e-3) / 1e9
+    tflops = flops_per_launch / (ms_step * 1e-3) / 1e12
+    peak_gbs = float(peaks["hbm_gbs"])
+    t_hbm = bytes_per_launch / (peak_gbs * 1e9)
+    t_tc = flops_per_launch / (float(peaks["bf16_tflops"]) * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    traffic = recorded_traffic("fused")
+
+    line = {
+        "metric": METRIC,
+        "value": nc * world / (ms * 1e-3 / args.steps),
+        "unit": "chunks/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": workload_config(w, nc),
+        "roofline": {
+            "bound": bound,
+            "achieved": achieved_gbs if bound == "hbm" else tflops,
+            "peak": peak_gbs if bound == "hbm" else float(peaks["bf16_tflops"]),
+            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": (achieved_gbs / peak_gbs) if bound == "hbm"
+            else tflops / float(peaks["bf16_tflops"]),
+            "traffic": traffic,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback",
+            "roofline_frac": max(t_hbm, t_tc) / (ms_step * 1e-3),
+            "tflops": tflops,
+            "bytes_per_launch": bytes_per_launch,
+            "flops_per_launch": flops_per_launch,
+        },
+        "clocks": clocks.summary(),
+        "e2e": {"value": nc * world / (e2e_ms * 1e-3), "unit": "chunks/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, threads, _ = cpu_oracle_sample(w, args.sample_chunks)
+        line["cpu_baseline"] = {"value": args.sample_chunks / dt, "unit": "chunks/s",
+                                "cores": threads, "kind": "oracle",
+                                "sample": f"first {args.sample_chunks} of {nc} chunks, fp64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

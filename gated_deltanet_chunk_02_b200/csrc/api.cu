@@ -1,0 +1,250 @@
+// api.cu — the C ABI of libgdn: argument checks, dispatch, status word.
+//
+// Every entry point validates its arguments on the host before launching
+// anything; on failure it returns a negative code, launches nothing and keeps
+// a message for gdn_last_error().  Kernels report device-side failures by
+// OR-ing bits into a per-device status word (never by trapping).
+#include <cstdio>
+#include <cstdarg>
+#include <string>
+
+#include "../../include/gdn.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.h"
+
+namespace gdn {
+__device__ int g_status = 0;
+}  // namespace gdn
+
+namespace {
+
+thread_local std::string t_last_error;
+thread_local int64_t t_launches = 0;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(GDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by all entry points; *nc receives the chunk count.
+int check_shape(const gdn_shape& s, int64_t* nc) {
+    if (s.B < 0 || s.H < 0 || s.T < 0) return fail(GDN_ERR_ARG, "negative B, H or T");
+    if (s.k != 32 && s.k != 64 && s.k != 128 && s.k != 256)
+        return fail(GDN_ERR_ARG, "chunk size k=%d not in {32, 64, 128, 256}", s.k);
+    if (s.T % s.k) return fail(GDN_ERR_ARG, "T=%lld is not a multiple of k=%d", (long long)s.T, s.k);
+    if (s.d != 128) return fail(GDN_ERR_UNSUPPORTED, "head dim d=%d (only 128 is built)", s.d);
+    const int64_t n = s.B * s.H * (s.T / s.k);
+    if (n > 0x7fffffffLL) return fail(GDN_ERR_ARG, "too many chunks (%lld)", (long long)n);
+    *nc = n;
+    return GDN_OK;
+}
+
+int check_ptrs(std::initializer_list<std::pair<const void*, const char*>> ps) {
+    for (auto& p : ps) {
+        if (!p.first) return fail(GDN_ERR_ARG, "%s is NULL", p.second);
+        if (!aligned16(p.first)) return fail(GDN_ERR_ALIGN, "%s is not 16-byte aligned", p.second);
+    }
+    return GDN_OK;
+}
+
+int check_opt_ptr(const void* p, const char* name) {
+    if (p && !aligned16(p)) return fail(GDN_ERR_ALIGN, "%s is not 16-byte aligned", name);
+    return GDN_OK;
+}
+
+int check_dtype(gdn_dtype dt) {
+    if (dt != GDN_F32 && dt != GDN_BF16) return fail(GDN_ERR_ARG, "unknown dtype %d", (int)dt);
+    return GDN_OK;
+}
+
+int check_NS(int N, int mask, int S, int k) {
+    if (N < 1 || N > k - 1) return fail(GDN_ERR_ARG, "Neumann order N=%d outside [1, k-1]", N);
+    if (mask != 0 && mask != 1) return fail(GDN_ERR_ARG, "mask must be 0 or 1");
+    if (S < 0 || S > 64) return fail(GDN_ERR_ARG, "residual steps S=%d outside [0, 64]", S);
+    return GDN_OK;
+}
+
+int launched(cudaError_t e, const char* what) {
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    ++t_launches;
+    return GDN_OK;
+}
+
+}  // namespace
+
+#define GDN_TRY(x)                  \
+    do {                            \
+        int _rc = (x);              \
+        if (_rc != GDN_OK) return _rc; \
+    } while (0)
+
+extern "C" {
+
+int gdn_build_A(const void* K, const float* beta, const float* g, float* A, gdn_shape s,
+                gdn_dtype dtype, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_dtype(dtype));
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{K, "K"}, {beta, "beta"}, {g, "g"}, {A, "A"}}));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == GDN_BF16 && gdn::tc_available())
+        return launched(gdn::launch_build_A_tc(K, beta, g, A, nc, s.k, st), "build_A (tcgen05)");
+    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "build_A: k=256 needs the bf16 tensor-core path");
+    return launched(gdn::launch_build_A_simt(K, beta, g, A, nc, s.k, dtype == GDN_BF16, st),
+                    "build_A");
+}
+
+int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask, int S,
+                       gdn_prec prec, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_NS(N, mask, S, s.k));
+    if (prec != GDN_PREC_F32 && prec != GDN_PREC_F16) return fail(GDN_ERR_ARG, "unknown precision");
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (prec == GDN_PREC_F16) {
+        if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
+        if (s.k == 256 && !(mask == 1 && S == 0))
+            return fail(GDN_ERR_UNSUPPORTED, "k=256 on tensor cores supports mask=1, S=0 only");
+        return launched(gdn::launch_neumann_tc(A, T, nc, s.k, N, mask, S, st), "neumann (tcgen05)");
+    }
+    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "float32 Neumann chain supports k <= 128");
+    return launched(gdn::launch_neumann_simt(A, T, nc, s.k, N, mask, S, st), "neumann");
+}
+
+int gdn_invert_fwdsub(const float* A, float* T, gdn_shape s, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    return launched(gdn::launch_fwdsub(A, T, nc, s.k, (cudaStream_t)stream), "fwdsub");
+}
+
+int gdn_wy(const float* T, const void* K, const void* V, const float* beta, const float* g,
+           void* W, void* U, gdn_shape s, gdn_dtype dtype, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_dtype(dtype));
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{T, "T"}, {K, "K"}, {V, "V"}, {beta, "beta"}, {W, "W"}, {U, "U"}}));
+    GDN_TRY(check_opt_ptr(g, "g"));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == GDN_BF16 && gdn::tc_available())
+        return launched(gdn::launch_wy_tc(T, K, V, beta, g, W, U, nc, s.k, st), "wy (tcgen05)");
+    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "wy: k=256 needs the bf16 tensor-core path");
+    return launched(gdn::launch_wy_simt(T, K, V, beta, g, W, U, nc, s.k, dtype == GDN_BF16, st),
+                    "wy");
+}
+
+int gdn_invert_neumann_i8(const float* A, float* T, int N, int mask, int8_t* q_dbg,
+                          int32_t* acc_dbg, float* scale_dbg, gdn_shape s, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    if (s.k != 64) return fail(GDN_ERR_UNSUPPORTED, "INT8 path is built for k=64");
+    if (N < 1 || N > 8) return fail(GDN_ERR_ARG, "INT8 path: N=%d outside [1, 8]", N);
+    if (mask != 0 && mask != 1) return fail(GDN_ERR_ARG, "mask must be 0 or 1");
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    GDN_TRY(check_opt_ptr(q_dbg, "q_dbg"));
+    GDN_TRY(check_opt_ptr(acc_dbg, "acc_dbg"));
+    GDN_TRY(check_opt_ptr(scale_dbg, "scale_dbg"));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (gdn::tc_available())
+        return launched(gdn::launch_neumann_i8_tc(A, T, N, mask, q_dbg, acc_dbg, scale_dbg, nc, st),
+                        "neumann_i8 (tcgen05)");
+    return launched(gdn::launch_neumann_i8_simt(A, T, N, mask, q_dbg, acc_dbg, scale_dbg, nc, st),
+                    "neumann_i8");
+}
+
+int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta, const float* g, int N,
+                       int mask, int S, int gated, void* W, void* U, float* T_out, gdn_shape s,
+                       gdn_dtype dtype, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_dtype(dtype));
+    GDN_TRY(check_NS(N, mask, S, s.k));
+    if (gated != 0 && gated != 1) return fail(GDN_ERR_ARG, "gated must be 0 or 1");
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{K, "K"}, {V, "V"}, {beta, "beta"}, {g, "g"}, {W, "W"}, {U, "U"}}));
+    GDN_TRY(check_opt_ptr(T_out, "T_out"));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (dtype == GDN_BF16 && gdn::tc_available()) {
+        if (s.k == 256 && !(mask == 1 && S == 0))
+            return fail(GDN_ERR_UNSUPPORTED, "k=256 on tensor cores supports mask=1, S=0 only");
+        return launched(gdn::launch_fused_tc(K, V, beta, g, N, mask, S, gated, W, U, T_out, nc,
+                                             s.k, st),
+                        "chunk_wy_fused (tcgen05)");
+    }
+    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "fused CUDA-core path supports k <= 128");
+    return launched(gdn::launch_fused_simt(K, V, beta, g, N, mask, S, gated, W, U, T_out, nc,
+                                           s.k, dtype == GDN_BF16, st),
+                    "chunk_wy_fused");
+}
+
+int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype) {
+    int64_t nc;
+    if (check_shape(s, &nc) != GDN_OK) return -1;
+    const int64_t elem = dtype == GDN_BF16 ? 2 : 4;
+    return 2 * nc * (int64_t)s.k * s.d * elem;
+}
+
+int gdn_forward(const void* Q, const void* K, const void* V, const float* beta, const float* g,
+                const float* S0, int N, int mask, int S, int exact, void* O, float* S_final,
+                void* workspace, int64_t workspace_bytes, gdn_shape s, gdn_dtype dtype,
+                void* stream) {
+    (void)Q; (void)K; (void)V; (void)beta; (void)g; (void)S0; (void)N; (void)mask; (void)S;
+    (void)exact; (void)O; (void)S_final; (void)workspace; (void)workspace_bytes; (void)s;
+    (void)dtype; (void)stream;
+    return fail(GDN_ERR_UNSUPPORTED, "gdn_forward is not built yet");
+}
+
+int gdn_get_status(void* stream) {
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronise");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, gdn::g_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "read status");
+    const int z = 0;
+    e = cudaMemcpyToSymbol(gdn::g_status, &z, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status");
+    if (v & gdn::kStatusTimeout) return fail(GDN_ERR_TIMEOUT, "a bounded device wait ran out");
+    return GDN_OK;
+}
+
+const char* gdn_last_error(void) { return t_last_error.c_str(); }
+
+int64_t gdn_launch_count(void) { return t_launches; }
+
+}  // extern "C"
+
+// Device address of the status word for kernels in other translation units.
+namespace gdn {
+int* status_ptr() {
+    static thread_local int dev = -1;
+    static thread_local int* ptr = nullptr;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (cur != dev || !ptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        ptr = (int*)p;
+        dev = cur;
+    }
+    return ptr;
+}
+}  // namespace gdn

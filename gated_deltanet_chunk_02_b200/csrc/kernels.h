@@ -1,0 +1,24 @@
+// kernels.h — internal launchers of libgdn (host side, not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// CUDA-core kernels (simt.cu); k in {32, 64, 128} unless stated.
+cudaError_t launch_build_A_simt(const void* K, const float* beta, const float* g, float* A,
+                                int64_t nc, int k, bool bf16, cudaStream_t st);
+cudaError_t launch_neumann_simt(const float* A, float* T, int64_t nc, int k, int N, int mask,
+                                int S, cudaStream_t st);
+cudaError_t launch_wy_simt(const float* T, const void* K, const void* V, const float* beta,
+                           const float* g, void* W, void* U, int64_t nc, int k, bool bf16,
+                           cudaStream_t st);
+cudaError_t launch_fused_simt(const void* K, const void* V, const float* beta, const float* g,
+                              int N, int mask, int S, int gated, void* W, void* U, float* Tout,
+                              int64_t nc, int k, bool bf16, cudaStream_t st);
+cudaError_t launch_fwdsub(const float* A, float* T, int64_t nc, int k, cudaStream_t st);  // k <= 256
+cudaError_t launch_neumann_i8_simt(const float* A, float* T, int N, int mask, int8_t* q,
+                                   int32_t* acc, float* sc, int64_t nc, cudaStream_t st);
+
+}  // namespace gdn

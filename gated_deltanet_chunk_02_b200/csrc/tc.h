@@ -1,0 +1,24 @@
+// tc.h — internal launchers of the tcgen05 (tensor-core) kernels of libgdn.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+int* status_ptr();     // device address of the status word (api.cu)
+bool tc_available();   // true when this build carries the sm_100a tensor-core kernels
+
+cudaError_t launch_build_A_tc(const void* K, const float* beta, const float* g, float* A,
+                              int64_t nc, int k, cudaStream_t st);
+cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int S,
+                              cudaStream_t st);
+cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const float* beta,
+                         const float* g, void* W, void* U, int64_t nc, int k, cudaStream_t st);
+cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8_t* q,
+                                 int32_t* acc, float* sc, int64_t nc, cudaStream_t st);
+cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, const float* g,
+                            int N, int mask, int S, int gated, void* W, void* U, float* Tout,
+                            int64_t nc, int k, cudaStream_t st);
+
+}  // namespace gdn

@@ -1,0 +1,171 @@
+/*
+ * gdn.h — C ABI of libgdn: the per-chunk hot path of chunk-wise Gated DeltaNet
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method: "When Good Enough Is Optimal: Multiplication-Only Matrix
+ * Inversion Approximation for Quantized Gated DeltaNet" (arXiv 2606.06034),
+ * as summarised on gist.science (sections "Énoncé du Problème",
+ * "Méthodologie" §1-§3, "Adaptation à la Quantification").  Each chunk of k
+ * tokens needs T = (I - A)^{-1} for a strictly lower-triangular A; T is
+ * approximated with matrix products only (truncated Neumann series, a
+ * structural band mask and a parallel residual correction) and then applied
+ * to form the WY factors.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.  Head-major and chunk-contiguous: K, V, Q, W, U, O are
+ *   [B, H, T, d] row-major (d = 128); beta, g are [B, H, T] float32;
+ *   A, T are [B, H, T/k, k, k] float32 row-major.  Chunk c of the flattened
+ *   [B*H*T/k] sequence owns rows [c*k, (c+1)*k) of every [.., T, ..] array.
+ *   nc = B*H*T/k is the number of chunks.
+ * Pointers.  All data pointers are DEVICE pointers owned by the caller, who
+ *   allocates them; the library never allocates device memory in a call.
+ *   Every pointer must be 16-byte aligned (tensor-memory-access rule).
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Every call is asynchronous on that stream; none synchronises,
+ *   except gdn_get_status.
+ * Errors.  Arguments are checked on the host before any launch; a failing
+ *   check returns a negative code, launches nothing and records a message for
+ *   gdn_last_error().  Device-side failures (a bounded wait that ran out) set a
+ *   per-device status word read by gdn_get_status(); kernels never trap.
+ * Values.  NaN/Inf inputs are not checked.  g must be the chunk-local
+ *   cumulative sum of the per-token log-gates (g_i includes token i's gate);
+ *   within a chunk g is then non-increasing, and exp(g_i - g_j) is evaluated
+ *   only for i > j, so it never overflows.
+ * Precision.  A and T are float32 in memory.  `dtype` fixes the type of
+ *   K, V, Q, W, U, O.  bf16 data run their contractions on the tcgen05 tensor
+ *   cores (bf16 x bf16 for K K^T and WY, fp16 x fp16 for the k x k chain, all
+ *   accumulating in fp32); float32 data run on CUDA cores in fp32.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct gdn_shape {
+    int64_t B, H, T;   /* batch, heads, tokens per sequence (T % k == 0)   */
+    int32_t k;         /* chunk size: 32, 64, 128 or 256                    */
+    int32_t d;         /* head dim d_k = d_v; 128 is the supported value    */
+} gdn_shape;
+
+typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Arithmetic of the k x k product chain in gdn_invert_neumann. */
+typedef enum gdn_prec {
+    GDN_PREC_F32 = 0,  /* float32 FMA on CUDA cores (k <= 128)               */
+    GDN_PREC_F16 = 1   /* tcgen05 tensor cores, fp16 operands, fp32 accumulate */
+} gdn_prec;
+
+enum {
+    GDN_OK = 0,
+    GDN_ERR_ARG = -1,          /* null pointer, bad size, N/S out of range   */
+    GDN_ERR_ALIGN = -2,        /* a pointer is not 16-byte aligned           */
+    GDN_ERR_UNSUPPORTED = -3,  /* valid request this build does not serve    */
+    GDN_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed          */
+    GDN_ERR_TIMEOUT = -5       /* device status: a bounded wait ran out      */
+};
+
+/*
+ * A_ij = -beta_i (k_i . k_j) exp(g_i - g_j) for i > j, 0 for i <= j, per chunk.
+ * The summary's problem statement ("Énoncé du Problème") fixes A as strictly
+ * lower triangular; its entries are those of the gated delta-rule chunk
+ * system.  In: K [B,H,T,d] (dtype), beta, g [B,H,T] f32.  Out: A [nc,k,k] f32.
+ */
+int gdn_build_A(const void* K, const float* beta, const float* g, float* A,
+                gdn_shape s, gdn_dtype dtype, void* stream);
+
+/*
+ * Multiplication-only approximate inverse T ~ (I - A)^{-1} per chunk
+ * ("Méthodologie" §1-§3): T0 = sum_{n=0}^{N} A^n (N >= 1 highest power), with
+ * the band mask M_ij = [i - j <= N] applied to every power when mask != 0;
+ * then, if S > 0, E = I - (I - A) T0 and T = T0 sum_{s=0}^{S} E^s (S >= 0).
+ * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.  1 <= N <= k-1, 0 <= S <= 64.
+ * GDN_PREC_F16 at k = 256 supports mask = 1 with S = 0 only.
+ */
+int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask,
+                       int S, gdn_prec prec, void* stream);
+
+/*
+ * Exact T = (I - A)^{-1} by forward substitution ("Énoncé du Problème": the
+ * k-1 sequential row steps the method replaces).  fp32 on CUDA cores.
+ * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.
+ */
+int gdn_invert_fwdsub(const float* A, float* T, gdn_shape s, void* stream);
+
+/*
+ * WY factors W = T diag(beta) K and U = T diag(beta) V per chunk.  If g is
+ * non-NULL, W is the gated factor T diag(beta * exp(g)) K used by the chunk
+ * recurrence (U unchanged).  In: T [nc,k,k] f32, K, V [B,H,T,d] (dtype),
+ * beta, g [B,H,T] f32.  Out: W, U [B,H,T,d] (dtype).
+ */
+int gdn_wy(const float* T, const void* K, const void* V, const float* beta,
+           const float* g, void* W, void* U, gdn_shape s, gdn_dtype dtype,
+           void* stream);
+
+/*
+ * INT8 truncated Neumann series ("Adaptation à la Quantification"): A and every
+ * power held as int8 codes with one symmetric fp32 scale per chunk and power,
+ * int32 accumulation on the tensor cores, band mask applied to each power
+ * before it is quantised, dequantised T0 = I + sum_n s_n q_n in fp32.  The
+ * fixed float32 operation order (IEEE, round-to-nearest-even, no FMA) is:
+ *   P1 = M.A; a = max|P1|; q1 = clamp(rint(P1 * (127/a)), +-127); s1 = a/127;
+ *   acc_n = q_{n-1} q1 (masked); m = max|acc_n|;
+ *   q_n = clamp(rint(float(acc_n) * (127/float(m))), +-127);
+ *   s_n = (s_{n-1} * s1) * (float(m)/127); zero maxima give q = 0, s = 0;
+ *   T0 = I + s_1 q_1 + ... + s_N q_N, summed left to right.
+ * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.  Optional debug outputs (NULL to
+ * skip): q [nc,N,k,k] int8, acc [nc,N,k,k] int32 (slot 0 zero), scale [nc,N]
+ * f32.  k = 64, 1 <= N <= 8.
+ */
+int gdn_invert_neumann_i8(const float* A, float* T, int N, int mask,
+                          int8_t* q_dbg, int32_t* acc_dbg, float* scale_dbg,
+                          gdn_shape s, void* stream);
+
+/*
+ * Fused per-chunk pipeline: A from K, beta, g; T by the Neumann + mask +
+ * residual method (as gdn_invert_neumann); then W, U (gated W if gated != 0).
+ * Only K, V, beta, g are read and only W, U (and T when T_out is non-NULL)
+ * written.  bf16: tensor-core path; f32: CUDA-core path (k <= 128).
+ */
+int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta,
+                       const float* g, int N, int mask, int S, int gated,
+                       void* W, void* U, float* T_out, gdn_shape s,
+                       gdn_dtype dtype, void* stream);
+
+/*
+ * Full chunk-wise Gated DeltaNet forward.  Per chunk: V~ = U - W_g S0^T,
+ * O = diag(exp g) Q S0^T + (Q K^T . Gamma . L) V~,
+ * S' = exp(g_last) S0 + V~^T diag(exp(g_last - g)) K, with
+ * Gamma_ij = exp(g_i - g_j) and L the lower triangle with diagonal.  T per
+ * chunk comes from the Neumann method (exact = 0) or forward substitution
+ * (exact = 1).  In: Q, K, V [B,H,T,d] (dtype), beta, g [B,H,T] f32, S0
+ * [B,H,d,d] f32 (d_v x d_k, NULL = zero).  Out: O [B,H,T,d] (dtype),
+ * S_final [B,H,d,d] f32.  `workspace` is caller-owned device memory of at
+ * least gdn_forward_workspace_bytes(s, dtype) bytes (W_g and U for every
+ * chunk); its contents on entry do not matter.
+ */
+int gdn_forward(const void* Q, const void* K, const void* V, const float* beta,
+                const float* g, const float* S0, int N, int mask, int S,
+                int exact, void* O, float* S_final, void* workspace,
+                int64_t workspace_bytes, gdn_shape s, gdn_dtype dtype,
+                void* stream);
+int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype);
+
+/* Synchronises `stream`, returns the device status word of the current
+ * device (GDN_OK or GDN_ERR_TIMEOUT) and clears it. */
+int gdn_get_status(void* stream);
+
+/* Message for the most recent nonzero return on this host thread. */
+const char* gdn_last_error(void);
+
+/* Number of kernels this library launched on this host thread since load. */
+int64_t gdn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_H */

@@ -1,0 +1,187 @@
+"""GPU parity: every C-ABI entry point against the CPU oracle, element by element,
+on the same seeded inputs.
+
+Tolerances (relative Frobenius error per output tensor): 1e-5 for float32
+data (float32 arithmetic), 1e-2 for bf16 data (tensor-core products with fp32
+accumulation); the INT8 codes, accumulators, scales and the dequantised T are
+compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gated_deltanet_chunk_02_b200 import gdn
+from gated_deltanet_chunk_02_b200.inputs import Workload, make_inputs
+
+from helpers import (TOL_F32, A_tensor, chunked, oracle_A32, per_chunk_max_rel, rel, to_dev,
+                     tol_for)
+
+pytestmark = pytest.mark.gpu
+
+
+def dev_inputs(inp):
+    return {k: to_dev(v) for k, v in inp.items()}
+
+
+def check_status():
+    assert gdn.gdn_get_status() == gdn.GDN_OK
+
+
+# --------------------------------------------------------------------------- #
+# A
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("k", [32, 64, 128])
+def test_build_A(dtype, k):
+    w = Workload(B=1, H=3, T=4 * k, k=k, dtype=dtype)        # 12 chunks
+    inp = make_inputs(w, seed=1)
+    d = dev_inputs(inp)
+    A = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_build_A(d["K"], d["beta"], d["g"], A, k)
+    check_status()
+    c = chunked(inp, w)
+    ref = O.build_A(c["K"], c["beta"], c["g"])
+    assert rel(A, ref) <= tol_for(dtype) * (0.1 if dtype == "bf16" else 1)
+    Ah = A.cpu().numpy().reshape(ref.shape)
+    assert np.all(np.triu(Ah) == 0)
+
+
+# --------------------------------------------------------------------------- #
+# inverses
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("k", [32, 64, 128, 256])
+def test_fwdsub(k):
+    w = Workload(B=1, H=2, T=3 * k, k=k, dtype="f32")
+    A32 = oracle_A32(make_inputs(w, seed=2), w)
+    T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_invert_fwdsub(to_dev(A_tensor(A32, w)), T)
+    check_status()
+    ref = O.invert_fwdsub(A32.astype(np.float64))
+    assert rel(T, ref) <= TOL_F32
+    assert per_chunk_max_rel(T, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("k", [32, 64, 128])
+@pytest.mark.parametrize("N", [1, 2, 3, 4])
+@pytest.mark.parametrize("mask", [0, 1])
+@pytest.mark.parametrize("S", [0, 1, 8])
+def test_neumann_f32(k, N, mask, S):
+    w = Workload(B=1, H=2, T=2 * k, k=k, dtype="f32")
+    A32 = oracle_A32(make_inputs(w, seed=3), w)
+    T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_invert_neumann(to_dev(A_tensor(A32, w)), T, N, mask, S, gdn.GDN_PREC_F32)
+    check_status()
+    ref = O.invert_neumann(A32.astype(np.float64), N, bool(mask), S)
+    assert rel(T, ref) <= TOL_F32
+
+
+# --------------------------------------------------------------------------- #
+# WY
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("k", [32, 64, 128])
+@pytest.mark.parametrize("gated", [False, True])
+def test_wy(dtype, k, gated):
+    w = Workload(B=1, H=2, T=3 * k, k=k, dtype=dtype)
+    inp = make_inputs(w, seed=4)
+    d = dev_inputs(inp)
+    c = chunked(inp, w)
+    T32 = O.invert_fwdsub(O.build_A(c["K"], c["beta"], c["g"])).astype(np.float32)
+    Td = to_dev(A_tensor(T32, w))
+    W = torch.empty_like(d["K"])
+    U = torch.empty_like(d["V"])
+    gdn.gdn_wy(Td, d["K"], d["V"], d["beta"], d["g"] if gated else None, W, U)
+    check_status()
+    Wr, Ur = O.wy(T32.astype(np.float64), c["K"], c["V"], c["beta"], c["g"] if gated else None)
+    assert rel(W, Wr) <= tol_for(dtype)
+    assert rel(U, Ur) <= tol_for(dtype)
+
+
+# --------------------------------------------------------------------------- #
+# fused
+# --------------------------------------------------------------------------- #
+def fused_reference(c, N, mask, S, gated):
+    A = O.build_A(c["K"], c["beta"], c["g"])
+    T = O.invert_neumann(A, N, bool(mask), S)
+    W, U = O.wy(T, c["K"], c["V"], c["beta"], c["g"] if gated else None)
+    return T, W, U
+
+
+@pytest.mark.parametrize("S", [0, 8])
+def test_fused_c1_f32(S):
+    """B=1, H=1, T=256, k=64 (4 chunks), float32, N=3 with mask, seed 0."""
+    w = Workload(B=1, H=1, T=256, k=64, dtype="f32")
+    inp = make_inputs(w, seed=0)
+    d = dev_inputs(inp)
+    W = torch.empty_like(d["K"])
+    U = torch.empty_like(d["V"])
+    T = torch.empty(1, 1, 4, 64, 64, device="cuda")
+    gdn.gdn_chunk_wy_fused(d["K"], d["V"], d["beta"], d["g"], 3, 1, S, 0, W, U, T, k=64)
+    check_status()
+    Tr, Wr, Ur = fused_reference(chunked(inp, w), 3, 1, S, False)
+    assert rel(T, Tr) <= TOL_F32
+    assert rel(W, Wr) <= TOL_F32
+    assert rel(U, Ur) <= TOL_F32
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("k", [32, 64, 128])
+@pytest.mark.parametrize("N,mask,S,gated", [(3, 1, 8, False), (2, 0, 0, True), (4, 1, 1, False),
+                                            (1, 1, 3, True)])
+def test_fused_small(dtype, k, N, mask, S, gated):
+    w = Workload(B=1, H=3, T=3 * k, k=k, dtype=dtype)       # 9 chunks: ragged vs any pairing
+    inp = make_inputs(w, seed=5)
+    d = dev_inputs(inp)
+    W = torch.empty_like(d["K"])
+    U = torch.empty_like(d["V"])
+    T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_chunk_wy_fused(d["K"], d["V"], d["beta"], d["g"], N, mask, S, int(gated), W, U, T, k=k)
+    check_status()
+    Tr, Wr, Ur = fused_reference(chunked(inp, w), N, mask, S, gated)
+    tol = tol_for(dtype)
+    assert rel(T, Tr) <= tol
+    assert rel(W, Wr) <= tol
+    assert rel(U, Ur) <= tol
+    assert per_chunk_max_rel(W, Wr.reshape(Wr.shape[0], -1)) <= 2 * tol
+
+
+def test_fused_without_T_output_matches():
+    w = Workload(B=2, H=2, T=256, k=64, dtype="bf16")
+    inp = make_inputs(w, seed=6)
+    d = dev_inputs(inp)
+    W1, U1, W2, U2 = (torch.empty_like(d["K"]) for _ in range(4))
+    T = torch.empty(2, 2, 4, 64, 64, device="cuda")
+    gdn.gdn_chunk_wy_fused(d["K"], d["V"], d["beta"], d["g"], 3, 1, 8, 0, W1, U1, T, k=64)
+    gdn.gdn_chunk_wy_fused(d["K"], d["V"], d["beta"], d["g"], 3, 1, 8, 0, W2, U2, None, k=64)
+    check_status()
+    assert torch.equal(W1, W2) and torch.equal(U1, U2)
+
+
+# --------------------------------------------------------------------------- #
+# INT8
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("N", [1, 2, 3, 4])
+@pytest.mark.parametrize("mask", [0, 1])
+def test_int8_bit_exact(N, mask):
+    w = Workload(B=1, H=4, T=1024, k=64, dtype="bf16")        # 64 chunks
+    A32 = oracle_A32(make_inputs(w, seed=7), w)
+    nc = A32.shape[0]
+    Ad = to_dev(A_tensor(A32, w))
+    T = torch.empty_like(Ad)
+    q = torch.empty(nc, N, 64, 64, dtype=torch.int8, device="cuda")
+    acc = torch.empty(nc, N, 64, 64, dtype=torch.int32, device="cuda")
+    sc = torch.empty(nc, N, dtype=torch.float32, device="cuda")
+    gdn.gdn_invert_neumann_i8(Ad, T, N, mask, q, acc, sc)
+    check_status()
+    r = O.int8_neumann(A32, N, bool(mask))
+    np.testing.assert_array_equal(q.cpu().numpy(), r["q"])
+    np.testing.assert_array_equal(acc.cpu().numpy(), r["acc"])
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), r["scale"].view(np.uint32))
+    np.testing.assert_array_equal(T.cpu().numpy().reshape(nc, 64, 64).view(np.uint32),
+                                  r["T"].view(np.uint32))
+    # without the debug outputs the same T comes out
+    T2 = torch.empty_like(Ad)
+    gdn.gdn_invert_neumann_i8(Ad, T2, N, mask)
+    check_status()
+    assert torch.equal(T, T2)
