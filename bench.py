@@ -20,7 +20,6 @@ import argparse
 import hashlib
 import json
 import os
-import subprocess
 import sys
 import threading
 import time
@@ -85,62 +84,86 @@ def recorded_traffic(kernel: str) -> float | None:
 
 
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML
+    every ~2 ms while the timed region runs (reading only; no setting is
+    touched)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown")]
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines: list[str] = []
-        self.thread = None
+        self.period = period_s
+        self.samples: list[tuple[int, int]] = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            h = pynvml.nvmlDeviceGetHandleByIndex(self._physical_index())
+            self._h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception:            # NVML missing: report no samples
+            self._nvml = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _physical_index(self) -> int:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                return int(vis.split(",")[self.gpu])
+            except (ValueError, IndexError):
+                pass
+        return self.gpu
+
+    def _sample(self):
+        n = self._nvml
+        mhz = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+        rs = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        self.samples.append((mhz, rs))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                break
+            time.sleep(self.period)
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+        if self._nvml is not None:
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-            if self.thread is not None:
-                self.thread.join(timeout=2)
+                self._sample()
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = sorted(m for m, _ in self.samples)
+        reasons = set()
+        for _, rs in self.samples:
+            for name, const in self.REASONS:
+                bit = getattr(self._nvml, const, 0) if self._nvml else 0
+                if rs & bit:
                     reasons.add(name)
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(mhz)}
 
 
 def dist_setup():
@@ -225,24 +248,27 @@ def run_reference(args, world, rank):
     return 0
 
 
-def workload_config(w: dict, nc: int) -> dict:
+def workload_config(w: dict, nc: int, rotate: int = ROTATE) -> dict:
     return {"workload": "fused chunk inverse+WY (A=KK^T gated, Neumann N=3 + band mask, "
                         "S=8 residual, W/U), B=4 H=16 T=4096 k=64 d=128 bf16",
             "B": w["B"], "H": w["H"], "T": w["T"], "k": w["k"], "d": w["d"], "N": w["N"],
             "mask": w["mask"], "S": w["S"], "chunks": nc,
-            "l2": f"inputs larger than L2: {ROTATE} rotating input/output sets of 270 MB"}
+            "l2": f"inputs larger than L2: {rotate} rotating input/output sets of 270 MB"}
 
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sample-chunks", type=int, default=512,
                     help="chunks per step for the CPU oracle timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling)")
+    ap.add_argument("--rotate", type=int, default=ROTATE,
+                    help="input/output sets cycled through the timed steps")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -267,7 +293,7 @@ def main(argv=None) -> int:
     k, d = w["k"], w["d"]
     elem = 2
     sets = []
-    for r in range(ROTATE):
+    for r in range(args.rotate):
         inp = make_inputs(wl, seed=1000 * rank + r)
         s = {key: inp[key].to(dev) for key in ("K", "V", "beta", "g")}
         s["W"] = torch.empty_like(s["K"])
@@ -276,7 +302,7 @@ def main(argv=None) -> int:
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
-        s = sets[i % ROTATE]
+        s = sets[i % len(sets)]
         gdn.gdn_chunk_wy_fused(s["K"], s["V"], s["beta"], s["g"], w["N"], w["mask"], w["S"],
                                w["gated"], s["W"], s["U"], None, k=k, stream=stream)
 
@@ -304,6 +330,8 @@ def main(argv=None) -> int:
     assert status == gdn.GDN_OK, status
 
     # end to end through the public API: pinned host inputs in, host outputs back
+    if args.no_e2e:
+        args.e2e_steps = 0
     host = {key: sets[0][key].cpu().pin_memory() for key in ("K", "V", "beta", "g")}
     hostW = torch.empty(sets[0]["W"].shape, dtype=sets[0]["W"].dtype).pin_memory()
     hostU = torch.empty_like(hostW).pin_memory()
@@ -317,7 +345,7 @@ def main(argv=None) -> int:
         hostW.copy_(dbuf["W"], non_blocking=True)
         hostU.copy_(dbuf["U"], non_blocking=True)
 
-    for _ in range(3):
+    for _ in range(3 if args.e2e_steps else 0):
         e2e_step()
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -328,7 +356,7 @@ def main(argv=None) -> int:
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / max(args.e2e_steps, 1), world, dev)
     h2d = sum(host[key].numel() * host[key].element_size() for key in host)
     d2h = 2 * hostW.numel() * hostW.element_size()
 
@@ -357,7 +385,7 @@ def main(argv=None) -> int:
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": workload_config(w, nc),
+        "config": workload_config(w, nc, args.rotate),
         "roofline": {
             "bound": bound,
             "achieved": achieved_gbs if bound == "hbm" else tflops,
@@ -374,8 +402,9 @@ def main(argv=None) -> int:
             "flops_per_launch": flops_per_launch,
         },
         "clocks": clocks.summary(),
-        "e2e": {"value": nc * world / (e2e_ms * 1e-3), "unit": "chunks/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": ({"value": nc * world / (e2e_ms * 1e-3), "unit": "chunks/s",
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                if args.e2e_steps else None),
         "gpu_launches": launches,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -163,7 +163,7 @@ int gdn_invert_neumann_i8(const float* A, float* T, int N, int mask, int8_t* q_d
     GDN_TRY(check_opt_ptr(acc_dbg, "acc_dbg"));
     GDN_TRY(check_opt_ptr(scale_dbg, "scale_dbg"));
     cudaStream_t st = (cudaStream_t)stream;
-    if (gdn::tc_available())
+    if (gdn::tc_i8_available())
         return launched(gdn::launch_neumann_i8_tc(A, T, N, mask, q_dbg, acc_dbg, scale_dbg, nc, st),
                         "neumann_i8 (tcgen05)");
     return launched(gdn::launch_neumann_i8_simt(A, T, N, mask, q_dbg, acc_dbg, scale_dbg, nc, st),

@@ -7,7 +7,8 @@
 namespace gdn {
 
 int* status_ptr();     // device address of the status word (api.cu)
-bool tc_available();   // true when this build carries the sm_100a tensor-core kernels
+bool tc_available();     // true when this build carries the sm_100a tensor-core kernels
+bool tc_i8_available();  // true when the INT8 tensor-core kernel is built
 
 cudaError_t launch_build_A_tc(const void* K, const float* beta, const float* g, float* A,
                               int64_t nc, int k, cudaStream_t st);

@@ -14,7 +14,7 @@ import oracle as O
 from gated_deltanet_chunk_02_b200 import gdn
 from gated_deltanet_chunk_02_b200.inputs import Workload, make_inputs
 
-from helpers import (TOL_F32, A_tensor, chunked, oracle_A32, per_chunk_max_rel, rel, to_dev,
+from helpers import (TOL_BF16, TOL_F32, A_tensor, chunked, oracle_A32, per_chunk_max_rel, rel, to_dev,
                      tol_for)
 
 pytestmark = pytest.mark.gpu
@@ -185,3 +185,25 @@ def test_int8_bit_exact(N, mask):
     gdn.gdn_invert_neumann_i8(Ad, T2, N, mask)
     check_status()
     assert torch.equal(T, T2)
+
+
+@pytest.mark.parametrize("k", [32, 64, 128])
+@pytest.mark.parametrize("N", [1, 2, 3, 4])
+@pytest.mark.parametrize("mask", [0, 1])
+@pytest.mark.parametrize("S", [0, 1, 2, 8])
+def test_neumann_tensor_cores(k, N, mask, S):
+    """The tcgen05 chain (fp16 operands, fp32 accumulation) on 9 chunks."""
+    w = Workload(B=1, H=3, T=3 * k, k=k, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=8), w)
+    T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_invert_neumann(to_dev(A_tensor(A32, w)), T, N, mask, S, gdn.GDN_PREC_F16)
+    check_status()
+    ref = O.invert_neumann(A32.astype(np.float64), N, bool(mask), S)
+    assert rel(T, ref) <= TOL_BF16
+    assert per_chunk_max_rel(T, ref) <= TOL_BF16
+    Th = T.cpu().numpy().reshape(ref.shape)
+    assert np.all(np.triu(Th, 1) == 0)                       # strictly lower + unit diagonal
+    if mask:
+        dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+        if S == 0:
+            assert np.all(Th[:, dist > N] == 0)
