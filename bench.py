@@ -249,8 +249,9 @@ def run_reference(args, world, rank):
 
 
 def workload_config(w: dict, nc: int, rotate: int = ROTATE) -> dict:
-    return {"workload": "fused chunk inverse+WY (A=KK^T gated, Neumann N=3 + band mask, "
-                        "S=8 residual, W/U), B=4 H=16 T=4096 k=64 d=128 bf16",
+    mask = "band mask" if w["mask"] else "no mask"
+    return {"workload": f"fused chunk inverse+WY (A=KK^T gated, Neumann N={w['N']} + {mask}, "
+                        f"S={w['S']} residual, W/U), B=4 H=16 T=4096 k=64 d=128 bf16",
             "B": w["B"], "H": w["H"], "T": w["T"], "k": w["k"], "d": w["d"], "N": w["N"],
             "mask": w["mask"], "S": w["S"], "chunks": nc,
             "l2": f"inputs larger than L2: {rotate} rotating input/output sets of 270 MB"}
@@ -267,6 +268,9 @@ def main(argv=None) -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (profiling)")
+    ap.add_argument("--N", type=int, default=WORKLOAD["N"], help="Neumann order")
+    ap.add_argument("--S", type=int, default=WORKLOAD["S"], help="residual steps")
+    ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="input/output sets cycled through the timed steps")
     args = ap.parse_args(argv)
@@ -287,7 +291,7 @@ def main(argv=None) -> int:
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = dict(WORKLOAD)
+    w = dict(WORKLOAD, N=args.N, S=args.S, mask=args.mask)
     wl = Workload(B=w["B"], H=w["H"], T=w["T"], k=w["k"], d=w["d"], dtype=w["dtype"])
     nc = wl.n_chunks
     k, d = w["k"], w["d"]

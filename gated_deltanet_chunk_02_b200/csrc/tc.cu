@@ -5,23 +5,27 @@
 // WY alone.  Design:
 //
 // * A "tile" is 128 consecutive rows of the flattened [B*H*T, d] arrays, i.e.
-//   128/KB chunks of KB tokens (KB = 64 or 128; k = 32 is run as 64-token
-//   blocks holding two 32-token chunks block-diagonally).  Every k x k product
-//   of the method is one M=128 tcgen05.mma over the tile: the left operand
-//   stacks the tile's chunks along M, the right operand places them side by
-//   side along N, and each chunk reads only its own diagonal block of the
-//   128 x 128 fp32 accumulator in tensor memory (TMEM).
-// * Warp 0 is the TMA producer (K, V tiles with 128-byte swizzle, beta and g).
-//   Each further 4-warp group ("slot") owns one tile at a time: one elected
-//   thread issues its MMAs, all 128 threads run the epilogues (TMEM -> registers
-//   -> mask / accumulate / convert -> swizzled shared-memory operand).  Two slots
-//   per CTA keep the tensor pipe busy while the other slot's epilogue runs.
-// * Thread r of a slot owns row r of the tile: the TMEM lane it may read
-//   (lane quarter = warp % 4) is the row it computes.
-// * The WY step is computed transposed, W^T = K^T (T diag(beta))^T, so that it
-//   is a full-rate M=128 (= d) product; its epilogue writes W, U row-wise.
-// * Every wait is bounded (2 s); on expiry the kernel sets the status word,
-//   stops issuing work, waits for its own copies/MMAs (bounded) and frees TMEM.
+//   128/KB blocks of KB tokens (KB = 64 or 128; chunks of k = 32 run as 64-token
+//   blocks holding two chunks block-diagonally).  Every k x k product of the
+//   method is ONE M=128 tcgen05.mma over the tile: the left operand stacks the
+//   tile's blocks along M, the right operand places them side by side along N,
+//   and each row reads only its own diagonal block of the 128 x 128 fp32
+//   accumulator in tensor memory (TMEM).
+// * Warp 0 is the TMA producer: K and V tiles (128-byte swizzle), beta and g.
+//   Each "slot" of 8 warps owns one tile at a time; its elected thread issues
+//   the tile's MMAs and TMA stores, and its 256 threads run the epilogues
+//   (TMEM -> registers -> mask / accumulate / convert -> swizzled shared-memory
+//   operand).  Thread (r, h) owns row r of the tile (its TMEM lane; the lane
+//   quarter is warp % 4) and the column half h.  Two slots per CTA keep the
+//   tensor pipe busy while the other slot runs an epilogue.
+// * T0 (then T) stays in TMEM columns [128, 128 + KB) of the slot, next to the
+//   product accumulator in columns [0, 128).
+// * WY is computed transposed, W^T = K^T (T diag(beta))^T, a full-rate M=128
+//   (= d) product; its epilogue transposes through the (now free) K/V tiles in
+//   shared memory and leaves with TMA bulk stores.
+// * Every wait is bounded (2 s).  On expiry the kernel sets the status word,
+//   stops issuing work, waits (bounded) for its own copies and MMAs and frees
+//   TMEM before returning.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -33,25 +37,29 @@ namespace tcg {
 constexpr int kD = 128;
 constexpr int kRows = 128;                       // rows per tile
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
+constexpr int kStatusSmemAlign = 2;              // dynamic shared memory not 1024-aligned
 
 enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3 };
 
 __host__ __device__ constexpr bool uses_K(int m) { return m == kFused || m == kBuildA || m == kWY; }
 __host__ __device__ constexpr bool uses_V(int m) { return m == kFused || m == kWY; }
-__host__ __device__ constexpr bool uses_ops(int m) { return m != kBuildA; }
+__host__ __device__ constexpr int block_of(int kc) { return kc < 64 ? 64 : kc; }
 
-// Per-slot shared-memory layout (bytes); every region is 1024-byte aligned.
+// Per-slot shared-memory layout (bytes).  The 1024-byte aligned operand
+// regions of all slots come first, then each slot's beta/g, then control.
 template <int KB, int MODE>
 struct SlotLayout {
     static constexpr int kK = uses_K(MODE) ? kRows * kD * 2 : 0;        // bf16 [2][128][64]
     static constexpr int kV = uses_V(MODE) ? kRows * kD * 2 : 0;
-    static constexpr int kOp = uses_ops(MODE) ? kRows * KB * 2 : 0;     // 16-bit [KB/64][128][64]
+    static constexpr int kAop = (MODE == kFused || MODE == kNeumann) ? kRows * KB * 2 : 0;
+    static constexpr int kXY = (MODE == kBuildA) ? 0 : kRows * KB * 2;  // 16-bit [KB/64][128][64]
     static constexpr int offK = 0;
     static constexpr int offV = offK + kK;
     static constexpr int offAop = offV + kV;
-    static constexpr int offX = offAop + (MODE == kWY ? 0 : kOp);
-    static constexpr int offY = offX + kOp;
-    static constexpr int bytes = offY + kOp;
+    static constexpr int offX = offAop + kAop;
+    static constexpr int offY = offX + kXY;
+    static constexpr int bytes = offY + kXY;
+    static constexpr int bg_bytes = uses_K(MODE) ? 2 * kRows * 4 : 0;  // beta[128], g[128]
 };
 
 // ------------------------------------------------------------------------- //
@@ -218,19 +226,66 @@ __device__ __forceinline__ void st_op32(uint8_t* buf, int r, int p, const float 
     }
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ void tma_load_1d(void* dst, const CUtensorMap* m, int x, uint64_t* b) {
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2}], [%3];" ::"r"(su32(dst)), "l"(m), "r"(x), "r"(su32(b))
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, int x, int y, const void* src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(m),
+                 "r"(x), "r"(y), "r"(su32(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// 32 consecutive TMEM columns of this thread's lane -> 32 raw words, no wait.
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// two 32-column pieces (e.g. an accumulator piece and a T0 piece) with one wait
+__device__ __forceinline__ void tmem_ld2(uint32_t a0, float (&v0)[32], uint32_t a1, float (&v1)[32]) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32_async(a0, r0);
+    tmem_ld32_async(a1, r1);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        v0[i] = __uint_as_float(r0[i]);
+        v1[i] = __uint_as_float(r1[i]);
+    }
+}
+
 struct Params {
     int64_t rows;        // B*H*T
     int ntiles;
-    int k;               // user chunk size (32, 64, 128)
     int N, mask, S, gated;
-    const float* beta;   // [rows]
-    const float* g;      // [rows]
     const float* Ain;    // kNeumann
     const float* Tin;    // kWY
     float* Aout;         // kBuildA
     float* Tout;         // kFused (optional), kNeumann
-    __nv_bfloat16* W;
-    __nv_bfloat16* U;
     int* status;
 };
 
@@ -242,22 +297,38 @@ struct __align__(8) Ctrl {
     int abort;
 };
 
+template <int KC, int MODE, int NS>
+struct KernelShape {
+    static constexpr int KB = block_of(KC);
+    using L = SlotLayout<KB, MODE>;
+    static constexpr int threads = 32 + 256 * NS;
+    static constexpr int smem = NS * L::bytes + NS * L::bg_bytes + (int)sizeof(Ctrl);
+};
+
 // ------------------------------------------------------------------------- //
 // the kernel
 // ------------------------------------------------------------------------- //
-template <int KB, int MODE, int NS>
-__global__ void __launch_bounds__(32 + 128 * NS, 1)
+template <int KC, int MODE, int NS>
+__global__ void __launch_bounds__(32 + 256 * NS, 1)
 k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+           const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mU,
+           const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mG,
            const Params p) {
+    constexpr int KB = block_of(KC);
+    constexpr bool SUB = KC < KB;                  // two 32-token chunks per 64 block
     using L = SlotLayout<KB, MODE>;
-    constexpr int NP = KB / 32;                    // 32-column pieces per row of a block
+    constexpr int NP = KB / 32;                    // 32-column pieces per block row
+    constexpr int PPT = NP / 2;                    // pieces per thread (two threads per row)
     constexpr int NCH = kRows / KB;                // blocks per tile
     constexpr uint32_t kTmemCols = NS == 2 ? 512 : 256;
 
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem);
-    uint8_t* slots = smem + 1024;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((su32(smem) & 1023u) != 0) {              // swizzled operands need 1024-byte alignment
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    uint8_t* bg_base = smem + NS * L::bytes;
+    Ctrl* ctrl = reinterpret_cast<Ctrl*>(bg_base + NS * L::bg_bytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -281,7 +352,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         // ------------------------------ producer ----------------------------
         if (uses_K(MODE) && lane == 0) {
             constexpr uint32_t kBytes = (uses_K(MODE) ? kRows * kD * 2 : 0) +
-                                        (uses_V(MODE) ? kRows * kD * 2 : 0);
+                                        (uses_V(MODE) ? kRows * kD * 2 : 0) + 2 * kRows * 4;
             int issued[2] = {0, 0};
             for (int n = 0;; ++n) {
                 const int tile = blockIdx.x + n * gridDim.x;
@@ -289,10 +360,12 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 const int s = n % NS, use = n / NS;
                 if (use > 0 && !mbar_wait(&ctrl->kvfree[s], (use - 1) & 1)) {
                     atomicExch(&ctrl->abort, 1);
+                    raise_status(p.status, kStatusTimeout);
                     break;
                 }
                 if (*(volatile int*)&ctrl->abort) break;
-                uint8_t* base = slots + s * L::bytes;
+                uint8_t* base = smem + s * L::bytes;
+                float* bg = reinterpret_cast<float*>(bg_base + s * L::bg_bytes);
                 const int y = tile * kRows;
                 mbar_expect_tx(&ctrl->full[s], kBytes);
                 tma_load_2d(base + L::offK, &mK, 0, y, &ctrl->full[s]);
@@ -301,6 +374,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     tma_load_2d(base + L::offV, &mV, 0, y, &ctrl->full[s]);
                     tma_load_2d(base + L::offV + kRows * 128, &mV, 64, y, &ctrl->full[s]);
                 }
+                tma_load_1d(bg, &mB, y, &ctrl->full[s]);
+                tma_load_1d(bg + kRows, &mG, y, &ctrl->full[s]);
                 issued[s] = use + 1;
             }
             // every copy this warp issued lands before the CTA exits
@@ -309,43 +384,49 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         }
     } else {
         // ------------------------------ slot s ------------------------------
-        // T0 (then T) lives in TMEM columns [128, 128 + KB) of the slot, row r
-        // in lane r, so the epilogues carry only 32-column pieces in registers.
-        const int s = (warp - 1) / 4;
+        const int s = (warp - 1) / 8;
+        const int h = ((warp - 1) % 8) / 4;            // column half of the row
         const int r = ((warp & 3) << 5) | lane;       // tile row == TMEM lane
         const int blk = r / KB;                        // block of this row in the tile
         const int i = r % KB;                          // row inside the block
-        const int sub = (p.k < KB) ? (i / p.k) : 0;    // 32-token chunk inside a 64 block
-        const int cl = (p.k < KB) ? sub * p.k : 0;     // first column of that chunk
-        const int ch = cl + (p.k < KB ? p.k : KB);     // one past its last column
-        uint8_t* base = slots + s * L::bytes;
+        const int cl = SUB ? (i / KC) * KC : 0;        // first column of this row's chunk
+        const int ch = cl + KC;                        // one past its last column
+        const int jmin = p.mask ? i - p.N : -KB;       // band mask keeps columns j >= jmin
+        uint8_t* base = smem + s * L::bytes;
         uint8_t* sK = base + L::offK;
         uint8_t* sV = base + L::offV;
         uint8_t* sAop = base + L::offAop;
         uint8_t* sX = base + L::offX;
         uint8_t* sY = base + L::offY;
+        const float* sb = reinterpret_cast<const float*>(bg_base + s * L::bg_bytes);
+        const float* sg = sb + kRows;
         const uint32_t tm = tmem_base + (uint32_t)(s * 256);
         const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);   // this warp's lanes
         const uint32_t tD = tl + blk * KB;            // this row's diagonal block of D
         const uint32_t tT = tl + 128;                 // this row's T0 / T
-        const bool leader = ((warp - 1) & 3) == 0 && lane == 0;
+        const bool leader = ((warp - 1) % 8) == 0 && lane == 0;
         const int bar_id = 1 + s;
+        const int pc0 = h * PPT;
         uint32_t mma_phase = 0;
         bool ok = true;
 
+        auto fail_wait = [&]() {
+            atomicExch(&ctrl->abort, 1);
+            raise_status(p.status, kStatusTimeout);
+        };
         auto wait_mma = [&]() -> bool {
             bool good = mbar_wait(&ctrl->mma[s], mma_phase);
             mma_phase ^= 1;
-            if (!good) { atomicExch(&ctrl->abort, 1); raise_status(p.status, kStatusTimeout); }
+            if (!good) fail_wait();
             tc_fence_after();
             return good;
         };
         // hand the operands written by this slot to the tensor pipe
         auto publish = [&]() {
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
-            bar_sync(bar_id, 128);
+            bar_sync(bar_id, 256);
             tc_fence_after();
         };
         // k x k chain product D = a_buf[128 x KB] * b_buf[KB x 128] (b: MN-major)
@@ -362,7 +443,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 mma_commit(&ctrl->mma[s]);
             }
         };
-        auto in_chunk = [&](int j) { return j >= cl && j < ch; };
+        auto in_chunk = [&](int j) { return SUB ? (j >= cl && j < ch) : true; };
         auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
 
         for (int n = s;; n += NS) {
@@ -372,14 +453,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             const int64_t row0 = (int64_t)tile * kRows;
             const int64_t grow = row0 + r;
             const bool valid = grow < p.rows;
-            const int64_t cidx = grow / p.k;                 // chunk of this row
-            const int64_t rin = grow % p.k;                  // row inside the chunk
-            const int64_t jrow0 = row0 + blk * KB;           // global row of block column 0
-            if (uses_K(MODE)) {
-                bool good = mbar_wait(&ctrl->full[s], use & 1);
-                if (!good) { atomicExch(&ctrl->abort, 1); raise_status(p.status, kStatusTimeout); }
-            }
-            bar_sync(bar_id, 128);
+            const int64_t cidx = grow / KC;                  // chunk of this row
+            const int64_t rin = grow % KC;                   // row inside the chunk
+            if (uses_K(MODE) && !mbar_wait(&ctrl->full[s], use & 1)) fail_wait();
+            bar_sync(bar_id, 256);
             if (*(volatile int*)&ctrl->abort) { ok = false; break; }
 
             if (MODE == kFused || MODE == kBuildA) {
@@ -394,25 +471,24 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         mma_ss(tm, a, a, id, kk > 0);
                     }
                     mma_commit(&ctrl->mma[s]);
-                    if (MODE == kBuildA) mma_commit(&ctrl->kvfree[s]);
                 }
                 if (!wait_mma()) { ok = false; break; }
-                const float bi = valid ? __ldg(p.beta + grow) : 0.f;
-                const float gi = valid ? __ldg(p.g + grow) : 0.f;
-#pragma unroll 1
-                for (int pc = 0; pc < NP; ++pc) {
+                const float bi = sb[r], gi = sg[r];
+                const float* gcol = sg + blk * KB;
+#pragma unroll
+                for (int pp = 0; pp < PPT; ++pp) {
+                    const int pc = pc0 + pp;
                     float v[32];
                     tmem_ld32(tD + pc * 32, v);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
                         const bool in = in_chunk(j) && j < i;
-                        const float gj = (in && jrow0 + j < p.rows) ? __ldg(p.g + jrow0 + j) : 0.f;
-                        v[jj] = in ? -bi * v[jj] * expf(gi - gj) : 0.f;
+                        v[jj] = in ? -bi * v[jj] * expf(gi - gcol[j]) : 0.f;
                     }
                     if (MODE == kBuildA) {
-                        if (valid && pc * 32 >= cl && pc * 32 < ch) {
-                            float* dst = p.Aout + cidx * p.k * p.k + rin * p.k + (pc * 32 - cl);
+                        if (valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch))) {
+                            float* dst = p.Aout + cidx * KC * KC + rin * KC + (pc * 32 - cl);
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
                                 reinterpret_cast<float4*>(dst)[q] =
@@ -424,7 +500,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) {
                             const int j = pc * 32 + jj;
-                            v[jj] = (p.mask && i - j > p.N) ? 0.f : v[jj];
+                            v[jj] = j >= jmin ? v[jj] : 0.f;
                             t[jj] = eye(j) + v[jj];
                         }
                         st_op32<false>(sAop, r, pc, v);           // P_1 = M . A
@@ -433,18 +509,20 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
                 if (MODE == kBuildA) {
                     tc_fence_before();
-                    bar_sync(bar_id, 128);
+                    bar_sync(bar_id, 256);                 // beta/g read, accumulator read
+                    if (leader) mbar_arrive(&ctrl->kvfree[s]);
                     continue;
                 }
             } else if (MODE == kNeumann) {
                 // ---- A row from global memory ----
-#pragma unroll 1
-                for (int pc = 0; pc < NP; ++pc) {
+#pragma unroll
+                for (int pp = 0; pp < PPT; ++pp) {
+                    const int pc = pc0 + pp;
                     float v[32], t[32];
-                    const bool have = valid && pc * 32 >= cl && pc * 32 < ch;
+                    const bool have = valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch));
                     if (have) {
                         const float4* src = reinterpret_cast<const float4*>(
-                            p.Ain + cidx * p.k * p.k + rin * p.k + (pc * 32 - cl));
+                            p.Ain + cidx * KC * KC + rin * KC + (pc * 32 - cl));
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             float4 a = __ldg(src + q);
@@ -458,7 +536,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
-                        v[jj] = (p.mask && i - j > p.N) ? 0.f : v[jj];
+                        v[jj] = j >= jmin ? v[jj] : 0.f;
                         t[jj] = eye(j) + v[jj];
                     }
                     st_op32<false>(sAop, r, pc, v);
@@ -466,13 +544,14 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
             } else {
                 // ---- kWY: T row from global memory ----
-#pragma unroll 1
-                for (int pc = 0; pc < NP; ++pc) {
+#pragma unroll
+                for (int pp = 0; pp < PPT; ++pp) {
+                    const int pc = pc0 + pp;
                     float t[32];
-                    const bool have = valid && pc * 32 >= cl && pc * 32 < ch;
+                    const bool have = valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch));
                     if (have) {
                         const float4* src = reinterpret_cast<const float4*>(
-                            p.Tin + cidx * p.k * p.k + rin * p.k + (pc * 32 - cl));
+                            p.Tin + cidx * KC * KC + rin * KC + (pc * 32 - cl));
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
                             float4 a = __ldg(src + q);
@@ -492,15 +571,15 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     publish();
                     mma_chain(sAop, sX);                                   // P_{n-1} A
                     if (!wait_mma()) { ok = false; break; }
-#pragma unroll 1
-                    for (int pc = 0; pc < NP; ++pc) {
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
                         float v[32], t[32];
-                        tmem_ld32(tD + pc * 32, v);
-                        tmem_ld32(tT + pc * 32, t);
+                        tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) {
                             const int j = pc * 32 + jj;
-                            v[jj] = (!in_chunk(j) || (p.mask && i - j > p.N)) ? 0.f : v[jj];
+                            v[jj] = (in_chunk(j) && j >= jmin) ? v[jj] : 0.f;
                             t[jj] += v[jj];
                         }
                         tmem_st32(tT + pc * 32, t);
@@ -510,8 +589,9 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 if (!ok) break;
                 // ---- parallel residual correction ----
                 if (p.S > 0) {
-#pragma unroll 1
-                    for (int pc = 0; pc < NP; ++pc) {
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
                         float t[32];
                         tmem_ld32(tT + pc * 32, t);
                         st_op32<false>(sY, r, pc, t);                      // T0
@@ -519,11 +599,11 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     publish();
                     mma_chain(sX, sY);                                      // A T0
                     if (!wait_mma()) { ok = false; break; }
-#pragma unroll 1
-                    for (int pc = 0; pc < NP; ++pc) {
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
                         float v[32], t[32];
-                        tmem_ld32(tD + pc * 32, v);
-                        tmem_ld32(tT + pc * 32, t);
+                        tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) {
                             const int j = pc * 32 + jj;
@@ -544,21 +624,25 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         mma_chain(sAop, sX);                                // (I + Q_m) E
                         if (!wait_mma()) { ok = false; break; }
                         const bool last = (m == p.S - 1);
-#pragma unroll 1
-                        for (int pc = 0; pc < NP; ++pc) {
-                            float v[32];
-                            tmem_ld32(tD + pc * 32, v);
 #pragma unroll
-                            for (int jj = 0; jj < 32; ++jj)
-                                if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
+                        for (int pp = 0; pp < PPT; ++pp) {
+                            const int pc = pc0 + pp;
+                            float v[32];
                             if (last) {
                                 float t[32];
+                                tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj)
+                                    if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
                                 st_op32<false>(sY, r, pc, v);               // Q_S
-                                tmem_ld32(tT + pc * 32, t);
                                 st_op32<false>(sAop, r, pc, t);             // T0
                             } else {
+                                tmem_ld32(tD + pc * 32, v);
 #pragma unroll
-                                for (int jj = 0; jj < 32; ++jj) v[jj] += eye(pc * 32 + jj);
+                                for (int jj = 0; jj < 32; ++jj) {
+                                    const int j = pc * 32 + jj;
+                                    v[jj] = in_chunk(j) ? v[jj] + eye(j) : 0.f;
+                                }
                                 st_op32<false>(sAop, r, pc, v);             // I + Q_{m+1}
                             }
                         }
@@ -567,25 +651,26 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     publish();
                     mma_chain(sAop, sY);                                    // T0 Q_S
                     if (!wait_mma()) { ok = false; break; }
-#pragma unroll 1
-                    for (int pc = 0; pc < NP; ++pc) {
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
                         float v[32], t[32];
-                        tmem_ld32(tD + pc * 32, v);
-                        tmem_ld32(tT + pc * 32, t);
+                        tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
-                            if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];         // T = T0 + T0 Q
+                            if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];     // T = T0 + T0 Q
                         tmem_st32(tT + pc * 32, t);
                     }
                 }
                 // ---- T out ----
                 if (p.Tout) {
-#pragma unroll 1
-                    for (int pc = 0; pc < NP; ++pc) {
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
                         float t[32];
                         tmem_ld32(tT + pc * 32, t);
-                        if (valid && pc * 32 >= cl && pc * 32 < ch) {
-                            float* dst = p.Tout + cidx * p.k * p.k + rin * p.k + (pc * 32 - cl);
+                        if (valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch))) {
+                            float* dst = p.Tout + cidx * KC * KC + rin * KC + (pc * 32 - cl);
 #pragma unroll
                             for (int q = 0; q < 8; ++q)
                                 reinterpret_cast<float4*>(dst)[q] =
@@ -597,17 +682,18 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 
             if (MODE == kFused || MODE == kWY) {
                 // ---- WY: T diag(beta [exp g]) -> X (bf16), T diag(beta) -> Y ----
-#pragma unroll 1
-                for (int pc = 0; pc < NP; ++pc) {
+                const float* bcol = sb + blk * KB;
+                const float* gcol = sg + blk * KB;
+#pragma unroll
+                for (int pp = 0; pp < PPT; ++pp) {
+                    const int pc = pc0 + pp;
                     float t[32], v[32];
                     tmem_ld32(tT + pc * 32, t);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
-                        const bool jv = jrow0 + j < p.rows;
-                        const float b = jv ? __ldg(p.beta + jrow0 + j) : 0.f;
-                        const float bw = p.gated ? b * expf(jv ? __ldg(p.g + jrow0 + j) : 0.f) : b;
-                        v[jj] = t[jj] * bw;
+                        const float b = bcol[j];
+                        v[jj] = p.gated ? t[jj] * (b * expf(gcol[j])) : t[jj] * b;
                         t[jj] = t[jj] * b;
                     }
                     st_op32<true>(sX, r, pc, v);
@@ -632,37 +718,54 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         }
                     }
                     mma_commit(&ctrl->mma[s]);
-                    mma_commit(&ctrl->kvfree[s]);
                 }
                 if (!wait_mma()) { ok = false; break; }
-                // lane r of the W^T / U^T accumulators is head-dim column d = r
-                const int d = r;
-#pragma unroll 1
-                for (int c = 0; c < NCH; ++c) {
-#pragma unroll 1
-                    for (int pc = 0; pc < NP; ++pc) {
+                // Lane r of the W^T / U^T accumulators is head-dim column d = r and
+                // accumulator column x is tile row x.  Thread half h transposes
+                // rows [64h, 64h + 64) through the K (W) and V (U) tiles, which
+                // the finished MMAs no longer read, in the TMA load layout.
+                {
+                    const int d = r;
+                    const uint32_t dbase = (uint32_t)((d >> 6) * (kRows * 128) + (d & 7) * 2);
+                    const int c16 = (d & 63) >> 3;
+#pragma unroll
+                    for (int pp = 0; pp < 2; ++pp) {
+                        const int x0 = h * 64 + pp * 32;
                         float w[32], u[32];
-                        tmem_ld32(tl + c * KB + pc * 32, w);
-                        tmem_ld32(tl + 128 + c * KB + pc * 32, u);
-                        const int64_t t0 = row0 + c * KB + pc * 32;
+                        tmem_ld2(tl + x0, w, tl + 128 + x0, u);
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) {
-                            if (t0 + jj < p.rows) {
-                                p.W[(t0 + jj) * kD + d] = __float2bfloat16_rn(w[jj]);
-                                p.U[(t0 + jj) * kD + d] = __float2bfloat16_rn(u[jj]);
-                            }
+                            const int x = x0 + jj;
+                            const uint32_t off = dbase + x * 128 + ((c16 ^ (x & 7)) << 4);
+                            *reinterpret_cast<__nv_bfloat16*>(sK + off) = __float2bfloat16_rn(w[jj]);
+                            *reinterpret_cast<__nv_bfloat16*>(sV + off) = __float2bfloat16_rn(u[jj]);
                         }
                     }
                 }
+                fence_async_smem();
+                tc_fence_before();
+                bar_sync(bar_id, 256);
+                if (leader) {
+                    const int y = (int)row0;
+                    tma_store_2d(&mW, 0, y, sK);
+                    tma_store_2d(&mW, 64, y, sK + kRows * 128);
+                    tma_store_2d(&mU, 0, y, sV);
+                    tma_store_2d(&mU, 64, y, sV + kRows * 128);
+                    bulk_commit();
+                    bulk_wait_read();                       // tiles may be reloaded now
+                    mbar_arrive(&ctrl->kvfree[s]);
+                }
+                continue;
             }
             tc_fence_before();
-            bar_sync(bar_id, 128);                 // accumulators free for the next tile
+            bar_sync(bar_id, 256);                 // accumulators free for the next tile
         }
         if (!ok) {
             atomicExch(&ctrl->abort, 1);
             // outstanding MMAs of this slot finish before TMEM is released
             mbar_wait(&ctrl->mma[s], mma_phase);
         }
+        if (leader) bulk_wait_all();               // W, U stores complete
     }
     tc_fence_before();
     __syncthreads();
@@ -683,12 +786,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 static EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
-        void* p = nullptr;
+        void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = (EncodeTiledFn)p;
+            fn = (EncodeTiledFn)ptr;
     }
     return fn;
 }
@@ -706,6 +809,19 @@ static bool map_kd(CUtensorMap* m, const void* base, int64_t rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows] fp32, box 128 (rows past the end read as zero)
+static bool map_vec(CUtensorMap* m, const void* base, int64_t rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[1] = {(cuuint64_t)rows};
+    cuuint64_t strides[1] = {4};
+    cuuint32_t box[1] = {(cuuint32_t)kRows};
+    cuuint32_t es[1] = {1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int num_sms() {
     int dev = 0, n = 148;
     cudaGetDevice(&dev);
@@ -713,26 +829,45 @@ static int num_sms() {
     return n;
 }
 
-template <int KB, int MODE, int NS>
-static cudaError_t launch(const void* K, const void* V, const float* beta, const float* g,
-                          const Params& p0, cudaStream_t st) {
-    using L = SlotLayout<KB, MODE>;
-    CUtensorMap mK, mV;
+struct IO {
+    const void* K = nullptr;
+    const void* V = nullptr;
+    const float* beta = nullptr;
+    const float* g = nullptr;
+    void* W = nullptr;
+    void* U = nullptr;
+};
+
+template <int KC, int MODE, int NS>
+static cudaError_t launch(const IO& io, const Params& p0, cudaStream_t st) {
+    using KS = KernelShape<KC, MODE, NS>;
+    static_assert(KS::smem <= 232448, "shared memory budget");
+    CUtensorMap mK, mV, mW, mU, mB, mG;
     memset(&mK, 0, sizeof mK);
     memset(&mV, 0, sizeof mV);
-    if (uses_K(MODE) && !map_kd(&mK, K, p0.rows)) return cudaErrorInvalidValue;
-    if (uses_V(MODE) && !map_kd(&mV, V, p0.rows)) return cudaErrorInvalidValue;
+    memset(&mW, 0, sizeof mW);
+    memset(&mU, 0, sizeof mU);
+    memset(&mB, 0, sizeof mB);
+    memset(&mG, 0, sizeof mG);
+    if (uses_K(MODE)) {
+        if (!map_kd(&mK, io.K, p0.rows) || !map_vec(&mB, io.beta, p0.rows) ||
+            !map_vec(&mG, io.g ? io.g : io.beta, p0.rows))
+            return cudaErrorInvalidValue;
+    }
+    if (uses_V(MODE)) {
+        if (!map_kd(&mV, io.V, p0.rows) || !map_kd(&mW, io.W, p0.rows) ||
+            !map_kd(&mU, io.U, p0.rows))
+            return cudaErrorInvalidValue;
+    }
     Params p = p0;
-    p.beta = beta;
-    p.g = g;
     p.status = status_ptr();
-    size_t smem = 1024 + 1024 + (size_t)NS * L::bytes;
+    size_t smem = KS::smem;
     if (smem < 120 * 1024) smem = 120 * 1024;     // one CTA per SM: it owns the SM's TMEM
-    cudaError_t e = cudaFuncSetAttribute(k_chunk_tc<KB, MODE, NS>,
+    cudaError_t e = cudaFuncSetAttribute(k_chunk_tc<KC, MODE, NS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = p.ntiles < num_sms() ? p.ntiles : num_sms();
-    k_chunk_tc<KB, MODE, NS><<<grid, 32 + 128 * NS, smem, st>>>(mK, mV, p);
+    k_chunk_tc<KC, MODE, NS><<<grid, KS::threads, smem, st>>>(mK, mV, mW, mU, mB, mG, p);
     return cudaGetLastError();
 }
 
@@ -741,8 +876,18 @@ static Params base_params(int64_t nc, int k) {
     memset(&p, 0, sizeof p);
     p.rows = nc * k;
     p.ntiles = (int)((p.rows + kRows - 1) / kRows);
-    p.k = k;
     return p;
+}
+
+// chunk size -> kernel instance; NS128 = slots per CTA at k = 128
+template <int MODE, int NS128>
+static cudaError_t dispatch(int k, const IO& io, const Params& p, cudaStream_t st) {
+    switch (k) {
+        case 32: return launch<32, MODE, 2>(io, p, st);
+        case 64: return launch<64, MODE, 2>(io, p, st);
+        case 128: return launch<128, MODE, NS128>(io, p, st);
+        default: return cudaErrorNotSupported;
+    }
 }
 
 }  // namespace tcg
@@ -750,39 +895,41 @@ static Params base_params(int64_t nc, int k) {
 bool tc_available() { return true; }
 bool tc_i8_available() { return false; }
 
-#define GDN_TC_DISPATCH(k, MODE, NS128, ...)                                       \
-    (k == 128 ? tcg::launch<128, MODE, NS128>(__VA_ARGS__)                           \
-              : tcg::launch<64, MODE, 2>(__VA_ARGS__))
-
 cudaError_t launch_build_A_tc(const void* K, const float* beta, const float* g, float* A,
                               int64_t nc, int k, cudaStream_t st) {
-    if (k > 128) return cudaErrorNotSupported;
     tcg::Params p = tcg::base_params(nc, k);
     p.Aout = A;
-    return GDN_TC_DISPATCH(k, tcg::kBuildA, 2, K, nullptr, beta, g, p, st);
+    tcg::IO io;
+    io.K = K;
+    io.beta = beta;
+    io.g = g;
+    return tcg::dispatch<tcg::kBuildA, 2>(k, io, p, st);
 }
 
 cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int S,
                               cudaStream_t st) {
-    if (k > 128) return cudaErrorNotSupported;
     tcg::Params p = tcg::base_params(nc, k);
     p.Ain = A;
     p.Tout = T;
     p.N = N;
     p.mask = mask;
     p.S = S;
-    return GDN_TC_DISPATCH(k, tcg::kNeumann, 2, nullptr, nullptr, nullptr, nullptr, p, st);
+    return tcg::dispatch<tcg::kNeumann, 2>(k, tcg::IO(), p, st);
 }
 
 cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const float* beta,
                          const float* g, void* W, void* U, int64_t nc, int k, cudaStream_t st) {
-    if (k > 128) return cudaErrorNotSupported;
     tcg::Params p = tcg::base_params(nc, k);
     p.Tin = T;
     p.gated = g != nullptr;
-    p.W = (__nv_bfloat16*)W;
-    p.U = (__nv_bfloat16*)U;
-    return GDN_TC_DISPATCH(k, tcg::kWY, 1, K, V, beta, g, p, st);
+    tcg::IO io;
+    io.K = K;
+    io.V = V;
+    io.beta = beta;
+    io.g = g;
+    io.W = W;
+    io.U = U;
+    return tcg::dispatch<tcg::kWY, 1>(k, io, p, st);
 }
 
 cudaError_t launch_neumann_i8_tc(const float*, float*, int, int, int8_t*, int32_t*, float*,
@@ -793,16 +940,20 @@ cudaError_t launch_neumann_i8_tc(const float*, float*, int, int, int8_t*, int32_
 cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, const float* g,
                             int N, int mask, int S, int gated, void* W, void* U, float* Tout,
                             int64_t nc, int k, cudaStream_t st) {
-    if (k > 128) return cudaErrorNotSupported;
     tcg::Params p = tcg::base_params(nc, k);
     p.N = N;
     p.mask = mask;
     p.S = S;
     p.gated = gated;
-    p.W = (__nv_bfloat16*)W;
-    p.U = (__nv_bfloat16*)U;
     p.Tout = Tout;
-    return GDN_TC_DISPATCH(k, tcg::kFused, 1, K, V, beta, g, p, st);
+    tcg::IO io;
+    io.K = K;
+    io.V = V;
+    io.beta = beta;
+    io.g = g;
+    io.W = W;
+    io.U = U;
+    return tcg::dispatch<tcg::kFused, 1>(k, io, p, st);
 }
 
 }  // namespace gdn
