@@ -198,18 +198,51 @@ int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta, const fl
 int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype) {
     int64_t nc;
     if (check_shape(s, &nc) != GDN_OK) return -1;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return -1;
     const int64_t elem = dtype == GDN_BF16 ? 2 : 4;
-    return 2 * nc * (int64_t)s.k * s.d * elem;
+    const int64_t rows = nc * s.k;
+    // W_g and U for every chunk, then A and T (exact path)
+    return 2 * rows * s.d * elem + 2 * nc * (int64_t)s.k * s.k * 4;
 }
 
 int gdn_forward(const void* Q, const void* K, const void* V, const float* beta, const float* g,
                 const float* S0, int N, int mask, int S, int exact, void* O, float* S_final,
                 void* workspace, int64_t workspace_bytes, gdn_shape s, gdn_dtype dtype,
                 void* stream) {
-    (void)Q; (void)K; (void)V; (void)beta; (void)g; (void)S0; (void)N; (void)mask; (void)S;
-    (void)exact; (void)O; (void)S_final; (void)workspace; (void)workspace_bytes; (void)s;
-    (void)dtype; (void)stream;
-    return fail(GDN_ERR_UNSUPPORTED, "gdn_forward is not built yet");
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_dtype(dtype));
+    if (s.k != 64) return fail(GDN_ERR_UNSUPPORTED, "gdn_forward is built for k=64");
+    if (exact != 0 && exact != 1) return fail(GDN_ERR_ARG, "exact must be 0 or 1");
+    if (!exact) GDN_TRY(check_NS(N, mask, S, s.k));
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{Q, "Q"}, {K, "K"}, {V, "V"}, {beta, "beta"}, {g, "g"}, {O, "O"},
+                        {S_final, "S_final"}, {workspace, "workspace"}}));
+    GDN_TRY(check_opt_ptr(S0, "S0"));
+    const int64_t need = gdn_forward_workspace_bytes(s, dtype);
+    if (workspace_bytes < need)
+        return fail(GDN_ERR_ARG, "workspace of %lld bytes is below the %lld needed",
+                    (long long)workspace_bytes, (long long)need);
+    cudaStream_t st = (cudaStream_t)stream;
+    const bool bf16 = dtype == GDN_BF16;
+    const int64_t elem = bf16 ? 2 : 4;
+    const int64_t rows = nc * s.k;
+    uint8_t* ws = (uint8_t*)workspace;
+    void* Wg = ws;
+    void* U = ws + rows * s.d * elem;
+    float* Abuf = (float*)(ws + 2 * rows * s.d * elem);
+    float* Tbuf = Abuf + nc * (int64_t)s.k * s.k;
+    if (exact) {
+        GDN_TRY(gdn_build_A(K, beta, g, Abuf, s, dtype, stream));
+        GDN_TRY(gdn_invert_fwdsub(Abuf, Tbuf, s, stream));
+        GDN_TRY(gdn_wy(Tbuf, K, V, beta, g, Wg, U, s, dtype, stream));
+    } else {
+        GDN_TRY(gdn_chunk_wy_fused(K, V, beta, g, N, mask, S, 1, Wg, U, nullptr, s, dtype,
+                                   stream));
+    }
+    return launched(gdn::launch_scan(Q, K, Wg, U, g, S0, O, S_final, s.B * s.H, s.T / s.k, bf16,
+                                     st),
+                    "forward scan");
 }
 
 int gdn_get_status(void* stream) {
@@ -223,6 +256,7 @@ int gdn_get_status(void* stream) {
     e = cudaMemcpyToSymbol(gdn::g_status, &z, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "clear status");
     if (v & gdn::kStatusTimeout) return fail(GDN_ERR_TIMEOUT, "a bounded device wait ran out");
+    if (v) return fail(GDN_ERR_CUDA, "device status bits 0x%x", v);
     return GDN_OK;
 }
 

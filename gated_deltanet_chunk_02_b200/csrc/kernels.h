@@ -21,4 +21,9 @@ cudaError_t launch_fwdsub(const float* A, float* T, int64_t nc, int k, cudaStrea
 cudaError_t launch_neumann_i8_simt(const float* A, float* T, int N, int mask, int8_t* q,
                                    int32_t* acc, float* sc, int64_t nc, cudaStream_t st);
 
+// Inter-chunk state scan of the forward (scan.cu); k = 64, d = 128.
+cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, const void* U, const float* g,
+                        const float* S0, void* O, float* Sfin, int64_t BH, int64_t nchunk,
+                        bool bf16, cudaStream_t st);
+
 }  // namespace gdn

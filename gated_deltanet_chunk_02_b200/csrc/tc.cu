@@ -11,15 +11,16 @@
 //   tile's blocks along M, the right operand places them side by side along N,
 //   and each row reads only its own diagonal block of the 128 x 128 fp32
 //   accumulator in tensor memory (TMEM).
-// * Warp 0 is the TMA producer: K and V tiles (128-byte swizzle), beta and g.
-//   Each "slot" of 8 warps owns one tile at a time; its elected thread issues
-//   the tile's MMAs and TMA stores, and its 256 threads run the epilogues
-//   (TMEM -> registers -> mask / accumulate / convert -> swizzled shared-memory
-//   operand).  Thread (r, h) owns row r of the tile (its TMEM lane; the lane
-//   quarter is warp % 4) and the column half h.  Two slots per CTA keep the
-//   tensor pipe busy while the other slot runs an epilogue.
-// * T0 (then T) stays in TMEM columns [128, 128 + KB) of the slot, next to the
-//   product accumulator in columns [0, 128).
+// * Each "slot" of 8 warps owns one tile at a time.  Its elected thread issues
+//   the tile's TMA loads (K with beta and g on one barrier, V on another, so
+//   the K K^T product starts before V lands), its MMAs and its TMA stores, and
+//   loads the slot's next tile as soon as the stores have read the staging
+//   tiles.  Its 256 threads run the epilogues (TMEM -> registers -> mask /
+//   accumulate / convert -> swizzled shared-memory operand).  Thread (r, h)
+//   owns row r of the tile (its TMEM lane; the lane quarter is warp % 4) and
+//   the column half h, and keeps its part of T0 (then T) in registers.  Two
+//   slots per CTA keep the tensor pipe busy while the other slot runs an
+//   epilogue.
 // * WY is computed transposed, W^T = K^T (T diag(beta))^T, a full-rate M=128
 //   (= d) product; its epilogue transposes through the (now free) K/V tiles in
 //   shared memory and leaves with TMA bulk stores.
@@ -290,9 +291,9 @@ struct Params {
 };
 
 struct __align__(8) Ctrl {
-    uint64_t full[2];
-    uint64_t kvfree[2];
-    uint64_t mma[2];
+    uint64_t fullK[2];   // K tile, beta, g landed
+    uint64_t fullV[2];   // V tile landed
+    uint64_t mma[2];     // the slot's MMAs completed
     uint32_t tmem;
     int abort;
 };
@@ -301,7 +302,7 @@ template <int KC, int MODE, int NS>
 struct KernelShape {
     static constexpr int KB = block_of(KC);
     using L = SlotLayout<KB, MODE>;
-    static constexpr int threads = 32 + 256 * NS;
+    static constexpr int threads = 256 * NS;
     static constexpr int smem = NS * L::bytes + NS * L::bg_bytes + (int)sizeof(Ctrl);
 };
 
@@ -309,7 +310,7 @@ struct KernelShape {
 // the kernel
 // ------------------------------------------------------------------------- //
 template <int KC, int MODE, int NS>
-__global__ void __launch_bounds__(32 + 256 * NS, 1)
+__global__ void __launch_bounds__(256 * NS, 1)
 k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
            const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mU,
            const __grid_constant__ CUtensorMap mB, const __grid_constant__ CUtensorMap mG,
@@ -335,8 +336,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&ctrl->full[s], 1);
-            mbar_init(&ctrl->kvfree[s], 1);
+            mbar_init(&ctrl->fullK[s], 1);
+            mbar_init(&ctrl->fullV[s], 1);
             mbar_init(&ctrl->mma[s], 1);
         }
         ctrl->abort = 0;
@@ -348,133 +349,211 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     tc_fence_after();
     const uint32_t tmem_base = ctrl->tmem;
 
-    if (warp == 0) {
-        // ------------------------------ producer ----------------------------
-        if (uses_K(MODE) && lane == 0) {
-            constexpr uint32_t kBytes = (uses_K(MODE) ? kRows * kD * 2 : 0) +
-                                        (uses_V(MODE) ? kRows * kD * 2 : 0) + 2 * kRows * 4;
-            int issued[2] = {0, 0};
-            for (int n = 0;; ++n) {
-                const int tile = blockIdx.x + n * gridDim.x;
-                if (tile >= p.ntiles) break;
-                const int s = n % NS, use = n / NS;
-                if (use > 0 && !mbar_wait(&ctrl->kvfree[s], (use - 1) & 1)) {
-                    atomicExch(&ctrl->abort, 1);
-                    raise_status(p.status, kStatusTimeout);
-                    break;
-                }
-                if (*(volatile int*)&ctrl->abort) break;
-                uint8_t* base = smem + s * L::bytes;
-                float* bg = reinterpret_cast<float*>(bg_base + s * L::bg_bytes);
-                const int y = tile * kRows;
-                mbar_expect_tx(&ctrl->full[s], kBytes);
-                tma_load_2d(base + L::offK, &mK, 0, y, &ctrl->full[s]);
-                tma_load_2d(base + L::offK + kRows * 128, &mK, 64, y, &ctrl->full[s]);
-                if (uses_V(MODE)) {
-                    tma_load_2d(base + L::offV, &mV, 0, y, &ctrl->full[s]);
-                    tma_load_2d(base + L::offV + kRows * 128, &mV, 64, y, &ctrl->full[s]);
-                }
-                tma_load_1d(bg, &mB, y, &ctrl->full[s]);
-                tma_load_1d(bg + kRows, &mG, y, &ctrl->full[s]);
-                issued[s] = use + 1;
-            }
-            // every copy this warp issued lands before the CTA exits
-            for (int s = 0; s < NS; ++s)
-                if (issued[s] > 0) mbar_wait(&ctrl->full[s], (issued[s] - 1) & 1);
-        }
-    } else {
-        // ------------------------------ slot s ------------------------------
-        const int s = (warp - 1) / 8;
-        const int h = ((warp - 1) % 8) / 4;            // column half of the row
-        const int r = ((warp & 3) << 5) | lane;       // tile row == TMEM lane
-        const int blk = r / KB;                        // block of this row in the tile
-        const int i = r % KB;                          // row inside the block
-        const int cl = SUB ? (i / KC) * KC : 0;        // first column of this row's chunk
-        const int ch = cl + KC;                        // one past its last column
-        const int jmin = p.mask ? i - p.N : -KB;       // band mask keeps columns j >= jmin
-        uint8_t* base = smem + s * L::bytes;
-        uint8_t* sK = base + L::offK;
-        uint8_t* sV = base + L::offV;
-        uint8_t* sAop = base + L::offAop;
-        uint8_t* sX = base + L::offX;
-        uint8_t* sY = base + L::offY;
-        const float* sb = reinterpret_cast<const float*>(bg_base + s * L::bg_bytes);
-        const float* sg = sb + kRows;
-        const uint32_t tm = tmem_base + (uint32_t)(s * 256);
-        const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);   // this warp's lanes
-        const uint32_t tD = tl + blk * KB;            // this row's diagonal block of D
-        const uint32_t tT = tl + 128;                 // this row's T0 / T
-        const bool leader = ((warp - 1) % 8) == 0 && lane == 0;
-        const int bar_id = 1 + s;
-        const int pc0 = h * PPT;
-        uint32_t mma_phase = 0;
-        bool ok = true;
+    // ------------------------------ slot s ------------------------------
+    // Slot s = warps [8s, 8s + 8).  Thread (r, h) owns tile row r (= its TMEM
+    // lane) and the column half h of that row's block; T0 / T of its half row
+    // lives in its registers.
+    const int s = warp / 8;
+    const int h = (warp % 8) / 4;
+    const int r = ((warp & 3) << 5) | lane;
+    const int blk = r / KB;                        // block of this row in the tile
+    const int i = r % KB;                          // row inside the block
+    const int cl = SUB ? (i / KC) * KC : 0;        // first column of this row's chunk
+    const int ch = cl + KC;                        // one past its last column
+    const int jmin = p.mask ? i - p.N : -KB;       // band mask keeps columns j >= jmin
+    uint8_t* base = smem + s * L::bytes;
+    uint8_t* sK = base + L::offK;
+    uint8_t* sV = base + L::offV;
+    uint8_t* sAop = base + L::offAop;
+    uint8_t* sX = base + L::offX;
+    uint8_t* sY = base + L::offY;
+    float* sb = reinterpret_cast<float*>(bg_base + s * L::bg_bytes);
+    float* sg = sb + kRows;
+    const uint32_t tm = tmem_base + (uint32_t)(s * 256);
+    const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);   // this warp's lanes
+    const uint32_t tD = tl + blk * KB;            // this row's diagonal block of D
+    const bool leader = (warp % 8) == 0 && lane == 0;
+    const int bar_id = 1 + s;
+    const int pc0 = h * PPT;
+    uint32_t mma_phase = 0;
+    bool ok = true;
 
-        auto fail_wait = [&]() {
-            atomicExch(&ctrl->abort, 1);
-            raise_status(p.status, kStatusTimeout);
-        };
-        auto wait_mma = [&]() -> bool {
-            bool good = mbar_wait(&ctrl->mma[s], mma_phase);
-            mma_phase ^= 1;
-            if (!good) fail_wait();
-            tc_fence_after();
-            return good;
-        };
-        // hand the operands written by this slot to the tensor pipe
-        auto publish = [&]() {
-            tmem_wait_st();
-            fence_async_smem();
-            tc_fence_before();
-            bar_sync(bar_id, 256);
-            tc_fence_after();
-        };
-        // k x k chain product D = a_buf[128 x KB] * b_buf[KB x 128] (b: MN-major)
-        auto mma_chain = [&](const uint8_t* a_buf, const uint8_t* b_buf) {
-            if (leader) {
-                constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
+    auto fail_wait = [&]() {
+        atomicExch(&ctrl->abort, 1);
+        raise_status(p.status, kStatusTimeout);
+    };
+    auto wait_mma = [&]() -> bool {
+        bool good = mbar_wait(&ctrl->mma[s], mma_phase);
+        mma_phase ^= 1;
+        if (!good) fail_wait();
+        tc_fence_after();
+        return good;
+    };
+    // hand the operands written by this slot to the tensor pipe
+    auto publish = [&]() {
+        fence_async_smem();
+        tc_fence_before();
+        bar_sync(bar_id, 256);
+        tc_fence_after();
+    };
+    // k x k chain product D = a_buf[128 x KB] * b_buf[KB x 128] (b: MN-major)
+    auto mma_chain = [&](const uint8_t* a_buf, const uint8_t* b_buf) {
+        if (leader) {
+            constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
 #pragma unroll
-                for (int kk = 0; kk < KB / 16; ++kk) {
-                    uint64_t a = sdesc(su32(a_buf) + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16,
-                                       1024);
-                    uint64_t b = sdesc(su32(b_buf) + kk * 2048, KB * 128, 1024);
-                    mma_ss(tm, a, b, id, kk > 0);
+            for (int kk = 0; kk < KB / 16; ++kk) {
+                uint64_t a = sdesc(su32(a_buf) + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16,
+                                   1024);
+                uint64_t b = sdesc(su32(b_buf) + kk * 2048, KB * 128, 1024);
+                mma_ss(tm, a, b, id, kk > 0);
+            }
+            mma_commit(&ctrl->mma[s]);
+        }
+    };
+    // the slot's leader loads its own tiles: K, beta, g on fullK, V on fullV
+    auto issue_loads = [&](int n) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (!uses_K(MODE) || tile >= p.ntiles) return;
+        const int y = tile * kRows;
+        mbar_expect_tx(&ctrl->fullK[s], kRows * kD * 2 + 2 * kRows * 4);
+        tma_load_2d(sK, &mK, 0, y, &ctrl->fullK[s]);
+        tma_load_2d(sK + kRows * 128, &mK, 64, y, &ctrl->fullK[s]);
+        tma_load_1d(sb, &mB, y, &ctrl->fullK[s]);
+        tma_load_1d(sg, &mG, y, &ctrl->fullK[s]);
+        if (uses_V(MODE)) {
+            mbar_expect_tx(&ctrl->fullV[s], kRows * kD * 2);
+            tma_load_2d(sV, &mV, 0, y, &ctrl->fullV[s]);
+            tma_load_2d(sV + kRows * 128, &mV, 64, y, &ctrl->fullV[s]);
+        }
+    };
+    auto in_chunk = [&](int j) { return SUB ? (j >= cl && j < ch) : true; };
+#define T0P(pp) (*reinterpret_cast<float(*)[32]>(&T0[(pp) * 32]))
+    auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
+    auto piece_in_chunk = [&](int pc) { return !SUB || (pc * 32 >= cl && pc * 32 < ch); };
+
+    if (leader) issue_loads(s);
+
+    for (int n = s;; n += NS) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (tile >= p.ntiles) break;
+        const uint32_t use_par = (uint32_t)((n / NS) & 1);
+        const int64_t row0 = (int64_t)tile * kRows;
+        const int64_t grow = row0 + r;
+        const bool valid = grow < p.rows;
+        const int64_t cidx = grow / KC;                  // chunk of this row
+        const int64_t rin = grow % KC;                   // row inside the chunk
+        float T0[PPT * 32];                              // this thread's part of row r of T0 / T
+
+        if (uses_K(MODE) && !mbar_wait(&ctrl->fullK[s], use_par)) fail_wait();
+        bar_sync(bar_id, 256);
+        if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+
+        if (MODE == kFused || MODE == kBuildA) {
+            // ---- G = K K^T over the tile, then A = -beta_i G_ij exp(g_i - g_j) ----
+            if (leader) {
+                tc_fence_after();
+                constexpr uint32_t id = idesc_f16(1, 0, 0, 128, 128);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    uint64_t a = sdesc(su32(sK) + (kk >> 2) * (kRows * 128) + (kk & 3) * 32,
+                                       16, 1024);
+                    mma_ss(tm, a, a, id, kk > 0);
                 }
                 mma_commit(&ctrl->mma[s]);
             }
-        };
-        auto in_chunk = [&](int j) { return SUB ? (j >= cl && j < ch) : true; };
-        auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
-
-        for (int n = s;; n += NS) {
-            const int tile = blockIdx.x + n * gridDim.x;
-            if (tile >= p.ntiles) break;
-            const int use = n / NS;
-            const int64_t row0 = (int64_t)tile * kRows;
-            const int64_t grow = row0 + r;
-            const bool valid = grow < p.rows;
-            const int64_t cidx = grow / KC;                  // chunk of this row
-            const int64_t rin = grow % KC;                   // row inside the chunk
-            if (uses_K(MODE) && !mbar_wait(&ctrl->full[s], use & 1)) fail_wait();
-            bar_sync(bar_id, 256);
-            if (*(volatile int*)&ctrl->abort) { ok = false; break; }
-
-            if (MODE == kFused || MODE == kBuildA) {
-                // ---- G = K K^T over the tile, then A = -beta_i G_ij exp(g_i - g_j) ----
-                if (leader) {
-                    tc_fence_after();
-                    constexpr uint32_t id = idesc_f16(1, 0, 0, 128, 128);
+            if (!wait_mma()) { ok = false; break; }
+            const float bi = sb[r], gi = sg[r];
+            const float* gcol = sg + blk * KB;
 #pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        uint64_t a = sdesc(su32(sK) + (kk >> 2) * (kRows * 128) + (kk & 3) * 32,
-                                           16, 1024);
-                        mma_ss(tm, a, a, id, kk > 0);
-                    }
-                    mma_commit(&ctrl->mma[s]);
+            for (int pp = 0; pp < PPT; ++pp) {
+                const int pc = pc0 + pp;
+                float v[32];
+                tmem_ld32(tD + pc * 32, v);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = pc * 32 + jj;
+                    const bool in = in_chunk(j) && j < i;
+                    v[jj] = in ? -bi * v[jj] * expf(gi - gcol[j]) : 0.f;
                 }
+                if (MODE == kBuildA) {
+                    if (valid && piece_in_chunk(pc)) {
+                        float* dst = p.Aout + cidx * KC * KC + rin * KC + (pc * 32 - cl);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            reinterpret_cast<float4*>(dst)[q] =
+                                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                    }
+                } else {
+                    st_op32<false>(sX, r, pc, v);             // A (chain's right operand)
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = pc * 32 + jj;
+                        v[jj] = j >= jmin ? v[jj] : 0.f;
+                        T0[pp * 32 + jj] = eye(j) + v[jj];
+                    }
+                    st_op32<false>(sAop, r, pc, v);           // P_1 = M . A
+                }
+            }
+            if (MODE == kBuildA) {
+                tc_fence_before();
+                bar_sync(bar_id, 256);                 // beta/g and the accumulator are read
+                if (leader) issue_loads(n + NS);
+                continue;
+            }
+        } else if (MODE == kNeumann) {
+            // ---- A row from global memory ----
+#pragma unroll
+            for (int pp = 0; pp < PPT; ++pp) {
+                const int pc = pc0 + pp;
+                float v[32];
+                if (valid && piece_in_chunk(pc)) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.Ain + cidx * KC * KC + rin * KC + (pc * 32 - cl));
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 a = __ldg(src + q);
+                        v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
+                }
+                st_op32<false>(sX, r, pc, v);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = pc * 32 + jj;
+                    v[jj] = j >= jmin ? v[jj] : 0.f;
+                    T0[pp * 32 + jj] = eye(j) + v[jj];
+                }
+                st_op32<false>(sAop, r, pc, v);
+            }
+        } else {
+            // ---- kWY: T row from global memory ----
+#pragma unroll
+            for (int pp = 0; pp < PPT; ++pp) {
+                const int pc = pc0 + pp;
+                if (valid && piece_in_chunk(pc)) {
+                    const float4* src = reinterpret_cast<const float4*>(
+                        p.Tin + cidx * KC * KC + rin * KC + (pc * 32 - cl));
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 a = __ldg(src + q);
+                        T0[pp * 32 + 4 * q] = a.x; T0[pp * 32 + 4 * q + 1] = a.y;
+                        T0[pp * 32 + 4 * q + 2] = a.z; T0[pp * 32 + 4 * q + 3] = a.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) T0[pp * 32 + jj] = 0.f;
+                }
+            }
+        }
+
+        if (MODE == kFused || MODE == kNeumann) {
+            // ---- truncated Neumann series, band mask on every power ----
+            for (int pw = 2; pw <= p.N; ++pw) {
+                publish();
+                mma_chain(sAop, sX);                                   // P_{n-1} A
                 if (!wait_mma()) { ok = false; break; }
-                const float bi = sb[r], gi = sg[r];
-                const float* gcol = sg + blk * KB;
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
@@ -483,295 +562,451 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
-                        const bool in = in_chunk(j) && j < i;
-                        v[jj] = in ? -bi * v[jj] * expf(gi - gcol[j]) : 0.f;
+                        v[jj] = (in_chunk(j) && j >= jmin) ? v[jj] : 0.f;
+                        T0[pp * 32 + jj] += v[jj];
                     }
-                    if (MODE == kBuildA) {
-                        if (valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch))) {
-                            float* dst = p.Aout + cidx * KC * KC + rin * KC + (pc * 32 - cl);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                reinterpret_cast<float4*>(dst)[q] =
-                                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                        }
-                    } else {
-                        float t[32];
-                        st_op32<false>(sX, r, pc, v);             // A (chain's right operand)
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int j = pc * 32 + jj;
-                            v[jj] = j >= jmin ? v[jj] : 0.f;
-                            t[jj] = eye(j) + v[jj];
-                        }
-                        st_op32<false>(sAop, r, pc, v);           // P_1 = M . A
-                        tmem_st32(tT + pc * 32, t);                // T0 = I + P_1
-                    }
+                    if (pw < p.N) st_op32<false>(sAop, r, pc, v);
                 }
-                if (MODE == kBuildA) {
-                    tc_fence_before();
-                    bar_sync(bar_id, 256);                 // beta/g read, accumulator read
-                    if (leader) mbar_arrive(&ctrl->kvfree[s]);
-                    continue;
-                }
-            } else if (MODE == kNeumann) {
-                // ---- A row from global memory ----
+            }
+            if (!ok) break;
+            // ---- parallel residual correction ----
+            if (p.S > 0) {
+#pragma unroll
+                for (int pp = 0; pp < PPT; ++pp) st_op32<false>(sY, r, pc0 + pp, T0P(pp));   // T0
+                publish();
+                mma_chain(sX, sY);                                      // A T0
+                if (!wait_mma()) { ok = false; break; }
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
-                    float v[32], t[32];
-                    const bool have = valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch));
-                    if (have) {
-                        const float4* src = reinterpret_cast<const float4*>(
-                            p.Ain + cidx * KC * KC + rin * KC + (pc * 32 - cl));
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 a = __ldg(src + q);
-                            v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
-                    }
-                    st_op32<false>(sX, r, pc, v);
+                    float v[32];
+                    tmem_ld32(tD + pc * 32, v);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
-                        v[jj] = j >= jmin ? v[jj] : 0.f;
-                        t[jj] = eye(j) + v[jj];
+                        v[jj] = in_chunk(j) ? eye(j) - T0[pp * 32 + jj] + v[jj] : 0.f;   // E
                     }
-                    st_op32<false>(sAop, r, pc, v);
-                    tmem_st32(tT + pc * 32, t);
-                }
-            } else {
-                // ---- kWY: T row from global memory ----
-#pragma unroll
-                for (int pp = 0; pp < PPT; ++pp) {
-                    const int pc = pc0 + pp;
-                    float t[32];
-                    const bool have = valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch));
-                    if (have) {
-                        const float4* src = reinterpret_cast<const float4*>(
-                            p.Tin + cidx * KC * KC + rin * KC + (pc * 32 - cl));
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float4 a = __ldg(src + q);
-                            t[4 * q] = a.x; t[4 * q + 1] = a.y; t[4 * q + 2] = a.z; t[4 * q + 3] = a.w;
-                        }
+                    if (p.S == 1) {
+                        st_op32<false>(sY, r, pc, v);                   // Q = E
+                        st_op32<false>(sAop, r, pc, T0P(pp));           // T0
                     } else {
+                        st_op32<false>(sX, r, pc, v);                   // E
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) t[jj] = 0.f;
+                        for (int jj = 0; jj < 32; ++jj) v[jj] += eye(pc * 32 + jj);
+                        st_op32<false>(sAop, r, pc, v);                 // I + Q_1
                     }
-                    tmem_st32(tT + pc * 32, t);
                 }
-            }
-
-            if (MODE == kFused || MODE == kNeumann) {
-                // ---- truncated Neumann series, band mask on every power ----
-                for (int pw = 2; pw <= p.N; ++pw) {
+                for (int m = 1; m < p.S; ++m) {
                     publish();
-                    mma_chain(sAop, sX);                                   // P_{n-1} A
+                    mma_chain(sAop, sX);                                // (I + Q_m) E
                     if (!wait_mma()) { ok = false; break; }
+                    const bool last = (m == p.S - 1);
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
-                        float v[32], t[32];
-                        tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
+                        float v[32];
+                        tmem_ld32(tD + pc * 32, v);
+                        if (last) {
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int j = pc * 32 + jj;
-                            v[jj] = (in_chunk(j) && j >= jmin) ? v[jj] : 0.f;
-                            t[jj] += v[jj];
+                            for (int jj = 0; jj < 32; ++jj)
+                                if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
+                            st_op32<false>(sY, r, pc, v);               // Q_S
+                            st_op32<false>(sAop, r, pc, T0P(pp));       // T0
+                        } else {
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) {
+                                const int j = pc * 32 + jj;
+                                v[jj] = in_chunk(j) ? v[jj] + eye(j) : 0.f;
+                            }
+                            st_op32<false>(sAop, r, pc, v);             // I + Q_{m+1}
                         }
-                        tmem_st32(tT + pc * 32, t);
-                        if (pw < p.N) st_op32<false>(sAop, r, pc, v);
                     }
                 }
                 if (!ok) break;
-                // ---- parallel residual correction ----
-                if (p.S > 0) {
-#pragma unroll
-                    for (int pp = 0; pp < PPT; ++pp) {
-                        const int pc = pc0 + pp;
-                        float t[32];
-                        tmem_ld32(tT + pc * 32, t);
-                        st_op32<false>(sY, r, pc, t);                      // T0
-                    }
-                    publish();
-                    mma_chain(sX, sY);                                      // A T0
-                    if (!wait_mma()) { ok = false; break; }
-#pragma unroll
-                    for (int pp = 0; pp < PPT; ++pp) {
-                        const int pc = pc0 + pp;
-                        float v[32], t[32];
-                        tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int j = pc * 32 + jj;
-                            v[jj] = in_chunk(j) ? eye(j) - t[jj] + v[jj] : 0.f;   // E
-                        }
-                        if (p.S == 1) {
-                            st_op32<false>(sY, r, pc, v);                   // Q = E
-                            st_op32<false>(sAop, r, pc, t);                 // T0
-                        } else {
-                            st_op32<false>(sX, r, pc, v);                   // E
-#pragma unroll
-                            for (int jj = 0; jj < 32; ++jj) v[jj] += eye(pc * 32 + jj);
-                            st_op32<false>(sAop, r, pc, v);                 // I + Q_1
-                        }
-                    }
-                    for (int m = 1; m < p.S; ++m) {
-                        publish();
-                        mma_chain(sAop, sX);                                // (I + Q_m) E
-                        if (!wait_mma()) { ok = false; break; }
-                        const bool last = (m == p.S - 1);
-#pragma unroll
-                        for (int pp = 0; pp < PPT; ++pp) {
-                            const int pc = pc0 + pp;
-                            float v[32];
-                            if (last) {
-                                float t[32];
-                                tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
-#pragma unroll
-                                for (int jj = 0; jj < 32; ++jj)
-                                    if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
-                                st_op32<false>(sY, r, pc, v);               // Q_S
-                                st_op32<false>(sAop, r, pc, t);             // T0
-                            } else {
-                                tmem_ld32(tD + pc * 32, v);
-#pragma unroll
-                                for (int jj = 0; jj < 32; ++jj) {
-                                    const int j = pc * 32 + jj;
-                                    v[jj] = in_chunk(j) ? v[jj] + eye(j) : 0.f;
-                                }
-                                st_op32<false>(sAop, r, pc, v);             // I + Q_{m+1}
-                            }
-                        }
-                    }
-                    if (!ok) break;
-                    publish();
-                    mma_chain(sAop, sY);                                    // T0 Q_S
-                    if (!wait_mma()) { ok = false; break; }
-#pragma unroll
-                    for (int pp = 0; pp < PPT; ++pp) {
-                        const int pc = pc0 + pp;
-                        float v[32], t[32];
-                        tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj)
-                            if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];     // T = T0 + T0 Q
-                        tmem_st32(tT + pc * 32, t);
-                    }
-                }
-                // ---- T out ----
-                if (p.Tout) {
-#pragma unroll
-                    for (int pp = 0; pp < PPT; ++pp) {
-                        const int pc = pc0 + pp;
-                        float t[32];
-                        tmem_ld32(tT + pc * 32, t);
-                        if (valid && (!SUB || (pc * 32 >= cl && pc * 32 < ch))) {
-                            float* dst = p.Tout + cidx * KC * KC + rin * KC + (pc * 32 - cl);
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                reinterpret_cast<float4*>(dst)[q] =
-                                    make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
-                        }
-                    }
-                }
-            }
-
-            if (MODE == kFused || MODE == kWY) {
-                // ---- WY: T diag(beta [exp g]) -> X (bf16), T diag(beta) -> Y ----
-                const float* bcol = sb + blk * KB;
-                const float* gcol = sg + blk * KB;
+                publish();
+                mma_chain(sAop, sY);                                    // T0 Q_S
+                if (!wait_mma()) { ok = false; break; }
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
-                    float t[32], v[32];
-                    tmem_ld32(tT + pc * 32, t);
+                    float v[32];
+                    tmem_ld32(tD + pc * 32, v);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (in_chunk(pc * 32 + jj)) T0[pp * 32 + jj] += v[jj];   // T = T0 + T0 Q
+                }
+            }
+            // ---- T out ----
+            if (p.Tout) {
+#pragma unroll
+                for (int pp = 0; pp < PPT; ++pp) {
+                    const int pc = pc0 + pp;
+                    if (valid && piece_in_chunk(pc)) {
+                        float* dst = p.Tout + cidx * KC * KC + rin * KC + (pc * 32 - cl);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            reinterpret_cast<float4*>(dst)[q] =
+                                make_float4(T0[pp * 32 + 4 * q], T0[pp * 32 + 4 * q + 1],
+                                            T0[pp * 32 + 4 * q + 2], T0[pp * 32 + 4 * q + 3]);
+                    }
+                }
+            }
+        }
+
+        if (MODE == kFused || MODE == kWY) {
+            // ---- WY: T diag(beta [exp g]) -> X (bf16), T diag(beta) -> Y ----
+            const float* bcol = sb + blk * KB;
+            const float* gcol = sg + blk * KB;
+#pragma unroll
+            for (int pp = 0; pp < PPT; ++pp) {
+                const int pc = pc0 + pp;
+                float t[32], v[32];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = pc * 32 + jj;
+                    const float b = bcol[j];
+                    const float tv = T0[pp * 32 + jj];
+                    v[jj] = p.gated ? tv * (b * expf(gcol[j])) : tv * b;
+                    t[jj] = tv * b;
+                }
+                st_op32<true>(sX, r, pc, v);
+                if (p.gated) st_op32<true>(sY, r, pc, t);
+            }
+            if (uses_V(MODE) && !mbar_wait(&ctrl->fullV[s], use_par)) fail_wait();
+            publish();
+            if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+            if (leader) {
+                constexpr uint32_t id = idesc_f16(1, 1, 0, KB, 128);
+                const uint8_t* bu = p.gated ? sY : sX;
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+#pragma unroll
+                    for (int kk = 0; kk < KB / 16; ++kk) {
+                        const uint32_t ka = su32(sK) + (c * KB + kk * 16) * 128;
+                        const uint32_t va = su32(sV) + (c * KB + kk * 16) * 128;
+                        const uint32_t bo = (c * KB) * 128 + (kk >> 2) * (kRows * 128) +
+                                            (kk & 3) * 32;
+                        mma_ss(tm + c * KB, sdesc(ka, kRows * 128, 1024),
+                               sdesc(su32(sX) + bo, 16, 1024), id, kk > 0);
+                        mma_ss(tm + 128 + c * KB, sdesc(va, kRows * 128, 1024),
+                               sdesc(su32(bu) + bo, 16, 1024), id, kk > 0);
+                    }
+                }
+                mma_commit(&ctrl->mma[s]);
+            }
+            if (!wait_mma()) { ok = false; break; }
+            // Lane r of the W^T / U^T accumulators is head-dim column d = r and
+            // accumulator column x is tile row x.  Thread half h transposes
+            // rows [64h, 64h + 64) through the K (W) and V (U) tiles, which
+            // the finished MMAs no longer read, in the TMA load layout.
+            {
+                const int d = r;
+                const uint32_t dbase = (uint32_t)((d >> 6) * (kRows * 128) + (d & 7) * 2);
+                const int c16 = (d & 63) >> 3;
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp) {
+                    const int x0 = h * 64 + pp * 32;
+                    float w[32], u[32];
+                    tmem_ld2(tl + x0, w, tl + 128 + x0, u);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
-                        const int j = pc * 32 + jj;
-                        const float b = bcol[j];
-                        v[jj] = p.gated ? t[jj] * (b * expf(gcol[j])) : t[jj] * b;
-                        t[jj] = t[jj] * b;
-                    }
-                    st_op32<true>(sX, r, pc, v);
-                    if (p.gated) st_op32<true>(sY, r, pc, t);
-                }
-                publish();
-                if (leader) {
-                    constexpr uint32_t id = idesc_f16(1, 1, 0, KB, 128);
-                    const uint8_t* bu = p.gated ? sY : sX;
-#pragma unroll
-                    for (int c = 0; c < NCH; ++c) {
-#pragma unroll
-                        for (int kk = 0; kk < KB / 16; ++kk) {
-                            const uint32_t ka = su32(sK) + (c * KB + kk * 16) * 128;
-                            const uint32_t va = su32(sV) + (c * KB + kk * 16) * 128;
-                            const uint32_t bo = (c * KB) * 128 + (kk >> 2) * (kRows * 128) +
-                                                (kk & 3) * 32;
-                            mma_ss(tm + c * KB, sdesc(ka, kRows * 128, 1024),
-                                   sdesc(su32(sX) + bo, 16, 1024), id, kk > 0);
-                            mma_ss(tm + 128 + c * KB, sdesc(va, kRows * 128, 1024),
-                                   sdesc(su32(bu) + bo, 16, 1024), id, kk > 0);
-                        }
-                    }
-                    mma_commit(&ctrl->mma[s]);
-                }
-                if (!wait_mma()) { ok = false; break; }
-                // Lane r of the W^T / U^T accumulators is head-dim column d = r and
-                // accumulator column x is tile row x.  Thread half h transposes
-                // rows [64h, 64h + 64) through the K (W) and V (U) tiles, which
-                // the finished MMAs no longer read, in the TMA load layout.
-                {
-                    const int d = r;
-                    const uint32_t dbase = (uint32_t)((d >> 6) * (kRows * 128) + (d & 7) * 2);
-                    const int c16 = (d & 63) >> 3;
-#pragma unroll
-                    for (int pp = 0; pp < 2; ++pp) {
-                        const int x0 = h * 64 + pp * 32;
-                        float w[32], u[32];
-                        tmem_ld2(tl + x0, w, tl + 128 + x0, u);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) {
-                            const int x = x0 + jj;
-                            const uint32_t off = dbase + x * 128 + ((c16 ^ (x & 7)) << 4);
-                            *reinterpret_cast<__nv_bfloat16*>(sK + off) = __float2bfloat16_rn(w[jj]);
-                            *reinterpret_cast<__nv_bfloat16*>(sV + off) = __float2bfloat16_rn(u[jj]);
-                        }
+                        const int x = x0 + jj;
+                        const uint32_t off = dbase + x * 128 + ((c16 ^ (x & 7)) << 4);
+                        *reinterpret_cast<__nv_bfloat16*>(sK + off) = __float2bfloat16_rn(w[jj]);
+                        *reinterpret_cast<__nv_bfloat16*>(sV + off) = __float2bfloat16_rn(u[jj]);
                     }
                 }
-                fence_async_smem();
-                tc_fence_before();
-                bar_sync(bar_id, 256);
-                if (leader) {
-                    const int y = (int)row0;
-                    tma_store_2d(&mW, 0, y, sK);
-                    tma_store_2d(&mW, 64, y, sK + kRows * 128);
-                    tma_store_2d(&mU, 0, y, sV);
-                    tma_store_2d(&mU, 64, y, sV + kRows * 128);
-                    bulk_commit();
-                    bulk_wait_read();                       // tiles may be reloaded now
-                    mbar_arrive(&ctrl->kvfree[s]);
-                }
-                continue;
             }
+            fence_async_smem();
             tc_fence_before();
-            bar_sync(bar_id, 256);                 // accumulators free for the next tile
+            bar_sync(bar_id, 256);
+            if (leader) {
+                const int y = (int)row0;
+                tma_store_2d(&mW, 0, y, sK);
+                tma_store_2d(&mW, 64, y, sK + kRows * 128);
+                tma_store_2d(&mU, 0, y, sV);
+                tma_store_2d(&mU, 64, y, sV + kRows * 128);
+                bulk_commit();
+                bulk_wait_read();                       // tiles may be reloaded now
+                issue_loads(n + NS);
+            }
+            continue;
         }
-        if (!ok) {
-            atomicExch(&ctrl->abort, 1);
-            // outstanding MMAs of this slot finish before TMEM is released
-            mbar_wait(&ctrl->mma[s], mma_phase);
-        }
-        if (leader) bulk_wait_all();               // W, U stores complete
+        tc_fence_before();
+        bar_sync(bar_id, 256);                 // accumulators free for the next tile
     }
+    if (!ok) {
+        atomicExch(&ctrl->abort, 1);
+        // outstanding MMAs of this slot finish before TMEM is released
+        mbar_wait(&ctrl->mma[s], mma_phase);
+    }
+#undef T0P
+    if (leader) bulk_wait_all();                   // W, U stores complete
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------------- //
+// INT8 truncated Neumann series on the tensor cores (k = 64)
+// ------------------------------------------------------------------------- //
+// Same tile / slot structure as k_chunk_tc: a tile stacks two 64-token chunks,
+// acc_n = q_{n-1} q_1 is one M=128, N=128, K=64 tcgen05.mma of kind::i8
+// (s8 x s8 -> s32 in TMEM), and each row reads its chunk's diagonal block.  The
+// per-chunk maxima are reduced across the 4 warps that hold a chunk through
+// shared memory.  Every float32 operation is the IEEE-rounded one of the scheme
+// in gdn.h, in that order, so codes, accumulators, scales and T are bit-exact.
+__host__ __device__ constexpr uint32_t idesc_i8(int N, int M) {
+    // D s32 (2), A and B signed 8-bit (1), A K-major, B MN-major
+    return (2u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ int quant_i8(float x, float r) {
+    float y = rintf(__fmul_rn(x, r));
+    y = fminf(fmaxf(y, -127.f), 127.f);
+    return (int)y;
+}
+// 32 int8 codes -> two 16-byte groups of a 128-byte swizzled row
+__device__ __forceinline__ void st_i8x32(uint8_t* buf, int row, int q0, const int (&c)[32]) {
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int b = 16 * g + 4 * k;
+            w[k] = (uint32_t)(c[b] & 0xff) | ((uint32_t)(c[b + 1] & 0xff) << 8) |
+                   ((uint32_t)(c[b + 2] & 0xff) << 16) | ((uint32_t)(c[b + 3] & 0xff) << 24);
+        }
+        const int q = q0 + g;
+        *reinterpret_cast<uint4*>(buf + row * 128 + (((q & 7) ^ (row & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+struct ParamsI8 {
+    int64_t rows;
+    int ntiles;
+    int N, mask;
+    const float* A;
+    float* T;
+    int8_t* q;
+    int32_t* acc;
+    float* scale;
+    int* status;
+};
+
+constexpr int kI8Slots = 2;
+constexpr int kI8OpBytes = kRows * 128;            // 16 KB, rows at a 128-byte pitch
+constexpr int kI8BBytes = 64 * 128;                // 8 KB: K = 64 rows of 128 codes
+
+__global__ void __launch_bounds__(256 * kI8Slots, 1)
+k_neumann_i8_tc(const ParamsI8 p) {
+    constexpr int KC = 64;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((su32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    struct __align__(8) CtrlI8 {
+        uint64_t mma[kI8Slots];
+        uint32_t tmem;
+        int abort;
+        float red_f[kI8Slots][2][4];
+        int red_i[kI8Slots][2][4];
+    };
+    CtrlI8* ctrl = reinterpret_cast<CtrlI8*>(smem + kI8Slots * (kI8OpBytes + kI8BBytes));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kI8Slots; ++s) mbar_init(&ctrl->mma[s], 1);
+        ctrl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tmem_alloc(&ctrl->tmem, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ctrl->tmem;
+
+    const int s = warp / 8;
+    const int h = (warp % 8) / 4;
+    const int r = ((warp & 3) << 5) | lane;
+    const int c = r / KC;                          // chunk of this row in the tile
+    const int i = r % KC;
+    const int wq = ((warp & 3) & 1) * 2 + h;       // this warp's slot among its chunk's 4 warps
+    const int jmin = p.mask ? i - p.N : -KC;
+    uint8_t* sA = smem + s * (kI8OpBytes + kI8BBytes);
+    uint8_t* sB = sA + kI8OpBytes;
+    const uint32_t tm = tmem_base + (uint32_t)(s * 128);
+    const uint32_t tD = tm + ((uint32_t)((warp & 3) * 32) << 16) + c * KC + 32 * h;
+    const bool leader = (warp % 8) == 0 && lane == 0;
+    const int bar_id = 1 + s;
+    uint32_t mma_phase = 0;
+    bool ok = true;
+
+    // maximum over the chunk held by this row's 4 warps
+    auto chunk_max_f = [&](float v) {
+        for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) ctrl->red_f[s][c][wq] = v;
+        bar_sync(bar_id, 256);
+        const float m = fmaxf(fmaxf(ctrl->red_f[s][c][0], ctrl->red_f[s][c][1]),
+                              fmaxf(ctrl->red_f[s][c][2], ctrl->red_f[s][c][3]));
+        return m;
+    };
+    auto chunk_max_i = [&](int v) {
+        for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) ctrl->red_i[s][c][wq] = v;
+        bar_sync(bar_id, 256);
+        return max(max(ctrl->red_i[s][c][0], ctrl->red_i[s][c][1]),
+                   max(ctrl->red_i[s][c][2], ctrl->red_i[s][c][3]));
+    };
+
+    for (int n = s;; n += kI8Slots) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (tile >= p.ntiles) break;
+        const int64_t grow = (int64_t)tile * kRows + r;
+        const bool valid = grow < p.rows;
+        const int64_t cidx = grow / KC, rin = grow % KC;
+        bar_sync(bar_id, 256);                     // previous tile's reads of sA, sB, red done
+        float a[32];
+        if (valid) {
+            const float4* src = reinterpret_cast<const float4*>(p.A + cidx * KC * KC + rin * KC + 32 * h);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float4 t = __ldg(src + q);
+                a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
+            }
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) a[jj] = 0.f;
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            const int j = 32 * h + jj;
+            if (j < jmin) a[jj] = 0.f;                 // P_1 = M . A
+            amax = fmaxf(amax, fabsf(a[jj]));
+        }
+        amax = chunk_max_f(amax);
+        const float r1 = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+        const float s1 = amax > 0.f ? __fdiv_rn(amax, 127.f) : 0.f;
+        int q[32];
+        float t[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            const int j = 32 * h + jj;
+            q[jj] = amax > 0.f ? quant_i8(a[jj], r1) : 0;
+            t[jj] = __fadd_rn(i == j ? 1.f : 0.f, __fmul_rn(s1, (float)q[jj]));
+        }
+        st_i8x32(sA, r, 2 * h, q);                     // q_1 as the left operand
+        st_i8x32(sB, i, 4 * c + 2 * h, q);             // q_1 as the right operand
+        if (valid) {
+            const int64_t base = (cidx * p.N * KC + rin) * KC + 32 * h;
+            if (p.q) {
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 4)
+                    *reinterpret_cast<char4*>(p.q + base + jj) =
+                        make_char4((signed char)q[jj], (signed char)q[jj + 1],
+                                   (signed char)q[jj + 2], (signed char)q[jj + 3]);
+            }
+            if (p.acc) {
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 4)
+                    *reinterpret_cast<int4*>(p.acc + base + jj) = make_int4(0, 0, 0, 0);
+            }
+            if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N] = s1;
+        }
+        float sprev = s1;
+        for (int pw = 1; pw < p.N; ++pw) {
+            fence_async_smem();
+            tc_fence_before();
+            bar_sync(bar_id, 256);
+            tc_fence_after();
+            if (leader) {
+                constexpr uint32_t id = idesc_i8(128, 128);
+#pragma unroll
+                for (int kk = 0; kk < KC / 32; ++kk) {
+                    const uint64_t ad = sdesc(su32(sA) + kk * 32, 16, 1024);
+                    const uint64_t bd = sdesc(su32(sB) + kk * 32 * 128, 16, 1024);
+                    mma_i8(tm, ad, bd, id, kk > 0);
+                }
+                mma_commit(&ctrl->mma[s]);
+            }
+            bool good = mbar_wait(&ctrl->mma[s], mma_phase);
+            mma_phase ^= 1;
+            if (!good) {
+                atomicExch(&ctrl->abort, 1);
+                raise_status(p.status, kStatusTimeout);
+            }
+            tc_fence_after();
+            uint32_t raw[32];
+            tmem_ld32_async(tD, raw);
+            tmem_wait_ld();
+            int accv[32];
+            int m = 0;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                const int j = 32 * h + jj;
+                accv[jj] = (j < jmin) ? 0 : (int)raw[jj];
+                m = max(m, abs(accv[jj]));
+            }
+            m = chunk_max_i(m);
+            if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+            const float mf = (float)m;
+            const float rn = m > 0 ? __fdiv_rn(127.f, mf) : 0.f;
+            const float sn = m > 0 ? __fmul_rn(__fmul_rn(sprev, s1), __fdiv_rn(mf, 127.f)) : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                q[jj] = m > 0 ? quant_i8((float)accv[jj], rn) : 0;
+                t[jj] = __fadd_rn(t[jj], __fmul_rn(sn, (float)q[jj]));
+            }
+            if (pw + 1 < p.N) st_i8x32(sA, r, 2 * h, q);
+            if (valid) {
+                const int64_t base = ((cidx * p.N + pw) * KC + rin) * KC + 32 * h;
+                if (p.q) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 4)
+                        *reinterpret_cast<char4*>(p.q + base + jj) =
+                            make_char4((signed char)q[jj], (signed char)q[jj + 1],
+                                       (signed char)q[jj + 2], (signed char)q[jj + 3]);
+                }
+                if (p.acc) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 4)
+                        *reinterpret_cast<int4*>(p.acc + base + jj) =
+                            make_int4(accv[jj], accv[jj + 1], accv[jj + 2], accv[jj + 3]);
+                }
+                if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N + pw] = sn;
+            }
+            sprev = sn;
+        }
+        if (!ok) break;
+        if (valid) {
+            float* dst = p.T + cidx * KC * KC + rin * KC + 32 * h;
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+                reinterpret_cast<float4*>(dst)[q4] =
+                    make_float4(t[4 * q4], t[4 * q4 + 1], t[4 * q4 + 2], t[4 * q4 + 3]);
+        }
+        tc_fence_before();
+    }
+    if (!ok) mbar_wait(&ctrl->mma[s], mma_phase);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 256);
     }
 }
 
@@ -893,7 +1128,7 @@ static cudaError_t dispatch(int k, const IO& io, const Params& p, cudaStream_t s
 }  // namespace tcg
 
 bool tc_available() { return true; }
-bool tc_i8_available() { return false; }
+bool tc_i8_available() { return true; }
 
 cudaError_t launch_build_A_tc(const void* K, const float* beta, const float* g, float* A,
                               int64_t nc, int k, cudaStream_t st) {
@@ -932,9 +1167,29 @@ cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const flo
     return tcg::dispatch<tcg::kWY, 1>(k, io, p, st);
 }
 
-cudaError_t launch_neumann_i8_tc(const float*, float*, int, int, int8_t*, int32_t*, float*,
-                                 int64_t, cudaStream_t) {
-    return cudaErrorNotSupported;
+cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8_t* q,
+                                 int32_t* acc, float* sc, int64_t nc, cudaStream_t st) {
+    tcg::ParamsI8 p;
+    memset(&p, 0, sizeof p);
+    p.rows = nc * 64;
+    p.ntiles = (int)((p.rows + tcg::kRows - 1) / tcg::kRows);
+    p.N = N;
+    p.mask = mask;
+    p.A = A;
+    p.T = T;
+    p.q = q;
+    p.acc = acc;
+    p.scale = sc;
+    p.status = status_ptr();
+    // two CTAs per SM at most: each holds 256 of the SM's 512 TMEM columns
+    const size_t smem = 80 * 1024;
+    cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int cap = 2 * tcg::num_sms();
+    const int grid = p.ntiles < cap ? p.ntiles : cap;
+    tcg::k_neumann_i8_tc<<<grid, 256 * tcg::kI8Slots, smem, st>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, const float* g,

@@ -146,7 +146,9 @@ int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta,
  * [B,H,d,d] f32 (d_v x d_k, NULL = zero).  Out: O [B,H,T,d] (dtype),
  * S_final [B,H,d,d] f32.  `workspace` is caller-owned device memory of at
  * least gdn_forward_workspace_bytes(s, dtype) bytes (W_g and U for every
- * chunk); its contents on entry do not matter.
+ * chunk in dtype, then A and T in f32); its contents on entry do not matter.
+ * k = 64.  The inter-chunk scan splits the d_v rows of the state across CTAs
+ * (rows of S never mix), each CTA walking its head's chunks in order.
  */
 int gdn_forward(const void* Q, const void* K, const void* V, const float* beta,
                 const float* g, const float* S0, int N, int mask, int S,
@@ -156,7 +158,8 @@ int gdn_forward(const void* Q, const void* K, const void* V, const float* beta,
 int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype);
 
 /* Synchronises `stream`, returns the device status word of the current
- * device (GDN_OK or GDN_ERR_TIMEOUT) and clears it. */
+ * device (GDN_OK, GDN_ERR_TIMEOUT, or GDN_ERR_CUDA when a kernel found its
+ * shared memory misaligned) and clears it. */
 int gdn_get_status(void* stream);
 
 /* Message for the most recent nonzero return on this host thread. */

@@ -122,5 +122,6 @@ def test_empty_inputs_are_noops(lib):
 def test_workspace_size(lib):
     s = sh(B=2, H=3, T=512, k=64)
     nc = 2 * 3 * 8
-    assert lib.gdn_forward_workspace_bytes(s, 1) == 2 * nc * 64 * 128 * 2
+    # W_g and U (bf16) plus A and T (fp32) for every chunk
+    assert lib.gdn_forward_workspace_bytes(s, 1) == 2 * nc * 64 * 128 * 2 + 2 * nc * 64 * 64 * 4
     assert lib.gdn_forward_workspace_bytes(sh(k=48), 1) == -1
