@@ -268,6 +268,11 @@ int64_t gdn_launch_count(void) { return t_launches; }
 
 // Device address of the status word for kernels in other translation units.
 namespace gdn {
+void record_error(int code, const char* msg) {
+    (void)code;
+    t_last_error = msg;
+}
+
 int* status_ptr() {
     static thread_local int dev = -1;
     static thread_local int* ptr = nullptr;

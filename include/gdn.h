@@ -157,6 +157,29 @@ int gdn_forward(const void* Q, const void* K, const void* V, const float* beta,
                 void* stream);
 int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype);
 
+/*
+ * gdn_forward without a workspace argument: it allocates nothing.  The pages
+ * have no counterpart to this call; it exists for callers that may not
+ * allocate device memory while they run (for example a plug-in inside a
+ * serving process that owns the whole GPU memory pool and hands out no
+ * allocator, or a deployment whose memory budget is fixed at start-up), for
+ * whom a cudaMalloc mid-request is forbidden or would synchronise the device.
+ * The scratch (W_g, U, A, T) lives in a 64 MiB device array inside the
+ * library, held on every GPU that loads it until the library is unloaded.
+ * Problems needing more than that (gdn_forward_workspace_bytes(s, dtype) >
+ * 64 MiB, about 680 chunks of 64 bf16 tokens) return GDN_ERR_ARG.  All calls
+ * on a device share the array and leave their data in it; nothing needs to
+ * start at zero, but calls whose kernels may overlap on the GPU race on it, so
+ * order them on one stream.  The first call on each device (made with that
+ * device current) looks up the array's address: make it before any stream
+ * capture.  Arguments and results are otherwise those of gdn_forward.
+ */
+int gdn_forward_static(const void* Q, const void* K, const void* V,
+                       const float* beta, const float* g, const float* S0,
+                       int N, int mask, int S, int exact, void* O,
+                       float* S_final, gdn_shape s, gdn_dtype dtype,
+                       void* stream);
+
 /* Synchronises `stream`, returns the device status word of the current
  * device (GDN_OK, GDN_ERR_TIMEOUT, or GDN_ERR_CUDA when a kernel found its
  * shared memory misaligned) and clears it. */
