@@ -411,27 +411,39 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         }
     };
     // the slot's leader loads its own tiles: K, beta, g on fullK, V on fullV
-    auto issue_loads = [&](int n) {
+    int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
+    auto issue_k = [&](int n) {
         const int tile = blockIdx.x + n * gridDim.x;
         if (!uses_K(MODE) || tile >= p.ntiles) return;
+        ++k_issued;
         const int y = tile * kRows;
         mbar_expect_tx(&ctrl->fullK[s], kRows * kD * 2 + 2 * kRows * 4);
         tma_load_2d(sK, &mK, 0, y, &ctrl->fullK[s]);
         tma_load_2d(sK + kRows * 128, &mK, 64, y, &ctrl->fullK[s]);
         tma_load_1d(sb, &mB, y, &ctrl->fullK[s]);
         tma_load_1d(sg, &mG, y, &ctrl->fullK[s]);
-        if (uses_V(MODE)) {
-            mbar_expect_tx(&ctrl->fullV[s], kRows * kD * 2);
-            tma_load_2d(sV, &mV, 0, y, &ctrl->fullV[s]);
-            tma_load_2d(sV + kRows * 128, &mV, 64, y, &ctrl->fullV[s]);
-        }
     };
+    auto issue_v = [&](int n) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (!uses_V(MODE) || tile >= p.ntiles) return;
+        ++v_issued;
+        const int y = tile * kRows;
+        mbar_expect_tx(&ctrl->fullV[s], kRows * kD * 2);
+        tma_load_2d(sV, &mV, 0, y, &ctrl->fullV[s]);
+        tma_load_2d(sV + kRows * 128, &mV, 64, y, &ctrl->fullV[s]);
+    };
+    // W leaves through the operand buffers (free once the WY products are done),
+    // U through the V tile; K is reloaded for the next tile meanwhile.
+    uint8_t* sWst = (MODE == kWY) ? sX : sAop;
     auto in_chunk = [&](int j) { return SUB ? (j >= cl && j < ch) : true; };
 #define T0P(pp) (*reinterpret_cast<float(*)[32]>(&T0[(pp) * 32]))
     auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
     auto piece_in_chunk = [&](int pc) { return !SUB || (pc * 32 >= cl && pc * 32 < ch); };
 
-    if (leader) issue_loads(s);
+    if (leader) {
+        issue_k(s);
+        issue_v(s);
+    }
 
     for (int n = s;; n += NS) {
         const int tile = blockIdx.x + n * gridDim.x;
@@ -444,6 +456,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         const int64_t rin = grow % KC;                   // row inside the chunk
         float T0[PPT * 32];                              // this thread's part of row r of T0 / T
 
+        if (MODE == kWY && leader && n != s) {
+            bulk_wait_read();                        // previous W/U stores have read X, Y, V
+            issue_v(n);
+        }
         if (uses_K(MODE) && !mbar_wait(&ctrl->fullK[s], use_par)) fail_wait();
         bar_sync(bar_id, 256);
         if (*(volatile int*)&ctrl->abort) { ok = false; break; }
@@ -460,8 +476,13 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     mma_ss(tm, a, a, id, kk > 0);
                 }
                 mma_commit(&ctrl->mma[s]);
+                if (MODE == kFused && n != s) {
+                    bulk_wait_read();                // previous W/U stores have read Aop, X, V
+                    issue_v(n);
+                }
             }
             if (!wait_mma()) { ok = false; break; }
+            if (MODE == kFused) bar_sync(bar_id, 256);   // staging free before operands are written
             const float bi = sb[r], gi = sg[r];
             const float* gcol = sg + blk * KB;
 #pragma unroll
@@ -473,7 +494,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
                     const bool in = in_chunk(j) && j < i;
-                    v[jj] = in ? -bi * v[jj] * expf(gi - gcol[j]) : 0.f;
+                    v[jj] = in ? -bi * v[jj] * __expf(gi - gcol[j]) : 0.f;
                 }
                 if (MODE == kBuildA) {
                     if (valid && piece_in_chunk(pc)) {
@@ -497,7 +518,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             if (MODE == kBuildA) {
                 tc_fence_before();
                 bar_sync(bar_id, 256);                 // beta/g and the accumulator are read
-                if (leader) issue_loads(n + NS);
+                if (leader) issue_k(n + NS);
                 continue;
             }
         } else if (MODE == kNeumann) {
@@ -666,7 +687,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     const int j = pc * 32 + jj;
                     const float b = bcol[j];
                     const float tv = T0[pp * 32 + jj];
-                    v[jj] = p.gated ? tv * (b * expf(gcol[j])) : tv * b;
+                    v[jj] = p.gated ? tv * (b * __expf(gcol[j])) : tv * b;
                     t[jj] = tv * b;
                 }
                 st_op32<true>(sX, r, pc, v);
@@ -695,10 +716,11 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 mma_commit(&ctrl->mma[s]);
             }
             if (!wait_mma()) { ok = false; break; }
+            if (leader) issue_k(n + NS);                 // K, beta, g are no longer read
             // Lane r of the W^T / U^T accumulators is head-dim column d = r and
             // accumulator column x is tile row x.  Thread half h transposes
-            // rows [64h, 64h + 64) through the K (W) and V (U) tiles, which
-            // the finished MMAs no longer read, in the TMA load layout.
+            // rows [64h, 64h + 64) into the W staging tile and the V tile, in
+            // the TMA load layout.
             {
                 const int d = r;
                 const uint32_t dbase = (uint32_t)((d >> 6) * (kRows * 128) + (d & 7) * 2);
@@ -712,7 +734,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     for (int jj = 0; jj < 32; ++jj) {
                         const int x = x0 + jj;
                         const uint32_t off = dbase + x * 128 + ((c16 ^ (x & 7)) << 4);
-                        *reinterpret_cast<__nv_bfloat16*>(sK + off) = __float2bfloat16_rn(w[jj]);
+                        *reinterpret_cast<__nv_bfloat16*>(sWst + off) = __float2bfloat16_rn(w[jj]);
                         *reinterpret_cast<__nv_bfloat16*>(sV + off) = __float2bfloat16_rn(u[jj]);
                     }
                 }
@@ -722,13 +744,11 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             bar_sync(bar_id, 256);
             if (leader) {
                 const int y = (int)row0;
-                tma_store_2d(&mW, 0, y, sK);
-                tma_store_2d(&mW, 64, y, sK + kRows * 128);
+                tma_store_2d(&mW, 0, y, sWst);
+                tma_store_2d(&mW, 64, y, sWst + kRows * 128);
                 tma_store_2d(&mU, 0, y, sV);
                 tma_store_2d(&mU, 64, y, sV + kRows * 128);
                 bulk_commit();
-                bulk_wait_read();                       // tiles may be reloaded now
-                issue_loads(n + NS);
             }
             continue;
         }
@@ -737,8 +757,13 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     }
     if (!ok) {
         atomicExch(&ctrl->abort, 1);
-        // outstanding MMAs of this slot finish before TMEM is released
+        // outstanding MMAs of this slot finish before TMEM is released, and the
+        // copies it issued land before the CTA's shared memory goes away
         mbar_wait(&ctrl->mma[s], mma_phase);
+        if (leader) {
+            if (k_issued > 0) mbar_wait(&ctrl->fullK[s], (uint32_t)((k_issued - 1) & 1));
+            if (v_issued > 0) mbar_wait(&ctrl->fullV[s], (uint32_t)((v_issued - 1) & 1));
+        }
     }
 #undef T0P
     if (leader) bulk_wait_all();                   // W, U stores complete
