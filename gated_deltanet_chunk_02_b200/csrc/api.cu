@@ -100,9 +100,9 @@ int gdn_build_A(const void* K, const float* beta, const float* g, float* A, gdn_
     if (nc == 0) return GDN_OK;
     GDN_TRY(check_ptrs({{K, "K"}, {beta, "beta"}, {g, "g"}, {A, "A"}}));
     cudaStream_t st = (cudaStream_t)stream;
+    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "build_A serves k <= 128");
     if (dtype == GDN_BF16 && gdn::tc_available())
         return launched(gdn::launch_build_A_tc(K, beta, g, A, nc, s.k, st), "build_A (tcgen05)");
-    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "build_A: k=256 needs the bf16 tensor-core path");
     return launched(gdn::launch_build_A_simt(K, beta, g, A, nc, s.k, dtype == GDN_BF16, st),
                     "build_A");
 }
@@ -118,8 +118,7 @@ int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask, i
     cudaStream_t st = (cudaStream_t)stream;
     if (prec == GDN_PREC_F16) {
         if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
-        if (s.k == 256 && !(mask == 1 && S == 0))
-            return fail(GDN_ERR_UNSUPPORTED, "k=256 on tensor cores supports mask=1, S=0 only");
+        if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "tensor-core Neumann chain serves k <= 128");
         return launched(gdn::launch_neumann_tc(A, T, nc, s.k, N, mask, S, st), "neumann (tcgen05)");
     }
     if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "float32 Neumann chain supports k <= 128");
@@ -143,9 +142,9 @@ int gdn_wy(const float* T, const void* K, const void* V, const float* beta, cons
     GDN_TRY(check_ptrs({{T, "T"}, {K, "K"}, {V, "V"}, {beta, "beta"}, {W, "W"}, {U, "U"}}));
     GDN_TRY(check_opt_ptr(g, "g"));
     cudaStream_t st = (cudaStream_t)stream;
+    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "wy serves k <= 128");
     if (dtype == GDN_BF16 && gdn::tc_available())
         return launched(gdn::launch_wy_tc(T, K, V, beta, g, W, U, nc, s.k, st), "wy (tcgen05)");
-    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "wy: k=256 needs the bf16 tensor-core path");
     return launched(gdn::launch_wy_simt(T, K, V, beta, g, W, U, nc, s.k, dtype == GDN_BF16, st),
                     "wy");
 }
@@ -183,8 +182,7 @@ int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta, const fl
     GDN_TRY(check_opt_ptr(T_out, "T_out"));
     cudaStream_t st = (cudaStream_t)stream;
     if (dtype == GDN_BF16 && gdn::tc_available()) {
-        if (s.k == 256 && !(mask == 1 && S == 0))
-            return fail(GDN_ERR_UNSUPPORTED, "k=256 on tensor cores supports mask=1, S=0 only");
+        if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "fused tensor-core path serves k <= 128");
         return launched(gdn::launch_fused_tc(K, V, beta, g, N, mask, S, gated, W, U, T_out, nc,
                                              s.k, st),
                         "chunk_wy_fused (tcgen05)");

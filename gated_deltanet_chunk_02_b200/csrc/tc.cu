@@ -56,9 +56,9 @@ struct SlotLayout {
     static constexpr int kXY = (MODE == kBuildA) ? 0 : kRows * KB * 2;  // 16-bit [KB/64][128][64]
     static constexpr int offK = 0;
     static constexpr int offV = offK + kK;
-    static constexpr int offAop = offV + kV;
-    static constexpr int offX = offAop + kAop;
-    static constexpr int offY = offX + kXY;
+    static constexpr int offX = offV + kV;
+    static constexpr int offAop = offX + kXY;
+    static constexpr int offY = offAop + kAop;
     static constexpr int bytes = offY + kXY;
     static constexpr int bg_bytes = uses_K(MODE) ? 2 * kRows * 4 : 0;  // beta[128], g[128]
 };
@@ -136,6 +136,32 @@ __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint3
         "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// 32 fp16 values (columns 32p .. 32p+31 of this lane's row) -> 16 packed TMEM columns
+__device__ __forceinline__ void tmem_st_h16(uint32_t taddr, const float (&v)[32]) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+        "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+        "r"(w[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t* b) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      su32(b))
@@ -206,9 +232,18 @@ __device__ __forceinline__ uint32_t pack_b2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 u) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(u.x), "r"(u.y),
+                 "r"(u.z), "r"(u.w)
+                 : "memory");
+}
+__device__ __forceinline__ void sts16(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
 // Store 32 values (columns 32p .. 32p+31 of row r) into an operand buffer.
 template <bool BF16>
 __device__ __forceinline__ void st_op32(uint8_t* buf, int r, int p, const float (&v)[32]) {
+    const uint32_t base = su32(buf);
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         uint4 u;
@@ -223,7 +258,7 @@ __device__ __forceinline__ void st_op32(uint8_t* buf, int r, int p, const float 
             u.z = pack_h2(v[8 * g + 4], v[8 * g + 5]);
             u.w = pack_h2(v[8 * g + 6], v[8 * g + 7]);
         }
-        *reinterpret_cast<uint4*>(buf + op_off(r, 4 * p + g)) = u;
+        sts128(base + op_off(r, 4 * p + g), u);
     }
 }
 
@@ -265,6 +300,31 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// two 16-column pieces with one wait
+__device__ __forceinline__ void tmem_ld2x16(uint32_t a0, float (&v0)[16], uint32_t a1,
+                                            float (&v1)[16]) {
+    uint32_t r0[16], r1[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]), "=r"(r0[5]),
+          "=r"(r0[6]), "=r"(r0[7]), "=r"(r0[8]), "=r"(r0[9]), "=r"(r0[10]), "=r"(r0[11]),
+          "=r"(r0[12]), "=r"(r0[13]), "=r"(r0[14]), "=r"(r0[15])
+        : "r"(a0));
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r1[0]), "=r"(r1[1]), "=r"(r1[2]), "=r"(r1[3]), "=r"(r1[4]), "=r"(r1[5]),
+          "=r"(r1[6]), "=r"(r1[7]), "=r"(r1[8]), "=r"(r1[9]), "=r"(r1[10]), "=r"(r1[11]),
+          "=r"(r1[12]), "=r"(r1[13]), "=r"(r1[14]), "=r"(r1[15])
+        : "r"(a1));
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        v0[i] = __uint_as_float(r0[i]);
+        v1[i] = __uint_as_float(r1[i]);
+    }
 }
 // two 32-column pieces (e.g. an accumulator piece and a T0 piece) with one wait
 __device__ __forceinline__ void tmem_ld2(uint32_t a0, float (&v0)[32], uint32_t a1, float (&v1)[32]) {
@@ -391,6 +451,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     };
     // hand the operands written by this slot to the tensor pipe
     auto publish = [&]() {
+        tmem_wait_st();
         fence_async_smem();
         tc_fence_before();
         bar_sync(bar_id, 256);
@@ -400,16 +461,30 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     auto mma_chain = [&](const uint8_t* a_buf, const uint8_t* b_buf) {
         if (leader) {
             constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
-#pragma unroll
+            const uint32_t ab = su32(a_buf), bb = su32(b_buf);
+#pragma unroll 1
             for (int kk = 0; kk < KB / 16; ++kk) {
-                uint64_t a = sdesc(su32(a_buf) + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16,
-                                   1024);
-                uint64_t b = sdesc(su32(b_buf) + kk * 2048, KB * 128, 1024);
+                uint64_t a = sdesc(ab + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
+                uint64_t b = sdesc(bb + kk * 2048, KB * 128, 1024);
                 mma_ss(tm, a, b, id, kk > 0);
             }
             mma_commit(&ctrl->mma[s]);
         }
     };
+    // k x k chain product D = Aop[128 x KB] (TMEM, fp16 pairs) * b_buf[KB x 128] (MN-major)
+    auto mma_chain_t = [&](const uint8_t* b_buf) {
+        if (leader) {
+            constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
+            const uint32_t bb = su32(b_buf);
+#pragma unroll 1
+            for (int kk = 0; kk < KB / 16; ++kk) {
+                uint64_t b = sdesc(bb + kk * 2048, KB * 128, 1024);
+                mma_ts(tm, tm + 128 + kk * 8, b, id, kk > 0);
+            }
+            mma_commit(&ctrl->mma[s]);
+        }
+    };
+    const uint32_t tA = tl + 128;                 // this row's A operand (fp16 pairs)
     // the slot's leader loads its own tiles: K, beta, g on fullK, V on fullV
     int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
     auto issue_k = [&](int n) {
@@ -434,7 +509,19 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     };
     // W leaves through the operand buffers (free once the WY products are done),
     // U through the V tile; K is reloaded for the next tile meanwhile.
-    uint8_t* sWst = (MODE == kWY) ? sX : sAop;
+    uint8_t* sWst = (MODE == kWY) ? sX : sAop;   // followed by Y: 32 KB at KB = 64
+    bool staged_free = true;                       // previous tile's stores have read Aop/Y/V
+    // The previous tile's W/U stores read Aop+Y and V; before this tile first
+    // writes Y (or V is reloaded) the leader waits for those reads to finish.
+    auto release_staging = [&](int n) {
+        if (staged_free) return;
+        if (leader) {
+            bulk_wait_read();
+            issue_v(n);
+        }
+        bar_sync(bar_id, 256);
+        staged_free = true;
+    };
     auto in_chunk = [&](int j) { return SUB ? (j >= cl && j < ch) : true; };
 #define T0P(pp) (*reinterpret_cast<float(*)[32]>(&T0[(pp) * 32]))
     auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
@@ -456,10 +543,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         const int64_t rin = grow % KC;                   // row inside the chunk
         float T0[PPT * 32];                              // this thread's part of row r of T0 / T
 
-        if (MODE == kWY && leader && n != s) {
-            bulk_wait_read();                        // previous W/U stores have read X, Y, V
-            issue_v(n);
-        }
         if (uses_K(MODE) && !mbar_wait(&ctrl->fullK[s], use_par)) fail_wait();
         bar_sync(bar_id, 256);
         if (*(volatile int*)&ctrl->abort) { ok = false; break; }
@@ -469,20 +552,15 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             if (leader) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_f16(1, 0, 0, 128, 128);
-#pragma unroll
+                const uint32_t kbase = su32(sK);
+#pragma unroll 1
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    uint64_t a = sdesc(su32(sK) + (kk >> 2) * (kRows * 128) + (kk & 3) * 32,
-                                       16, 1024);
+                    uint64_t a = sdesc(kbase + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024);
                     mma_ss(tm, a, a, id, kk > 0);
                 }
                 mma_commit(&ctrl->mma[s]);
-                if (MODE == kFused && n != s) {
-                    bulk_wait_read();                // previous W/U stores have read Aop, X, V
-                    issue_v(n);
-                }
             }
             if (!wait_mma()) { ok = false; break; }
-            if (MODE == kFused) bar_sync(bar_id, 256);   // staging free before operands are written
             const float bi = sb[r], gi = sg[r];
             const float* gcol = sg + blk * KB;
 #pragma unroll
@@ -512,7 +590,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         v[jj] = j >= jmin ? v[jj] : 0.f;
                         T0[pp * 32 + jj] = eye(j) + v[jj];
                     }
-                    st_op32<false>(sAop, r, pc, v);           // P_1 = M . A
+                    tmem_st_h16(tA + pc * 16, v);           // P_1 = M . A
                 }
             }
             if (MODE == kBuildA) {
@@ -546,10 +624,11 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     v[jj] = j >= jmin ? v[jj] : 0.f;
                     T0[pp * 32 + jj] = eye(j) + v[jj];
                 }
-                st_op32<false>(sAop, r, pc, v);
+                tmem_st_h16(tA + pc * 16, v);
             }
         } else {
             // ---- kWY: T row from global memory ----
+            release_staging(n);
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
@@ -569,11 +648,12 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             }
         }
 
+        if (MODE == kFused) release_staging(n);
         if (MODE == kFused || MODE == kNeumann) {
             // ---- truncated Neumann series, band mask on every power ----
             for (int pw = 2; pw <= p.N; ++pw) {
                 publish();
-                mma_chain(sAop, sX);                                   // P_{n-1} A
+                mma_chain_t(sX);                                       // P_{n-1} A
                 if (!wait_mma()) { ok = false; break; }
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
@@ -586,7 +666,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         v[jj] = (in_chunk(j) && j >= jmin) ? v[jj] : 0.f;
                         T0[pp * 32 + jj] += v[jj];
                     }
-                    if (pw < p.N) st_op32<false>(sAop, r, pc, v);
+                    if (pw < p.N) tmem_st_h16(tA + pc * 16, v);
                 }
             }
             if (!ok) break;
@@ -609,17 +689,17 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                     if (p.S == 1) {
                         st_op32<false>(sY, r, pc, v);                   // Q = E
-                        st_op32<false>(sAop, r, pc, T0P(pp));           // T0
+                        tmem_st_h16(tA + pc * 16, T0P(pp));           // T0
                     } else {
                         st_op32<false>(sX, r, pc, v);                   // E
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj) v[jj] += eye(pc * 32 + jj);
-                        st_op32<false>(sAop, r, pc, v);                 // I + Q_1
+                        tmem_st_h16(tA + pc * 16, v);                 // I + Q_1
                     }
                 }
                 for (int m = 1; m < p.S; ++m) {
                     publish();
-                    mma_chain(sAop, sX);                                // (I + Q_m) E
+                    mma_chain_t(sX);                                    // (I + Q_m) E
                     if (!wait_mma()) { ok = false; break; }
                     const bool last = (m == p.S - 1);
 #pragma unroll
@@ -632,20 +712,20 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             for (int jj = 0; jj < 32; ++jj)
                                 if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
                             st_op32<false>(sY, r, pc, v);               // Q_S
-                            st_op32<false>(sAop, r, pc, T0P(pp));       // T0
+                            tmem_st_h16(tA + pc * 16, T0P(pp));       // T0
                         } else {
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj) {
                                 const int j = pc * 32 + jj;
                                 v[jj] = in_chunk(j) ? v[jj] + eye(j) : 0.f;
                             }
-                            st_op32<false>(sAop, r, pc, v);             // I + Q_{m+1}
+                            tmem_st_h16(tA + pc * 16, v);             // I + Q_{m+1}
                         }
                     }
                 }
                 if (!ok) break;
                 publish();
-                mma_chain(sAop, sY);                                    // T0 Q_S
+                mma_chain_t(sY);                                        // T0 Q_S
                 if (!wait_mma()) { ok = false; break; }
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
@@ -676,41 +756,44 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 
         if (MODE == kFused || MODE == kWY) {
             // ---- WY: T diag(beta [exp g]) -> X (bf16), T diag(beta) -> Y ----
+            release_staging(n);
             const float* bcol = sb + blk * KB;
             const float* gcol = sg + blk * KB;
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
-                float t[32], v[32];
+                float v[32];
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
                     const float b = bcol[j];
-                    const float tv = T0[pp * 32 + jj];
-                    v[jj] = p.gated ? tv * (b * __expf(gcol[j])) : tv * b;
-                    t[jj] = tv * b;
+                    v[jj] = T0[pp * 32 + jj] * (p.gated ? b * __expf(gcol[j]) : b);
                 }
                 st_op32<true>(sX, r, pc, v);
-                if (p.gated) st_op32<true>(sY, r, pc, t);
+                if (p.gated) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) v[jj] = T0[pp * 32 + jj] * bcol[pc * 32 + jj];
+                    st_op32<true>(sY, r, pc, v);
+                }
             }
             if (uses_V(MODE) && !mbar_wait(&ctrl->fullV[s], use_par)) fail_wait();
             publish();
             if (*(volatile int*)&ctrl->abort) { ok = false; break; }
             if (leader) {
                 constexpr uint32_t id = idesc_f16(1, 1, 0, KB, 128);
-                const uint8_t* bu = p.gated ? sY : sX;
-#pragma unroll
+                const uint32_t kb0 = su32(sK), vb0 = su32(sV), xb0 = su32(sX);
+                const uint32_t ub0 = su32(p.gated ? sY : sX);
+#pragma unroll 1
                 for (int c = 0; c < NCH; ++c) {
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < KB / 16; ++kk) {
-                        const uint32_t ka = su32(sK) + (c * KB + kk * 16) * 128;
-                        const uint32_t va = su32(sV) + (c * KB + kk * 16) * 128;
+                        const uint32_t ao = (c * KB + kk * 16) * 128;
                         const uint32_t bo = (c * KB) * 128 + (kk >> 2) * (kRows * 128) +
                                             (kk & 3) * 32;
-                        mma_ss(tm + c * KB, sdesc(ka, kRows * 128, 1024),
-                               sdesc(su32(sX) + bo, 16, 1024), id, kk > 0);
-                        mma_ss(tm + 128 + c * KB, sdesc(va, kRows * 128, 1024),
-                               sdesc(su32(bu) + bo, 16, 1024), id, kk > 0);
+                        mma_ss(tm + c * KB, sdesc(kb0 + ao, kRows * 128, 1024),
+                               sdesc(xb0 + bo, 16, 1024), id, kk > 0);
+                        mma_ss(tm + 128 + c * KB, sdesc(vb0 + ao, kRows * 128, 1024),
+                               sdesc(ub0 + bo, 16, 1024), id, kk > 0);
                     }
                 }
                 mma_commit(&ctrl->mma[s]);
@@ -723,19 +806,20 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             // the TMA load layout.
             {
                 const int d = r;
+                const uint32_t wst = su32(sWst), vst = su32(sV);
                 const uint32_t dbase = (uint32_t)((d >> 6) * (kRows * 128) + (d & 7) * 2);
                 const int c16 = (d & 63) >> 3;
+#pragma unroll 1
+                for (int pp = 0; pp < 4; ++pp) {
+                    const int x0 = h * 64 + pp * 16;
+                    float w[16], u[16];
+                    tmem_ld2x16(tl + x0, w, tl + 128 + x0, u);
 #pragma unroll
-                for (int pp = 0; pp < 2; ++pp) {
-                    const int x0 = h * 64 + pp * 32;
-                    float w[32], u[32];
-                    tmem_ld2(tl + x0, w, tl + 128 + x0, u);
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
+                    for (int jj = 0; jj < 16; ++jj) {
                         const int x = x0 + jj;
                         const uint32_t off = dbase + x * 128 + ((c16 ^ (x & 7)) << 4);
-                        *reinterpret_cast<__nv_bfloat16*>(sWst + off) = __float2bfloat16_rn(w[jj]);
-                        *reinterpret_cast<__nv_bfloat16*>(sV + off) = __float2bfloat16_rn(u[jj]);
+                        sts16(wst + off, __bfloat16_as_ushort(__float2bfloat16_rn(w[jj])));
+                        sts16(vst + off, __bfloat16_as_ushort(__float2bfloat16_rn(u[jj])));
                     }
                 }
             }
@@ -750,6 +834,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 tma_store_2d(&mU, 64, y, sV + kRows * 128);
                 bulk_commit();
             }
+            staged_free = false;
             continue;
         }
         tc_fence_before();

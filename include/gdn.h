@@ -84,7 +84,8 @@ int gdn_build_A(const void* K, const float* beta, const float* g, float* A,
  * the band mask M_ij = [i - j <= N] applied to every power when mask != 0;
  * then, if S > 0, E = I - (I - A) T0 and T = T0 sum_{s=0}^{S} E^s (S >= 0).
  * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.  1 <= N <= k-1, 0 <= S <= 64.
- * GDN_PREC_F16 at k = 256 supports mask = 1 with S = 0 only.
+ * GDN_PREC_F16 serves k <= 128; GDN_PREC_F32 serves k <= 128; k = 256
+ * returns GDN_ERR_UNSUPPORTED in this build.
  */
 int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask,
                        int S, gdn_prec prec, void* stream);
