@@ -485,6 +485,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         }
     };
     const uint32_t tA = tl + 128;                 // this row's A operand (fp16 pairs)
+    // T0 / T: in TMEM columns [160, 224) at KB = 64 (two threads per row, 32
+    // columns each), in registers at KB = 128.
+    constexpr bool kT0Tmem = (KB == 64);
+    const uint32_t tT = tl + 160;
     // the slot's leader loads its own tiles: K, beta, g on fullK, V on fullV
     int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
     auto issue_k = [&](int n) {
@@ -523,7 +527,23 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         staged_free = true;
     };
     auto in_chunk = [&](int j) { return SUB ? (j >= cl && j < ch) : true; };
-#define T0P(pp) (*reinterpret_cast<float(*)[32]>(&T0[(pp) * 32]))
+    // read / write this thread's 32-column piece pp of T0
+    auto t0_get = [&](int pp, float (&t)[32], float* T0r) {
+        if (kT0Tmem) {
+            tmem_ld32(tT + (pc0 + pp) * 32, t);
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) t[jj] = T0r[pp * 32 + jj];
+        }
+    };
+    auto t0_put = [&](int pp, const float (&t)[32], float* T0r) {
+        if (kT0Tmem) {
+            tmem_st32(tT + (pc0 + pp) * 32, t);
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) T0r[pp * 32 + jj] = t[jj];
+        }
+    };
     auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
     auto piece_in_chunk = [&](int pc) { return !SUB || (pc * 32 >= cl && pc * 32 < ch); };
 
@@ -541,7 +561,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         const bool valid = grow < p.rows;
         const int64_t cidx = grow / KC;                  // chunk of this row
         const int64_t rin = grow % KC;                   // row inside the chunk
-        float T0[PPT * 32];                              // this thread's part of row r of T0 / T
+        float T0[kT0Tmem ? 1 : PPT * 32];                // this thread's part of row r of T0 / T
 
         if (uses_K(MODE) && !mbar_wait(&ctrl->fullK[s], use_par)) fail_wait();
         bar_sync(bar_id, 256);
@@ -584,12 +604,14 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                 } else {
                     st_op32<false>(sX, r, pc, v);             // A (chain's right operand)
+                    float t[32];
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
                         v[jj] = j >= jmin ? v[jj] : 0.f;
-                        T0[pp * 32 + jj] = eye(j) + v[jj];
+                        t[jj] = eye(j) + v[jj];
                     }
+                    t0_put(pp, t, T0);
                     tmem_st_h16(tA + pc * 16, v);           // P_1 = M . A
                 }
             }
@@ -618,12 +640,14 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
                 }
                 st_op32<false>(sX, r, pc, v);
+                float t[32];
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
                     v[jj] = j >= jmin ? v[jj] : 0.f;
-                    T0[pp * 32 + jj] = eye(j) + v[jj];
+                    t[jj] = eye(j) + v[jj];
                 }
+                t0_put(pp, t, T0);
                 tmem_st_h16(tA + pc * 16, v);
             }
         } else {
@@ -632,19 +656,20 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
+                float t[32];
                 if (valid && piece_in_chunk(pc)) {
                     const float4* src = reinterpret_cast<const float4*>(
                         p.Tin + cidx * KC * KC + rin * KC + (pc * 32 - cl));
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         float4 a = __ldg(src + q);
-                        T0[pp * 32 + 4 * q] = a.x; T0[pp * 32 + 4 * q + 1] = a.y;
-                        T0[pp * 32 + 4 * q + 2] = a.z; T0[pp * 32 + 4 * q + 3] = a.w;
+                        t[4 * q] = a.x; t[4 * q + 1] = a.y; t[4 * q + 2] = a.z; t[4 * q + 3] = a.w;
                     }
                 } else {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) T0[pp * 32 + jj] = 0.f;
+                    for (int jj = 0; jj < 32; ++jj) t[jj] = 0.f;
                 }
+                t0_put(pp, t, T0);
             }
         }
 
@@ -658,14 +683,16 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
-                    float v[32];
+                    float v[32], t[32];
                     tmem_ld32(tD + pc * 32, v);
+                    t0_get(pp, t, T0);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
                         v[jj] = (in_chunk(j) && j >= jmin) ? v[jj] : 0.f;
-                        T0[pp * 32 + jj] += v[jj];
+                        t[jj] += v[jj];
                     }
+                    t0_put(pp, t, T0);
                     if (pw < p.N) tmem_st_h16(tA + pc * 16, v);
                 }
             }
@@ -673,23 +700,28 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             // ---- parallel residual correction ----
             if (p.S > 0) {
 #pragma unroll
-                for (int pp = 0; pp < PPT; ++pp) st_op32<false>(sY, r, pc0 + pp, T0P(pp));   // T0
+                for (int pp = 0; pp < PPT; ++pp) {
+                    float t[32];
+                    t0_get(pp, t, T0);
+                    st_op32<false>(sY, r, pc0 + pp, t);                // T0
+                }
                 publish();
                 mma_chain(sX, sY);                                      // A T0
                 if (!wait_mma()) { ok = false; break; }
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
-                    float v[32];
+                    float v[32], t[32];
                     tmem_ld32(tD + pc * 32, v);
+                    t0_get(pp, t, T0);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
-                        v[jj] = in_chunk(j) ? eye(j) - T0[pp * 32 + jj] + v[jj] : 0.f;   // E
+                        v[jj] = in_chunk(j) ? eye(j) - t[jj] + v[jj] : 0.f;   // E
                     }
                     if (p.S == 1) {
                         st_op32<false>(sY, r, pc, v);                   // Q = E
-                        tmem_st_h16(tA + pc * 16, T0P(pp));           // T0
+                        tmem_st_h16(tA + pc * 16, t);                 // T0
                     } else {
                         st_op32<false>(sX, r, pc, v);                   // E
 #pragma unroll
@@ -712,7 +744,9 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             for (int jj = 0; jj < 32; ++jj)
                                 if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
                             st_op32<false>(sY, r, pc, v);               // Q_S
-                            tmem_st_h16(tA + pc * 16, T0P(pp));       // T0
+                            float t[32];
+                            t0_get(pp, t, T0);
+                            tmem_st_h16(tA + pc * 16, t);             // T0
                         } else {
 #pragma unroll
                             for (int jj = 0; jj < 32; ++jj) {
@@ -730,11 +764,13 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
-                    float v[32];
+                    float v[32], t[32];
                     tmem_ld32(tD + pc * 32, v);
+                    t0_get(pp, t, T0);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj)
-                        if (in_chunk(pc * 32 + jj)) T0[pp * 32 + jj] += v[jj];   // T = T0 + T0 Q
+                        if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];          // T = T0 + T0 Q
+                    t0_put(pp, t, T0);
                 }
             }
             // ---- T out ----
@@ -743,12 +779,13 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
                     if (valid && piece_in_chunk(pc)) {
+                        float t[32];
+                        t0_get(pp, t, T0);
                         float* dst = p.Tout + cidx * KC * KC + rin * KC + (pc * 32 - cl);
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             reinterpret_cast<float4*>(dst)[q] =
-                                make_float4(T0[pp * 32 + 4 * q], T0[pp * 32 + 4 * q + 1],
-                                            T0[pp * 32 + 4 * q + 2], T0[pp * 32 + 4 * q + 3]);
+                                make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
                     }
                 }
             }
@@ -762,17 +799,18 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
-                float v[32];
+                float v[32], t[32];
+                t0_get(pp, t, T0);
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
                     const float b = bcol[j];
-                    v[jj] = T0[pp * 32 + jj] * (p.gated ? b * __expf(gcol[j]) : b);
+                    v[jj] = t[jj] * (p.gated ? b * __expf(gcol[j]) : b);
                 }
                 st_op32<true>(sX, r, pc, v);
                 if (p.gated) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) v[jj] = T0[pp * 32 + jj] * bcol[pc * 32 + jj];
+                    for (int jj = 0; jj < 32; ++jj) v[jj] = t[jj] * bcol[pc * 32 + jj];
                     st_op32<true>(sY, r, pc, v);
                 }
             }
@@ -850,7 +888,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             if (v_issued > 0) mbar_wait(&ctrl->fullV[s], (uint32_t)((v_issued - 1) & 1));
         }
     }
-#undef T0P
     if (leader) bulk_wait_all();                   // W, U stores complete
     tc_fence_before();
     __syncthreads();
