@@ -257,6 +257,123 @@ def workload_config(w: dict, nc: int, rotate: int = ROTATE) -> dict:
             "l2": f"inputs larger than L2: {rotate} rotating input/output sets of 270 MB"}
 
 
+
+def run_component(args, world, rank, local, dev) -> int:
+    """Device-timed run of one component kernel (A, Neumann, fwdsub, INT8, WY
+    or the full forward) on its own workload; same JSON keys as the headline."""
+    import torch
+    from gated_deltanet_chunk_02_b200 import gdn
+    from gated_deltanet_chunk_02_b200.inputs import Workload, make_inputs
+    kern = args.kernel
+    if kern == "forward":
+        wl = Workload(B=1, H=16, T=65536, k=64, dtype="bf16")
+    else:
+        k = args.k or 64
+        wl = Workload(B=1, H=32, T=16384, k=k, dtype="bf16")
+    k, d, nc = wl.k, wl.d, wl.n_chunks
+    stream = torch.cuda.current_stream(dev)
+    sets = []
+    for r in range(args.rotate):
+        inp = make_inputs(wl, seed=1000 * rank + r, with_q=(kern == "forward"))
+        st = {key: v.to(dev) for key, v in inp.items()}
+        st["A"] = torch.empty(wl.B, wl.H, wl.T // k, k, k, device=dev)
+        st["T"] = torch.empty_like(st["A"])
+        if kern in ("neumann", "fwdsub", "int8", "wy"):
+            gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
+        if kern == "wy":
+            gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
+        if kern in ("wy", "forward"):
+            st["W"] = torch.empty_like(st["K"])
+            st["U"] = torch.empty_like(st["V"])
+        if kern == "forward":
+            st["O"] = torch.empty_like(st["Q"])
+            st["Sf"] = torch.empty(wl.B, wl.H, d, d, device=dev)
+            st["ws"] = torch.empty(gdn.gdn_forward_workspace_bytes(st["K"], k), dtype=torch.uint8,
+                                   device=dev)
+        sets.append(st)
+
+    def step(i):
+        st = sets[i % len(sets)]
+        if kern == "neumann":
+            gdn.gdn_invert_neumann(st["A"], st["T"], args.N, args.mask, args.S, gdn.GDN_PREC_F16,
+                                   stream=stream)
+        elif kern == "fwdsub":
+            gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
+        elif kern == "int8":
+            gdn.gdn_invert_neumann_i8(st["A"], st["T"], args.N, args.mask, stream=stream)
+        elif kern == "build_A":
+            gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
+        elif kern == "wy":
+            gdn.gdn_wy(st["T"], st["K"], st["V"], st["beta"], None, st["W"], st["U"], stream=stream)
+        else:
+            gdn.gdn_forward(st["Q"], st["K"], st["V"], st["beta"], st["g"], None, args.N,
+                            args.mask, args.S, 0, st["O"], st["Sf"], st["ws"], k=k, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert gdn.gdn_get_status(stream) == gdn.GDN_OK
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launches0 = gdn.gdn_launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = gdn.gdn_launch_count() - launches0
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    assert gdn.gdn_get_status(stream) == gdn.GDN_OK
+    ms_step = ms / args.steps
+    # algorithmic bytes and dense-product flops per chunk
+    kk2 = k * k * 4
+    kd = k * d * 2
+    chain = (args.N - 1 + (args.S + 1 if args.S > 0 else 0)) * 2 * k ** 3
+    per = {
+        "neumann": (2 * kk2, chain),
+        "fwdsub": (2 * kk2, 2 * k ** 3 // 6),
+        "int8": (2 * kk2, (args.N - 1) * 2 * k ** 3),
+        "build_A": (kd + 8 * k + kk2, 2 * k * k * d),
+        "wy": (kk2 + 2 * kd + 4 * k + 2 * kd, 4 * k * k * d),
+        "forward": (4 * kd + 8 * k, algorithmic_flops_per_chunk(k, d, args.N, args.S)
+                    + 2 * (4 * k * d * d + k * k * d + k * k * d)),
+    }[kern]
+    bytes_l, flops_l = per[0] * nc, per[1] * nc
+    peaks, peak_kind = load_peaks()
+    gbs = bytes_l / (ms_step * 1e-3) / 1e9
+    tfl = flops_l / (ms_step * 1e-3) / 1e12
+    t_hbm = bytes_l / (float(peaks["hbm_gbs"]) * 1e9)
+    t_tc = flops_l / (float(peaks["bf16_tflops"]) * 1e12)
+    bound = "hbm" if (t_hbm >= t_tc or kern == "fwdsub") else "tensor"
+    line = {
+        "metric": f"{kern} kernel: chunks/s (k={k}, d={d}, bf16 data)",
+        "value": nc * world / (ms_step * 1e-3), "unit": "chunks/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{kern}, B={wl.B} H={wl.H} T={wl.T} k={k} d={d} N={args.N} "
+                               f"mask={args.mask} S={args.S}", "chunks": nc},
+        "roofline": {"bound": bound, "achieved": gbs if bound == "hbm" else tfl,
+                     "peak": float(peaks["hbm_gbs"]) if bound == "hbm" else float(peaks["bf16_tflops"]),
+                     "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                     "frac": gbs / float(peaks["hbm_gbs"]) if bound == "hbm"
+                     else tfl / float(peaks["bf16_tflops"]),
+                     "traffic": recorded_traffic(kern), "peak_source": peak_kind,
+                     "roofline_frac": max(t_hbm, t_tc) / (ms_step * 1e-3), "tflops": tfl,
+                     "bytes_per_launch": bytes_l, "flops_per_launch": flops_l},
+        "clocks": clocks.summary(), "e2e": None, "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -271,6 +388,10 @@ def main(argv=None) -> int:
     ap.add_argument("--N", type=int, default=WORKLOAD["N"], help="Neumann order")
     ap.add_argument("--S", type=int, default=WORKLOAD["S"], help="residual steps")
     ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
+    ap.add_argument("--kernel", default="fused",
+                    choices=["fused", "neumann", "fwdsub", "int8", "build_A", "wy", "forward"],
+                    help="time one component instead of the fused step (not the headline)")
+    ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="input/output sets cycled through the timed steps")
     args = ap.parse_args(argv)
@@ -291,6 +412,8 @@ def main(argv=None) -> int:
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.kernel != "fused":
+        return run_component(args, world, rank, local, dev)
     w = dict(WORKLOAD, N=args.N, S=args.S, mask=args.mask)
     wl = Workload(B=w["B"], H=w["H"], T=w["T"], k=w["k"], d=w["d"], dtype=w["dtype"])
     nc = wl.n_chunks

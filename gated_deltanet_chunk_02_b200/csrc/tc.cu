@@ -206,6 +206,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         : "memory");
 }
 
+// e^x = 2^(x log2 e), with the PTX base-2 exponential ex2.approx.ftz (relative
+// error about 2^-22 by the PTX ISA; inputs here are <= 0, results in (0, 1]).
+__device__ __forceinline__ float exp_e(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+    return y;
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm100 layout: version 1).
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
@@ -592,7 +600,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
                     const bool in = in_chunk(j) && j < i;
-                    v[jj] = in ? -bi * v[jj] * __expf(gi - gcol[j]) : 0.f;
+                    v[jj] = in ? -bi * v[jj] * exp_e(gi - gcol[j]) : 0.f;
                 }
                 if (MODE == kBuildA) {
                     if (valid && piece_in_chunk(pc)) {
@@ -805,7 +813,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
                     const float b = bcol[j];
-                    v[jj] = t[jj] * (p.gated ? b * __expf(gcol[j]) : b);
+                    v[jj] = t[jj] * (p.gated ? b * exp_e(gcol[j]) : b);
                 }
                 st_op32<true>(sX, r, pc, v);
                 if (p.gated) {
