@@ -56,10 +56,23 @@ def load_peaks() -> tuple[dict, str]:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "fused": ["tc.cu", "tc.h", "common.cuh"],
+    "neumann": ["tc.cu", "tc.h", "common.cuh"],
+    "int8": ["tc.cu", "tc.h", "common.cuh"],
+    "build_A": ["tc.cu", "tc.h", "common.cuh"],
+    "wy": ["tc.cu", "tc.h", "common.cuh"],
+    "fwdsub": ["simt.cu", "kernels.h", "common.cuh"],
+    "forward": ["tc.cu", "scan.cu", "simt.cu", "common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str = "fused") -> str:
+    """Hash of the CUDA sources the kernel is built from (ties a recorded ncu
+    traffic figure to the code it was measured on)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_deltanet_chunk_02_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES.get(kernel, sorted(os.listdir(csrc))):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -77,7 +90,7 @@ def recorded_traffic(kernel: str) -> float | None:
             if ":" in line and not line.startswith("#"):
                 key, v = line.split(":", 1)
                 vals[key.strip()] = v.strip()
-    if vals.get("source_hash") != kernel_source_hash():
+    if vals.get(f"{kernel}.source_hash") != kernel_source_hash(kernel):
         return None
     v = vals.get(f"{kernel}.dram_bytes_per_launch")
     return float(v) if v else None
