@@ -1,5 +1,5 @@
 // scan.cu — the inter-chunk state recurrence of the chunk-wise Gated DeltaNet
-// forward (CUDA cores, fp32 state).
+// forward (fp32 state).
 //
 // With W_g = T diag(beta e^g) K and U = T diag(beta) V per chunk (computed in
 // parallel beforehand), the chunk-wise form of the gated delta rule is, for a
@@ -11,8 +11,13 @@
 // (L: lower triangle with the diagonal).  Row v of S only ever meets column v
 // of V~, U and O, so the d_v rows split across CTAs with no exchange: grid =
 // (B*H, d_v / DV), each CTA walks its head's chunks in order holding a DV x d_k
-// slice of S in shared memory.  The chunk's Q, K, W_g tiles are staged in
-// shared memory as fp32; the intra-chunk scores Q K^T are recomputed per slice.
+// slice of S in shared memory.
+//
+// Per chunk: the next chunk's Q, K, W_g, U and g tiles are fetched with
+// cp.async while this one is processed (double buffer); the scores Q K^T are
+// one 64 x 64 x 128 product, on the tensor cores (mma.sync, bf16 inputs, fp32
+// accumulation) for bf16 data and in fp32 FMA for fp32 data; the state
+// products run as register-blocked fp32 FMA loops.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -20,14 +25,126 @@ namespace gdn {
 
 constexpr int kScanThreads = 256;
 constexpr int kSD = 128;          // d_k = d_v
-constexpr int kSLd = kSD + 1;     // padded pitch
 constexpr int kDV = 16;           // state rows per CTA
 constexpr int kSK = 64;           // chunk size served by the scan
 
 template <typename TI>
-__device__ __forceinline__ void stage_tile(float* dst, const TI* src) {
-    for (int e = threadIdx.x; e < kSK * kSD; e += kScanThreads)
-        dst[(e / kSD) * kSLd + e % kSD] = ld_elem(src, e);
+struct ScanTile {
+    static constexpr int kPitch = (sizeof(TI) == 2) ? kSD + 8 : kSD + 4;   // elements, 16-B rows
+    static constexpr int kTileBytes = kSK * kPitch * (int)sizeof(TI);
+    static constexpr int kUBytes = kSK * kDV * (int)sizeof(TI);
+    // one stage: Q, K, W tiles, the U slice and g
+    static constexpr int kStage = 3 * kTileBytes + kUBytes + kSK * 4;
+    static constexpr int kStages = (sizeof(TI) == 2) ? 2 : 1;   // fp32 tiles: single buffer
+};
+
+// e^x = 2^(x log2 e), with the PTX base-2 exponential ex2.approx.ftz
+// (relative error about 2^-22 by the PTX ISA); arguments here are <= 0.
+__device__ __forceinline__ float exp_e(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+    return y;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Fetch chunk `row0`'s tiles into stage buffer `st` (all threads; async).
+template <typename TI>
+__device__ __forceinline__ void fetch_chunk(uint8_t* st, const TI* Q, const TI* K, const TI* Wg,
+                                            const TI* U, const float* g, int64_t row0, int v0) {
+    using L = ScanTile<TI>;
+    constexpr int kVec = 16 / sizeof(TI);                 // elements per 16-byte copy
+    constexpr int kPerRow = kSD / kVec;
+    const TI* src[3] = {Q + row0 * kSD, K + row0 * kSD, Wg + row0 * kSD};
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+        TI* dst = reinterpret_cast<TI*>(st + m * L::kTileBytes);
+        for (int e = threadIdx.x; e < kSK * kPerRow; e += kScanThreads) {
+            const int r = e / kPerRow, c = (e % kPerRow) * kVec;
+            cp_async16(dst + r * L::kPitch + c, src[m] + r * kSD + c);
+        }
+    }
+    {
+        constexpr int kUVec = kDV / kVec;                 // 16-byte copies per U row slice
+        TI* dst = reinterpret_cast<TI*>(st + 3 * L::kTileBytes);
+        for (int e = threadIdx.x; e < kSK * kUVec; e += kScanThreads) {
+            const int r = e / kUVec, c = (e % kUVec) * kVec;
+            cp_async16(dst + r * kDV + c, U + (row0 + r) * kSD + v0 + c);
+        }
+        float* gd = reinterpret_cast<float*>(st + 3 * L::kTileBytes + L::kUBytes);
+        if (threadIdx.x < kSK / 4) cp_async16(gd + threadIdx.x * 4, g + row0 + threadIdx.x * 4);
+    }
+}
+
+// sA[t][j] = (q_t . k_j) e^{g_t - g_j} for j <= t, else 0 (pitch 65).
+__device__ __forceinline__ void chunk_scores(const __nv_bfloat16* Qs, const __nv_bfloat16* Ks,
+                                             const float* gs, float* sA) {
+    // 8 warps: warp w owns rows 16*(w/2) .. +16 and columns 32*(w%2) .. +32
+    constexpr int P = ScanTile<__nv_bfloat16>::kPitch;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = 16 * (warp >> 1), n0 = 32 * (warp & 1);
+    const int gr = lane >> 2, gc = 2 * (lane & 3);
+    float acc[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < kSD; k0 += 16) {
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr) * P + k0 + gc);
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr + 8) * P + k0 + gc);
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr) * P + k0 + gc + 8);
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr + 8) * P + k0 + gc + 8);
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int nb = n0 + 8 * n;
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(Ks + (nb + gr) * P + k0 + gc);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(Ks + (nb + gr) * P + k0 + gc + 8);
+            asm volatile(
+                "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+                "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+                : "+f"(acc[n][0]), "+f"(acc[n][1]), "+f"(acc[n][2]), "+f"(acc[n][3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+    const int t0 = m0 + gr, t1 = m0 + gr + 8;
+    const float g0 = gs[t0], g1 = gs[t1];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+        const int c = n0 + 8 * n + gc;
+        const float gc0 = gs[c], gc1 = gs[c + 1];
+        sA[t0 * (kSK + 1) + c] = c <= t0 ? acc[n][0] * exp_e(g0 - gc0) : 0.f;
+        sA[t0 * (kSK + 1) + c + 1] = c + 1 <= t0 ? acc[n][1] * exp_e(g0 - gc1) : 0.f;
+        sA[t1 * (kSK + 1) + c] = c <= t1 ? acc[n][2] * exp_e(g1 - gc0) : 0.f;
+        sA[t1 * (kSK + 1) + c + 1] = c + 1 <= t1 ? acc[n][3] * exp_e(g1 - gc1) : 0.f;
+    }
+}
+__device__ __forceinline__ void chunk_scores(const float* Qs, const float* Ks, const float* gs,
+                                             float* sA) {
+    constexpr int P = ScanTile<float>::kPitch;
+    for (int e = threadIdx.x; e < kSK * kSK; e += kScanThreads) {
+        const int t = e / kSK, j = e % kSK;
+        float a = 0.f;
+        if (j <= t) {
+            const float* qr = Qs + t * P;
+            const float* kr = Ks + j * P;
+#pragma unroll 8
+            for (int c = 0; c < kSD; ++c) a = fmaf(qr[c], kr[c], a);
+            a *= exp_e(gs[t] - gs[j]);
+        }
+        sA[t * (kSK + 1) + j] = a;
+    }
 }
 
 template <typename TI>
@@ -35,100 +152,133 @@ __global__ void __launch_bounds__(kScanThreads)
 k_scan(const TI* __restrict__ Q, const TI* __restrict__ K, const TI* __restrict__ Wg,
        const TI* __restrict__ U, const float* __restrict__ g, const float* __restrict__ S0,
        TI* __restrict__ O, float* __restrict__ Sfin, int64_t nchunk) {
-    extern __shared__ float sm[];
-    float* sQ = sm;                         // [64][129]
-    float* sK = sQ + kSK * kSLd;            // [64][129]
-    float* sW = sK + kSK * kSLd;            // [64][129]
-    float* sS = sW + kSK * kSLd;            // [DV][129]   state slice
-    float* sVt = sS + kDV * kSLd;           // [64][DV]    V~ slice
-    float* sP = sVt + kSK * kDV;            // [64][DV]    Q S^T slice
-    float* sA = sP + kSK * kDV;             // [64][65]    scores . Gamma . L
-    float* sg = sA + kSK * (kSK + 1);       // [64] g
-    float* sgam = sg + kSK;                 // [64] e^{g_t}
+    using L = ScanTile<TI>;
+    constexpr int P = L::kPitch;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t* stage[2] = {smem, smem + (L::kStages - 1) * L::kStage};
+    float* sS = reinterpret_cast<float*>(smem + L::kStages * L::kStage);   // [DV][129] state
+    constexpr int kSP = kSD + 1;
+    float* sVt = sS + kDV * kSP;            // [64][DV]  V~ slice (times e^{g_last - g_t} later)
+    float* sP = sVt + kSK * kDV;            // [64][DV]  Q S^T slice
+    float* sA = sP + kSK * kDV;             // [64][65]  scores . Gamma . L
+    float* sgam = sA + kSK * (kSK + 1);     // [64] e^{g_t}
     float* sdec = sgam + kSK;               // [64] e^{g_last - g_t}
     const int64_t bh = blockIdx.x;
     const int v0 = blockIdx.y * kDV;
     const int tid = threadIdx.x;
 
-    // state slice
     for (int e = tid; e < kDV * kSD; e += kScanThreads) {
         const int v = e / kSD, c = e % kSD;
-        sS[v * kSLd + c] = S0 ? S0[(bh * kSD + v0 + v) * kSD + c] : 0.f;
+        sS[v * kSP + c] = S0 ? S0[(bh * kSD + v0 + v) * kSD + c] : 0.f;
     }
+    if (L::kStages == 2) {
+        fetch_chunk(stage[0], Q, K, Wg, U, g, bh * nchunk * kSK, v0);
+        cp_async_commit();
+    }
+
+    // thread -> (token t, 4 state rows) for the 64 x DV products
+    const int pt = tid >> 2, pv = (tid & 3) * 4;
+    // thread -> (state row v, 8 columns) for the DV x 128 state update
+    const int uv = tid >> 4, uc = (tid & 15) * 8;
+
     for (int64_t ci = 0; ci < nchunk; ++ci) {
         const int64_t row0 = (bh * nchunk + ci) * kSK;
+        uint8_t* cur = stage[ci & 1];
+        if (L::kStages == 1) {
+            fetch_chunk(cur, Q, K, Wg, U, g, row0, v0);
+            cp_async_commit();
+            cp_async_wait0();
+        } else if (ci + 1 < nchunk) {
+            fetch_chunk(stage[(ci + 1) & 1], Q, K, Wg, U, g, row0 + kSK, v0);
+            cp_async_commit();
+            cp_async_wait1();
+        } else {
+            cp_async_wait0();
+        }
         __syncthreads();
-        stage_tile(sQ, Q + row0 * kSD);
-        stage_tile(sK, K + row0 * kSD);
-        stage_tile(sW, Wg + row0 * kSD);
-        if (tid < kSK) sg[tid] = g[row0 + tid];
-        __syncthreads();
+        const TI* Qs = reinterpret_cast<const TI*>(cur);
+        const TI* Ks = reinterpret_cast<const TI*>(cur + L::kTileBytes);
+        const TI* Ws = reinterpret_cast<const TI*>(cur + 2 * L::kTileBytes);
+        const TI* Us = reinterpret_cast<const TI*>(cur + 3 * L::kTileBytes);
+        const float* gs = reinterpret_cast<const float*>(cur + 3 * L::kTileBytes + L::kUBytes);
         if (tid < kSK) {
-            sgam[tid] = expf(sg[tid]);
-            sdec[tid] = expf(sg[kSK - 1] - sg[tid]);
+            sgam[tid] = exp_e(gs[tid]);
+            sdec[tid] = exp_e(gs[kSK - 1] - gs[tid]);
         }
-        // scores: A[t][j] = (q_t . k_j) e^{g_t - g_j} for j <= t; thread -> 16 entries
-        for (int e = tid; e < kSK * kSK; e += kScanThreads) {
-            const int t = e / kSK, j = e % kSK;
-            float a = 0.f;
-            if (j <= t) {
-                const float* qr = sQ + t * kSLd;
-                const float* kr = sK + j * kSLd;
-#pragma unroll 8
-                for (int c = 0; c < kSD; ++c) a = fmaf(qr[c], kr[c], a);
-                a *= expf(sg[t] - sg[j]);
-            }
-            sA[t * (kSK + 1) + j] = a;
-        }
-        // V~ = U - W_g S^T and P = Q S^T on the slice: 64 x DV each, 4 per thread
-        for (int e = tid; e < kSK * kDV; e += kScanThreads) {
-            const int t = e / kDV, v = e % kDV;
-            const float* wr = sW + t * kSLd;
-            const float* qr = sQ + t * kSLd;
-            const float* sr = sS + v * kSLd;
-            float ws = 0.f, qs = 0.f;
-#pragma unroll 8
+        chunk_scores(Qs, Ks, gs, sA);
+        // V~ = U - W_g S^T and P = Q S^T on the slice
+        {
+            float w[4] = {0.f, 0.f, 0.f, 0.f}, q[4] = {0.f, 0.f, 0.f, 0.f};
+            const TI* wr = Ws + pt * P;
+            const TI* qr = Qs + pt * P;
+#pragma unroll 4
             for (int c = 0; c < kSD; ++c) {
-                ws = fmaf(wr[c], sr[c], ws);
-                qs = fmaf(qr[c], sr[c], qs);
+                const float wc = to_f(wr[c]), qc = to_f(qr[c]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float sv = sS[(pv + i) * kSP + c];
+                    w[i] = fmaf(wc, sv, w[i]);
+                    q[i] = fmaf(qc, sv, q[i]);
+                }
             }
-            sVt[t * kDV + v] = ld_elem(U, (row0 + t) * kSD + v0 + v) - ws;
-            sP[t * kDV + v] = qs;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                sVt[pt * kDV + pv + i] = to_f(Us[pt * kDV + pv + i]) - w[i];
+                sP[pt * kDV + pv + i] = q[i];
+            }
         }
         __syncthreads();
-        // O = diag(gamma) P + A V~
-        for (int e = tid; e < kSK * kDV; e += kScanThreads) {
-            const int t = e / kDV, v = e % kDV;
-            float o = sgam[t] * sP[t * kDV + v];
-            const float* ar = sA + t * (kSK + 1);
-            for (int j = 0; j <= t; ++j) o = fmaf(ar[j], sVt[j * kDV + v], o);
-            st_elem(O, (row0 + t) * kSD + v0 + v, o);
+        // O = diag(gamma) P + (scores . Gamma . L) V~
+        {
+            const float* ar = sA + pt * (kSK + 1);
+            float o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = sgam[pt] * sP[pt * kDV + pv + i];
+            for (int j = 0; j <= pt; ++j) {
+                const float a = ar[j];
+                const float4 vv = *reinterpret_cast<const float4*>(sVt + j * kDV + pv);
+                o[0] = fmaf(a, vv.x, o[0]);
+                o[1] = fmaf(a, vv.y, o[1]);
+                o[2] = fmaf(a, vv.z, o[2]);
+                o[3] = fmaf(a, vv.w, o[3]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) st_elem(O, (row0 + pt) * kSD + v0 + pv + i, o[i]);
         }
-        // S' = gamma_last S + V~^T diag(e^{g_last - g}) K: DV x 128, 8 per thread
-        const float gam = sgam[kSK - 1];
-        for (int e = tid; e < kDV * kSD; e += kScanThreads) {
-            const int v = e / kSD, c = e % kSD;
-            float acc = gam * sS[v * kSLd + c];
-            for (int t = 0; t < kSK; ++t)
-                acc = fmaf(sVt[t * kDV + v] * sdec[t], sK[t * kSLd + c], acc);
-            sS[v * kSLd + c] = acc;
+        // S' = gamma_last S + V~^T diag(e^{g_last - g}) K
+        {
+            float acc[8];
+            const float gam = sgam[kSK - 1];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] = gam * sS[uv * kSP + uc + c];
+            for (int t = 0; t < kSK; ++t) {
+                const float a = sVt[t * kDV + uv] * sdec[t];
+                const TI* kr = Ks + t * P + uc;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[c] = fmaf(a, to_f(kr[c]), acc[c]);
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sS[uv * kSP + uc + c] = acc[c];
         }
+        __syncthreads();                // stage buffer and state free for the next chunk
     }
-    __syncthreads();
     for (int e = tid; e < kDV * kSD; e += kScanThreads) {
         const int v = e / kSD, c = e % kSD;
-        Sfin[(bh * kSD + v0 + v) * kSD + c] = sS[v * kSLd + c];
+        Sfin[(bh * kSD + v0 + v) * kSD + c] = sS[v * kSP + c];
     }
 }
 
 cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, const void* U, const float* g,
                         const float* S0, void* O, float* Sfin, int64_t BH, int64_t nchunk,
                         bool bf16, cudaStream_t st) {
-    const size_t smem = (size_t)(3 * kSK * kSLd + kDV * kSLd + 2 * kSK * kDV +
-                                 kSK * (kSK + 1) + 3 * kSK) * sizeof(float);
     dim3 grid((unsigned)BH, kSD / kDV);
+    auto smem_for = [](int stage, int nstages) {
+        return (size_t)(nstages * stage) + (size_t)(kDV * (kSD + 1) + 2 * kSK * kDV +
+                                                    kSK * (kSK + 1) + 2 * kSK) * sizeof(float);
+    };
     cudaError_t e;
     if (bf16) {
+        const size_t smem = smem_for(ScanTile<__nv_bfloat16>::kStage, 2);
         e = cudaFuncSetAttribute(k_scan<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
@@ -136,6 +286,7 @@ cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, const void
             (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)Wg,
             (const __nv_bfloat16*)U, g, S0, (__nv_bfloat16*)O, Sfin, nchunk);
     } else {
+        const size_t smem = smem_for(ScanTile<float>::kStage, 1);
         e = cudaFuncSetAttribute(k_scan<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
