@@ -100,8 +100,7 @@ int gdn_build_A(const void* K, const float* beta, const float* g, float* A, gdn_
     if (nc == 0) return GDN_OK;
     GDN_TRY(check_ptrs({{K, "K"}, {beta, "beta"}, {g, "g"}, {A, "A"}}));
     cudaStream_t st = (cudaStream_t)stream;
-    if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "build_A serves k <= 128");
-    if (dtype == GDN_BF16 && gdn::tc_available())
+    if (dtype == GDN_BF16 && gdn::tc_available() && s.k <= 128)
         return launched(gdn::launch_build_A_tc(K, beta, g, A, nc, s.k, st), "build_A (tcgen05)");
     return launched(gdn::launch_build_A_simt(K, beta, g, A, nc, s.k, dtype == GDN_BF16, st),
                     "build_A");
@@ -118,7 +117,12 @@ int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask, i
     cudaStream_t st = (cudaStream_t)stream;
     if (prec == GDN_PREC_F16) {
         if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
-        if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "tensor-core Neumann chain serves k <= 128");
+        if (s.k == 256) {
+            if (S != 0)
+                return fail(GDN_ERR_UNSUPPORTED, "tensor-core Neumann chain at k=256 serves S=0");
+            return launched(gdn::launch_neumann256_tc(A, T, nc, N, mask, st),
+                            "neumann k=256 (tcgen05)");
+        }
         return launched(gdn::launch_neumann_tc(A, T, nc, s.k, N, mask, S, st), "neumann (tcgen05)");
     }
     if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "float32 Neumann chain supports k <= 128");

@@ -8,7 +8,7 @@ namespace gdn {
 
 // CUDA-core kernels (simt.cu); k in {32, 64, 128} unless stated.
 cudaError_t launch_build_A_simt(const void* K, const float* beta, const float* g, float* A,
-                                int64_t nc, int k, bool bf16, cudaStream_t st);
+                                int64_t nc, int k, bool bf16, cudaStream_t st);  // k <= 256
 cudaError_t launch_neumann_simt(const float* A, float* T, int64_t nc, int k, int N, int mask,
                                 int S, cudaStream_t st);
 cudaError_t launch_wy_simt(const float* T, const void* K, const void* V, const float* beta,

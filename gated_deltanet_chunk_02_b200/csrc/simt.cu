@@ -221,6 +221,47 @@ k_build_A_simt(const TI* __restrict__ Kp, const float* __restrict__ beta,
     for (int e = threadIdx.x; e < K * K; e += kSimtThreads) Ac[e] = X[(e / K) * (K + 1) + e % K];
 }
 
+// k = 256: K K^T by 128 x 128 quadrants (upper quadrant is zero), A written
+// straight to global memory.
+template <typename TI>
+__global__ void __launch_bounds__(kSimtThreads)
+k_build_A_simt256(const TI* __restrict__ Kp, const float* __restrict__ beta,
+                  const float* __restrict__ g, float* __restrict__ A) {
+    constexpr int K = 256, R = 8;
+    extern __shared__ float sm[];
+    float* Ks = sm;                       // [256][129]
+    float* sb = Ks + K * kLdK;
+    float* sg = sb + K;
+    const int64_t c = blockIdx.x;
+    const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+    load_tile_kd<K>(Ks, Kp + c * K * kD, (const float*)nullptr);
+    for (int i = threadIdx.x; i < K; i += kSimtThreads) {
+        sb[i] = beta[c * K + i];
+        sg[i] = g[c * K + i];
+    }
+    __syncthreads();
+    float* Ac = A + c * K * K;
+    for (int q = 0; q < 4; ++q) {
+        const int qi = q >> 1, qj = q & 1;
+        if (qj > qi) {
+            for (int ii = 0; ii < R; ++ii)
+                for (int jj = 0; jj < R; ++jj)
+                    Ac[(128 * qi + ty + 16 * ii) * K + 128 * qj + tx + 16 * jj] = 0.f;
+            continue;
+        }
+        float G[R][R];
+        zero(G);
+        mm_nt<R, R>(Ks + 128 * qi * kLdK, kLdK, Ks + 128 * qj * kLdK, kLdK, kD, G, ty, tx);
+#pragma unroll
+        for (int ii = 0; ii < R; ++ii)
+#pragma unroll
+            for (int jj = 0; jj < R; ++jj) {
+                const int i = 128 * qi + ty + 16 * ii, j = 128 * qj + tx + 16 * jj;
+                Ac[i * K + j] = (i > j) ? -sb[i] * G[ii][jj] * expf(sg[i] - sg[j]) : 0.f;
+            }
+    }
+}
+
 template <int K>
 __global__ void __launch_bounds__(kSimtThreads)
 k_neumann_simt(const float* __restrict__ A, float* __restrict__ T, int N, int mask, int S) {
@@ -528,6 +569,22 @@ static cudaError_t build_A_t(const TI* K, const float* beta, const float* g, flo
 
 cudaError_t launch_build_A_simt(const void* K, const float* beta, const float* g, float* A,
                                 int64_t nc, int k, bool bf16, cudaStream_t st) {
+    if (k == 256) {
+        const size_t smem = (256 * kLdK + 2 * 256) * sizeof(float);
+        cudaError_t e;
+        if (bf16) {
+            e = prep(k_build_A_simt256<__nv_bfloat16>, smem);
+            if (e != cudaSuccess) return e;
+            k_build_A_simt256<__nv_bfloat16><<<(unsigned)nc, kSimtThreads, smem, st>>>(
+                (const __nv_bfloat16*)K, beta, g, A);
+        } else {
+            e = prep(k_build_A_simt256<float>, smem);
+            if (e != cudaSuccess) return e;
+            k_build_A_simt256<float><<<(unsigned)nc, kSimtThreads, smem, st>>>((const float*)K,
+                                                                              beta, g, A);
+        }
+        return cudaGetLastError();
+    }
     return bf16 ? build_A_t((const __nv_bfloat16*)K, beta, g, A, nc, k, st)
                 : build_A_t((const float*)K, beta, g, A, nc, k, st);
 }

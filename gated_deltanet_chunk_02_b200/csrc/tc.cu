@@ -1166,6 +1166,204 @@ k_neumann_i8_tc(const ParamsI8 p) {
 }
 
 // ------------------------------------------------------------------------- //
+// k = 256: the truncated Neumann series on the tensor cores, S = 0
+// ------------------------------------------------------------------------- //
+// The chunk is a 2 x 2 block matrix of 128 x 128 blocks (the upper-right block
+// of a strictly lower-triangular A is zero).  The series is summed in Horner
+// form, X_1 = I + M.A and X_m = I + M.(X_{m-1} A), so that X_N = M.(sum of
+// A^n, n = 0..N).  Keeping only the band of X_{m-1} changes nothing inside the
+// band: entry (i, j) of X A reads X only at (i, l) with j < l <= i, and
+// i - l < i - j.  One step is four 128 x 128 x 128 products:
+//   D00 = X00 A00,  D10 = X10 A00 + X11 A10,  D11 = X11 A11
+// with the X blocks as K-major left operands, the A blocks as MN-major right
+// operands (both fp16 in shared memory, row-major with the 128-byte swizzle)
+// and the three accumulators in TMEM columns [0, 384).  Warp group q (warps
+// 4q .. 4q + 3) owns block q of {D00, D10, D11}: thread row = its TMEM lane.
+// One chunk per CTA at a time (persistent grid); the 192 KB of operands leave
+// no room for a second chunk.
+struct Params256 {
+    int64_t nc;
+    int N;
+    int mask;
+    const float* A;
+    float* T;
+    int* status;
+};
+
+constexpr int k256Threads = 384;
+constexpr int k256Blk = kRows * 128 * 2;            // one 128 x 128 fp16 operand block
+constexpr int k256Smem = 6 * k256Blk + 64;
+
+// Byte offset of element (r, c) of a 128 x 128 fp16 operand block.
+__device__ __forceinline__ uint32_t el_off256(int r, int c) {
+    return op_off(r, c >> 3) + (uint32_t)((c & 7) * 2);
+}
+
+// T entries of the 32 x 32 tile (rows 32 rg .., columns c0 ..) that are zero
+// whatever A holds: above the diagonal, or outside the band.
+__device__ __forceinline__ bool zero_tile256(int rg, int c0, int mask, int N) {
+    return c0 > 32 * rg + 31 || (mask && c0 + 31 < 32 * rg - N);
+}
+
+__global__ void __launch_bounds__(k256Threads, 1)
+k_neumann256_tc(const Params256 p) {
+    constexpr int KC = 256;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((su32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    // right operands A00, A10, A11; left operands X00, X10, X11
+    auto sA = [&](int b) { return smem + b * k256Blk; };
+    auto sX = [&](int b) { return smem + (3 + b) * k256Blk; };
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + 6 * k256Blk);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + 6 * k256Blk + 8);
+    int* abort_flag = reinterpret_cast<int*>(smem + 6 * k256Blk + 16);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(mbar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tmem_alloc(tslot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tslot;
+
+    const int gq = warp >> 2;                        // 0: D00, 1: D10, 2: D11
+    const int rr = ((warp & 3) << 5) | lane;         // row inside the block = TMEM lane
+    const int row = (gq ? 128 : 0) + rr;             // row inside the chunk
+    const int col0 = gq == 2 ? 128 : 0;              // first column of the block
+    const int rg = row >> 5;                         // this warp's 32-row group
+    const uint32_t tD = tm + ((uint32_t)((warp & 3) * 32) << 16) + 128 * gq;
+    const bool leader = threadIdx.x == 0;
+    const int N = p.N, mask = p.mask;
+    const int jmin = mask ? row - N : -KC;           // band: columns j >= jmin
+    uint32_t phase = 0;
+    bool ok = true, timed_out = false;
+
+    // one step's products, issued by one thread
+    auto issue = [&]() {
+        constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
+        auto blk = [&](uint32_t dcol, const uint8_t* xa, const uint8_t* ab, bool acc) {
+            const uint32_t xb = su32(xa), bb = su32(ab);
+#pragma unroll 1
+            for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tm + dcol, sdesc(xb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024),
+                       sdesc(bb + kk * 2048, kRows * 128, 1024), id, (acc || kk > 0) ? 1u : 0u);
+        };
+        blk(0, sX(0), sA(0), false);
+        blk(128, sX(1), sA(0), false);
+        blk(128, sX(2), sA(1), true);
+        blk(256, sX(2), sA(2), false);
+        mma_commit(mbar);
+    };
+    auto publish = [&]() {
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    };
+
+    for (int64_t c = blockIdx.x; c < p.nc; c += gridDim.x) {
+        const float* Ac = p.A + c * KC * KC;
+        float* Tc = p.T + c * KC * KC;
+        // ---- A -> operands, X_1 = I + M.A; rows read whole by one warp (coalesced).
+        // T entries that stay zero are written here; at N = 1 all of T is.
+#pragma unroll 1
+        for (int r0 = warp; r0 < KC; r0 += 4 * 12) {
+            float4 a[4][2];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int rw = r0 + 12 * u;
+                if (rw < KC) {
+                    const float4* src = reinterpret_cast<const float4*>(Ac + (int64_t)rw * KC);
+                    a[u][0] = __ldg(src + lane);
+                    a[u][1] = __ldg(src + 32 + lane);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int rw = r0 + 12 * u;
+                if (rw >= KC) continue;
+                const int jm = mask ? rw - N : -KC;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int j0 = 128 * hf + 4 * lane;
+                    const float av[4] = {a[u][hf].x, a[u][hf].y, a[u][hf].z, a[u][hf].w};
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        x[e] = (j0 + e == rw ? 1.f : 0.f) + (j0 + e >= jm ? av[e] : 0.f);
+                    const bool upper = hf == 1 && rw < 128;
+                    if (!upper) {
+                        const int b = (rw >= 128) + hf;          // 0: (0,0), 1: (1,0), 2: (1,1)
+                        const uint32_t off = el_off256(rw & 127, j0 & 127);
+                        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(su32(sA(b)) + off),
+                                     "r"(pack_h2(av[0], av[1])), "r"(pack_h2(av[2], av[3]))
+                                     : "memory");
+                        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(su32(sX(b)) + off),
+                                     "r"(pack_h2(x[0], x[1])), "r"(pack_h2(x[2], x[3]))
+                                     : "memory");
+                    }
+                    float4* dst = reinterpret_cast<float4*>(Tc + (int64_t)rw * KC + j0);
+                    if (N == 1 && !upper)
+                        *dst = make_float4(x[0], x[1], x[2], x[3]);
+                    else if (upper || zero_tile256(rw >> 5, j0 & ~31, mask, N))
+                        *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+        }
+        publish();
+        if (*(volatile int*)abort_flag) { ok = false; break; }
+        // ---- steps 2 .. N
+        for (int m = 2; m <= N; ++m) {
+            if (leader) issue();
+            if (mbar_wait(mbar, phase)) {
+                phase ^= 1;
+            } else {                                 // the products are still in flight
+                timed_out = true;
+                atomicExch(abort_flag, 1);
+                raise_status(p.status, kStatusTimeout);
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int pc = 0; pc < 4; ++pc) {
+                const int c0 = col0 + 32 * pc;
+                if (zero_tile256(rg, c0, mask, N)) continue;   // warp-uniform
+                float v[32];
+                tmem_ld32(tD + 32 * pc, v);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = c0 + jj;
+                    v[jj] = (j == row ? 1.f : 0.f) + (j >= jmin ? v[jj] : 0.f);
+                }
+                if (m < N) {
+                    st_op32<false>(sX(gq), rr, pc, v);
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(Tc + (int64_t)row * KC + c0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                }
+            }
+            publish();
+            if (*(volatile int*)abort_flag) { ok = false; break; }
+        }
+        if (!ok) break;
+    }
+    if (timed_out) mbar_wait(mbar, phase);          // bounded: let the products finish
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+// ------------------------------------------------------------------------- //
 // host side
 // ------------------------------------------------------------------------- //
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1344,6 +1542,25 @@ cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8
     const int cap = 2 * tcg::num_sms();
     const int grid = p.ntiles < cap ? p.ntiles : cap;
     tcg::k_neumann_i8_tc<<<grid, 256 * tcg::kI8Slots, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, int mask,
+                                cudaStream_t st) {
+    tcg::Params256 p;
+    p.nc = nc;
+    p.N = N;
+    p.mask = mask;
+    p.A = A;
+    p.T = T;
+    p.status = status_ptr();
+    cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann256_tc,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tcg::k256Smem);
+    if (e != cudaSuccess) return e;
+    const int sms = tcg::num_sms();
+    const int grid = nc < sms ? (int)nc : sms;
+    tcg::k_neumann256_tc<<<grid, tcg::k256Threads, tcg::k256Smem, st>>>(p);
     return cudaGetLastError();
 }
 

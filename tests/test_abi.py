@@ -109,6 +109,18 @@ def test_float32_chain_limit_and_bad_enums(lib):
     assert lib.gdn_build_A(P(FAKE), P(FAKE), P(FAKE), P(FAKE), sh(), 5, None) == gdn.GDN_ERR_ARG
 
 
+def test_k256_chain_limits(lib):
+    # the k=256 tensor-core chain sums the series without the residual step
+    rc = lib.gdn_invert_neumann(P(FAKE), P(FAKE), sh(T=512, k=256), 3, 1, 8, 1, None)
+    assert rc == gdn.GDN_ERR_UNSUPPORTED and "S=0" in last(lib)
+    # N runs up to k - 1
+    assert lib.gdn_invert_neumann(P(FAKE), P(FAKE), sh(T=512, k=256), 256, 1, 0, 1,
+                                  None) == gdn.GDN_ERR_ARG
+    # the fused and WY kernels stop at k=128
+    assert lib.gdn_chunk_wy_fused(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 3, 1, 0, 0, P(FAKE), P(FAKE),
+                                  None, sh(T=512, k=256), 1, None) == gdn.GDN_ERR_UNSUPPORTED
+
+
 def test_empty_inputs_are_noops(lib):
     n0 = lib.gdn_launch_count()
     for s in (sh(B=0), sh(H=0), sh(T=0)):

@@ -79,7 +79,7 @@ def test_c1_f32_full():
     assert rel(T.cpu().double().numpy().reshape(Tr.shape), Tr) <= TOL_F32
 
 
-@pytest.mark.parametrize("k", [32, 64, 128])
+@pytest.mark.parametrize("k", [32, 64, 128, 256])
 def test_c3_chunk_sweep(k):
     w = Workload(B=1, H=32, T=16384, k=k, dtype="bf16")
     inp = make_inputs(w, seed=0)
