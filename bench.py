@@ -208,6 +208,17 @@ def barrier(world: int):
         dist.barrier()
 
 
+def shard_seed(rank: int, copy: int) -> int:
+    """Seed of input copy `copy` on rank `rank`: every rank draws its own batch
+    (weak scaling: the units of work are independent chunks, no exchange)."""
+    return 1000 * rank + copy
+
+
+def aggregate_throughput(units_per_rank: int, world: int, ms_total: float, steps: int) -> float:
+    """Whole-job units/s: the units all ranks processed over the max-over-ranks time."""
+    return units_per_rank * world / (ms_total * 1e-3 / steps)
+
+
 def cpu_oracle_sample(w: dict, n_sample: int, seed: int = 0) -> tuple[float, int, dict]:
     """Time the oracle (as it stands) on the first n_sample chunks of the
     workload; returns (seconds, threads used, info)."""
@@ -287,7 +298,7 @@ def run_component(args, world, rank, local, dev) -> int:
     stream = torch.cuda.current_stream(dev)
     sets = []
     for r in range(args.rotate):
-        inp = make_inputs(wl, seed=1000 * rank + r, with_q=(kern == "forward"))
+        inp = make_inputs(wl, seed=shard_seed(rank, r), with_q=(kern == "forward"))
         st = {key: v.to(dev) for key, v in inp.items()}
         st["A"] = torch.empty(wl.B, wl.H, wl.T // k, k, k, device=dev)
         st["T"] = torch.empty_like(st["A"])
@@ -364,7 +375,8 @@ def run_component(args, world, rank, local, dev) -> int:
     bound = "hbm" if (t_hbm >= t_tc or kern == "fwdsub") else "tensor"
     line = {
         "metric": f"{kern} kernel: chunks/s (k={k}, d={d}, bf16 data)",
-        "value": nc * world / (ms_step * 1e-3), "unit": "chunks/s", "n_gpus": world,
+        "value": aggregate_throughput(nc, world, ms, args.steps), "unit": "chunks/s",
+        "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
@@ -434,7 +446,7 @@ def main(argv=None) -> int:
     elem = 2
     sets = []
     for r in range(args.rotate):
-        inp = make_inputs(wl, seed=1000 * rank + r)
+        inp = make_inputs(wl, seed=shard_seed(rank, r))
         s = {key: inp[key].to(dev) for key in ("K", "V", "beta", "g")}
         s["W"] = torch.empty_like(s["K"])
         s["U"] = torch.empty_like(s["V"])
@@ -514,7 +526,7 @@ def main(argv=None) -> int:
 
     line = {
         "metric": METRIC,
-        "value": nc * world / (ms * 1e-3 / args.steps),
+        "value": aggregate_throughput(nc, world, ms, args.steps),
         "unit": "chunks/s",
         "n_gpus": world,
         "steps": args.steps,
