@@ -334,6 +334,24 @@ __device__ __forceinline__ void tmem_ld2x16(uint32_t a0, float (&v0)[16], uint32
         v1[i] = __uint_as_float(r1[i]);
     }
 }
+// 16 TMEM columns of fp16 pairs (32 values) of this thread's lane -> 32 floats
+__device__ __forceinline__ void tmem_ld_h16(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
 // two 32-column pieces (e.g. an accumulator piece and a T0 piece) with one wait
 __device__ __forceinline__ void tmem_ld2(uint32_t a0, float (&v0)[32], uint32_t a1, float (&v1)[32]) {
     uint32_t r0[32], r1[32];
@@ -497,6 +515,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     // columns each), in registers at KB = 128.
     constexpr bool kT0Tmem = (KB == 64);
     const uint32_t tT = tl + 160;
+    const uint32_t tF = tl + (KB == 64 ? 224 : 192);  // F = E + E^2 of the residual (fp16 pairs)
     // the slot's leader loads its own tiles: K, beta, g on fullK, V on fullV
     int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
     auto issue_k = [&](int n) {
@@ -555,6 +574,39 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
     auto piece_in_chunk = [&](int pc) { return !SUB || (pc * 32 >= cl && pc * 32 < ch); };
 
+    // products of one residual round: D[0,128) = X X, D[128,256) = Y X
+    auto mma_pair = [&](bool sq, bool gp) {
+        if (leader) {
+            constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
+            const uint32_t xb = su32(sX), yb = su32(sY);
+#pragma unroll 1
+            for (int kk = 0; kk < KB / 16; ++kk) {
+                const uint32_t ko = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+                const uint64_t bx = sdesc(xb + kk * 2048, KB * 128, 1024);
+                if (sq) mma_ss(tm, sdesc(xb + ko, 16, 1024), bx, id, kk > 0);
+                if (gp) mma_ss(tm + 128, sdesc(yb + ko, 16, 1024), bx, id, kk > 0);
+            }
+            mma_commit(&ctrl->mma[s]);
+        }
+    };
+    // 8 fp16 values of row rr, columns 8q .. 8q + 7, of an operand buffer
+    auto ld_h8 = [&](const uint8_t* buf, int rr, int q, float (&o)[8]) {
+        uint4 u;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+                     : "r"(su32(buf) + op_off(rr, q)));
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[c]));
+            o[2 * c] = f.x;
+            o[2 * c + 1] = f.y;
+        }
+    };
+    auto st_h8 = [&](uint8_t* buf, int rr, int q, const float (&v)[8]) {
+        sts128(su32(buf) + op_off(rr, q), make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]),
+                                                     pack_h2(v[4], v[5]), pack_h2(v[6], v[7])));
+    };
     if (leader) {
         issue_k(s);
         issue_v(s);
@@ -705,80 +757,273 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
             }
             if (!ok) break;
-            // ---- parallel residual correction ----
+            // ---- parallel residual correction: T = T0 G, G = sum_{s<=S} E^s ----
+            // Two schedules.  Horner keeps (I + Q_m) in TMEM as the left operand
+            // of Q_{m+1} = (I + Q_m) E (S - 1 products, one per round) and T0 in
+            // fp32; it is the faster one while S is small.  Doubling (below)
+            // needs only ~log2(S) rounds of two shared-memory products, and
+            // serves the standalone inverse and S >= 15.
+            // Doubling applies when S + 1 is 2^m or 2^m + 1: with a = 2^r,
+            // G(2a) - I = (G(a) - I) + E^a + (G(a) - I) E^a and E^2a = E^a E^a,
+            // two products per round sharing the right operand E^a.  T0 - I
+            // (fp16) goes to the Aop buffer, E = I - T0 + A + A (T0 - I) to X,
+            // G - I to Y, and T = T0 + (G - I) + (T0 - I)(G - I).  Both
+            // accumulators of a round fill the slot's TMEM, so T0 survives the
+            // rounds as its fp16 copy at KB = 64.
             if (p.S > 0) {
+                const int S = p.S;
+                int K2 = 0;
+                while ((2 << K2) <= S + 1) ++K2;
+                const bool p2p1 = (1 << K2) + 1 == S + 1;
+                const bool dbl = (1 << K2) == S + 1 || p2p1;
+                // doubling is built into the standalone inverse only: in the
+                // fused kernel its registers would cost every other phase
+                if (!(MODE == kNeumann && dbl)) {
+                    // Horner with stride 2: Q_1 = E, E^2 = E E, F = E + E^2,
+                    // Q_{m+2} = F + Q_m E^2, and Q_{m+1} = E + Q_m E when one
+                    // step is left; Q_m (no identity) is the left operand in
+                    // TMEM, E in X, E^2 then Q_S in Y, F in TMEM as fp16.
 #pragma unroll
-                for (int pp = 0; pp < PPT; ++pp) {
-                    float t[32];
-                    t0_get(pp, t, T0);
-                    st_op32<false>(sY, r, pc0 + pp, t);                // T0
-                }
-                publish();
-                mma_chain(sX, sY);                                      // A T0
-                if (!wait_mma()) { ok = false; break; }
-#pragma unroll
-                for (int pp = 0; pp < PPT; ++pp) {
-                    const int pc = pc0 + pp;
-                    float v[32], t[32];
-                    tmem_ld32(tD + pc * 32, v);
-                    t0_get(pp, t, T0);
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = pc * 32 + jj;
-                        v[jj] = in_chunk(j) ? eye(j) - t[jj] + v[jj] : 0.f;   // E
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        float t[32];
+                        t0_get(pp, t, T0);
+                        st_op32<false>(sY, r, pc0 + pp, t);                // T0
                     }
-                    if (p.S == 1) {
-                        st_op32<false>(sY, r, pc, v);                   // Q = E
-                        tmem_st_h16(tA + pc * 16, t);                 // T0
-                    } else {
-                        st_op32<false>(sX, r, pc, v);                   // E
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) v[jj] += eye(pc * 32 + jj);
-                        tmem_st_h16(tA + pc * 16, v);                 // I + Q_1
-                    }
-                }
-                for (int m = 1; m < p.S; ++m) {
                     publish();
-                    mma_chain_t(sX);                                    // (I + Q_m) E
+                    mma_chain(sX, sY);                                      // A T0
                     if (!wait_mma()) { ok = false; break; }
-                    const bool last = (m == p.S - 1);
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
-                        float v[32];
+                        float v[32], t[32];
                         tmem_ld32(tD + pc * 32, v);
-                        if (last) {
+                        t0_get(pp, t, T0);
 #pragma unroll
-                            for (int jj = 0; jj < 32; ++jj)
-                                if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
-                            st_op32<false>(sY, r, pc, v);               // Q_S
-                            float t[32];
-                            t0_get(pp, t, T0);
-                            tmem_st_h16(tA + pc * 16, t);             // T0
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int j = pc * 32 + jj;
+                            v[jj] = in_chunk(j) ? eye(j) - t[jj] + v[jj] : 0.f;   // E
+                        }
+                        if (p.S == 1) {
+                            st_op32<false>(sY, r, pc, v);                   // Q_1 = E
+                            tmem_st_h16(tA + pc * 16, t);                 // T0
                         } else {
-#pragma unroll
-                            for (int jj = 0; jj < 32; ++jj) {
-                                const int j = pc * 32 + jj;
-                                v[jj] = in_chunk(j) ? v[jj] + eye(j) : 0.f;
-                            }
-                            tmem_st_h16(tA + pc * 16, v);             // I + Q_{m+1}
+                            st_op32<false>(sX, r, pc, v);                   // E
+                            tmem_st_h16(tA + pc * 16, v);                 // Q_1 = E
                         }
                     }
-                }
-                if (!ok) break;
-                publish();
-                mma_chain_t(sY);                                        // T0 Q_S
-                if (!wait_mma()) { ok = false; break; }
+                    // this row's E from X, 8 columns at a time
+                    auto e_row = [&](int pc, float (&e)[32]) {
 #pragma unroll
-                for (int pp = 0; pp < PPT; ++pp) {
-                    const int pc = pc0 + pp;
-                    float v[32], t[32];
-                    tmem_ld32(tD + pc * 32, v);
-                    t0_get(pp, t, T0);
+                        for (int g = 0; g < 4; ++g) {
+                            float h8[8];
+                            ld_h8(sX, r, 4 * pc + g, h8);
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
-                        if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];          // T = T0 + T0 Q
-                    t0_put(pp, t, T0);
+                            for (int c = 0; c < 8; ++c) e[8 * g + c] = h8[c];
+                        }
+                    };
+                    // Q_S is final: Q_S -> Y (right operand), T0 -> TMEM (left)
+                    auto finish_q = [&](int pp, float (&q)[32]) {
+                        const int pc = pc0 + pp;
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (!in_chunk(pc * 32 + jj)) q[jj] = 0.f;
+                        st_op32<false>(sY, r, pc, q);
+                        float t[32];
+                        t0_get(pp, t, T0);
+                        tmem_st_h16(tA + pc * 16, t);
+                    };
+                    if (p.S >= 2) {
+                        publish();
+                        mma_chain_t(sX);                                    // E E
+                        if (!wait_mma()) { ok = false; break; }
+#pragma unroll
+                        for (int pp = 0; pp < PPT; ++pp) {
+                            const int pc = pc0 + pp;
+                            float v[32], e[32];
+                            tmem_ld32(tD + pc * 32, v);
+                            e_row(pc, e);
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) e[jj] += v[jj];     // F
+                            if (p.S == 2) {
+                                finish_q(pp, e);                            // Q_2 = F
+                            } else {
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj)
+                                    if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
+                                st_op32<false>(sY, r, pc, v);               // E^2
+                                tmem_st_h16(tF + pc * 16, e);             // F
+                            }
+                        }
+                        int m = 1;
+                        while (p.S >= 3 && m + 2 <= p.S) {
+                            publish();
+                            mma_chain_t(sY);                                // Q_m E^2
+                            if (!wait_mma()) { ok = false; break; }
+                            m += 2;
+#pragma unroll
+                            for (int pp = 0; pp < PPT; ++pp) {
+                                const int pc = pc0 + pp;
+                                float v[32], f[32];
+                                tmem_ld32(tD + pc * 32, v);
+                                tmem_ld_h16(tF + pc * 16, f);
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj) v[jj] += f[jj];     // Q_m
+                                if (m == p.S) {
+                                    finish_q(pp, v);
+                                } else {
+#pragma unroll
+                                    for (int jj = 0; jj < 32; ++jj)
+                                        if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
+                                    tmem_st_h16(tA + pc * 16, v);
+                                }
+                            }
+                        }
+                        if (!ok) break;
+                        if (p.S >= 3 && m < p.S) {                          // one step left
+                            publish();
+                            mma_chain_t(sX);                                // Q_m E
+                            if (!wait_mma()) { ok = false; break; }
+#pragma unroll
+                            for (int pp = 0; pp < PPT; ++pp) {
+                                const int pc = pc0 + pp;
+                                float v[32], e[32];
+                                tmem_ld32(tD + pc * 32, v);
+                                e_row(pc, e);
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj) v[jj] += e[jj];     // Q_S
+                                finish_q(pp, v);
+                            }
+                        }
+                    }
+                    publish();
+                    mma_chain_t(sY);                                        // T0 Q_S
+                    if (!wait_mma()) { ok = false; break; }
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
+                        float v[32], t[32];
+                        tmem_ld32(tD + pc * 32, v);
+                        t0_get(pp, t, T0);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];          // T = T0 + T0 Q
+                        t0_put(pp, t, T0);
+                    }
+                } else if constexpr (MODE == kNeumann) {
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
+                        float t[32];
+                        t0_get(pp, t, T0);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) t[jj] -= eye(pc * 32 + jj);
+                        st_op32<false>(sAop, r, pc, t);                    // T0 - I
+                    }
+                    publish();
+                    mma_chain(sX, sAop);                                    // A (T0 - I)
+                    if (!wait_mma()) { ok = false; break; }
+                    const int rounds = K2;
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
+                        float v[32], t[32];
+                        tmem_ld32(tD + pc * 32, v);
+                        t0_get(pp, t, T0);
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            float a8[8], e8[8], z8[8];
+                            ld_h8(sX, r, 4 * pc + g, a8);                    // A
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const int jj = 8 * g + c, j = pc * 32 + jj;
+                                e8[c] = in_chunk(j) ? eye(j) - t[jj] + a8[c] + v[jj] : 0.f;
+                                z8[c] = 0.f;
+                            }
+                            st_h8(sX, r, 4 * pc + g, e8);                    // E^1
+                            st_h8(sY, r, 4 * pc + g, z8);                    // G(1) - I = 0
+                        }
+                    }
+                    for (int rd = 1; rd <= rounds; ++rd) {
+                        const bool sq = rd < K2 || p2p1;                   // E^a E^a
+                        const bool gp = rd > 1;                            // (G - I) E^a
+                        const bool add_sq = rd == K2 && p2p1;              // + E^(2^m)
+                        const bool ea_out = sq && rd < K2;
+                        if (sq || gp) {
+                            publish();
+                            mma_pair(sq, gp);
+                            if (!wait_mma()) { ok = false; break; }
+                        }
+#pragma unroll
+                        for (int pp = 0; pp < PPT; ++pp) {
+                            const int pc = pc0 + pp;
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                float da[16], db[16];
+                                const uint32_t c0 = tD + pc * 32 + 16 * hh;
+                                if (sq && gp) {
+                                    tmem_ld2x16(c0, da, c0 + 128, db);
+                                } else if (sq) {
+                                    tmem_ld2x16(c0, da, c0, db);
+                                } else if (gp) {
+                                    tmem_ld2x16(c0 + 128, db, c0 + 128, da);
+                                } else {
+#pragma unroll
+                                    for (int c = 0; c < 16; ++c) da[c] = db[c] = 0.f;
+                                }
+#pragma unroll
+                                for (int g2 = 0; g2 < 2; ++g2) {
+                                    const int q = 4 * pc + 2 * hh + g2;
+                                    float ea[8], gb[8], go[8], eo[8];
+                                    ld_h8(sX, r, q, ea);
+                                    ld_h8(sY, r, q, gb);
+#pragma unroll
+                                    for (int c = 0; c < 8; ++c) {
+                                        float x = ea[c];
+                                        x += gb[c];
+                                        if (gp) x += db[8 * g2 + c];
+                                        if (add_sq) x += da[8 * g2 + c];
+                                        go[c] = in_chunk(8 * q + c) ? x : 0.f;
+                                        eo[c] = in_chunk(8 * q + c) ? da[8 * g2 + c] : 0.f;
+                                    }
+                                    st_h8(sY, r, q, go);
+                                    if (ea_out) st_h8(sX, r, q, eo);
+                                }
+                            }
+                        }
+                    }
+                    if (!ok) break;
+                    publish();
+                    mma_chain(sAop, sY);                                    // (T0 - I)(G - I)
+                    if (!wait_mma()) { ok = false; break; }
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
+                        float v[32], t[32];
+                        tmem_ld32(tD + pc * 32, v);
+                        if (kT0Tmem) {                                      // T0 from its fp16 copy
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                float h8[8];
+                                ld_h8(sAop, r, 4 * pc + g, h8);
+#pragma unroll
+                                for (int c = 0; c < 8; ++c)
+                                    t[8 * g + c] = eye(pc * 32 + 8 * g + c) + h8[c];
+                            }
+                        } else {
+                            t0_get(pp, t, T0);
+                        }
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            float g8[8];
+                            ld_h8(sY, r, 4 * pc + g, g8);                    // G - I
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const int jj = 8 * g + c;
+                                t[jj] = in_chunk(pc * 32 + jj) ? t[jj] + g8[c] + v[jj] : 0.f;
+                            }
+                        }
+                        t0_put(pp, t, T0);
+                    }
                 }
             }
             // ---- T out ----
@@ -1502,7 +1747,7 @@ cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N
     p.N = N;
     p.mask = mask;
     p.S = S;
-    return tcg::dispatch<tcg::kNeumann, 2>(k, tcg::IO(), p, st);
+    return tcg::dispatch<tcg::kNeumann, 1>(k, tcg::IO(), p, st);
 }
 
 cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const float* beta,

@@ -146,6 +146,33 @@ def test_fused_small(dtype, k, N, mask, S, gated):
     assert per_chunk_max_rel(W, Wr.reshape(Wr.shape[0], -1)) <= 2 * tol
 
 
+@pytest.mark.parametrize("k", [32, 64, 128])
+@pytest.mark.parametrize("N,mask", [(1, 1), (3, 1), (4, 1), (3, 0)])
+@pytest.mark.parametrize("S", [0, 1, 2, 3, 4, 5, 7, 8, 9, 16])
+def test_fused_residual_schedules(k, N, mask, S):
+    """The residual sum G = sum E^s by doubling (S + 1 = 2^m or 2^m + 1) and by
+    Horner (the other S), on 9 chunks."""
+    gated = (S % 2 == 1)
+    w = Workload(B=1, H=3, T=3 * k, k=k, dtype="bf16")
+    inp = make_inputs(w, seed=11 + S)
+    d = dev_inputs(inp)
+    W = torch.empty_like(d["K"])
+    U = torch.empty_like(d["V"])
+    T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_chunk_wy_fused(d["K"], d["V"], d["beta"], d["g"], N, mask, S, int(gated), W, U, T, k=k)
+    check_status()
+    Tr, Wr, Ur = fused_reference(chunked(inp, w), N, mask, S, gated)
+    assert rel(T, Tr) <= TOL_BF16
+    assert per_chunk_max_rel(T, Tr) <= TOL_BF16
+    assert rel(W, Wr) <= TOL_BF16
+    assert rel(U, Ur) <= TOL_BF16
+    Th = T.cpu().numpy().reshape(Tr.shape)
+    assert np.all(np.triu(Th, 1) == 0)
+    if S == 0 and mask:
+        dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+        assert np.all(Th[:, dist > N] == 0)
+
+
 def test_fused_without_T_output_matches():
     w = Workload(B=2, H=2, T=256, k=64, dtype="bf16")
     inp = make_inputs(w, seed=6)
@@ -190,7 +217,7 @@ def test_int8_bit_exact(N, mask):
 @pytest.mark.parametrize("k", [32, 64, 128])
 @pytest.mark.parametrize("N", [1, 2, 3, 4])
 @pytest.mark.parametrize("mask", [0, 1])
-@pytest.mark.parametrize("S", [0, 1, 2, 8])
+@pytest.mark.parametrize("S", [0, 1, 2, 3, 5, 8])
 def test_neumann_tensor_cores(k, N, mask, S):
     """The tcgen05 chain (fp16 operands, fp32 accumulation) on 9 chunks."""
     w = Workload(B=1, H=3, T=3 * k, k=k, dtype="bf16")
