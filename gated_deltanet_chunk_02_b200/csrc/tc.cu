@@ -334,6 +334,22 @@ __device__ __forceinline__ void tmem_ld2x16(uint32_t a0, float (&v0)[16], uint32
         v1[i] = __uint_as_float(r1[i]);
     }
 }
+// 16 lanes x 8 columns in the mma accumulator fragment layout: thread t gets
+// lane (t / 4) columns 2 (t % 4) + {0, 1} in r[0..1] and lane (8 + t / 4) in
+// r[2..3], lanes counted from taddr's; no wait.
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, uint32_t (&r)[4]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+// Four 8 x 8 b16 blocks, stored transposed; threads 8m .. 8m + 7 give the row
+// addresses of block m (16-byte aligned).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1,
+                                                  uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
 // 16 TMEM columns of fp16 pairs (32 values) of this thread's lane -> 32 floats
 __device__ __forceinline__ void tmem_ld_h16(uint32_t taddr, float (&v)[32]) {
     uint32_t r[16];
@@ -1091,27 +1107,38 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             }
             if (!wait_mma()) { ok = false; break; }
             if (leader) issue_k(n + NS);                 // K, beta, g are no longer read
-            // Lane r of the W^T / U^T accumulators is head-dim column d = r and
-            // accumulator column x is tile row x.  Thread half h transposes
-            // rows [64h, 64h + 64) into the W staging tile and the V tile, in
-            // the TMA load layout.
+            // Lane d of the W^T / U^T accumulators is head-dim column d and
+            // accumulator column x is tile row x.  Warp (quarter q, half h)
+            // moves d in [32q, 32q + 32) x rows [64h, 64h + 64): 16x256b TMEM
+            // loads give each thread (d, x..x+1) pairs of 8 x 8 blocks, and
+            // stmatrix .trans writes the blocks transposed, one 16-byte row
+            // segment (8 d of one tile row) per address, into the W staging
+            // tile and the V tile in the TMA layout.
             {
-                const int d = r;
                 const uint32_t wst = su32(sWst), vst = su32(sV);
-                const uint32_t dbase = (uint32_t)((d >> 6) * (kRows * 128) + (d & 7) * 2);
-                const int c16 = (d & 63) >> 3;
+                const int mq = lane >> 3, mr = lane & 7;   // stmatrix: matrix, row of this address
 #pragma unroll 1
-                for (int pp = 0; pp < 4; ++pp) {
-                    const int x0 = h * 64 + pp * 16;
-                    float w[16], u[16];
-                    tmem_ld2x16(tl + x0, w, tl + 128 + x0, u);
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const int x = x0 + jj;
-                        const uint32_t off = dbase + x * 128 + ((c16 ^ (x & 7)) << 4);
-                        sts16(wst + off, __bfloat16_as_ushort(__float2bfloat16_rn(w[jj])));
-                        sts16(vst + off, __bfloat16_as_ushort(__float2bfloat16_rn(u[jj])));
-                    }
+                for (int it = 0; it < 8; ++it) {
+                    const int hb = it & 1;
+                    const int x0 = h * 64 + (it >> 1) * 16;
+                    const int db = (warp & 3) * 32 + 16 * hb;
+                    const uint32_t ta = tl + ((uint32_t)(16 * hb) << 16) + x0;
+                    uint32_t wa[4], wb[4], ua[4], ub[4];
+                    tmem_ld_16x256b(ta, wa);
+                    tmem_ld_16x256b(ta + 8, wb);
+                    tmem_ld_16x256b(ta + 128, ua);
+                    tmem_ld_16x256b(ta + 136, ub);
+                    tmem_wait_ld();
+                    const int x = x0 + 8 * (mq >> 1) + mr, d = db + 8 * (mq & 1);
+                    const uint32_t off = (uint32_t)((d >> 6) * (kRows * 128) + x * 128 +
+                                                    ((((d & 63) >> 3) ^ (x & 7)) << 4));
+                    auto pk = [](uint32_t lo, uint32_t hi) {
+                        return pack_b2(__uint_as_float(lo), __uint_as_float(hi));
+                    };
+                    stmatrix_x4_trans(wst + off, pk(wa[0], wa[1]), pk(wa[2], wa[3]), pk(wb[0], wb[1]),
+                                      pk(wb[2], wb[3]));
+                    stmatrix_x4_trans(vst + off, pk(ua[0], ua[1]), pk(ua[2], ua[3]), pk(ub[0], ub[1]),
+                                      pk(ub[2], ub[3]));
                 }
             }
             fence_async_smem();
