@@ -492,9 +492,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         return good;
     };
     // hand the operands written by this slot to the tensor pipe
-    auto publish = [&]() {
+    // smem: generic shared-memory stores since the last publish feed the MMA
+    auto publish = [&](bool smem) {
         tmem_wait_st();
-        fence_async_smem();
+        if (smem) fence_async_smem();
         tc_fence_before();
         bar_sync(bar_id, 256);
         tc_fence_after();
@@ -663,12 +664,18 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
                 float v[32];
-                tmem_ld32(tD + pc * 32, v);
+                // pieces above the diagonal or in another chunk for the whole warp
+                if (pc * 32 > (i | 31) || !piece_in_chunk(pc)) {
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = pc * 32 + jj;
-                    const bool in = in_chunk(j) && j < i;
-                    v[jj] = in ? -bi * v[jj] * exp_e(gi - gcol[j]) : 0.f;
+                    for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
+                } else {
+                    tmem_ld32(tD + pc * 32, v);
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = pc * 32 + jj;
+                        const bool in = in_chunk(j) && j < i;
+                        v[jj] = in ? -bi * v[jj] * exp_e(gi - gcol[j]) : 0.f;
+                    }
                 }
                 if (MODE == kBuildA) {
                     if (valid && piece_in_chunk(pc)) {
@@ -684,11 +691,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
-                        v[jj] = j >= jmin ? v[jj] : 0.f;
-                        t[jj] = eye(j) + v[jj];
+                        t[jj] = eye(j) + (j >= jmin ? v[jj] : 0.f);   // X_1 = I + M.A
                     }
-                    t0_put(pp, t, T0);
-                    tmem_st_h16(tA + pc * 16, v);           // P_1 = M . A
+                    if (p.N == 1) t0_put(pp, t, T0);
+                    else tmem_st_h16(tA + pc * 16, t);
                 }
             }
             if (MODE == kBuildA) {
@@ -720,11 +726,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
-                    v[jj] = j >= jmin ? v[jj] : 0.f;
-                    t[jj] = eye(j) + v[jj];
+                    t[jj] = eye(j) + (j >= jmin ? v[jj] : 0.f);       // X_1 = I + M.A
                 }
-                t0_put(pp, t, T0);
-                tmem_st_h16(tA + pc * 16, v);
+                if (p.N == 1) t0_put(pp, t, T0);
+                else tmem_st_h16(tA + pc * 16, t);
             }
         } else {
             // ---- kWY: T row from global memory ----
@@ -751,25 +756,26 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 
         if (MODE == kFused) release_staging(n);
         if (MODE == kFused || MODE == kNeumann) {
-            // ---- truncated Neumann series, band mask on every power ----
+            // ---- truncated Neumann series in Horner form ----
+            // X_1 = I + M.A, X_n = I + M.(X_{n-1} A), T0 = X_N: inside the band
+            // X_{n-1} A reads only in-band entries of X_{n-1}, so masking every
+            // step gives M.(sum_{n<=N} A^n) exactly.
             for (int pw = 2; pw <= p.N; ++pw) {
-                publish();
-                mma_chain_t(sX);                                       // P_{n-1} A
+                publish(pw == 2);
+                mma_chain_t(sX);                                       // X_{n-1} A
                 if (!wait_mma()) { ok = false; break; }
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
-                    float v[32], t[32];
+                    float v[32];
                     tmem_ld32(tD + pc * 32, v);
-                    t0_get(pp, t, T0);
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
-                        v[jj] = (in_chunk(j) && j >= jmin) ? v[jj] : 0.f;
-                        t[jj] += v[jj];
+                        v[jj] = eye(j) + ((in_chunk(j) && j >= jmin) ? v[jj] : 0.f);
                     }
-                    t0_put(pp, t, T0);
-                    if (pw < p.N) tmem_st_h16(tA + pc * 16, v);
+                    if (pw == p.N) t0_put(pp, v, T0);
+                    else tmem_st_h16(tA + pc * 16, v);
                 }
             }
             if (!ok) break;
@@ -805,7 +811,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         t0_get(pp, t, T0);
                         st_op32<false>(sY, r, pc0 + pp, t);                // T0
                     }
-                    publish();
+                    publish(true);
                     mma_chain(sX, sY);                                      // A T0
                     if (!wait_mma()) { ok = false; break; }
 #pragma unroll
@@ -849,7 +855,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         tmem_st_h16(tA + pc * 16, t);
                     };
                     if (p.S >= 2) {
-                        publish();
+                        publish(true);
                         mma_chain_t(sX);                                    // E E
                         if (!wait_mma()) { ok = false; break; }
 #pragma unroll
@@ -872,7 +878,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         }
                         int m = 1;
                         while (p.S >= 3 && m + 2 <= p.S) {
-                            publish();
+                            publish(m == 1);
                             mma_chain_t(sY);                                // Q_m E^2
                             if (!wait_mma()) { ok = false; break; }
                             m += 2;
@@ -896,7 +902,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         }
                         if (!ok) break;
                         if (p.S >= 3 && m < p.S) {                          // one step left
-                            publish();
+                            publish(false);
                             mma_chain_t(sX);                                // Q_m E
                             if (!wait_mma()) { ok = false; break; }
 #pragma unroll
@@ -911,7 +917,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             }
                         }
                     }
-                    publish();
+                    publish(true);
                     mma_chain_t(sY);                                        // T0 Q_S
                     if (!wait_mma()) { ok = false; break; }
 #pragma unroll
@@ -935,7 +941,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         for (int jj = 0; jj < 32; ++jj) t[jj] -= eye(pc * 32 + jj);
                         st_op32<false>(sAop, r, pc, t);                    // T0 - I
                     }
-                    publish();
+                    publish(true);
                     mma_chain(sX, sAop);                                    // A (T0 - I)
                     if (!wait_mma()) { ok = false; break; }
                     const int rounds = K2;
@@ -965,7 +971,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         const bool add_sq = rd == K2 && p2p1;              // + E^(2^m)
                         const bool ea_out = sq && rd < K2;
                         if (sq || gp) {
-                            publish();
+                            publish(true);
                             mma_pair(sq, gp);
                             if (!wait_mma()) { ok = false; break; }
                         }
@@ -1008,7 +1014,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         }
                     }
                     if (!ok) break;
-                    publish();
+                    publish(true);
                     mma_chain(sAop, sY);                                    // (T0 - I)(G - I)
                     if (!wait_mma()) { ok = false; break; }
 #pragma unroll
@@ -1084,7 +1090,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
             }
             if (uses_V(MODE) && !mbar_wait(&ctrl->fullV[s], use_par)) fail_wait();
-            publish();
+            publish(true);
             if (*(volatile int*)&ctrl->abort) { ok = false; break; }
             if (leader) {
                 constexpr uint32_t id = idesc_f16(1, 1, 0, KB, 128);
