@@ -59,7 +59,11 @@ struct SlotLayout {
     static constexpr int offX = offV + kV;
     static constexpr int offAop = offX + kXY;
     static constexpr int offY = offAop + kAop;
-    static constexpr int bytes = offY + kXY;
+    // the standalone inverse stages the next tile's A (fp32, 128-byte swizzled
+    // boxes of 32 columns x 128 rows) while it works on the current one
+    static constexpr int kStage = (MODE == kNeumann) ? kRows * KB * 4 : 0;
+    static constexpr int offStage = offY + kXY;
+    static constexpr int bytes = offStage + kStage;
     static constexpr int bg_bytes = uses_K(MODE) ? 2 * kRows * 4 : 0;  // beta[128], g[128]
 };
 
@@ -469,6 +473,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     uint8_t* sAop = base + L::offAop;
     uint8_t* sX = base + L::offX;
     uint8_t* sY = base + L::offY;
+    uint8_t* sStage = base + L::offStage;
     float* sb = reinterpret_cast<float*>(bg_base + s * L::bg_bytes);
     float* sg = sb + kRows;
     const uint32_t tm = tmem_base + (uint32_t)(s * 256);
@@ -537,9 +542,16 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
     auto issue_k = [&](int n) {
         const int tile = blockIdx.x + n * gridDim.x;
-        if (!uses_K(MODE) || tile >= p.ntiles) return;
+        if (!(uses_K(MODE) || MODE == kNeumann) || tile >= p.ntiles) return;
         ++k_issued;
         const int y = tile * kRows;
+        if (MODE == kNeumann) {                        // A: KC / 32 boxes of 16 KB
+            mbar_expect_tx(&ctrl->fullK[s], (KC / 32) * 16384);
+#pragma unroll 1
+            for (int b = 0; b < KC / 32; ++b)
+                tma_load_2d(sStage + b * 16384, &mK, 32 * b, y, &ctrl->fullK[s]);
+            return;
+        }
         mbar_expect_tx(&ctrl->fullK[s], kRows * kD * 2 + 2 * kRows * 4);
         tma_load_2d(sK, &mK, 0, y, &ctrl->fullK[s]);
         tma_load_2d(sK + kRows * 128, &mK, 64, y, &ctrl->fullK[s]);
@@ -640,7 +652,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         const int64_t rin = grow % KC;                   // row inside the chunk
         float T0[kT0Tmem ? 1 : PPT * 32];                // this thread's part of row r of T0 / T
 
-        if (uses_K(MODE) && !mbar_wait(&ctrl->fullK[s], use_par)) fail_wait();
+        if ((uses_K(MODE) || MODE == kNeumann) && !mbar_wait(&ctrl->fullK[s], use_par))
+            fail_wait();
         bar_sync(bar_id, 256);
         if (*(volatile int*)&ctrl->abort) { ok = false; break; }
 
@@ -704,18 +717,24 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 continue;
             }
         } else if (MODE == kNeumann) {
-            // ---- A row from global memory ----
+            // ---- A rows from the staged tile ----
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
                 float v[32];
-                if (valid && piece_in_chunk(pc)) {
-                    const float4* src = reinterpret_cast<const float4*>(
-                        p.Ain + cidx * KC * KC + rin * KC + (pc * 32 - cl));
+                if (piece_in_chunk(pc)) {                 // rows past the end were zero-filled
+                    const uint32_t rb =
+                        su32(sStage) + (uint32_t)(((pc * 32 - cl) >> 5) * 16384 + r * 128);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 a = __ldg(src + q);
-                        v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        uint32_t u0, u1, u2, u3;
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(u0), "=r"(u1), "=r"(u2), "=r"(u3)
+                                     : "r"(rb + ((c4 ^ (r & 7)) << 4)));
+                        v[4 * c4] = __uint_as_float(u0);
+                        v[4 * c4 + 1] = __uint_as_float(u1);
+                        v[4 * c4 + 2] = __uint_as_float(u2);
+                        v[4 * c4 + 3] = __uint_as_float(u3);
                     }
                 } else {
 #pragma unroll
@@ -731,6 +750,12 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 if (p.N == 1) t0_put(pp, t, T0);
                 else tmem_st_h16(tA + pc * 16, t);
             }
+            // the stage is read: it takes the slot's next tile; the previous
+            // tile's T store has read the Aop / Y staging before it is reused
+            fence_async_smem();
+            if (leader) bulk_wait_read();
+            bar_sync(bar_id, 256);
+            if (leader) issue_k(n + NS);
         } else {
             // ---- kWY: T row from global memory ----
             release_staging(n);
@@ -1049,7 +1074,35 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
             }
             // ---- T out ----
-            if (p.Tout) {
+            if (MODE == kNeumann) {
+                // through the Aop | Y buffers as fp32 128-byte swizzled boxes, TMA store
+                bar_sync(bar_id, 256);                 // this tile's Aop / Y operands are read
+                const uint32_t st0 = su32(sAop);
+#pragma unroll
+                for (int pp = 0; pp < PPT; ++pp) {
+                    const int pc = pc0 + pp;
+                    if (piece_in_chunk(pc)) {
+                        float t[32];
+                        t0_get(pp, t, T0);
+                        const uint32_t rb = st0 + (uint32_t)(((pc * 32 - cl) >> 5) * 16384 + r * 128);
+#pragma unroll
+                        for (int c4 = 0; c4 < 8; ++c4)
+                            sts128(rb + ((c4 ^ (r & 7)) << 4),
+                                   make_uint4(__float_as_uint(t[4 * c4]), __float_as_uint(t[4 * c4 + 1]),
+                                              __float_as_uint(t[4 * c4 + 2]),
+                                              __float_as_uint(t[4 * c4 + 3])));
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                bar_sync(bar_id, 256);
+                if (leader) {
+#pragma unroll 1
+                    for (int b = 0; b < KC / 32; ++b)
+                        tma_store_2d(&mW, 32 * b, (int)row0, sAop + b * 16384);
+                    bulk_commit();
+                }
+            } else if (p.Tout) {
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
@@ -1675,6 +1728,19 @@ static bool map_kd(CUtensorMap* m, const void* base, int64_t rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, cols] fp32, box 32 columns x 128 rows, 128-byte swizzle
+static bool map_f32(CUtensorMap* m, const void* base, int64_t rows, int cols) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)kRows};
+    cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [rows] fp32, box 128 (rows past the end read as zero)
 static bool map_vec(CUtensorMap* m, const void* base, int64_t rows) {
     EncodeTiledFn f = encode_fn();
@@ -1723,6 +1789,10 @@ static cudaError_t launch(const IO& io, const Params& p0, cudaStream_t st) {
     if (uses_V(MODE)) {
         if (!map_kd(&mV, io.V, p0.rows) || !map_kd(&mW, io.W, p0.rows) ||
             !map_kd(&mU, io.U, p0.rows))
+            return cudaErrorInvalidValue;
+    }
+    if (MODE == kNeumann) {                        // A in through mK, T out through mW
+        if (!map_f32(&mK, p0.Ain, p0.rows, KC) || !map_f32(&mW, p0.Tout, p0.rows, KC))
             return cudaErrorInvalidValue;
     }
     Params p = p0;
