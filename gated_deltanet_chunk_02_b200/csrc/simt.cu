@@ -419,6 +419,75 @@ k_fwdsub(const float* __restrict__ A, float* __restrict__ T) {
     }
 }
 
+// Forward substitution for k <= 64: one warp per chunk.  The chunk's A is
+// copied to shared memory in one coalesced pass (cp.async); lane l owns the
+// columns j = l + 32c of T and keeps them in registers; the row sweep
+// T[i][j] = [i == j] + sum_{l < i} A[i][l] T[l][j] reads each row of A as
+// float4 broadcasts (every lane needs the same A[i][l]).  Column group c is
+// zero above row 32c, so its sweep starts there.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+
+constexpr int kFwdWarps = 4;                     // chunks per CTA (one per warp)
+
+template <int K>
+__global__ void __launch_bounds__(32 * kFwdWarps)
+k_fwdsub_warp(const float* __restrict__ A, float* __restrict__ T, int64_t nc) {
+    constexpr int NC = K / 32;                   // column groups per lane
+    extern __shared__ __align__(16) float smf[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* sA = smf + warp * K * K;
+    const int64_t stride = (int64_t)gridDim.x * kFwdWarps;
+    for (int64_t c = (int64_t)blockIdx.x * kFwdWarps + warp; c < nc; c += stride) {
+        const float* Ac = A + c * K * K;
+        __syncwarp();                            // the previous chunk's reads of sA are done
+#pragma unroll
+        for (int q = 0; q < K * K / 128; ++q) {
+            const int e = (q * 32 + lane) * 4;
+            cp_async16(sA + e, Ac + e);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncwarp();
+        float x[NC][K];
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc) {
+            const int cb = 32 * cc;
+            const int j = cb + lane;
+#pragma unroll
+            for (int i = cb; i < K; ++i) {
+                const float* ar = sA + i * K;
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                for (int l = cb; l + 4 <= i; l += 4) {
+                    const float4 a = *reinterpret_cast<const float4*>(ar + l);
+                    s0 = fmaf(a.x, x[cc][l], s0);
+                    s1 = fmaf(a.y, x[cc][l + 1], s1);
+                    s2 = fmaf(a.z, x[cc][l + 2], s2);
+                    s3 = fmaf(a.w, x[cc][l + 3], s3);
+                }
+                const int l0 = cb + ((i - cb) & ~3);
+                if (l0 < i) {
+                    const float4 a = *reinterpret_cast<const float4*>(ar + l0);
+                    s0 = fmaf(a.x, x[cc][l0], s0);
+                    if (l0 + 1 < i) s1 = fmaf(a.y, x[cc][l0 + 1], s1);
+                    if (l0 + 2 < i) s2 = fmaf(a.z, x[cc][l0 + 2], s2);
+                }
+                x[cc][i] = (i == j ? 1.f : 0.f) + ((s0 + s1) + (s2 + s3));
+            }
+        }
+        float* Tc = T + c * K * K;
+#pragma unroll
+        for (int cc = 0; cc < NC; ++cc)
+#pragma unroll
+            for (int i = 0; i < K; ++i) Tc[i * K + 32 * cc + lane] = i < 32 * cc ? 0.f : x[cc][i];
+    }
+}
+
 // INT8 truncated Neumann, k = 64 (see gdn_invert_neumann_i8 for the scheme).
 __device__ __forceinline__ float block_max_f(float v, float* red) {
     for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -645,6 +714,25 @@ cudaError_t launch_fused_simt(const void* K, const void* V, const float* beta, c
 }
 
 cudaError_t launch_fwdsub(const float* A, float* T, int64_t nc, int k, cudaStream_t st) {
+    if (k <= 64) {
+        const size_t smem = (size_t)kFwdWarps * k * k * sizeof(float);
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t need = (nc + kFwdWarps - 1) / kFwdWarps;
+        const int64_t cap = (int64_t)sms * 8;
+        const unsigned grid = (unsigned)(need < cap ? need : cap);
+        cudaError_t e;
+        if (k == 32) {
+            e = prep(k_fwdsub_warp<32>, smem);
+            if (!e) k_fwdsub_warp<32><<<grid, 32 * kFwdWarps, smem, st>>>(A, T, nc);
+        } else {
+            e = prep(k_fwdsub_warp<64>, smem);
+            if (!e) k_fwdsub_warp<64><<<grid, 32 * kFwdWarps, smem, st>>>(A, T, nc);
+        }
+        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
     const int CB = k < 128 ? k : 128;
     const int nb = k / CB;
     dim3 grid((unsigned)nc, (unsigned)nb);
