@@ -488,6 +488,129 @@ k_fwdsub_warp(const float* __restrict__ A, float* __restrict__ T, int64_t nc) {
     }
 }
 
+// Forward substitution for k = 128 by 64 x 64 blocks, exact in exact arithmetic:
+// T00 = (I - A00)^-1 and T11 = (I - A11)^-1 by the row sweep above (one warp
+// per 32-column group), then T10 = T11 (A10 T00) with both products on the
+// CUDA cores in fp32.  One chunk per 128-thread CTA at a time.
+template <int CB>
+__device__ __forceinline__ void fwd_sweep64(const float* sA, int pitch, int lane, float* sT,
+                                            float* Tg, int tpitch) {
+    // rows of the 64 x 64 block at sA (row pitch `pitch`), columns CB + lane
+    const int j = CB + lane;
+    float x[64];
+#pragma unroll
+    for (int i = CB; i < 64; ++i) {
+        const float* ar = sA + i * pitch;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+        for (int l = CB; l + 4 <= i; l += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(ar + l);
+            s0 = fmaf(a.x, x[l], s0);
+            s1 = fmaf(a.y, x[l + 1], s1);
+            s2 = fmaf(a.z, x[l + 2], s2);
+            s3 = fmaf(a.w, x[l + 3], s3);
+        }
+        const int l0 = CB + ((i - CB) & ~3);
+        if (l0 < i) {
+            const float4 a = *reinterpret_cast<const float4*>(ar + l0);
+            s0 = fmaf(a.x, x[l0], s0);
+            if (l0 + 1 < i) s1 = fmaf(a.y, x[l0 + 1], s1);
+            if (l0 + 2 < i) s2 = fmaf(a.z, x[l0 + 2], s2);
+        }
+        x[i] = (i == j ? 1.f : 0.f) + ((s0 + s1) + (s2 + s3));
+    }
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const float v = i < CB ? 0.f : x[i];
+        sT[i * 64 + j] = v;
+        Tg[(int64_t)i * tpitch + j] = v;
+    }
+}
+
+// acc[8][4] += P[r0 + rr][l] Q[l][c0 + cc] over l in [l_lo, l_hi), a multiple of
+// 4 wide: per 4 values of l, 8 float4 reads of P rows and 4 of Q rows.
+template <int PP, int QP>
+__device__ __forceinline__ void mm_tile84(const float* P, const float* Q, int r0, int c0, int l_lo,
+                                          int l_hi, float (&acc)[8][4]) {
+#pragma unroll 1
+    for (int l = l_lo; l < l_hi; l += 4) {
+        float4 q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = *reinterpret_cast<const float4*>(Q + (l + u) * QP + c0);
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            const float4 pv = *reinterpret_cast<const float4*>(P + (r0 + rr) * PP + l);
+            const float pu[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                acc[rr][0] = fmaf(pu[u], q[u].x, acc[rr][0]);
+                acc[rr][1] = fmaf(pu[u], q[u].y, acc[rr][1]);
+                acc[rr][2] = fmaf(pu[u], q[u].z, acc[rr][2]);
+                acc[rr][3] = fmaf(pu[u], q[u].w, acc[rr][3]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128)
+k_fwdsub128(const float* __restrict__ A, float* __restrict__ T, int64_t nc) {
+    constexpr int K = 128;
+    extern __shared__ __align__(16) float smf[];
+    float* sA = smf;                        // [128][128]
+    float* sT00 = sA + K * K;               // [64][64]
+    float* sT11 = sT00 + 64 * 64;
+    float* sX = sT11 + 64 * 64;             // A10 T00
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int64_t c = blockIdx.x; c < nc; c += gridDim.x) {
+        const float* Ac = A + c * K * K;
+        float* Tc = T + c * K * K;
+        __syncthreads();                    // the previous chunk is done with shared memory
+#pragma unroll
+        for (int q = 0; q < K * K / 4 / 128; ++q) {
+            const int e = (q * 128 + tid) * 4;
+            cp_async16(sA + e, Ac + e);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        // the upper-right block of T is zero
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int e = q * 128 + tid;        // 1024 float4 of rows 0..63, columns 64..127
+            reinterpret_cast<float4*>(Tc + (e >> 4) * K + 64)[e & 15] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+        switch (warp) {                     // diagonal blocks, 32 columns per warp
+            case 0: fwd_sweep64<0>(sA, K, lane, sT00, Tc, K); break;
+            case 1: fwd_sweep64<32>(sA, K, lane, sT00, Tc, K); break;
+            case 2: fwd_sweep64<0>(sA + 64 * K + 64, K, lane, sT11, Tc + 64 * K + 64, K); break;
+            default: fwd_sweep64<32>(sA + 64 * K + 64, K, lane, sT11, Tc + 64 * K + 64, K); break;
+        }
+        __syncthreads();
+        // 8 x 4 register tiles: rows 8 (tid / 16) .., columns 4 (tid % 16) ..
+        const int r0 = 8 * (tid >> 4), c0 = 4 * (tid & 15);
+        float acc[8][4];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) acc[rr][cc] = 0.f;
+        mm_tile84<K, 64>(sA + 64 * K, sT00, r0, c0, c0, 64, acc);   // X = A10 T00 (T00[l][c] = 0, l < c)
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+            *reinterpret_cast<float4*>(sX + (r0 + rr) * 64 + c0) =
+                make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+        __syncthreads();
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) acc[rr][cc] = 0.f;
+        mm_tile84<64, 64>(sT11, sX, r0, c0, 0, r0 + 8, acc);        // T10 = T11 X (T11[r][l] = 0, l > r)
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+            *reinterpret_cast<float4*>(Tc + (int64_t)(64 + r0 + rr) * K + c0) =
+                make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+    }
+}
+
 // INT8 truncated Neumann, k = 64 (see gdn_invert_neumann_i8 for the scheme).
 __device__ __forceinline__ float block_max_f(float v, float* red) {
     for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -731,6 +854,18 @@ cudaError_t launch_fwdsub(const float* A, float* T, int64_t nc, int k, cudaStrea
             if (!e) k_fwdsub_warp<64><<<grid, 32 * kFwdWarps, smem, st>>>(A, T, nc);
         }
         if (e != cudaSuccess) return e;
+        return cudaGetLastError();
+    }
+    if (k == 128) {
+        const size_t smem = (size_t)(128 * 128 + 3 * 64 * 64) * sizeof(float);
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t cap = (int64_t)sms * 2;
+        const unsigned grid = (unsigned)(nc < cap ? nc : cap);
+        cudaError_t e = prep(k_fwdsub128, smem);
+        if (e != cudaSuccess) return e;
+        k_fwdsub128<<<grid, 128, smem, st>>>(A, T, nc);
         return cudaGetLastError();
     }
     const int CB = k < 128 ? k : 128;
