@@ -1295,9 +1295,11 @@ struct ParamsI8 {
 constexpr int kI8Slots = 2;
 constexpr int kI8OpBytes = kRows * 128;            // 16 KB, rows at a 128-byte pitch
 constexpr int kI8BBytes = 64 * 128;                // 8 KB: K = 64 rows of 128 codes
+constexpr int kI8Stage = kRows * 64 * 4;           // 32 KB: the next tile's A (fp32, swizzled)
+constexpr int kI8SlotBytes = kI8OpBytes + kI8BBytes + kI8Stage;
 
 __global__ void __launch_bounds__(256 * kI8Slots, 1)
-k_neumann_i8_tc(const ParamsI8 p) {
+k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
     constexpr int KC = 64;
     extern __shared__ __align__(1024) uint8_t smem[];
     if ((su32(smem) & 1023u) != 0) {
@@ -1306,16 +1308,20 @@ k_neumann_i8_tc(const ParamsI8 p) {
     }
     struct __align__(8) CtrlI8 {
         uint64_t mma[kI8Slots];
+        uint64_t full[kI8Slots];                   // the slot's staged A landed
         uint32_t tmem;
         int abort;
         float red_f[kI8Slots][2][4];
         int red_i[kI8Slots][2][4];
     };
-    CtrlI8* ctrl = reinterpret_cast<CtrlI8*>(smem + kI8Slots * (kI8OpBytes + kI8BBytes));
+    CtrlI8* ctrl = reinterpret_cast<CtrlI8*>(smem + kI8Slots * kI8SlotBytes);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kI8Slots; ++s) mbar_init(&ctrl->mma[s], 1);
+        for (int s = 0; s < kI8Slots; ++s) {
+            mbar_init(&ctrl->mma[s], 1);
+            mbar_init(&ctrl->full[s], 1);
+        }
         ctrl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1332,8 +1338,9 @@ k_neumann_i8_tc(const ParamsI8 p) {
     const int i = r % KC;
     const int wq = ((warp & 3) & 1) * 2 + h;       // this warp's slot among its chunk's 4 warps
     const int jmin = p.mask ? i - p.N : -KC;
-    uint8_t* sA = smem + s * (kI8OpBytes + kI8BBytes);
+    uint8_t* sA = smem + s * kI8SlotBytes;
     uint8_t* sB = sA + kI8OpBytes;
+    uint8_t* sStage = sB + kI8BBytes;
     const uint32_t tm = tmem_base + (uint32_t)(s * 128);
     const uint32_t tD = tm + ((uint32_t)((warp & 3) * 32) << 16) + c * KC + 32 * h;
     const bool leader = (warp % 8) == 0 && lane == 0;
@@ -1358,25 +1365,47 @@ k_neumann_i8_tc(const ParamsI8 p) {
                    max(ctrl->red_i[s][c][2], ctrl->red_i[s][c][3]));
     };
 
+    // the slot's leader stages A of the slot's tile n: two 32-column boxes
+    int a_issued = 0;
+    auto issue_a = [&](int n) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (tile >= p.ntiles) return;
+        ++a_issued;
+        mbar_expect_tx(&ctrl->full[s], kI8Stage);
+        tma_load_2d(sStage, &mA, 0, tile * kRows, &ctrl->full[s]);
+        tma_load_2d(sStage + 16384, &mA, 32, tile * kRows, &ctrl->full[s]);
+    };
+    if (leader) issue_a(s);
+
     for (int n = s;; n += kI8Slots) {
         const int tile = blockIdx.x + n * gridDim.x;
         if (tile >= p.ntiles) break;
         const int64_t grow = (int64_t)tile * kRows + r;
         const bool valid = grow < p.rows;
         const int64_t cidx = grow / KC, rin = grow % KC;
-        bar_sync(bar_id, 256);                     // previous tile's reads of sA, sB, red done
-        float a[32];
-        if (valid) {
-            const float4* src = reinterpret_cast<const float4*>(p.A + cidx * KC * KC + rin * KC + 32 * h);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float4 t = __ldg(src + q);
-                a[4 * q] = t.x; a[4 * q + 1] = t.y; a[4 * q + 2] = t.z; a[4 * q + 3] = t.w;
-            }
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 32; ++jj) a[jj] = 0.f;
+        if (!mbar_wait(&ctrl->full[s], (uint32_t)((n / kI8Slots) & 1))) {
+            atomicExch(&ctrl->abort, 1);
+            raise_status(p.status, kStatusTimeout);
         }
+        float a[32];                                // rows past the end were zero-filled
+        {
+            const uint32_t rb = su32(sStage) + (uint32_t)(h * 16384 + r * 128);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+                uint32_t u0, u1, u2, u3;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(u0), "=r"(u1), "=r"(u2), "=r"(u3)
+                             : "r"(rb + ((c4 ^ (r & 7)) << 4)));
+                a[4 * c4] = __uint_as_float(u0);
+                a[4 * c4 + 1] = __uint_as_float(u1);
+                a[4 * c4 + 2] = __uint_as_float(u2);
+                a[4 * c4 + 3] = __uint_as_float(u3);
+            }
+        }
+        fence_async_smem();
+        bar_sync(bar_id, 256);                     // previous tile's reads of sA, sB, red and the stage done
+        if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+        if (leader) issue_a(n + kI8Slots);
         float amax = 0.f;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
@@ -1487,7 +1516,10 @@ k_neumann_i8_tc(const ParamsI8 p) {
         }
         tc_fence_before();
     }
-    if (!ok) mbar_wait(&ctrl->mma[s], mma_phase);
+    if (!ok) {
+        mbar_wait(&ctrl->mma[s], mma_phase);
+        if (leader && a_issued > 0) mbar_wait(&ctrl->full[s], (uint32_t)((a_issued - 1) & 1));
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -1882,14 +1914,17 @@ cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8
     p.acc = acc;
     p.scale = sc;
     p.status = status_ptr();
+    CUtensorMap mA;
+    memset(&mA, 0, sizeof mA);
+    if (!tcg::map_f32(&mA, A, p.rows, 64)) return cudaErrorInvalidValue;
     // two CTAs per SM at most: each holds 256 of the SM's 512 TMEM columns
-    const size_t smem = 80 * 1024;
+    const size_t smem = tcg::kI8Slots * tcg::kI8SlotBytes + 512;
     cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int cap = 2 * tcg::num_sms();
     const int grid = p.ntiles < cap ? p.ntiles : cap;
-    tcg::k_neumann_i8_tc<<<grid, 256 * tcg::kI8Slots, smem, st>>>(p);
+    tcg::k_neumann_i8_tc<<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
     return cudaGetLastError();
 }
 
