@@ -242,8 +242,10 @@ int gdn_forward(const void* Q, const void* K, const void* V, const float* beta, 
         GDN_TRY(gdn_chunk_wy_fused(K, V, beta, g, N, mask, S, 1, Wg, U, nullptr, s, dtype,
                                    stream));
     }
-    return launched(gdn::launch_scan(Q, K, Wg, U, g, S0, O, S_final, s.B * s.H, s.T / s.k, bf16,
-                                     st),
+    // the A / T region (2 k^2 f32 per chunk = d^2 fp16 at k = 64) takes the
+    // chunks' start states of the bf16 scan
+    return launched(gdn::launch_scan(Q, K, Wg, U, g, S0, O, S_final, Abuf, s.B * s.H, s.T / s.k,
+                                     bf16, st),
                     "forward scan");
 }
 

@@ -22,8 +22,10 @@ cudaError_t launch_neumann_i8_simt(const float* A, float* T, int N, int mask, in
                                    int32_t* acc, float* sc, int64_t nc, cudaStream_t st);
 
 // Inter-chunk state scan of the forward (scan.cu); k = 64, d = 128.
-cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, const void* U, const float* g,
-                        const float* S0, void* O, float* Sfin, int64_t BH, int64_t nchunk,
-                        bool bf16, cudaStream_t st);
+// bf16: U is overwritten by V~ (fp16) and Sstates ([B*H*nchunk][d][d] fp16) by
+// the chunks' start states; f32 uses neither.
+cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, const float* g,
+                        const float* S0, void* O, float* Sfin, void* Sstates, int64_t BH,
+                        int64_t nchunk, bool bf16, cudaStream_t st);
 
 }  // namespace gdn

@@ -525,10 +525,341 @@ k_scan_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__
     }
 }
 
-cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, const void* U, const float* g,
-                        const float* S0, void* O, float* Sfin, int64_t BH, int64_t nchunk,
-                        bool bf16, cudaStream_t st) {
+// ---------------------------------------------------------------------------
+// bf16 forward in two kernels.  The recurrence is the only serial part, so it
+// runs alone (k_state_tc: per chunk V~ = U - W_g S^T, written over U as fp16,
+// the chunk's start state S_c stored as fp16, S <- gamma_last S + (V~ dec)^T K),
+// and the output of every chunk follows in parallel (k_out_tc:
+// O = diag(gamma) Q S_c^T + (Q K^T . Gamma . L) V~, the scores once per chunk).
+// ---------------------------------------------------------------------------
+constexpr int kStThreads = 128;
+
+struct StTile {
+    static constexpr int kPitch = kSD + 8;                     // staged bf16 row, elements
+    static constexpr int kTile = kSK * kPitch * 2;
+    static constexpr int kU = kSK * kDV * 2;
+    static constexpr int kStage = 2 * kTile + kU + kSK * 4;    // K, W_g, U slice, g
+};
+
+__device__ __forceinline__ void fetch_state(uint8_t* st, const __nv_bfloat16* K,
+                                            const __nv_bfloat16* Wg, const __nv_bfloat16* U,
+                                            const float* g, int64_t row0, int v0) {
+    constexpr int kPerRow = kSD / 8;
+    const __nv_bfloat16* src[2] = {K + row0 * kSD, Wg + row0 * kSD};
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(st + m * StTile::kTile);
+        for (int e = threadIdx.x; e < kSK * kPerRow; e += kStThreads) {
+            const int r = e / kPerRow, c = (e % kPerRow) * 8;
+            cp_async16(dst + r * StTile::kPitch + c, src[m] + r * kSD + c);
+        }
+    }
+    __nv_bfloat16* ud = reinterpret_cast<__nv_bfloat16*>(st + 2 * StTile::kTile);
+    if (threadIdx.x < kSK * 2) {
+        const int r = threadIdx.x >> 1, c = (threadIdx.x & 1) * 8;
+        cp_async16(ud + r * kDV + c, U + (row0 + r) * kSD + v0 + c);
+    }
+    float* gd = reinterpret_cast<float*>(st + 2 * StTile::kTile + StTile::kU);
+    if (threadIdx.x < kSK / 4) cp_async16(gd + threadIdx.x * 4, g + row0 + threadIdx.x * 4);
+}
+
+__global__ void __launch_bounds__(kStThreads)
+k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ Wg,
+           __nv_bfloat16* __restrict__ U, const float* __restrict__ g, const float* __restrict__ S0,
+           __half* __restrict__ Sst, float* __restrict__ Sfin, int64_t nchunk) {
+    constexpr int P = StTile::kPitch;
+    constexpr int P16 = ScanMma::kP16;
+    constexpr int PS = ScanMma::kPS;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t* stage[2] = {smem, smem + StTile::kStage};
+    __half* sSh = reinterpret_cast<__half*>(smem + 2 * StTile::kStage);        // [16][136] S
+    __nv_bfloat16* sVd = reinterpret_cast<__nv_bfloat16*>(sSh + kDV * PS);      // [16][72]
+    float* sdec = reinterpret_cast<float*>(sVd + kDV * P16);                    // [64]
+    const int64_t bh = blockIdx.x;
+    const int v0 = blockIdx.y * kDV;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gr = lane >> 2, gc = (lane & 3) * 2;
+    const int mt = 16 * warp;                      // token rows of this warp (V~)
+
+    float Sacc[4][4];                              // columns 32w + 8nt + gc, rows gr, gr + 8
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const int c = 32 * warp + 8 * nt + gc;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int v = gr + 8 * hh;
+            const float s0 = S0 ? S0[(bh * kSD + v0 + v) * kSD + c] : 0.f;
+            const float s1 = S0 ? S0[(bh * kSD + v0 + v) * kSD + c + 1] : 0.f;
+            Sacc[nt][2 * hh] = s0;
+            Sacc[nt][2 * hh + 1] = s1;
+            *reinterpret_cast<uint32_t*>(sSh + v * PS + c) = pack_h2f(s0, s1);
+        }
+    }
+    fetch_state(stage[0], K, Wg, U, g, bh * nchunk * kSK, v0);
+    cp_async_commit();
+
+    for (int64_t ci = 0; ci < nchunk; ++ci) {
+        const int64_t row0 = (bh * nchunk + ci) * kSK;
+        uint8_t* cur = stage[ci & 1];
+        if (ci + 1 < nchunk) {
+            fetch_state(stage[(ci + 1) & 1], K, Wg, U, g, row0 + kSK, v0);
+            cp_async_commit();
+            cp_async_wait1();
+        } else {
+            cp_async_wait0();
+        }
+        __syncthreads();
+        const __nv_bfloat16* Ks = reinterpret_cast<const __nv_bfloat16*>(cur);
+        const __nv_bfloat16* Ws = reinterpret_cast<const __nv_bfloat16*>(cur + StTile::kTile);
+        const __nv_bfloat16* Us = reinterpret_cast<const __nv_bfloat16*>(cur + 2 * StTile::kTile);
+        const float* gs = reinterpret_cast<const float*>(cur + 2 * StTile::kTile + StTile::kU);
+        if (tid < kSK) sdec[tid] = exp_e(gs[kSK - 1] - gs[tid]);
+        // the chunk's start state, for the output pass
+        {
+            __half* dst = Sst + ((bh * nchunk + ci) * kSD + v0) * kSD;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int c = 32 * warp + 8 * nt + gc;
+                *reinterpret_cast<uint32_t*>(dst + gr * kSD + c) = pack_h2f(Sacc[nt][0], Sacc[nt][1]);
+                *reinterpret_cast<uint32_t*>(dst + (gr + 8) * kSD + c) =
+                    pack_h2f(Sacc[nt][2], Sacc[nt][3]);
+            }
+        }
+        __syncthreads();                           // sdec
+        // V~ = U - W_g S^T on rows mt .. mt + 15
+        {
+            float acc[2][4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+#pragma unroll
+            for (int k0 = 0; k0 < kSD; k0 += 16) {
+                const uint32_t a0 = bf2_to_h2(ld32(Ws + (mt + gr) * P + k0 + gc));
+                const uint32_t a1 = bf2_to_h2(ld32(Ws + (mt + gr + 8) * P + k0 + gc));
+                const uint32_t a2 = bf2_to_h2(ld32(Ws + (mt + gr) * P + k0 + gc + 8));
+                const uint32_t a3 = bf2_to_h2(ld32(Ws + (mt + gr + 8) * P + k0 + gc + 8));
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+                    mma_f16(acc[n], a0, a1, a2, a3, ld32(sSh + (8 * n + gr) * PS + k0 + gc),
+                            ld32(sSh + (8 * n + gr) * PS + k0 + gc + 8));
+            }
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                const int v = 8 * n + gc;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int t = mt + gr + 8 * hh;
+                    const float x0 = __bfloat162float(Us[t * kDV + v]) - acc[n][2 * hh];
+                    const float x1 = __bfloat162float(Us[t * kDV + v + 1]) - acc[n][2 * hh + 1];
+                    sVd[v * P16 + t] = __float2bfloat16_rn(x0 * sdec[t]);
+                    sVd[(v + 1) * P16 + t] = __float2bfloat16_rn(x1 * sdec[t]);
+                    // V~ replaces U (fp16 bits)
+                    *reinterpret_cast<uint32_t*>(U + (row0 + t) * kSD + v0 + v) = pack_h2f(x0, x1);
+                }
+            }
+        }
+        __syncthreads();
+        // S' = gamma_last S + (V~ dec)^T K, columns 32w .. 32w + 31
+        {
+            const float gl = exp_e(gs[kSK - 1]);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) Sacc[nt][i] *= gl;
+#pragma unroll
+            for (int k0 = 0; k0 < kSK; k0 += 16) {
+                const uint32_t a0 = ld32(sVd + gr * P16 + k0 + gc);
+                const uint32_t a1 = ld32(sVd + (gr + 8) * P16 + k0 + gc);
+                const uint32_t a2 = ld32(sVd + gr * P16 + k0 + gc + 8);
+                const uint32_t a3 = ld32(sVd + (gr + 8) * P16 + k0 + gc + 8);
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const int n0 = 32 * warp + 8 * nt;
+                    const int krow = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const uint32_t addr = (uint32_t)__cvta_generic_to_shared(Ks + krow * P + n0);
+                    uint32_t b0, b1;
+                    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                                 : "=r"(b0), "=r"(b1) : "r"(addr));
+                    mma_bf16(Sacc[nt], a0, a1, a2, a3, b0, b1);
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int c = 32 * warp + 8 * nt + gc;
+                *reinterpret_cast<uint32_t*>(sSh + gr * PS + c) = pack_h2f(Sacc[nt][0], Sacc[nt][1]);
+                *reinterpret_cast<uint32_t*>(sSh + (gr + 8) * PS + c) =
+                    pack_h2f(Sacc[nt][2], Sacc[nt][3]);
+            }
+        }
+        __syncthreads();                           // stage, sVd and the S copy free
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const int c = 32 * warp + 8 * nt + gc;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int v = gr + 8 * hh;
+            Sfin[(bh * kSD + v0 + v) * kSD + c] = Sacc[nt][2 * hh];
+            Sfin[(bh * kSD + v0 + v) * kSD + c + 1] = Sacc[nt][2 * hh + 1];
+        }
+    }
+}
+
+struct OutTile {
+    static constexpr int kP = kSD + 8;                         // staged row pitch, elements
+    static constexpr int kQ = kSK * kP * 2;                    // Q, K, V~ tiles
+    static constexpr int kS = kSD * kP * 2;                    // S_c (fp16)
+    static constexpr int kA = kSK * ScanMma::kP16 * 2;         // scores (fp16)
+    static constexpr int bytes = 3 * kQ + kS + kA + kSK * 4;
+};
+
+__global__ void __launch_bounds__(kStThreads)
+k_out_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+         const __half* __restrict__ Vt, const float* __restrict__ g, const __half* __restrict__ Sst,
+         __nv_bfloat16* __restrict__ O, int64_t nctot) {
+    constexpr int P = OutTile::kP;
+    constexpr int P16 = ScanMma::kP16;
+    extern __shared__ __align__(16) uint8_t smem[];
+    __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
+    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + OutTile::kQ);
+    __half* sV = reinterpret_cast<__half*>(smem + 2 * OutTile::kQ);
+    __half* sS = reinterpret_cast<__half*>(smem + 3 * OutTile::kQ);
+    __half* sA = reinterpret_cast<__half*>(smem + 3 * OutTile::kQ + OutTile::kS);
+    float* sg = reinterpret_cast<float*>(smem + 3 * OutTile::kQ + OutTile::kS + OutTile::kA);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gr = lane >> 2, gc = (lane & 3) * 2;
+    const int mt = 16 * warp;
+    for (int64_t ch = blockIdx.x; ch < nctot; ch += gridDim.x) {
+        const int64_t row0 = ch * kSK;
+        __syncthreads();                           // the previous chunk's tiles are read
+        for (int e = tid; e < kSK * 16; e += kStThreads) {
+            const int r = e >> 4, c = (e & 15) * 8;
+            cp_async16(sQ + r * P + c, Q + (row0 + r) * kSD + c);
+            cp_async16(sK + r * P + c, K + (row0 + r) * kSD + c);
+            cp_async16(sV + r * P + c, Vt + (row0 + r) * kSD + c);
+        }
+        for (int e = tid; e < kSD * 16; e += kStThreads) {
+            const int r = e >> 4, c = (e & 15) * 8;
+            cp_async16(sS + r * P + c, Sst + (ch * kSD + r) * kSD + c);
+        }
+        if (tid < kSK / 4) cp_async16(sg + tid * 4, g + row0 + tid * 4);
+        cp_async_commit();
+        cp_async_wait0();
+        __syncthreads();
+        const int t0 = mt + gr, t1 = t0 + 8;
+        const float g0 = sg[t0], g1 = sg[t1];
+        // scores . Gamma . L on this warp's rows (column tiles up to the diagonal)
+        {
+            float acc[8][4];
+#pragma unroll
+            for (int n = 0; n < 8; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+#pragma unroll
+            for (int k0 = 0; k0 < kSD; k0 += 16) {
+                const uint32_t a0 = ld32(sQ + t0 * P + k0 + gc);
+                const uint32_t a1 = ld32(sQ + t1 * P + k0 + gc);
+                const uint32_t a2 = ld32(sQ + t0 * P + k0 + gc + 8);
+                const uint32_t a3 = ld32(sQ + t1 * P + k0 + gc + 8);
+#pragma unroll
+                for (int n = 0; n < 8; ++n) {
+                    if (8 * n > mt + 15) continue;
+                    mma_bf16(acc[n], a0, a1, a2, a3, ld32(sK + (8 * n + gr) * P + k0 + gc),
+                             ld32(sK + (8 * n + gr) * P + k0 + gc + 8));
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const int c = 8 * n + gc;
+                const float x00 = c <= t0 ? acc[n][0] * exp_e(g0 - sg[c]) : 0.f;
+                const float x01 = c + 1 <= t0 ? acc[n][1] * exp_e(g0 - sg[c + 1]) : 0.f;
+                const float x10 = c <= t1 ? acc[n][2] * exp_e(g1 - sg[c]) : 0.f;
+                const float x11 = c + 1 <= t1 ? acc[n][3] * exp_e(g1 - sg[c + 1]) : 0.f;
+                *reinterpret_cast<uint32_t*>(sA + t0 * P16 + c) = pack_h2f(x00, x01);
+                *reinterpret_cast<uint32_t*>(sA + t1 * P16 + c) = pack_h2f(x10, x11);
+            }
+        }
+        __syncwarp();                              // sA rows of this warp
+        // P = Q S_c^T (all 128 state rows), times gamma
+        float pacc[16][4];
+#pragma unroll
+        for (int n = 0; n < 16; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pacc[n][i] = 0.f;
+#pragma unroll
+        for (int k0 = 0; k0 < kSD; k0 += 16) {
+            const uint32_t a0 = bf2_to_h2(ld32(sQ + t0 * P + k0 + gc));
+            const uint32_t a1 = bf2_to_h2(ld32(sQ + t1 * P + k0 + gc));
+            const uint32_t a2 = bf2_to_h2(ld32(sQ + t0 * P + k0 + gc + 8));
+            const uint32_t a3 = bf2_to_h2(ld32(sQ + t1 * P + k0 + gc + 8));
+#pragma unroll
+            for (int n = 0; n < 16; ++n)
+                mma_f16(pacc[n], a0, a1, a2, a3, ld32(sS + (8 * n + gr) * P + k0 + gc),
+                        ld32(sS + (8 * n + gr) * P + k0 + gc + 8));
+        }
+        const float gam0 = exp_e(g0), gam1 = exp_e(g1);
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            pacc[n][0] *= gam0;
+            pacc[n][1] *= gam0;
+            pacc[n][2] *= gam1;
+            pacc[n][3] *= gam1;
+        }
+        // O += scores V~ over the causal token tiles
+        for (int k0 = 0; k0 <= mt; k0 += 16) {
+            const uint32_t a0 = ld32(sA + t0 * P16 + k0 + gc);
+            const uint32_t a1 = ld32(sA + t1 * P16 + k0 + gc);
+            const uint32_t a2 = ld32(sA + t0 * P16 + k0 + gc + 8);
+            const uint32_t a3 = ld32(sA + t1 * P16 + k0 + gc + 8);
+            const int krow = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+                const uint32_t addr = (uint32_t)__cvta_generic_to_shared(sV + krow * P + 8 * n);
+                uint32_t b0, b1;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                             : "=r"(b0), "=r"(b1) : "r"(addr));
+                mma_f16(pacc[n], a0, a1, a2, a3, b0, b1);
+            }
+        }
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            const int v = 8 * n + gc;
+            *reinterpret_cast<__nv_bfloat162*>(O + (row0 + t0) * kSD + v) =
+                __floats2bfloat162_rn(pacc[n][0], pacc[n][1]);
+            *reinterpret_cast<__nv_bfloat162*>(O + (row0 + t1) * kSD + v) =
+                __floats2bfloat162_rn(pacc[n][2], pacc[n][3]);
+        }
+    }
+}
+
+cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, const float* g,
+                        const float* S0, void* O, float* Sfin, void* Sstates, int64_t BH,
+                        int64_t nchunk, bool bf16, cudaStream_t st) {
     dim3 grid((unsigned)BH, kSD / kDV);
+    if (bf16) {
+        const size_t s1 = 2 * StTile::kStage + (size_t)kDV * ScanMma::kPS * 2 +
+                          (size_t)kDV * ScanMma::kP16 * 2 + kSK * sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(k_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)s1);
+        if (e != cudaSuccess) return e;
+        k_state_tc<<<grid, kStThreads, s1, st>>>((const __nv_bfloat16*)K, (const __nv_bfloat16*)Wg,
+                                                 (__nv_bfloat16*)U, g, S0, (__half*)Sstates, Sfin,
+                                                 nchunk);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(k_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 OutTile::bytes);
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t nct = BH * nchunk, cap = (int64_t)sms * 2;
+        k_out_tc<<<(unsigned)(nct < cap ? nct : cap), kStThreads, OutTile::bytes, st>>>(
+            (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __half*)U, g,
+            (const __half*)Sstates, (__nv_bfloat16*)O, nct);
+        return cudaGetLastError();
+    }
     auto smem_for = [](int stage, int nstages) {
         return (size_t)(nstages * stage) + (size_t)(kDV * (kSD + 1) + 2 * kSK * kDV +
                                                     kSK * (kSK + 1) + 2 * kSK) * sizeof(float);
