@@ -533,6 +533,7 @@ k_scan_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__
 // O = diag(gamma) Q S_c^T + (Q K^T . Gamma . L) V~, the scores once per chunk).
 // ---------------------------------------------------------------------------
 constexpr int kStThreads = 128;
+constexpr int kStStages = 3;
 
 struct StTile {
     static constexpr int kPitch = kSD + 8;                     // staged bf16 row, elements
@@ -571,10 +572,10 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
     constexpr int P16 = ScanMma::kP16;
     constexpr int PS = ScanMma::kPS;
     extern __shared__ __align__(16) uint8_t smem[];
-    uint8_t* stage[2] = {smem, smem + StTile::kStage};
-    __half* sSh = reinterpret_cast<__half*>(smem + 2 * StTile::kStage);        // [16][136] S
+    // kStStages stages: the tiles of chunks ci + 1 .. ci + kStStages - 1 stream
+    // in while chunk ci is used
+    __half* sSh = reinterpret_cast<__half*>(smem + kStStages * StTile::kStage); // [16][136] S
     __nv_bfloat16* sVd = reinterpret_cast<__nv_bfloat16*>(sSh + kDV * PS);      // [16][72]
-    float* sdec = reinterpret_cast<float*>(sVd + kDV * P16);                    // [64]
     const int64_t bh = blockIdx.x;
     const int v0 = blockIdx.y * kDV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -595,25 +596,31 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
             *reinterpret_cast<uint32_t*>(sSh + v * PS + c) = pack_h2f(s0, s1);
         }
     }
-    fetch_state(stage[0], K, Wg, U, g, bh * nchunk * kSK, v0);
-    cp_async_commit();
+#pragma unroll
+    for (int q = 0; q < kStStages - 1; ++q) {
+        if (q < nchunk)
+            fetch_state(smem + q * StTile::kStage, K, Wg, U, g, (bh * nchunk + q) * kSK, v0);
+        cp_async_commit();
+    }
 
+    // Two barriers per chunk: the first makes this chunk's tiles and the
+    // previous S' (sSh) visible and frees the stage of chunk ci - 1 for the
+    // prefetch;
+    // the second makes V~ (sVd) visible to the state update.
     for (int64_t ci = 0; ci < nchunk; ++ci) {
         const int64_t row0 = (bh * nchunk + ci) * kSK;
-        uint8_t* cur = stage[ci & 1];
-        if (ci + 1 < nchunk) {
-            fetch_state(stage[(ci + 1) & 1], K, Wg, U, g, row0 + kSK, v0);
-            cp_async_commit();
-            cp_async_wait1();
-        } else {
-            cp_async_wait0();
-        }
+        uint8_t* cur = smem + (ci % kStStages) * StTile::kStage;
+        // this chunk's group is complete; the later ones may be in flight
+        asm volatile("cp.async.wait_group %0;" ::"n"(kStStages - 2) : "memory");
         __syncthreads();
+        if (ci + kStStages - 1 < nchunk)
+            fetch_state(smem + ((ci + kStStages - 1) % kStStages) * StTile::kStage, K, Wg, U, g,
+                        row0 + (kStStages - 1) * kSK, v0);
+        cp_async_commit();                         // (possibly empty) keeps the group count
         const __nv_bfloat16* Ks = reinterpret_cast<const __nv_bfloat16*>(cur);
         const __nv_bfloat16* Ws = reinterpret_cast<const __nv_bfloat16*>(cur + StTile::kTile);
         const __nv_bfloat16* Us = reinterpret_cast<const __nv_bfloat16*>(cur + 2 * StTile::kTile);
         const float* gs = reinterpret_cast<const float*>(cur + 2 * StTile::kTile + StTile::kU);
-        if (tid < kSK) sdec[tid] = exp_e(gs[kSK - 1] - gs[tid]);
         // the chunk's start state, for the output pass
         {
             __half* dst = Sst + ((bh * nchunk + ci) * kSD + v0) * kSD;
@@ -625,14 +632,13 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
                     pack_h2f(Sacc[nt][2], Sacc[nt][3]);
             }
         }
-        __syncthreads();                           // sdec
-        // V~ = U - W_g S^T on rows mt .. mt + 15
+        // V~ = U - W_g S^T on rows mt .. mt + 15 (two accumulation chains)
         {
-            float acc[2][4];
+            float acc[2][4], acc2[2][4];
 #pragma unroll
             for (int n = 0; n < 2; ++n)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+                for (int i = 0; i < 4; ++i) acc[n][i] = acc2[n][i] = 0.f;
 #pragma unroll
             for (int k0 = 0; k0 < kSD; k0 += 16) {
                 const uint32_t a0 = bf2_to_h2(ld32(Ws + (mt + gr) * P + k0 + gc));
@@ -641,19 +647,26 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
                 const uint32_t a3 = bf2_to_h2(ld32(Ws + (mt + gr + 8) * P + k0 + gc + 8));
 #pragma unroll
                 for (int n = 0; n < 2; ++n)
-                    mma_f16(acc[n], a0, a1, a2, a3, ld32(sSh + (8 * n + gr) * PS + k0 + gc),
+                    mma_f16(k0 < kSD / 2 ? acc[n] : acc2[n], a0, a1, a2, a3,
+                            ld32(sSh + (8 * n + gr) * PS + k0 + gc),
                             ld32(sSh + (8 * n + gr) * PS + k0 + gc + 8));
             }
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[n][i] += acc2[n][i];
+            const float gl1 = gs[kSK - 1];
 #pragma unroll
             for (int n = 0; n < 2; ++n) {
                 const int v = 8 * n + gc;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int t = mt + gr + 8 * hh;
+                    const float dec = exp_e(gl1 - gs[t]);
                     const float x0 = __bfloat162float(Us[t * kDV + v]) - acc[n][2 * hh];
                     const float x1 = __bfloat162float(Us[t * kDV + v + 1]) - acc[n][2 * hh + 1];
-                    sVd[v * P16 + t] = __float2bfloat16_rn(x0 * sdec[t]);
-                    sVd[(v + 1) * P16 + t] = __float2bfloat16_rn(x1 * sdec[t]);
+                    sVd[v * P16 + t] = __float2bfloat16_rn(x0 * dec);
+                    sVd[(v + 1) * P16 + t] = __float2bfloat16_rn(x1 * dec);
                     // V~ replaces U (fp16 bits)
                     *reinterpret_cast<uint32_t*>(U + (row0 + t) * kSD + v0 + v) = pack_h2f(x0, x1);
                 }
@@ -692,7 +705,6 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
                     pack_h2f(Sacc[nt][2], Sacc[nt][3]);
             }
         }
-        __syncthreads();                           // stage, sVd and the S copy free
     }
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
@@ -838,8 +850,8 @@ cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, c
                         int64_t nchunk, bool bf16, cudaStream_t st) {
     dim3 grid((unsigned)BH, kSD / kDV);
     if (bf16) {
-        const size_t s1 = 2 * StTile::kStage + (size_t)kDV * ScanMma::kPS * 2 +
-                          (size_t)kDV * ScanMma::kP16 * 2 + kSK * sizeof(float);
+        const size_t s1 = kStStages * StTile::kStage + (size_t)kDV * ScanMma::kPS * 2 +
+                          (size_t)kDV * ScanMma::kP16 * 2;
         cudaError_t e = cudaFuncSetAttribute(k_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)s1);
         if (e != cudaSuccess) return e;
