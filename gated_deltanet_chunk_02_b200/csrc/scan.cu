@@ -11,12 +11,14 @@
 // (L: lower triangle with the diagonal).  Row v of S only ever meets column v
 // of V~, U and O, so the d_v rows split across CTAs with no exchange: grid =
 // (B*H, d_v / DV), each CTA walks its head's chunks in order holding a DV x d_k
-// slice of S in shared memory.
+// slice of S.
 //
-// Per chunk the next chunk's Q, K, W_g, U and g tiles are fetched with
-// cp.async while this one is processed.  bf16 data run every product on the
-// tensor cores (k_scan_tc, mma.sync with fp32 accumulation, the state slice
-// held as fp32 accumulator fragments); fp32 data run fp32 FMA loops (k_scan).
+// bf16 data: only V~ and S' are on the serial path.  k_state_tc runs them
+// alone (tiles prefetched two chunks ahead with cp.async, the state slice
+// held as fp32 mma.sync accumulator fragments), writing V~ over U and each
+// chunk's start state S_c to the workspace; k_out_tc then forms O for every
+// chunk in parallel.  fp32 data: k_scan does the whole recurrence and O in
+// one pass with fp32 FMA loops.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -87,48 +89,6 @@ __device__ __forceinline__ void fetch_chunk(uint8_t* st, const TI* Q, const TI* 
 }
 
 // sA[t][j] = (q_t . k_j) e^{g_t - g_j} for j <= t, else 0 (pitch 65).
-__device__ __forceinline__ void chunk_scores(const __nv_bfloat16* Qs, const __nv_bfloat16* Ks,
-                                             const float* gs, float* sA) {
-    // 8 warps: warp w owns rows 16*(w/2) .. +16 and columns 32*(w%2) .. +32
-    constexpr int P = ScanTile<__nv_bfloat16>::kPitch;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = 16 * (warp >> 1), n0 = 32 * (warp & 1);
-    const int gr = lane >> 2, gc = 2 * (lane & 3);
-    float acc[4][4];
-#pragma unroll
-    for (int n = 0; n < 4; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-#pragma unroll
-    for (int k0 = 0; k0 < kSD; k0 += 16) {
-        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr) * P + k0 + gc);
-        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr + 8) * P + k0 + gc);
-        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr) * P + k0 + gc + 8);
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(Qs + (m0 + gr + 8) * P + k0 + gc + 8);
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            const int nb = n0 + 8 * n;
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(Ks + (nb + gr) * P + k0 + gc);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(Ks + (nb + gr) * P + k0 + gc + 8);
-            asm volatile(
-                "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-                "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-                : "+f"(acc[n][0]), "+f"(acc[n][1]), "+f"(acc[n][2]), "+f"(acc[n][3])
-                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-        }
-    }
-    const int t0 = m0 + gr, t1 = m0 + gr + 8;
-    const float g0 = gs[t0], g1 = gs[t1];
-#pragma unroll
-    for (int n = 0; n < 4; ++n) {
-        const int c = n0 + 8 * n + gc;
-        const float gc0 = gs[c], gc1 = gs[c + 1];
-        sA[t0 * (kSK + 1) + c] = c <= t0 ? acc[n][0] * exp_e(g0 - gc0) : 0.f;
-        sA[t0 * (kSK + 1) + c + 1] = c + 1 <= t0 ? acc[n][1] * exp_e(g0 - gc1) : 0.f;
-        sA[t1 * (kSK + 1) + c] = c <= t1 ? acc[n][2] * exp_e(g1 - gc0) : 0.f;
-        sA[t1 * (kSK + 1) + c + 1] = c + 1 <= t1 ? acc[n][3] * exp_e(g1 - gc1) : 0.f;
-    }
-}
 __device__ __forceinline__ void chunk_scores(const float* Qs, const float* Ks, const float* gs,
                                              float* sA) {
     constexpr int P = ScanTile<float>::kPitch;
@@ -268,13 +228,9 @@ k_scan(const TI* __restrict__ Q, const TI* __restrict__ K, const TI* __restrict_
 }
 
 // ------------------------------------------------------------------------- //
-// bf16 data: every per-chunk product on the tensor cores (mma.sync m16n8k16,
-// fp32 accumulation).  Warps 0-3 own the state slice S (16 x 128) as fp32
-// accumulator fragments (warp w: columns [32w, 32w + 32)); they form
-// V~ = U - W_g S^T and the state update.  Warps 4-7 form P = Q S^T and
-// O = diag(gamma) P + (scores . Gamma . L) V~.  All 8 warps share the scores.
-// Operands pass through shared memory as fp16 (W_g, Q converted exactly from
-// bf16; S, V~, scores rounded to fp16) or bf16 (K, V~ diag(decay)).
+// bf16 data: mma.sync m16n8k16 with fp32 accumulation.  Operands pass through
+// shared memory as fp16 (W_g, Q converted exactly from bf16; S, V~, scores
+// rounded to fp16) or bf16 (K, V~ diag(decay)).
 // ------------------------------------------------------------------------- //
 struct ScanMma {
     static constexpr int kP16 = kSK + 8;          // pitch of 64-wide fp16/bf16 rows
@@ -307,222 +263,6 @@ __device__ __forceinline__ uint32_t ld32(const void* p) { return *reinterpret_ca
 __device__ __forceinline__ uint32_t pack_h2f(float a, float b) {
     const __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-__global__ void __launch_bounds__(kScanThreads)
-k_scan_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-          const __nv_bfloat16* __restrict__ Wg, const __nv_bfloat16* __restrict__ U,
-          const float* __restrict__ g, const float* __restrict__ S0, __nv_bfloat16* __restrict__ O,
-          float* __restrict__ Sfin, int64_t nchunk) {
-    using L = ScanTile<__nv_bfloat16>;
-    constexpr int P = L::kPitch;                  // staged tile pitch (bf16 elements)
-    constexpr int P16 = ScanMma::kP16;
-    constexpr int PS = ScanMma::kPS;
-    extern __shared__ __align__(16) uint8_t smem[];
-    uint8_t* stage[2] = {smem, smem + L::kStage};
-    __half* sA = reinterpret_cast<__half*>(smem + 2 * L::kStage);          // [64][72] scores
-    __half* sSh = sA + kSK * P16;                                          // [16][136] S (fp16)
-    __half* sVt = sSh + kDV * PS;                                          // [16][72] V~^T (fp16)
-    __nv_bfloat16* sVd = reinterpret_cast<__nv_bfloat16*>(sVt + kDV * P16); // [16][72] (V~ dec)^T
-    float* sgam = reinterpret_cast<float*>(sVd + kDV * P16);               // [64]
-    float* sdec = sgam + kSK;                                              // [64]
-    const int64_t bh = blockIdx.x;
-    const int v0 = blockIdx.y * kDV;
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int gr = lane >> 2, gc = (lane & 3) * 2;
-
-    // state fragments (warps 0-3): n-tile nt covers columns 32w + 8nt .. +8
-    float Sacc[4][4];
-    if (warp < 4) {
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int c = 32 * warp + 8 * nt + gc;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int v = gr + 8 * hh;
-                const float s0 = S0 ? S0[(bh * kSD + v0 + v) * kSD + c] : 0.f;
-                const float s1 = S0 ? S0[(bh * kSD + v0 + v) * kSD + c + 1] : 0.f;
-                Sacc[nt][2 * hh] = s0;
-                Sacc[nt][2 * hh + 1] = s1;
-                *reinterpret_cast<uint32_t*>(sSh + v * PS + c) = pack_h2f(s0, s1);
-            }
-        }
-    }
-    fetch_chunk(stage[0], Q, K, Wg, U, g, bh * nchunk * kSK, v0);
-    cp_async_commit();
-
-    for (int64_t ci = 0; ci < nchunk; ++ci) {
-        const int64_t row0 = (bh * nchunk + ci) * kSK;
-        uint8_t* cur = stage[ci & 1];
-        if (ci + 1 < nchunk) {
-            fetch_chunk(stage[(ci + 1) & 1], Q, K, Wg, U, g, row0 + kSK, v0);
-            cp_async_commit();
-            cp_async_wait1();
-        } else {
-            cp_async_wait0();
-        }
-        __syncthreads();
-        const __nv_bfloat16* Qs = reinterpret_cast<const __nv_bfloat16*>(cur);
-        const __nv_bfloat16* Ks = reinterpret_cast<const __nv_bfloat16*>(cur + L::kTileBytes);
-        const __nv_bfloat16* Ws = reinterpret_cast<const __nv_bfloat16*>(cur + 2 * L::kTileBytes);
-        const __nv_bfloat16* Us = reinterpret_cast<const __nv_bfloat16*>(cur + 3 * L::kTileBytes);
-        const float* gs = reinterpret_cast<const float*>(cur + 3 * L::kTileBytes + L::kUBytes);
-        if (tid < kSK) {
-            sgam[tid] = exp_e(gs[tid]);
-            sdec[tid] = exp_e(gs[kSK - 1] - gs[tid]);
-        }
-        // ---- scores . Gamma . L (fp16) : warp w rows 16(w/2).., columns 32(w%2)..
-        {
-            const int m0 = 16 * (warp >> 1), n0 = 32 * (warp & 1);
-            float acc[4][4];
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-#pragma unroll
-            for (int k0 = 0; k0 < kSD; k0 += 16) {
-                const uint32_t a0 = ld32(Qs + (m0 + gr) * P + k0 + gc);
-                const uint32_t a1 = ld32(Qs + (m0 + gr + 8) * P + k0 + gc);
-                const uint32_t a2 = ld32(Qs + (m0 + gr) * P + k0 + gc + 8);
-                const uint32_t a3 = ld32(Qs + (m0 + gr + 8) * P + k0 + gc + 8);
-#pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    const int nb = n0 + 8 * n;
-                    mma_bf16(acc[n], a0, a1, a2, a3, ld32(Ks + (nb + gr) * P + k0 + gc),
-                             ld32(Ks + (nb + gr) * P + k0 + gc + 8));
-                }
-            }
-            const int t0 = m0 + gr, t1 = t0 + 8;
-            const float g0 = gs[t0], g1 = gs[t1];
-#pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const int c = n0 + 8 * n + gc;
-                const float x00 = c <= t0 ? acc[n][0] * exp_e(g0 - gs[c]) : 0.f;
-                const float x01 = c + 1 <= t0 ? acc[n][1] * exp_e(g0 - gs[c + 1]) : 0.f;
-                const float x10 = c <= t1 ? acc[n][2] * exp_e(g1 - gs[c]) : 0.f;
-                const float x11 = c + 1 <= t1 ? acc[n][3] * exp_e(g1 - gs[c + 1]) : 0.f;
-                *reinterpret_cast<uint32_t*>(sA + t0 * P16 + c) = pack_h2f(x00, x01);
-                *reinterpret_cast<uint32_t*>(sA + t1 * P16 + c) = pack_h2f(x10, x11);
-            }
-        }
-        __syncthreads();
-        float Pacc[2][4];                          // warps 4-7: P = Q S^T, then O
-        const int mt = (warp & 3) * 16;            // token tile of this warp
-        {
-            float acc[2][4];
-#pragma unroll
-            for (int n = 0; n < 2; ++n)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-            const __nv_bfloat16* Xs = warp < 4 ? Ws : Qs;
-#pragma unroll
-            for (int k0 = 0; k0 < kSD; k0 += 16) {
-                const uint32_t a0 = bf2_to_h2(ld32(Xs + (mt + gr) * P + k0 + gc));
-                const uint32_t a1 = bf2_to_h2(ld32(Xs + (mt + gr + 8) * P + k0 + gc));
-                const uint32_t a2 = bf2_to_h2(ld32(Xs + (mt + gr) * P + k0 + gc + 8));
-                const uint32_t a3 = bf2_to_h2(ld32(Xs + (mt + gr + 8) * P + k0 + gc + 8));
-#pragma unroll
-                for (int n = 0; n < 2; ++n)
-                    mma_f16(acc[n], a0, a1, a2, a3, ld32(sSh + (8 * n + gr) * PS + k0 + gc),
-                            ld32(sSh + (8 * n + gr) * PS + k0 + gc + 8));
-            }
-            if (warp < 4) {
-                // V~ = U - W_g S^T, stored transposed: fp16 and bf16 times decay
-#pragma unroll
-                for (int n = 0; n < 2; ++n) {
-                    const int v = 8 * n + gc;
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int t = mt + gr + 8 * hh;
-                        const float u0 = __bfloat162float(Us[t * kDV + v]);
-                        const float u1 = __bfloat162float(Us[t * kDV + v + 1]);
-                        const float x0 = u0 - acc[n][2 * hh], x1 = u1 - acc[n][2 * hh + 1];
-                        sVt[v * P16 + t] = __float2half_rn(x0);
-                        sVt[(v + 1) * P16 + t] = __float2half_rn(x1);
-                        sVd[v * P16 + t] = __float2bfloat16_rn(x0 * sdec[t]);
-                        sVd[(v + 1) * P16 + t] = __float2bfloat16_rn(x1 * sdec[t]);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int n = 0; n < 2; ++n)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        Pacc[n][i] = acc[n][i] * sgam[mt + gr + 8 * (i >> 1)];
-            }
-        }
-        __syncthreads();
-        if (warp >= 4) {
-            // O = diag(gamma) P + scores V~ ; causal: only k-tiles <= this token tile
-            for (int k0 = 0; k0 <= mt; k0 += 16) {
-                const uint32_t a0 = ld32(sA + (mt + gr) * P16 + k0 + gc);
-                const uint32_t a1 = ld32(sA + (mt + gr + 8) * P16 + k0 + gc);
-                const uint32_t a2 = ld32(sA + (mt + gr) * P16 + k0 + gc + 8);
-                const uint32_t a3 = ld32(sA + (mt + gr + 8) * P16 + k0 + gc + 8);
-#pragma unroll
-                for (int n = 0; n < 2; ++n)
-                    mma_f16(Pacc[n], a0, a1, a2, a3, ld32(sVt + (8 * n + gr) * P16 + k0 + gc),
-                            ld32(sVt + (8 * n + gr) * P16 + k0 + gc + 8));
-            }
-#pragma unroll
-            for (int n = 0; n < 2; ++n) {
-                const int v = v0 + 8 * n + gc;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int64_t t = row0 + mt + gr + 8 * hh;
-                    __nv_bfloat162 o2 = __floats2bfloat162_rn(Pacc[n][2 * hh], Pacc[n][2 * hh + 1]);
-                    *reinterpret_cast<__nv_bfloat162*>(O + t * kSD + v) = o2;
-                }
-            }
-        } else {
-            // S' = gamma_last S + (V~ decay)^T K: A = sVd [16 x 64], B = K tile (row-major,
-            // loaded transposed by ldmatrix)
-            const float gl = sgam[kSK - 1];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) Sacc[nt][i] *= gl;
-#pragma unroll
-            for (int k0 = 0; k0 < kSK; k0 += 16) {
-                const uint32_t a0 = ld32(sVd + gr * P16 + k0 + gc);
-                const uint32_t a1 = ld32(sVd + (gr + 8) * P16 + k0 + gc);
-                const uint32_t a2 = ld32(sVd + gr * P16 + k0 + gc + 8);
-                const uint32_t a3 = ld32(sVd + (gr + 8) * P16 + k0 + gc + 8);
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int n0 = 32 * warp + 8 * nt;
-                    const int krow = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const uint32_t addr =
-                        (uint32_t)__cvta_generic_to_shared(Ks + krow * P + n0);
-                    uint32_t b0, b1;
-                    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-                                 : "=r"(b0), "=r"(b1) : "r"(addr));
-                    mma_bf16(Sacc[nt], a0, a1, a2, a3, b0, b1);
-                }
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int c = 32 * warp + 8 * nt + gc;
-                *reinterpret_cast<uint32_t*>(sSh + gr * PS + c) = pack_h2f(Sacc[nt][0], Sacc[nt][1]);
-                *reinterpret_cast<uint32_t*>(sSh + (gr + 8) * PS + c) =
-                    pack_h2f(Sacc[nt][2], Sacc[nt][3]);
-            }
-        }
-        __syncthreads();                // stage buffer, V~, scores and S copy free
-    }
-    if (warp < 4) {
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int c = 32 * warp + 8 * nt + gc;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int v = gr + 8 * hh;
-                Sfin[(bh * kSD + v0 + v) * kSD + c] = Sacc[nt][2 * hh];
-                Sfin[(bh * kSD + v0 + v) * kSD + c + 1] = Sacc[nt][2 * hh + 1];
-            }
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -876,25 +616,13 @@ cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, c
         return (size_t)(nstages * stage) + (size_t)(kDV * (kSD + 1) + 2 * kSK * kDV +
                                                     kSK * (kSK + 1) + 2 * kSK) * sizeof(float);
     };
-    cudaError_t e;
-    if (bf16) {
-        const size_t smem = 2 * ScanTile<__nv_bfloat16>::kStage +
-                            (size_t)(kSK * ScanMma::kP16 + kDV * ScanMma::kPS + 2 * kDV * ScanMma::kP16) * 2 +
-                            2 * kSK * sizeof(float);
-        e = cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        k_scan_tc<<<grid, kScanThreads, smem, st>>>(
-            (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)Wg,
-            (const __nv_bfloat16*)U, g, S0, (__nv_bfloat16*)O, Sfin, nchunk);
-    } else {
-        const size_t smem = smem_for(ScanTile<float>::kStage, 1);
-        e = cudaFuncSetAttribute(k_scan<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        k_scan<float><<<grid, kScanThreads, smem, st>>>((const float*)Q, (const float*)K,
-                                                         (const float*)Wg, (const float*)U, g, S0,
-                                                         (float*)O, Sfin, nchunk);
-    }
+    const size_t smem = smem_for(ScanTile<float>::kStage, 1);
+    cudaError_t e = cudaFuncSetAttribute(k_scan<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    k_scan<float><<<grid, kScanThreads, smem, st>>>((const float*)Q, (const float*)K,
+                                                     (const float*)Wg, (const float*)U, g, S0,
+                                                     (float*)O, Sfin, nchunk);
     return cudaGetLastError();
 }
 

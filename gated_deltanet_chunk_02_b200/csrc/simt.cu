@@ -552,9 +552,13 @@ __device__ __forceinline__ void mm_tile84(const float* P, const float* Q, int r0
     }
 }
 
+// `nc` 128 x 128 diagonal blocks: block c is diagonal block (c % nb) of chunk
+// c / nb, rows `pitch` floats apart (k = 128: nb = 1, pitch 128; k = 256: nb = 2,
+// pitch 256, the off-diagonal block then comes from k_fwdsub256_off).
+template <int PITCH>
 __global__ void __launch_bounds__(128)
 k_fwdsub128(const float* __restrict__ A, float* __restrict__ T, int64_t nc) {
-    constexpr int K = 128;
+    constexpr int K = 128, pitch = PITCH, nb = PITCH / 128;
     extern __shared__ __align__(16) float smf[];
     float* sA = smf;                        // [128][128]
     float* sT00 = sA + K * K;               // [64][64]
@@ -562,28 +566,30 @@ k_fwdsub128(const float* __restrict__ A, float* __restrict__ T, int64_t nc) {
     float* sX = sT11 + 64 * 64;             // A10 T00
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     for (int64_t c = blockIdx.x; c < nc; c += gridDim.x) {
-        const float* Ac = A + c * K * K;
-        float* Tc = T + c * K * K;
+        const int64_t boff = (c / nb) * (int64_t)pitch * pitch + (c % nb) * ((int64_t)K * pitch + K);
+        const float* Ac = A + boff;
+        float* Tc = T + boff;
         __syncthreads();                    // the previous chunk is done with shared memory
 #pragma unroll
         for (int q = 0; q < K * K / 4 / 128; ++q) {
-            const int e = (q * 128 + tid) * 4;
-            cp_async16(sA + e, Ac + e);
+            const int e = q * 128 + tid;    // float4 index: row e / 32, column 4 (e % 32)
+            cp_async16(sA + e * 4, Ac + (int64_t)(e >> 5) * pitch + (e & 31) * 4);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         // the upper-right block of T is zero
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int e = q * 128 + tid;        // 1024 float4 of rows 0..63, columns 64..127
-            reinterpret_cast<float4*>(Tc + (e >> 4) * K + 64)[e & 15] = make_float4(0.f, 0.f, 0.f, 0.f);
+            reinterpret_cast<float4*>(Tc + (int64_t)(e >> 4) * pitch + 64)[e & 15] =
+                make_float4(0.f, 0.f, 0.f, 0.f);
         }
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
         switch (warp) {                     // diagonal blocks, 32 columns per warp
-            case 0: fwd_sweep64<0>(sA, K, lane, sT00, Tc, K); break;
-            case 1: fwd_sweep64<32>(sA, K, lane, sT00, Tc, K); break;
-            case 2: fwd_sweep64<0>(sA + 64 * K + 64, K, lane, sT11, Tc + 64 * K + 64, K); break;
-            default: fwd_sweep64<32>(sA + 64 * K + 64, K, lane, sT11, Tc + 64 * K + 64, K); break;
+            case 0: fwd_sweep64<0>(sA, K, lane, sT00, Tc, pitch); break;
+            case 1: fwd_sweep64<32>(sA, K, lane, sT00, Tc, pitch); break;
+            case 2: fwd_sweep64<0>(sA + 64 * K + 64, K, lane, sT11, Tc + 64 * pitch + 64, pitch); break;
+            default: fwd_sweep64<32>(sA + 64 * K + 64, K, lane, sT11, Tc + 64 * pitch + 64, pitch); break;
         }
         __syncthreads();
         // 8 x 4 register tiles: rows 8 (tid / 16) .., columns 4 (tid % 16) ..
@@ -606,8 +612,103 @@ k_fwdsub128(const float* __restrict__ A, float* __restrict__ T, int64_t nc) {
         mm_tile84<64, 64>(sT11, sX, r0, c0, 0, r0 + 8, acc);        // T10 = T11 X (T11[r][l] = 0, l > r)
 #pragma unroll
         for (int rr = 0; rr < 8; ++rr)
-            *reinterpret_cast<float4*>(Tc + (int64_t)(64 + r0 + rr) * K + c0) =
+            *reinterpret_cast<float4*>(Tc + (int64_t)(64 + r0 + rr) * pitch + c0) =
                 make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+    }
+}
+
+// k = 256 off-diagonal block: with T00, T11 (128 x 128) already in T,
+// T10 = T11 (A10 T00) and T01 = 0.  One chunk per 256-thread CTA; thread
+// (tr, tc) owns rows 8 tr .., columns 8 tc .. of each 128 x 128 product.
+__device__ __forceinline__ void mm128_tile(const float* P, const float* Q, int r0, int c0, int l_lo,
+                                           int l_hi, float (&acc)[8][8]) {
+#pragma unroll 1
+    for (int l = l_lo; l < l_hi; l += 4) {
+        float4 qa[4], qb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            qa[u] = *reinterpret_cast<const float4*>(Q + (l + u) * 128 + c0);
+            qb[u] = *reinterpret_cast<const float4*>(Q + (l + u) * 128 + c0 + 4);
+        }
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            const float4 pv = *reinterpret_cast<const float4*>(P + (r0 + rr) * 128 + l);
+            const float pu[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                acc[rr][0] = fmaf(pu[u], qa[u].x, acc[rr][0]);
+                acc[rr][1] = fmaf(pu[u], qa[u].y, acc[rr][1]);
+                acc[rr][2] = fmaf(pu[u], qa[u].z, acc[rr][2]);
+                acc[rr][3] = fmaf(pu[u], qa[u].w, acc[rr][3]);
+                acc[rr][4] = fmaf(pu[u], qb[u].x, acc[rr][4]);
+                acc[rr][5] = fmaf(pu[u], qb[u].y, acc[rr][5]);
+                acc[rr][6] = fmaf(pu[u], qb[u].z, acc[rr][6]);
+                acc[rr][7] = fmaf(pu[u], qb[u].w, acc[rr][7]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256)
+k_fwdsub256_off(const float* __restrict__ A, float* __restrict__ T, int64_t nc) {
+    constexpr int K = 256, H = 128;
+    extern __shared__ __align__(16) float smf[];
+    float* sP = smf;                        // A10, then T11   [128][128]
+    float* sQ = sP + H * H;                 // T00             [128][128]
+    float* sX = sQ + H * H;                 // A10 T00         [128][128]
+    const int tid = threadIdx.x;
+    const int r0 = 8 * (tid >> 4), c0 = 8 * (tid & 15);
+    auto load_block = [&](float* dst, const float* src) {   // 128 x 128 block, row pitch K
+#pragma unroll 4
+        for (int q = 0; q < H * H / 4 / 256; ++q) {
+            const int e = q * 256 + tid;
+            cp_async16(dst + e * 4, src + (int64_t)(e >> 5) * K + (e & 31) * 4);
+        }
+    };
+    for (int64_t c = blockIdx.x; c < nc; c += gridDim.x) {
+        const float* Ac = A + c * K * K;
+        float* Tc = T + c * K * K;
+        __syncthreads();
+        load_block(sP, Ac + H * K);                          // A10
+        load_block(sQ, Tc);                                  // T00
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        // T01 = 0
+#pragma unroll 4
+        for (int q = 0; q < H * H / 4 / 256; ++q) {
+            const int e = q * 256 + tid;
+            reinterpret_cast<float4*>(Tc + (int64_t)(e >> 5) * K + H)[e & 31] =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+        float acc[8][8];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) acc[rr][cc] = 0.f;
+        mm128_tile(sP, sQ, r0, c0, c0, H, acc);              // X = A10 T00 (T00[l][c] = 0, l < c)
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            float4* xr = reinterpret_cast<float4*>(sX + (r0 + rr) * H + c0);
+            xr[0] = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+            xr[1] = make_float4(acc[rr][4], acc[rr][5], acc[rr][6], acc[rr][7]);
+        }
+        __syncthreads();                                     // A10 is read: T11 takes its place
+        load_block(sP, Tc + H * K + H);                      // T11
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) acc[rr][cc] = 0.f;
+        mm128_tile(sP, sX, r0, c0, 0, r0 + 8, acc);          // T10 = T11 X (T11[r][l] = 0, l > r)
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+            float4* dst = reinterpret_cast<float4*>(Tc + (int64_t)(H + r0 + rr) * K + c0);
+            dst[0] = make_float4(acc[rr][0], acc[rr][1], acc[rr][2], acc[rr][3]);
+            dst[1] = make_float4(acc[rr][4], acc[rr][5], acc[rr][6], acc[rr][7]);
+        }
     }
 }
 
@@ -863,9 +964,27 @@ cudaError_t launch_fwdsub(const float* A, float* T, int64_t nc, int k, cudaStrea
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int64_t cap = (int64_t)sms * 2;
         const unsigned grid = (unsigned)(nc < cap ? nc : cap);
-        cudaError_t e = prep(k_fwdsub128, smem);
+        cudaError_t e = prep(k_fwdsub128<128>, smem);
         if (e != cudaSuccess) return e;
-        k_fwdsub128<<<grid, 128, smem, st>>>(A, T, nc);
+        k_fwdsub128<128><<<grid, 128, smem, st>>>(A, T, nc);
+        return cudaGetLastError();
+    }
+    if (k == 256) {                            // diagonal 128-blocks, then the off-diagonal one
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const size_t smem1 = (size_t)(128 * 128 + 3 * 64 * 64) * sizeof(float);
+        cudaError_t e = prep(k_fwdsub128<256>, smem1);
+        if (e != cudaSuccess) return e;
+        const int64_t nd = 2 * nc, cap1 = (int64_t)sms * 2;
+        k_fwdsub128<256><<<(unsigned)(nd < cap1 ? nd : cap1), 128, smem1, st>>>(A, T, nd);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        const size_t smem2 = (size_t)3 * 128 * 128 * sizeof(float);
+        e = prep(k_fwdsub256_off, smem2);
+        if (e != cudaSuccess) return e;
+        const int64_t cap2 = sms;
+        k_fwdsub256_off<<<(unsigned)(nc < cap2 ? nc : cap2), 256, smem2, st>>>(A, T, nc);
         return cudaGetLastError();
     }
     const int CB = k < 128 ? k : 128;
