@@ -13,17 +13,19 @@
 //   accumulator in tensor memory (TMEM).
 // * Each "slot" of 8 warps owns one tile at a time.  Its elected thread issues
 //   the tile's TMA loads (K with beta and g on one barrier, V on another, so
-//   the K K^T product starts before V lands), its MMAs and its TMA stores, and
-//   loads the slot's next tile as soon as the stores have read the staging
-//   tiles.  Its 256 threads run the epilogues (TMEM -> registers -> mask /
-//   accumulate / convert -> swizzled shared-memory operand).  Thread (r, h)
-//   owns row r of the tile (its TMEM lane; the lane quarter is warp % 4) and
-//   the column half h, and keeps its part of T0 (then T) in registers.  Two
-//   slots per CTA keep the tensor pipe busy while the other slot runs an
-//   epilogue.
+//   the K K^T product starts before V lands; in the standalone inverse, A one
+//   tile ahead), its MMAs and its TMA stores.  Its 256 threads run the
+//   epilogues (TMEM -> registers -> mask / accumulate / convert -> TMEM or
+//   swizzled shared-memory operand).  Thread (r, h) owns row r of the tile
+//   (its TMEM lane; the lane quarter is warp % 4) and the column half h.  The
+//   series runs in Horner form with the left operand in TMEM; T0 sits in TMEM
+//   at KB = 64 and in registers at KB = 128.  Two slots per CTA keep the
+//   tensor pipe busy while the other slot runs an epilogue.
+// * The residual sum uses Horner with stride 2 (Q_{m+2} = F + Q_m E^2) in the
+//   fused step and doubling in the standalone inverse.
 // * WY is computed transposed, W^T = K^T (T diag(beta))^T, a full-rate M=128
-//   (= d) product; its epilogue transposes through the (now free) K/V tiles in
-//   shared memory and leaves with TMA bulk stores.
+//   (= d) product; its epilogue transposes through the (now free) operand and
+//   V tiles with stmatrix .trans and leaves with TMA bulk stores.
 // * Every wait is bounded (2 s).  On expiry the kernel sets the status word,
 //   stops issuing work, waits (bounded) for its own copies and MMAs and frees
 //   TMEM before returning.

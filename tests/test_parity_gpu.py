@@ -260,3 +260,57 @@ def test_neumann_tensor_cores_k256(N, mask):
         assert np.all(Th[:, dist > N] == 0)
     if N == 1:                                               # T = I + M.A, no products
         assert np.array_equal(Th, ref.astype(np.float32))
+
+
+# --------------------------------------------------------------------------- #
+# degenerate inputs
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("k", [32, 64, 128])
+def test_neumann_full_order_is_exact_inverse(k):
+    """N = k - 1 keeps every power (A^k = 0): the truncated series is the exact
+    inverse, on the tensor-core and the fp32 chains alike."""
+    w = Workload(B=1, H=2, T=2 * k, k=k, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=21), w)
+    exact = O.invert_fwdsub(A32.astype(np.float64))
+    Ad = to_dev(A_tensor(A32, w))
+    for prec, tol in ((gdn.GDN_PREC_F16, TOL_BF16), (gdn.GDN_PREC_F32, TOL_F32)):
+        T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+        gdn.gdn_invert_neumann(Ad, T, k - 1, 0, 0, prec)
+        check_status()
+        assert rel(T, exact) <= tol
+
+
+@pytest.mark.parametrize("k", [32, 64, 128])
+def test_fused_beta_zero_gives_identity(k):
+    """beta = 0: A = 0, T = I and W = U = 0 exactly."""
+    w = Workload(B=1, H=2, T=2 * k, k=k, dtype="bf16")
+    d = dev_inputs(make_inputs(w, seed=22))
+    d["beta"].zero_()
+    W = torch.full_like(d["K"], 7.0)
+    U = torch.full_like(d["V"], 7.0)
+    T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_chunk_wy_fused(d["K"], d["V"], d["beta"], d["g"], 3, 1, 8, 1, W, U, T, k=k)
+    check_status()
+    eye = torch.eye(k, device="cuda").expand_as(T)
+    assert torch.equal(T, eye)
+    assert torch.count_nonzero(W) == 0 and torch.count_nonzero(U) == 0
+
+
+@pytest.mark.parametrize("gate", ["none", "strong"])
+def test_fused_gate_extremes(gate):
+    """No decay (g = 0) and a decay strong enough that most e^{g_i - g_j}
+    underflow: both match the oracle."""
+    k = 64
+    w = Workload(B=1, H=3, T=3 * k, k=k, dtype="bf16")
+    inp = make_inputs(w, seed=23, gate_scale=0.0 if gate == "none" else 40.0)
+    d = dev_inputs(inp)
+    W = torch.empty_like(d["K"])
+    U = torch.empty_like(d["V"])
+    T = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    gdn.gdn_chunk_wy_fused(d["K"], d["V"], d["beta"], d["g"], 3, 1, 8, 1, W, U, T, k=k)
+    check_status()
+    Tr, Wr, Ur = fused_reference(chunked(inp, w), 3, 1, 8, True)
+    assert torch.isfinite(T).all() and torch.isfinite(W.float()).all()
+    assert rel(T, Tr) <= TOL_BF16
+    assert rel(W, Wr) <= TOL_BF16
+    assert rel(U, Ur) <= TOL_BF16
