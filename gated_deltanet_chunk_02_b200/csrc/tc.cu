@@ -402,6 +402,7 @@ struct __align__(8) Ctrl {
     uint64_t fullK[2];   // K tile, beta, g landed
     uint64_t fullV[2];   // V tile landed
     uint64_t mma[2];     // the slot's MMAs completed
+    uint64_t wdone[2];   // the slot's W^T products completed (K no longer read)
     uint32_t tmem;
     int abort;
 };
@@ -447,6 +448,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             mbar_init(&ctrl->fullK[s], 1);
             mbar_init(&ctrl->fullV[s], 1);
             mbar_init(&ctrl->mma[s], 1);
+            mbar_init(&ctrl->wdone[s], 1);
         }
         ctrl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1151,6 +1153,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 constexpr uint32_t id = idesc_f16(1, 1, 0, KB, 128);
                 const uint32_t kb0 = su32(sK), vb0 = su32(sV), xb0 = su32(sX);
                 const uint32_t ub0 = su32(p.gated ? sY : sX);
+                // W^T first, with its own commit: the slot's next K tile can
+                // start loading while the U^T products still run
 #pragma unroll 1
                 for (int c = 0; c < NCH; ++c) {
 #pragma unroll 1
@@ -1160,14 +1164,25 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                                             (kk & 3) * 32;
                         mma_ss(tm + c * KB, sdesc(kb0 + ao, kRows * 128, 1024),
                                sdesc(xb0 + bo, 16, 1024), id, kk > 0);
+                    }
+                }
+                mma_commit(&ctrl->wdone[s]);
+#pragma unroll 1
+                for (int c = 0; c < NCH; ++c) {
+#pragma unroll 1
+                    for (int kk = 0; kk < KB / 16; ++kk) {
+                        const uint32_t ao = (c * KB + kk * 16) * 128;
+                        const uint32_t bo = (c * KB) * 128 + (kk >> 2) * (kRows * 128) +
+                                            (kk & 3) * 32;
                         mma_ss(tm + 128 + c * KB, sdesc(vb0 + ao, kRows * 128, 1024),
                                sdesc(ub0 + bo, 16, 1024), id, kk > 0);
                     }
                 }
                 mma_commit(&ctrl->mma[s]);
+                if (mbar_wait(&ctrl->wdone[s], use_par)) issue_k(n + NS);   // K is free
+                else fail_wait();
             }
             if (!wait_mma()) { ok = false; break; }
-            if (leader) issue_k(n + NS);                 // K, beta, g are no longer read
             // Lane d of the W^T / U^T accumulators is head-dim column d and
             // accumulator column x is tile row x.  Warp (quarter q, half h)
             // moves d in [32q, 32q + 32) x rows [64h, 64h + 64): 16x256b TMEM
@@ -1178,28 +1193,33 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             {
                 const uint32_t wst = su32(sWst), vst = su32(sV);
                 const int mq = lane >> 3, mr = lane & 7;   // stmatrix: matrix, row of this address
+                auto pk = [](uint32_t lo, uint32_t hi) {
+                    return pack_b2(__uint_as_float(lo), __uint_as_float(hi));
+                };
 #pragma unroll 1
-                for (int it = 0; it < 8; ++it) {
-                    const int hb = it & 1;
-                    const int x0 = h * 64 + (it >> 1) * 16;
-                    const int db = (warp & 3) * 32 + 16 * hb;
-                    const uint32_t ta = tl + ((uint32_t)(16 * hb) << 16) + x0;
-                    uint32_t wa[4], wb[4], ua[4], ub[4];
-                    tmem_ld_16x256b(ta, wa);
-                    tmem_ld_16x256b(ta + 8, wb);
-                    tmem_ld_16x256b(ta + 128, ua);
-                    tmem_ld_16x256b(ta + 136, ub);
+                for (int it2 = 0; it2 < 4; ++it2) {       // two 16-lane halves per TMEM wait
+                    const int x0 = h * 64 + it2 * 16;
+                    uint32_t wa[2][4], wb[2][4], ua[2][4], ub[2][4];
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const uint32_t ta = tl + ((uint32_t)(16 * hb) << 16) + x0;
+                        tmem_ld_16x256b(ta, wa[hb]);
+                        tmem_ld_16x256b(ta + 8, wb[hb]);
+                        tmem_ld_16x256b(ta + 128, ua[hb]);
+                        tmem_ld_16x256b(ta + 136, ub[hb]);
+                    }
                     tmem_wait_ld();
-                    const int x = x0 + 8 * (mq >> 1) + mr, d = db + 8 * (mq & 1);
-                    const uint32_t off = (uint32_t)((d >> 6) * (kRows * 128) + x * 128 +
-                                                    ((((d & 63) >> 3) ^ (x & 7)) << 4));
-                    auto pk = [](uint32_t lo, uint32_t hi) {
-                        return pack_b2(__uint_as_float(lo), __uint_as_float(hi));
-                    };
-                    stmatrix_x4_trans(wst + off, pk(wa[0], wa[1]), pk(wa[2], wa[3]), pk(wb[0], wb[1]),
-                                      pk(wb[2], wb[3]));
-                    stmatrix_x4_trans(vst + off, pk(ua[0], ua[1]), pk(ua[2], ua[3]), pk(ub[0], ub[1]),
-                                      pk(ub[2], ub[3]));
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb) {
+                        const int db = (warp & 3) * 32 + 16 * hb;
+                        const int x = x0 + 8 * (mq >> 1) + mr, d = db + 8 * (mq & 1);
+                        const uint32_t off = (uint32_t)((d >> 6) * (kRows * 128) + x * 128 +
+                                                        ((((d & 63) >> 3) ^ (x & 7)) << 4));
+                        stmatrix_x4_trans(wst + off, pk(wa[hb][0], wa[hb][1]), pk(wa[hb][2], wa[hb][3]),
+                                          pk(wb[hb][0], wb[hb][1]), pk(wb[hb][2], wb[hb][3]));
+                        stmatrix_x4_trans(vst + off, pk(ua[hb][0], ua[hb][1]), pk(ua[hb][2], ua[hb][3]),
+                                          pk(ub[hb][0], ub[hb][1]), pk(ub[hb][2], ub[hb][3]));
+                    }
                 }
             }
             fence_async_smem();
