@@ -181,6 +181,14 @@ int gdn_forward_static(const void* Q, const void* K, const void* V,
                        float* S_final, gdn_shape s, gdn_dtype dtype,
                        void* stream);
 
+/*
+ * Streams and graphs: every entry point enqueues its kernels on `stream`
+ * (NULL = the legacy default stream) and returns without synchronising; none
+ * allocates device memory (gdn_forward takes a caller workspace).  The calls
+ * can therefore be captured into CUDA graphs and replayed; make one eager
+ * call first (it sets kernel attributes and looks up the status word), and
+ * capture gdn_forward_static only after its first eager call on the device.
+ */
 /* Synchronises `stream`, returns the device status word of the current
  * device (GDN_OK, GDN_ERR_TIMEOUT, or GDN_ERR_CUDA when a kernel found its
  * shared memory misaligned) and clears it. */
