@@ -117,12 +117,9 @@ int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask, i
     cudaStream_t st = (cudaStream_t)stream;
     if (prec == GDN_PREC_F16) {
         if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
-        if (s.k == 256) {
-            if (S != 0)
-                return fail(GDN_ERR_UNSUPPORTED, "tensor-core Neumann chain at k=256 serves S=0");
-            return launched(gdn::launch_neumann256_tc(A, T, nc, N, mask, st),
+        if (s.k == 256)
+            return launched(gdn::launch_neumann256_tc(A, T, nc, N, mask, S, st),
                             "neumann k=256 (tcgen05)");
-        }
         return launched(gdn::launch_neumann_tc(A, T, nc, s.k, N, mask, S, st), "neumann (tcgen05)");
     }
     if (s.k > 128) return fail(GDN_ERR_UNSUPPORTED, "float32 Neumann chain supports k <= 128");

@@ -1628,6 +1628,7 @@ struct Params256 {
     int64_t nc;
     int N;
     int mask;
+    int S;
     const float* A;
     float* T;
     int* status;
@@ -1783,9 +1784,8 @@ k_neumann256_tc(const Params256 p) {
                     const int j = c0 + jj;
                     v[jj] = (j == row ? 1.f : 0.f) + (j >= jmin ? v[jj] : 0.f);
                 }
-                if (m < N) {
-                    st_op32<false>(sX(gq), rr, pc, v);
-                } else {
+                if (m < N || p.S > 0) st_op32<false>(sX(gq), rr, pc, v);   // X_m; T0 for the residual
+                if (m == N) {
                     float4* dst = reinterpret_cast<float4*>(Tc + (int64_t)row * KC + c0);
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
@@ -1796,6 +1796,108 @@ k_neumann256_tc(const Params256 p) {
             if (*(volatile int*)abort_flag) { ok = false; break; }
         }
         if (!ok) break;
+        // ---- residual (S > 0): E = I - T0 + A T0, Q_{m+1} = (I + Q_m) E,
+        // T = T0 + T0 Q_S.  T0 (fp32) waits in the output T and is re-read from
+        // there (each thread its own row pieces); the six operand blocks are
+        // reused: A's blocks take E, then Q_S; the X blocks hold T0, then
+        // I + Q_m, then T0 again for the last product.
+        if (p.S > 0) {
+            auto wait_products = [&]() {
+                if (mbar_wait(mbar, phase)) {
+                    phase ^= 1;
+                } else {
+                    timed_out = true;
+                    atomicExch(abort_flag, 1);
+                    raise_status(p.status, kStatusTimeout);
+                }
+                tc_fence_after();
+            };
+            auto t0_row = [&](int c0, float (&t)[32]) {
+                const float4* src = reinterpret_cast<const float4*>(Tc + (int64_t)row * KC + c0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 x = src[q];
+                    t[4 * q] = x.x; t[4 * q + 1] = x.y; t[4 * q + 2] = x.z; t[4 * q + 3] = x.w;
+                }
+            };
+            // A T0: left A blocks, right T0 blocks
+            if (leader) {
+                constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
+                auto blk = [&](uint32_t dcol, const uint8_t* xa, const uint8_t* ab, bool acc) {
+                    const uint32_t xb = su32(xa), bb = su32(ab);
+#pragma unroll 1
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tm + dcol, sdesc(xb + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024),
+                               sdesc(bb + kk * 2048, kRows * 128, 1024), id, (acc || kk > 0) ? 1u : 0u);
+                };
+                blk(0, sA(0), sX(0), false);
+                blk(128, sA(1), sX(0), false);
+                blk(128, sA(2), sX(1), true);
+                blk(256, sA(2), sX(2), false);
+                mma_commit(mbar);
+            }
+            wait_products();
+#pragma unroll 1
+            for (int pc = 0; pc < 4; ++pc) {
+                const int c0 = col0 + 32 * pc;
+                if (c0 > 32 * rg + 31) continue;        // above the diagonal for the whole warp
+                float v[32], t[32];
+                tmem_ld32(tD + 32 * pc, v);
+                t0_row(c0, t);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) v[jj] += (c0 + jj == row ? 1.f : 0.f) - t[jj];   // E
+                st_op32<false>(sA(gq), rr, pc, v);
+                if (p.S > 1) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) v[jj] += (c0 + jj == row ? 1.f : 0.f);
+                    st_op32<false>(sX(gq), rr, pc, v);                          // I + Q_1
+                }
+            }
+            publish();
+            if (*(volatile int*)abort_flag) { ok = false; break; }
+            for (int m = 1; m < p.S; ++m) {                                     // (I + Q_m) E
+                if (leader) issue();
+                wait_products();
+                const bool last = (m == p.S - 1);
+#pragma unroll 1
+                for (int pc = 0; pc < 4; ++pc) {
+                    const int c0 = col0 + 32 * pc;
+                    if (c0 > 32 * rg + 31) continue;
+                    float v[32];
+                    tmem_ld32(tD + 32 * pc, v);
+                    if (last) {
+                        st_op32<false>(sA(gq), rr, pc, v);                      // Q_S
+                        float t[32];
+                        t0_row(c0, t);
+                        st_op32<false>(sX(gq), rr, pc, t);                      // T0
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) v[jj] += (c0 + jj == row ? 1.f : 0.f);
+                        st_op32<false>(sX(gq), rr, pc, v);                      // I + Q_{m+1}
+                    }
+                }
+                publish();
+                if (*(volatile int*)abort_flag) { ok = false; break; }
+            }
+            if (!ok) break;
+            if (leader) issue();                                                // T0 Q_S
+            wait_products();
+#pragma unroll 1
+            for (int pc = 0; pc < 4; ++pc) {
+                const int c0 = col0 + 32 * pc;
+                if (c0 > 32 * rg + 31) continue;
+                float v[32], t[32];
+                tmem_ld32(tD + 32 * pc, v);
+                t0_row(c0, t);
+                float4* dst = reinterpret_cast<float4*>(Tc + (int64_t)row * KC + c0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    dst[q] = make_float4(t[4 * q] + v[4 * q], t[4 * q + 1] + v[4 * q + 1],
+                                         t[4 * q + 2] + v[4 * q + 2], t[4 * q + 3] + v[4 * q + 3]);
+            }
+            publish();
+            if (*(volatile int*)abort_flag) { ok = false; break; }
+        }
     }
     if (timed_out) mbar_wait(mbar, phase);          // bounded: let the products finish
     tc_fence_before();
@@ -2008,12 +2110,13 @@ cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8
     return cudaGetLastError();
 }
 
-cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, int mask,
+cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, int mask, int S,
                                 cudaStream_t st) {
     tcg::Params256 p;
     p.nc = nc;
     p.N = N;
     p.mask = mask;
+    p.S = S;
     p.A = A;
     p.T = T;
     p.status = status_ptr();

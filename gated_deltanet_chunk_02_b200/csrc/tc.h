@@ -14,8 +14,8 @@ cudaError_t launch_build_A_tc(const void* K, const float* beta, const float* g, 
                               int64_t nc, int k, cudaStream_t st);
 cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int S,
                               cudaStream_t st);
-// k = 256, S = 0: banded or full truncated series, one chunk per CTA
-cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, int mask,
+// k = 256: truncated series (Horner, by 128 x 128 blocks) and residual, one chunk per CTA
+cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, int mask, int S,
                                 cudaStream_t st);
 cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const float* beta,
                          const float* g, void* W, void* U, int64_t nc, int k, cudaStream_t st);

@@ -84,8 +84,9 @@ int gdn_build_A(const void* K, const float* beta, const float* g, float* A,
  * the band mask M_ij = [i - j <= N] applied to every power when mask != 0;
  * then, if S > 0, E = I - (I - A) T0 and T = T0 sum_{s=0}^{S} E^s (S >= 0).
  * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.  1 <= N <= k-1, 0 <= S <= 64.
- * GDN_PREC_F16 serves k <= 128; GDN_PREC_F32 serves k <= 128; k = 256
- * returns GDN_ERR_UNSUPPORTED in this build.
+ * GDN_PREC_F16 (tensor cores: fp16 operands, fp32 accumulation) serves
+ * every k; GDN_PREC_F32 (fp32 on CUDA cores) serves k <= 128 and returns
+ * GDN_ERR_UNSUPPORTED at k = 256.
  */
 int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask,
                        int S, gdn_prec prec, void* stream);

@@ -236,30 +236,32 @@ def test_neumann_tensor_cores(k, N, mask, S):
             assert np.all(Th[:, dist > N] == 0)
 
 
-@pytest.mark.parametrize("N,mask", [(1, 1), (2, 1), (3, 1), (4, 1), (3, 0), (8, 0), (40, 1),
-                                    (255, 1)])
-def test_neumann_tensor_cores_k256(N, mask):
-    """The k=256 tcgen05 chain (2 x 2 blocks of 128, Horner sum, S=0) on 6
-    chunks; N=40 puts the band across the block boundary of D10, N=255 keeps
-    every power."""
+@pytest.mark.parametrize("N,mask,S", [(1, 1, 0), (2, 1, 0), (3, 1, 0), (4, 1, 0), (3, 0, 0),
+                                      (8, 0, 0), (40, 1, 0), (255, 1, 0), (1, 1, 1), (3, 1, 1),
+                                      (3, 1, 2), (3, 1, 8), (2, 0, 3), (40, 1, 8)])
+def test_neumann_tensor_cores_k256(N, mask, S):
+    """The k=256 tcgen05 chain (2 x 2 blocks of 128, Horner sums) on 6 chunks;
+    N=40 puts the band across the block boundary of D10, N=255 keeps every
+    power, S > 0 runs the residual through the reused operand blocks."""
     k = 256
     w = Workload(B=1, H=2, T=3 * k, k=k, dtype="bf16")
     A32 = oracle_A32(make_inputs(w, seed=9), w)
     T = torch.full((w.B, w.H, w.T // k, k, k), float("nan"), device="cuda")
-    gdn.gdn_invert_neumann(to_dev(A_tensor(A32, w)), T, N, mask, 0, gdn.GDN_PREC_F16)
+    gdn.gdn_invert_neumann(to_dev(A_tensor(A32, w)), T, N, mask, S, gdn.GDN_PREC_F16)
     check_status()
-    ref = O.invert_neumann(A32.astype(np.float64), N, bool(mask), 0)
+    ref = O.invert_neumann(A32.astype(np.float64), N, bool(mask), S)
     assert torch.isfinite(T).all()                           # every entry written
     assert rel(T, ref) <= TOL_BF16
     assert per_chunk_max_rel(T, ref) <= TOL_BF16
     Th = T.cpu().numpy().reshape(ref.shape)
     assert np.all(np.triu(Th, 1) == 0)
-    assert np.all(np.diagonal(Th, axis1=1, axis2=2) == 1)
-    if mask:
-        dist = np.arange(k)[:, None] - np.arange(k)[None, :]
-        assert np.all(Th[:, dist > N] == 0)
-    if N == 1:                                               # T = I + M.A, no products
-        assert np.array_equal(Th, ref.astype(np.float32))
+    if S == 0:
+        assert np.all(np.diagonal(Th, axis1=1, axis2=2) == 1)
+        if mask:
+            dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+            assert np.all(Th[:, dist > N] == 0)
+        if N == 1:                                           # T = I + M.A, no products
+            assert np.array_equal(Th, ref.astype(np.float32))
 
 
 # --------------------------------------------------------------------------- #
