@@ -102,6 +102,8 @@ int gdn_build_A(const void* K, const float* beta, const float* g, float* A, gdn_
     cudaStream_t st = (cudaStream_t)stream;
     if (dtype == GDN_BF16 && gdn::tc_available() && s.k <= 128)
         return launched(gdn::launch_build_A_tc(K, beta, g, A, nc, s.k, st), "build_A (tcgen05)");
+    if (dtype == GDN_BF16 && gdn::tc_available() && s.k == 256)
+        return launched(gdn::launch_build_A256_tc(K, beta, g, A, nc, st), "build_A k=256 (tcgen05)");
     return launched(gdn::launch_build_A_simt(K, beta, g, A, nc, s.k, dtype == GDN_BF16, st),
                     "build_A");
 }

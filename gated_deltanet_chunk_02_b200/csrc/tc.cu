@@ -1909,6 +1909,147 @@ k_neumann256_tc(const Params256 p) {
 }
 
 // ------------------------------------------------------------------------- //
+// A for k = 256 chunks: G = K K^T as three 128 x 128 blocks (G00, G10, G11;
+// G01 is never needed), A_ij = -beta_i G_ij e^{g_i - g_j} for j < i.  One chunk
+// per CTA at a time; the chunk's K arrives by TMA as two 128-row tiles (bf16,
+// 128-byte swizzle) and the next chunk's K is loaded while this one's epilogue
+// writes A.  Warp group q (warps 4q .. 4q + 3) owns block q of {G00, G10, G11}.
+// ------------------------------------------------------------------------- //
+struct ParamsA256 {
+    int64_t nc;
+    const float* beta;
+    const float* g;
+    float* A;
+    int* status;
+};
+
+constexpr int kA256Smem = 2 * 2 * kRows * kD * 2 + 64;     // two stages of 2 K tiles, control
+
+__global__ void __launch_bounds__(384, 1)
+k_build_A256_tc(const __grid_constant__ CUtensorMap mK, const ParamsA256 p) {
+    constexpr int KC = 256;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((su32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    constexpr int kTile = kRows * kD * 2;                   // 32 KB: 128 rows of K
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + 4 * kTile);     // [2] stage landed
+    uint64_t* mbar = full + 2;                                          // products done
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(mbar + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(mbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tmem_alloc(tslot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tslot;
+    const int gq = warp >> 2;
+    const int rr = ((warp & 3) << 5) | lane;
+    const int row = (gq ? 128 : 0) + rr;
+    const int col0 = gq == 2 ? 128 : 0;
+    const uint32_t tD = tm + ((uint32_t)((warp & 3) * 32) << 16) + 128 * gq;
+    const bool leader = threadIdx.x == 0;
+    bool ok = true, timed_out = false;
+    uint32_t phase = 0;
+    int issued = 0;
+    auto issue = [&](int64_t c, int st) {
+        if (c >= p.nc) return;
+        ++issued;
+        uint8_t* base = smem + st * 2 * kTile;
+        mbar_expect_tx(&full[st], 2 * kTile);
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+            const int y = (int)(c * KC + 128 * b);
+            tma_load_2d(base + b * kTile, &mK, 0, y, &full[st]);
+            tma_load_2d(base + b * kTile + kRows * 128, &mK, 64, y, &full[st]);
+        }
+    };
+    if (leader) issue(blockIdx.x, 0);
+    int it = 0;
+    for (int64_t c = blockIdx.x; c < p.nc; c += gridDim.x, ++it) {
+        const int st = it & 1;
+        uint8_t* k0 = smem + st * 2 * kTile;
+        uint8_t* k1 = k0 + kTile;
+        if (!mbar_wait(&full[st], (uint32_t)((it >> 1) & 1))) {
+            raise_status(p.status, kStatusTimeout);
+            ok = false;
+        }
+        // the other stage is free (its products completed last iteration)
+        if (leader) issue(c + gridDim.x, st ^ 1);
+        tc_fence_after();
+        if (leader && ok) {
+            constexpr uint32_t id = idesc_f16(1, 0, 0, 128, 128);
+            auto blk = [&](uint32_t dcol, const uint8_t* xa, const uint8_t* xb) {
+                const uint32_t a0 = su32(xa), b0 = su32(xb);
+#pragma unroll 1
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t ko = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+                    mma_ss(tm + dcol, sdesc(a0 + ko, 16, 1024), sdesc(b0 + ko, 16, 1024), id, kk > 0);
+                }
+            };
+            blk(0, k0, k0);                                 // G00
+            blk(128, k1, k0);                               // G10
+            blk(256, k1, k1);                               // G11
+            mma_commit(mbar);
+        }
+        __syncwarp();
+        // (all threads) products done
+        if (ok && !mbar_wait(mbar, phase)) {
+            timed_out = true;
+            raise_status(p.status, kStatusTimeout);
+            ok = false;
+        }
+        if (ok) phase ^= 1;
+        tc_fence_after();
+        if (__syncthreads_or(!ok)) break;
+        const int64_t grow = c * KC + row;
+        const float bi = p.beta[grow], gi = p.g[grow];
+        const float* gcol = p.g + c * KC + col0;
+        float* Ar = p.A + (c * KC + row) * (int64_t)KC;
+#pragma unroll 1
+        for (int pc = 0; pc < 4; ++pc) {
+            const int c0 = col0 + 32 * pc;
+            float v[32];
+            if (c0 > (row | 31)) {                          // above the diagonal for the warp
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
+            } else {
+                tmem_ld32(tD + 32 * pc, v);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = c0 + jj;
+                    v[jj] = j < row ? -bi * v[jj] * exp_e(gi - gcol[32 * pc + jj]) : 0.f;
+                }
+            }
+            float4* dst = reinterpret_cast<float4*>(Ar + c0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        if (gq == 0) {                                      // the upper-right block is zero
+            float4* dst = reinterpret_cast<float4*>(Ar + 128);
+#pragma unroll 4
+            for (int q = 0; q < 32; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        tc_fence_before();
+        __syncthreads();                                    // accumulators free
+    }
+    if (timed_out) mbar_wait(mbar, phase);
+    if (leader && issued > 0) mbar_wait(&full[(issued - 1) & 1], (uint32_t)(((issued - 1) >> 1) & 1));
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+// ------------------------------------------------------------------------- //
 // host side
 // ------------------------------------------------------------------------- //
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -2054,6 +2195,26 @@ cudaError_t launch_build_A_tc(const void* K, const float* beta, const float* g, 
     io.beta = beta;
     io.g = g;
     return tcg::dispatch<tcg::kBuildA, 2>(k, io, p, st);
+}
+
+cudaError_t launch_build_A256_tc(const void* K, const float* beta, const float* g, float* A,
+                                 int64_t nc, cudaStream_t st) {
+    CUtensorMap mK;
+    memset(&mK, 0, sizeof mK);
+    if (!tcg::map_kd(&mK, K, nc * 256)) return cudaErrorInvalidValue;
+    tcg::ParamsA256 p;
+    p.nc = nc;
+    p.beta = beta;
+    p.g = g;
+    p.A = A;
+    p.status = status_ptr();
+    cudaError_t e = cudaFuncSetAttribute(tcg::k_build_A256_tc,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, tcg::kA256Smem);
+    if (e != cudaSuccess) return e;
+    const int sms = tcg::num_sms();
+    const int grid = nc < sms ? (int)nc : sms;
+    tcg::k_build_A256_tc<<<grid, 384, tcg::kA256Smem, st>>>(mK, p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int S,

@@ -12,6 +12,9 @@ bool tc_i8_available();  // true when the INT8 tensor-core kernel is built
 
 cudaError_t launch_build_A_tc(const void* K, const float* beta, const float* g, float* A,
                               int64_t nc, int k, cudaStream_t st);
+// k = 256, bf16 K: three 128 x 128 blocks of K K^T per chunk
+cudaError_t launch_build_A256_tc(const void* K, const float* beta, const float* g, float* A,
+                                 int64_t nc, cudaStream_t st);
 cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int S,
                               cudaStream_t st);
 // k = 256: truncated series (Horner, by 128 x 128 blocks) and residual, one chunk per CTA
