@@ -22,7 +22,8 @@
 //   at KB = 64 and in registers at KB = 128.  Two slots per CTA keep the
 //   tensor pipe busy while the other slot runs an epilogue.
 // * The residual sum uses Horner with stride 2 (Q_{m+2} = F + Q_m E^2) in the
-//   fused step and doubling in the standalone inverse.
+//   fused step and doubling in the standalone inverse (at KB = 64 one product
+//   per block and round: V_a stacked over E^a times E^a).
 // * WY is computed transposed, W^T = K^T (T diag(beta))^T, a full-rate M=128
 //   (= d) product; its epilogue transposes through the (now free) operand and
 //   V tiles with stmatrix .trans and leaves with TMA bulk stores.
@@ -866,27 +867,126 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             }
             if (!ok) break;
             // ---- parallel residual correction: T = T0 G, G = sum_{s<=S} E^s ----
-            // Two schedules.  Horner keeps (I + Q_m) in TMEM as the left operand
-            // of Q_{m+1} = (I + Q_m) E (S - 1 products, one per round) and T0 in
-            // fp32; it is the faster one while S is small.  Doubling (below)
-            // needs only ~log2(S) rounds of two shared-memory products, and
-            // serves the standalone inverse and S >= 15.
-            // Doubling applies when S + 1 is 2^m or 2^m + 1: with a = 2^r,
+            // Three schedules.  Horner keeps (I + Q_m) in TMEM as the left
+            // operand of Q_{m+1} = (I + Q_m) E (S - 1 products, one per round,
+            // in 64-row blocks that do not wait for each other) and T0 in fp32;
+            // it serves the fused step and every S the doubling forms do not.
+            // The standalone inverse doubles when S + 1 is 2^m or 2^m + 1:
+            // stacked at KB = 64 (below), with two products per round at KB =
+            // 128.  In the fused step the stacked form measured slower at S <= 8
+            // (its lockstep rounds and wider epilogues cost more than the two
+            // rounds it saves), so the fused step keeps Horner.
+            // Two-product doubling (KB = 128): with a = 2^r,
             // G(2a) - I = (G(a) - I) + E^a + (G(a) - I) E^a and E^2a = E^a E^a,
             // two products per round sharing the right operand E^a.  T0 - I
             // (fp16) goes to the Aop buffer, E = I - T0 + A + A (T0 - I) to X,
-            // G - I to Y, and T = T0 + (G - I) + (T0 - I)(G - I).  Both
-            // accumulators of a round fill the slot's TMEM, so T0 survives the
-            // rounds as its fp16 copy at KB = 64.
+            // G - I to Y, and T = T0 + (G - I) + (T0 - I)(G - I); T0 stays in
+            // registers.
             if (p.S > 0) {
                 const int S = p.S;
                 int K2 = 0;
                 while ((2 << K2) <= S + 1) ++K2;
                 const bool p2p1 = (1 << K2) + 1 == S + 1;
                 const bool dbl = (1 << K2) == S + 1 || p2p1;
-                // doubling is built into the standalone inverse only: in the
-                // fused kernel its registers would cost every other phase
-                if (!(MODE == kNeumann && dbl)) {
+                // Stacked doubling (64-row blocks, S + 1 = 2^J or 2^J + 1).
+                // With U_a = sum_{s<a} E^s and V_a = T0 U_a: V_2a = V_a + V_a E^a
+                // and E^2a = E^a E^a share the right operand E^a, so ONE M = 128
+                // product per block gives both when its left operand stacks V_a
+                // over E^a.  Block 0 stacks [V_0; E_0] (the X buffer), block 1
+                // [E_1; V_1] (the Aop buffer): each block's V rows land on its
+                // own TMEM lanes, where V_a stays in fp32 (the T0 columns), and
+                // its E rows on the other block's lanes, whose threads write
+                // them back.  Every thread therefore writes row r of X and of
+                // Aop.  T0 (fp16) waits in Y for the last product T0 E^(2^J)
+                // when S = 2^J.  S = 8 takes 5 dependent rounds (Horner: 7).
+                bool stacked = false;
+                if constexpr (KB == 64 && MODE == kNeumann) stacked = dbl;
+                if (stacked) {
+                    // this row's V_a; the other block's E^a row r; the other block's columns
+                    auto sVr = [&]() { return blk == 0 ? sX : sAop; };
+                    auto sEr = [&]() { return blk == 0 ? sAop : sX; };
+                    auto tE = [&]() { return tl + (uint32_t)((1 - blk) * 64); };
+                    // block 0's product into columns [0, 64), block 1's into [64, 128)
+                    auto mma_blocks = [&](const uint8_t* a0, const uint8_t* b0, const uint8_t* a1,
+                                          const uint8_t* b1) {
+                        if (leader) {
+                            constexpr uint32_t id = idesc_f16(0, 0, 1, 64, 128);
+                            const uint32_t x0 = su32(a0), y0 = su32(b0);
+                            const uint32_t x1 = su32(a1), y1 = su32(b1);
+#pragma unroll 1
+                            for (int kk = 0; kk < 4; ++kk) {
+                                mma_ss(tm, sdesc(x0 + kk * 32, 16, 1024),
+                                       sdesc(y0 + kk * 2048, 64 * 128, 1024), id, kk > 0);
+                                mma_ss(tm + 64, sdesc(x1 + kk * 32, 16, 1024),
+                                       sdesc(y1 + kk * 2048, 64 * 128, 1024), id, kk > 0);
+                            }
+                            mma_commit(&ctrl->mma[s]);
+                        }
+                    };
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        float t[32];
+                        t0_get(pp, t, T0);
+                        st_op32<false>(sY, r, pc0 + pp, t);                // T0
+                    }
+                    publish(true);
+                    mma_blocks(sX, sY, sX, sY + 64 * 128);                  // A T0
+                    if (!wait_mma()) { ok = false; break; }
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
+                        float v[32], t[32];
+                        tmem_ld2(tD + pc * 32, v, tT + pc * 32, t);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int j = pc * 32 + jj;
+                            v[jj] = in_chunk(j) ? eye(j) - t[jj] + v[jj] : 0.f;   // E
+                        }
+                        st_op32<false>(sVr(), r, pc, t);                   // V_1 = T0
+                        st_op32<false>(sVr(), r ^ 64, pc, v);              // E of this block
+                    }
+                    for (int rd = 1; rd <= K2; ++rd) {
+                        const bool last = rd == K2;
+                        publish(true);
+                        mma_blocks(sX, sX + 64 * 128, sAop, sAop);          // [V; E] E, [E; V] E
+                        if (!wait_mma()) { ok = false; break; }
+#pragma unroll
+                        for (int pp = 0; pp < PPT; ++pp) {
+                            const int pc = pc0 + pp;
+                            if (!last || p2p1) {
+                                float e[32];
+                                tmem_ld32(tE() + pc * 32, e);
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj)
+                                    if (!in_chunk(pc * 32 + jj)) e[jj] = 0.f;
+                                st_op32<false>(sEr(), r, pc, e);           // E^2a
+                            }
+                            float d[32], v[32];
+                            tmem_ld2(tD + pc * 32, d, tT + pc * 32, v);
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj)
+                                v[jj] = in_chunk(pc * 32 + jj) ? v[jj] + d[jj] : 0.f;   // V_2a
+                            t0_put(pp, v, T0);
+                            if (!last) st_op32<false>(sVr(), r, pc, v);
+                        }
+                    }
+                    if (!ok) break;
+                    if (p2p1) {
+                        publish(true);
+                        mma_blocks(sY, sX + 64 * 128, sY, sAop);            // T0 E^(2^J)
+                        if (!wait_mma()) { ok = false; break; }
+#pragma unroll
+                        for (int pp = 0; pp < PPT; ++pp) {
+                            const int pc = pc0 + pp;
+                            float d[32], v[32];
+                            tmem_ld2(tD + pc * 32, d, tT + pc * 32, v);
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj)
+                                if (in_chunk(pc * 32 + jj)) v[jj] += d[jj];      // T
+                            t0_put(pp, v, T0);
+                        }
+                    }
+                } else if (!(MODE == kNeumann && dbl)) {
                     // Horner with stride 2: Q_1 = E, E^2 = E E, F = E + E^2,
                     // Q_{m+2} = F + Q_m E^2, and Q_{m+1} = E + Q_m E when one
                     // step is left; Q_m (no identity) is the left operand in
@@ -1017,7 +1117,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];          // T = T0 + T0 Q
                         t0_put(pp, t, T0);
                     }
-                } else if constexpr (MODE == kNeumann) {
+                } else if constexpr (MODE == kNeumann && KB != 64) {
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
@@ -1108,18 +1208,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         const int pc = pc0 + pp;
                         float v[32], t[32];
                         tmem_ld32(tD + pc * 32, v);
-                        if (kT0Tmem) {                                      // T0 from its fp16 copy
-#pragma unroll
-                            for (int g = 0; g < 4; ++g) {
-                                float h8[8];
-                                ld_h8(sAop, r, 4 * pc + g, h8);
-#pragma unroll
-                                for (int c = 0; c < 8; ++c)
-                                    t[8 * g + c] = eye(pc * 32 + 8 * g + c) + h8[c];
-                            }
-                        } else {
-                            t0_get(pp, t, T0);
-                        }
+                        t0_get(pp, t, T0);
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
                             float g8[8];
