@@ -8,7 +8,9 @@ Sources.  The method is the one of "When Good Enough Is Optimal:
 Multiplication-Only Matrix Inversion Approximation for Quantized Gated
 DeltaNet" (arXiv 2606.06034), read through its gist.science technical summary
 (sections "Énoncé du Problème", "Méthodologie" §1-§3, "Adaptation à la
-Quantification", "Études d'Ablation") and its deepcamp.cc abstract page.  The
+Quantification", "Études d'Ablation") and its deepcamp.cc abstract page; the
+decode step follows the technical summary of "A Persistent-State Dataflow
+Accelerator for Memory-Bound Linear Attention Decode on FPGA".  The
 pages do not print A's entries nor the Gated DeltaNet recurrence; those come
 from the textbook gated delta rule
 
@@ -28,12 +30,14 @@ against invariants, closed forms and exact rational brute force; none is
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 __all__ = [
     "to_chunks", "from_chunks", "band_mask", "build_A", "invert_fwdsub",
     "neumann_powers_sum", "invert_neumann", "residual_matrix", "wy",
-    "int8_neumann", "chunk_forward", "token_recurrence", "rel_fro", "snr_db",
+    "int8_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
 ]
 
 
@@ -335,4 +339,44 @@ def token_recurrence(Q, K, V, beta, loggate, S0=None):
         H = eye - bt[:, None, None] * kt[:, :, None] * kt[:, None, :]
         S = at[:, None, None] * (S @ H) + bt[:, None, None] * vt[:, :, None] * kt[:, None, :]
         O[:, t] = np.einsum("bij,bj->bi", S, qt)
+    return O, S
+
+
+# --------------------------------------------------------------------------- #
+# decode: the recurrence advanced token by token from a carried state
+# --------------------------------------------------------------------------- #
+def decode(Q, K, V, beta, loggate, S0):
+    """Decode steps of the gated delta rule with grouped query/key heads.
+
+    "A Persistent-State Dataflow Accelerator for Memory-Bound Linear Attention
+    Decode on FPGA" (its technical summary, §1 and §2): per generated token
+    the whole d_v x d_k state of every value head is updated once, and pairs
+    of value heads share one query and one key vector (grouped value heads).
+    This is the plain definition, one token at a time:
+
+      S <- a_t S (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S q_t,
+      a_t = exp(loggate_t),
+
+    where value head h reads query/key head h // (Hv / Hk).  The summary's
+    two-pass rewrite of the step is the kernel's business, not the oracle's.
+
+    ``Q, K: [B, Hk, n, d_k]``, ``V: [B, Hv, n, d_v]``, ``beta, loggate:
+    [B, Hv, n]``, ``S0: [B, Hv, d_v, d_k]``.  Returns ``(O [B, Hv, n, d_v],
+    S [B, Hv, d_v, d_k])`` in float64.
+    """
+    Q, K, V, beta, lg, S = (np.array(x, np.float64) for x in (Q, K, V, beta, loggate, S0))
+    B, Hk, n, dk = K.shape
+    Hv = V.shape[1]
+    G = Hv // Hk
+    O = np.zeros(V.shape)
+    eye = np.eye(dk)
+    for b in range(B):
+        for h in range(Hv):
+            Sh = S[b, h]
+            for t in range(n):
+                k, q, v = K[b, h // G, t], Q[b, h // G, t], V[b, h, t]
+                bt, at = beta[b, h, t], math.exp(lg[b, h, t])
+                Sh = at * Sh @ (eye - bt * np.outer(k, k)) + bt * np.outer(v, k)
+                O[b, h, t] = Sh @ q
+            S[b, h] = Sh
     return O, S

@@ -320,6 +320,94 @@ def test_I8_chunk_form_equals_token_recurrence(T_len, d):
 
 
 # --------------------------------------------------------------------------- #
+# decode steps (grouped query/key heads)
+# --------------------------------------------------------------------------- #
+def test_decode_two_dim_closed_form():
+    """One step by hand: S = I, k = e_1, v = (2, 3), b = 1/2, a = e^-1, q = (1, 1):
+    S' = a (I - k k^T / 2) + v k^T / 2 = [[a/2 + 1, 0], [3/2, a]]."""
+    a = math.exp(-1.0)
+    Q = np.array([[[[1.0, 1.0]]]])
+    K = np.array([[[[1.0, 0.0]]]])
+    V = np.array([[[[2.0, 3.0]]]])
+    Ob, Sb = O.decode(Q, K, V, np.full((1, 1, 1), 0.5), np.full((1, 1, 1), -1.0),
+                      np.eye(2)[None, None])
+    S_ref = np.array([[a / 2 + 1.0, 0.0], [1.5, a]])
+    assert np.allclose(Sb[0, 0], S_ref, rtol=0, atol=1e-15)
+    assert np.allclose(Ob[0, 0, 0], S_ref @ np.array([1.0, 1.0]), rtol=0, atol=1e-15)
+
+
+def test_decode_full_write_retrieves_value():
+    """Delta-rule property: with a = 1, b = 1 and a unit key, the updated state
+    maps that key exactly onto its value (S' k = S k - S k + v)."""
+    rng = np.random.default_rng(21)
+    d = 16
+    k = rng.standard_normal(d)
+    k /= np.linalg.norm(k)
+    v = rng.standard_normal(d)
+    S0 = rng.standard_normal((1, 1, d, d))
+    _, S1 = O.decode(rng.standard_normal((1, 1, 1, d)), k[None, None, None], v[None, None, None],
+                     np.ones((1, 1, 1)), np.zeros((1, 1, 1)), S0)
+    assert np.allclose(S1[0, 0] @ k, v, rtol=0, atol=1e-12)
+
+
+def test_decode_zero_beta_only_decays():
+    rng = np.random.default_rng(22)
+    d, n = 8, 3
+    S0 = rng.standard_normal((1, 2, d, d))
+    Q = rng.standard_normal((1, 1, n, d))
+    lg = -np.abs(rng.standard_normal((1, 2, n)))
+    Ob, Sb = O.decode(Q, rng.standard_normal((1, 1, n, d)), rng.standard_normal((1, 2, n, d)),
+                      np.zeros((1, 2, n)), lg, S0)
+    for h in range(2):
+        decay = np.exp(np.cumsum(lg[0, h]))
+        for t in range(n):
+            assert np.allclose(Ob[0, h, t], decay[t] * S0[0, h] @ Q[0, 0, t], rtol=1e-13, atol=0)
+        assert np.allclose(Sb[0, h], decay[-1] * S0[0, h], rtol=1e-13, atol=0)
+
+
+def test_decode_equals_chunk_form():
+    """Decoding 128 tokens one at a time equals the chunk-wise forward with the
+    exact inverse (pinned above against the token recurrence)."""
+    k, n, d, H = 64, 128, 32, 2
+    rng = np.random.default_rng(23)
+    K, V, beta, _, lg = random_chunks(H * n // k, k, d, seed=23)
+    K, V = K.reshape(1, H, n, d), V.reshape(1, H, n, d)
+    beta, lg = beta.reshape(1, H, n), lg.reshape(1, H, n)
+    Q = rng.standard_normal((1, H, n, d))
+    Q /= np.linalg.norm(Q, axis=-1, keepdims=True)
+    S0 = 0.1 * rng.standard_normal((1, H, d, d))
+    Od, Sd = O.decode(Q, K, V, beta, lg, S0)
+    c = n // k
+    g = np.cumsum(lg.reshape(H, c, k), axis=-1)
+    Kc, Vc, Qc = (x.reshape(H, c, k, d) for x in (K, V, Q))
+    bc = beta.reshape(H, c, k)
+    T = O.invert_fwdsub(O.build_A(Kc, bc, g))
+    Oc, Sc = O.chunk_forward(Qc, Kc, Vc, bc, g, T, S0[0])
+    assert O.rel_fro(Od[0], Oc.reshape(H, n, d)) <= 1e-10
+    assert O.rel_fro(Sd[0], Sc) <= 1e-10
+
+
+def test_decode_value_heads_share_query_key_in_groups():
+    """Hv = 2 Hk: value heads 2j and 2j + 1 read query/key head j, i.e. the same
+    result as repeating each query/key head twice along the head axis."""
+    rng = np.random.default_rng(24)
+    B, Hk, Hv, n, d = 2, 2, 4, 3, 8
+    Q = rng.standard_normal((B, Hk, n, d))
+    K = rng.standard_normal((B, Hk, n, d))
+    K /= np.linalg.norm(K, axis=-1, keepdims=True)
+    V = rng.standard_normal((B, Hv, n, d))
+    beta = rng.uniform(0.1, 0.9, (B, Hv, n))
+    lg = -rng.uniform(0.0, 1.0, (B, Hv, n))
+    S0 = rng.standard_normal((B, Hv, d, d))
+    Og, Sg = O.decode(Q, K, V, beta, lg, S0)
+    Or, Sr = O.decode(np.repeat(Q, 2, axis=1), np.repeat(K, 2, axis=1), V, beta, lg, S0)
+    assert np.array_equal(Og, Or) and np.array_equal(Sg, Sr)
+    # and not the interleaved assignment h % Hk
+    Oi, _ = O.decode(np.tile(Q, (1, 2, 1, 1)), np.tile(K, (1, 2, 1, 1)), V, beta, lg, S0)
+    assert not np.allclose(Og, Oi)
+
+
+# --------------------------------------------------------------------------- #
 # INT8 scheme
 # --------------------------------------------------------------------------- #
 def test_I9_int8_codes_and_accumulators():
