@@ -399,6 +399,96 @@ def run_component(args, world, rank, local, dev) -> int:
         dist.destroy_process_group()
     return 0
 
+def run_decode(args, world, rank, local, dev) -> int:
+    """Device-timed decode steps: every sequence of the batch advances by
+    ``--tokens`` tokens through ``gdn_decode`` (16 query/key heads, 32 value
+    heads, d = 128, fp32 state).  State sets rotate so that the timed steps
+    touch more than L2 holds."""
+    import torch
+    from gated_deltanet_chunk_02_b200 import gdn
+    from gated_deltanet_chunk_02_b200.inputs import make_decode_inputs
+    B, Hk, Hv, n, d = args.batch, 16, 32, args.tokens, 128
+    elem = 2
+    per_set = B * Hv * d * d * 4
+    sets_n = max(args.rotate, -(-3 * 64 * 2 ** 20 // per_set))      # >= 192 MB in total
+    stream = torch.cuda.current_stream(dev)
+    base = make_decode_inputs(B, Hk, Hv, n, d=d, dtype="bf16", seed=shard_seed(rank, 0))
+    sets = []
+    for r in range(sets_n):
+        st = {key: v.to(dev) for key, v in base.items()}
+        st["O"] = torch.empty_like(st["V"])
+        sets.append(st)
+
+    def steps_all(st_):
+        for st in sets:
+            gdn.gdn_decode(st["Q"], st["K"], st["V"], st["beta"], st["loggate"], st["S0"],
+                           st["O"], stream=st_)
+
+    # one CUDA graph replays a decode step on every state set (a serving loop
+    # replays its captured step; at batch 1 host launch costs would otherwise
+    # be timed instead of the kernel)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        steps_all(side)
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    assert gdn.gdn_get_status(stream) == gdn.GDN_OK
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        steps_all(torch.cuda.current_stream(dev))
+    replays = max(1, args.steps // sets_n)
+    for _ in range(max(1, args.warmup // sets_n + 1)):
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    assert gdn.gdn_get_status(stream) == gdn.GDN_OK
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(replays):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = replays * sets_n
+    launches = steps                              # one kernel per decode step
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    assert gdn.gdn_get_status(stream) == gdn.GDN_OK
+    del graph
+    ms_step = ms / steps
+    # state read + written once per call; per token q, k (per key head), v, o
+    # (per value head), beta and the log-gate
+    bytes_l = B * Hv * 2 * d * d * 4 + B * n * (Hk * 2 * d * elem + Hv * (2 * d * elem + 8))
+    flops_l = B * Hv * n * 8 * d * d
+    peaks, peak_kind = load_peaks()
+    gbs = bytes_l / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": f"decode step: tokens/s (batch {B}, {n} token(s), 32 value heads, d=128)",
+        "value": world * B * n / (ms_step * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "us_per_step": ms_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"decode, B={B} Hk={Hk} Hv={Hv} n={n} d={d}, bf16 q/k/v, "
+                               "fp32 state in place",
+                   "l2": f"{sets_n} rotating state sets, {sets_n * per_set / 2**20:.0f} MB",
+                   "launch": "CUDA graph of one step per state set"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(peaks["hbm_gbs"]),
+                     "unit": "GB/s", "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
+                     "peak_source": peak_kind, "bytes_per_launch": bytes_l,
+                     "flops_per_launch": flops_l},
+        "clocks": clocks.summary(), "e2e": None, "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -414,9 +504,12 @@ def main(argv=None) -> int:
     ap.add_argument("--S", type=int, default=WORKLOAD["S"], help="residual steps")
     ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
     ap.add_argument("--kernel", default="fused",
-                    choices=["fused", "neumann", "fwdsub", "int8", "build_A", "wy", "forward"],
+                    choices=["fused", "neumann", "fwdsub", "int8", "build_A", "wy", "forward",
+                             "decode"],
                     help="time one component instead of the fused step (not the headline)")
     ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")
+    ap.add_argument("--batch", type=int, default=64, help="sequences per --kernel decode step")
+    ap.add_argument("--tokens", type=int, default=1, help="tokens per --kernel decode call")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="input/output sets cycled through the timed steps")
     args = ap.parse_args(argv)
@@ -437,6 +530,8 @@ def main(argv=None) -> int:
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.kernel == "decode":
+        return run_decode(args, world, rank, local, dev)
     if args.kernel != "fused":
         return run_component(args, world, rank, local, dev)
     w = dict(WORKLOAD, N=args.N, S=args.S, mask=args.mask)

@@ -248,6 +248,25 @@ int gdn_forward(const void* Q, const void* K, const void* V, const float* beta, 
                     "forward scan");
 }
 
+int gdn_decode(const void* Q, const void* K, const void* V, const float* beta,
+               const float* loggate, float* S, void* O, int64_t B, int64_t Hk, int64_t Hv,
+               int64_t n, int32_t d, gdn_dtype dtype, void* stream) {
+    GDN_TRY(check_dtype(dtype));
+    if (B < 0 || Hk < 0 || Hv < 0 || n < 0) return fail(GDN_ERR_ARG, "negative B, Hk, Hv or n");
+    if (d != 128) return fail(GDN_ERR_UNSUPPORTED, "head dim d=%d (only 128 is built)", d);
+    if (B == 0 || Hv == 0 || n == 0) return GDN_OK;
+    if (Hk == 0 || Hv % Hk)
+        return fail(GDN_ERR_ARG, "Hv=%lld is not a multiple of Hk=%lld", (long long)Hv,
+                    (long long)Hk);
+    if (B > 65535 || Hv > (1LL << 28) || n > 0x7fffffffLL)
+        return fail(GDN_ERR_ARG, "B, Hv or n too large");
+    GDN_TRY(check_ptrs({{Q, "Q"}, {K, "K"}, {V, "V"}, {beta, "beta"}, {loggate, "loggate"},
+                        {S, "S"}, {O, "O"}}));
+    return launched(gdn::launch_decode(Q, K, V, beta, loggate, S, O, B, Hk, Hv, n,
+                                       dtype == GDN_BF16, (cudaStream_t)stream),
+                    "decode");
+}
+
 int gdn_get_status(void* stream) {
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e = cudaStreamSynchronize(st);

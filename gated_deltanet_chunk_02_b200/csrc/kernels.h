@@ -28,4 +28,9 @@ cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, c
                         const float* S0, void* O, float* Sfin, void* Sstates, int64_t BH,
                         int64_t nchunk, bool bf16, cudaStream_t st);
 
+// Decode steps (decode.cu); d = 128, S [B][Hv][d][d] fp32 updated in place.
+cudaError_t launch_decode(const void* Q, const void* K, const void* V, const float* beta,
+                          const float* loggate, float* S, void* O, int64_t B, int64_t Hk,
+                          int64_t Hv, int64_t n, bool bf16, cudaStream_t st);
+
 }  // namespace gdn

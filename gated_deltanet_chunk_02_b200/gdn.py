@@ -25,8 +25,8 @@ GDN_OK, GDN_ERR_ARG, GDN_ERR_ALIGN, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_T
 EXPORTS = [
     "gdn_build_A", "gdn_invert_neumann", "gdn_invert_fwdsub", "gdn_wy",
     "gdn_invert_neumann_i8", "gdn_chunk_wy_fused", "gdn_forward",
-    "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_get_status", "gdn_last_error",
-    "gdn_launch_count",
+    "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_decode", "gdn_get_status",
+    "gdn_last_error", "gdn_launch_count",
 ]
 
 
@@ -68,6 +68,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gdn_forward": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I64, S, _I, _P],
         "gdn_forward_workspace_bytes": [S, _I],
         "gdn_forward_static": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, S, _I, _P],
+        "gdn_decode": [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int32, _I,
+                       _P],
         "gdn_get_status": [_P],
         "gdn_last_error": [],
         "gdn_launch_count": [],
@@ -178,6 +180,15 @@ def gdn_forward_static(Q, K, V, beta, g, S0, N, mask, S, exact, O, S_final, k=64
     _check(load().gdn_forward_static(_ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(g), _ptr(S0), N,
                                      int(mask), S, int(exact), _ptr(O), _ptr(S_final),
                                      shape_of(K, k), _dtype(K), _stream(stream)))
+
+
+def gdn_decode(Q, K, V, beta, loggate, S, O, stream=None):
+    """Decode n tokens: Q, K ``[B, Hk, n, d]``, V, O ``[B, Hv, n, d]``, beta,
+    loggate ``[B, Hv, n]``, state S ``[B, Hv, d, d]`` (float32, in place)."""
+    B, Hk, n, d = K.shape
+    Hv = V.shape[1]
+    _check(load().gdn_decode(_ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(loggate), _ptr(S),
+                             _ptr(O), B, Hk, Hv, n, d, _dtype(K), _stream(stream)))
 
 
 def gdn_get_status(stream=None) -> int:

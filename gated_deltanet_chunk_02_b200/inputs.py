@@ -17,6 +17,10 @@ Recipe (the distributions of the workloads the method is evaluated on):
 Draw order from one ``torch.Generator`` seeded with ``seed``: K, V,
 beta-logits, gate-logits, then Q.  K, V and Q are cast to the requested dtype
 after drawing; beta, g and the log-gates stay float32.
+
+Decode inputs (``make_decode_inputs``) use the same distributions for one or
+a few tokens per sequence, with grouped heads (``Hk`` query/key heads, ``Hv``
+value heads) and a carried float32 state ``S0 ~ N(0, 1/d)`` per value head.
 """
 from __future__ import annotations
 
@@ -83,6 +87,35 @@ def make_inputs(w: Workload, seed: int = 0, with_q: bool = False,
         Q = Q / Q.norm(dim=-1, keepdim=True)
         out["Q"] = Q.to(DTYPES[w.dtype]).contiguous()
     return out
+
+
+def make_decode_inputs(B: int, Hk: int, Hv: int, n: int, d: int = 128, dtype: str = "bf16",
+                       seed: int = 0) -> dict:
+    """Draw inputs of ``n`` decode steps on the CPU.
+
+    Draw order: K, V, beta-logits, gate-logits, Q, S0.  Returns ``Q, K``
+    (``[B,Hk,n,d]``, dtype), ``V`` (``[B,Hv,n,d]``, dtype), ``beta, loggate``
+    (``[B,Hv,n]`` float32, the per-token log-gates) and ``S0``
+    (``[B,Hv,d,d]`` float32).
+    """
+    gen = torch.Generator().manual_seed(seed)
+    K = torch.randn((B, Hk, n, d), generator=gen, dtype=torch.float32)
+    K = K / K.norm(dim=-1, keepdim=True)
+    V = torch.randn((B, Hv, n, d), generator=gen, dtype=torch.float32)
+    beta = torch.sigmoid(torch.randn((B, Hv, n), generator=gen, dtype=torch.float32))
+    loggate = -torch.nn.functional.softplus(
+        torch.randn((B, Hv, n), generator=gen, dtype=torch.float32))
+    Q = torch.randn((B, Hk, n, d), generator=gen, dtype=torch.float32)
+    Q = Q / Q.norm(dim=-1, keepdim=True)
+    S0 = torch.randn((B, Hv, d, d), generator=gen, dtype=torch.float32) / d ** 0.5
+    return {
+        "Q": Q.to(DTYPES[dtype]).contiguous(),
+        "K": K.to(DTYPES[dtype]).contiguous(),
+        "V": V.to(DTYPES[dtype]).contiguous(),
+        "beta": beta.contiguous(),
+        "loggate": loggate.contiguous(),
+        "S0": S0.contiguous(),
+    }
 
 
 def as_f64_numpy(t: torch.Tensor):

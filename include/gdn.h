@@ -183,6 +183,25 @@ int gdn_forward_static(const void* Q, const void* K, const void* V,
                        void* stream);
 
 /*
+ * Decode: the gated delta rule advanced token by token from a carried state,
+ * as in the technical summary of "A Persistent-State Dataflow Accelerator for
+ * Memory-Bound Linear Attention Decode on FPGA" (§1-§2).  For every batch b,
+ * value head h and token t = 0 .. n-1, with query/key head j = h / (Hv / Hk)
+ * (consecutive value heads share one query and one key):
+ *   S <- a_t S (I - b_t k_t k_t^T) + b_t v_t k_t^T,   o_t = S q_t,
+ *   a_t = exp(loggate_t)   (the token's own log-gate, not a cumulative sum).
+ * In: Q, K [B, Hk, n, d] (dtype), V [B, Hv, n, d] (dtype), beta, loggate
+ * [B, Hv, n] f32.  In/out: S [B, Hv, d, d] f32 (d_v x d_k, row-major),
+ * updated in place.  Out: O [B, Hv, n, d] (dtype).  d = 128, Hv a multiple of
+ * Hk, B <= 65535.  The state is read once and written once per call whatever
+ * n is (n = 1 is one decode step).  B, Hv or n = 0: nothing happens.  Errors
+ * as for every call; S is untouched on a nonzero return.
+ */
+int gdn_decode(const void* Q, const void* K, const void* V, const float* beta,
+               const float* loggate, float* S, void* O, int64_t B, int64_t Hk, int64_t Hv,
+               int64_t n, int32_t d, gdn_dtype dtype, void* stream);
+
+/*
  * Streams and graphs: every entry point enqueues its kernels on `stream`
  * (NULL = the legacy default stream) and returns without synchronising; none
  * allocates device memory (gdn_forward takes a caller workspace).  The calls

@@ -128,6 +128,21 @@ def test_empty_inputs_are_noops(lib):
     assert lib.gdn_launch_count() == n0
 
 
+def test_decode_argument_checks(lib):
+    n0 = lib.gdn_launch_count()
+    args = [P(FAKE)] * 7
+    # Hv not a multiple of Hk, head dim, bad dtype, misaligned state, empty
+    assert lib.gdn_decode(*args, 1, 3, 4, 1, 128, 1, None) == gdn.GDN_ERR_ARG
+    assert lib.gdn_decode(*args, 1, 2, 4, 1, 64, 1, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_decode(*args, 1, 2, 4, 1, 128, 9, None) == gdn.GDN_ERR_ARG
+    bad = args[:5] + [P(MISALIGNED), P(FAKE)]
+    assert lib.gdn_decode(*bad, 1, 2, 4, 1, 128, 1, None) == gdn.GDN_ERR_ALIGN
+    assert lib.gdn_decode(*[None] * 7, 1, 2, 4, 0, 128, 1, None) == gdn.GDN_OK
+    assert lib.gdn_decode(*[None] * 7, 0, 2, 4, 1, 128, 1, None) == gdn.GDN_OK
+    assert lib.gdn_decode(*[None] * 7, 1, 2, 4, 1, 128, 1, None) == gdn.GDN_ERR_ARG
+    assert lib.gdn_launch_count() == n0
+
+
 def test_workspace_size(lib):
     s = sh(B=2, H=3, T=512, k=64)
     nc = 2 * 3 * 8
