@@ -36,7 +36,7 @@ import numpy as np
 
 __all__ = [
     "to_chunks", "from_chunks", "band_mask", "build_A", "invert_fwdsub",
-    "neumann_powers_sum", "invert_neumann", "residual_matrix", "wy",
+    "neumann_powers_sum", "invert_neumann", "invert_newton", "residual_matrix", "wy",
     "int8_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
 ]
 
@@ -180,6 +180,24 @@ def invert_neumann(A: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
         Ep = Ep @ E
         acc = acc + Ep
     return T0 @ acc
+
+
+def invert_newton(A: np.ndarray, N: int, mask: bool, M: int) -> np.ndarray:
+    """Sequential residual correction, the comparison point of "When Good Enough
+    Is Optimal", Méthodologie §3: the iterative update T^(m+1) = T^(m) +
+    T^(m) R^(m) that the method replaces by its parallel sum, with the plain
+    reading R^(m) = I - (I - A) T^(m) (the residual of the current iterate).
+    T^(0) is the truncated, optionally masked series of ``invert_neumann``;
+    ``M`` steps are applied.
+    """
+    if M < 0:
+        raise ValueError("M must be >= 0")
+    A = np.asarray(A, np.float64)
+    T = invert_neumann(A, N, mask, 0)
+    for _ in range(M):
+        R = residual_matrix(A, T)
+        T = T + T @ R
+    return T
 
 
 def wy(T: np.ndarray, K: np.ndarray, V: np.ndarray, beta: np.ndarray,

@@ -320,6 +320,42 @@ def test_I8_chunk_form_equals_token_recurrence(T_len, d):
 
 
 # --------------------------------------------------------------------------- #
+# sequential correction (the comparison point of the parallel residual)
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("N,mask", [(1, True), (3, True), (3, False), (2, True)])
+def test_newton_steps_equal_parallel_residual_with_doubled_terms(N, mask):
+    """M sequential steps sum 2^M terms of the residual series: with R_m the
+    residual of T_m, R_{m+1} = R_m^2, so T_M = T0 (I + E + ... + E^(2^M - 1))."""
+    K, _, beta, g, _ = random_chunks(3, 16, 8, seed=31)
+    A = O.build_A(K, beta, g)
+    for M in range(4):
+        TN = O.invert_newton(A, N, mask, M)
+        TP = O.invert_neumann(A, N, mask, 2 ** M - 1)
+        assert np.allclose(TN, TP, rtol=0, atol=1e-12)
+
+
+def test_newton_residual_squares_each_step():
+    K, _, beta, g, _ = random_chunks(2, 16, 8, seed=32)
+    A = O.build_A(K, beta, g)
+    eye = np.eye(16)
+    prev = O.residual_matrix(A, O.invert_newton(A, 2, True, 0))
+    for M in range(1, 4):
+        R = eye - (eye - A) @ O.invert_newton(A, 2, True, M)
+        assert np.allclose(R, prev @ prev, rtol=0, atol=1e-13)
+        prev = R
+
+
+def test_newton_reaches_the_exact_inverse():
+    """2^M (N + 1) >= k: the residual's power vanishes, T_M is exact."""
+    K, _, beta, g, _ = random_chunks(2, 16, 8, seed=33)
+    A = O.build_A(K, beta, g)
+    T = O.invert_newton(A, 3, True, 2)                 # 4 * 4 >= 16
+    assert np.allclose((np.eye(16) - A) @ T, np.eye(16), rtol=0, atol=1e-13)
+    T1 = O.invert_newton(A, 3, True, 1)                # 2 * 4 < 16: not exact
+    assert not np.allclose((np.eye(16) - A) @ T1, np.eye(16), rtol=0, atol=1e-9)
+
+
+# --------------------------------------------------------------------------- #
 # decode steps (grouped query/key heads)
 # --------------------------------------------------------------------------- #
 def test_decode_two_dim_closed_form():
