@@ -302,7 +302,7 @@ def run_component(args, world, rank, local, dev) -> int:
         st = {key: v.to(dev) for key, v in inp.items()}
         st["A"] = torch.empty(wl.B, wl.H, wl.T // k, k, k, device=dev)
         st["T"] = torch.empty_like(st["A"])
-        if kern in ("neumann", "fwdsub", "int8", "wy"):
+        if kern in ("neumann", "newton", "fwdsub", "int8", "wy"):
             gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
         if kern == "wy":
             gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
@@ -321,6 +321,8 @@ def run_component(args, world, rank, local, dev) -> int:
         if kern == "neumann":
             gdn.gdn_invert_neumann(st["A"], st["T"], args.N, args.mask, args.S, gdn.GDN_PREC_F16,
                                    stream=stream)
+        elif kern == "newton":
+            gdn.gdn_invert_newton(st["A"], st["T"], args.N, args.mask, args.M, stream=stream)
         elif kern == "fwdsub":
             gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
         elif kern == "int8":
@@ -359,6 +361,7 @@ def run_component(args, world, rank, local, dev) -> int:
     chain = (args.N - 1 + (args.S + 1 if args.S > 0 else 0)) * 2 * k ** 3
     per = {
         "neumann": (2 * kk2, chain),
+        "newton": (2 * kk2, (args.N - 1 + 2 * args.M) * 2 * k ** 3),
         "fwdsub": (2 * kk2, 2 * k ** 3 // 6),
         "int8": (2 * kk2, (args.N - 1) * 2 * k ** 3),
         "build_A": (kd + 8 * k + kk2, 2 * k * k * d),
@@ -381,7 +384,9 @@ def run_component(args, world, rank, local, dev) -> int:
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": f"{kern}, B={wl.B} H={wl.H} T={wl.T} k={k} d={d} N={args.N} "
-                               f"mask={args.mask} S={args.S}", "chunks": nc},
+                               f"mask={args.mask} "
+                               + (f"M={args.M}" if kern == "newton" else f"S={args.S}"),
+                   "chunks": nc},
         "roofline": {"bound": bound, "achieved": gbs if bound == "hbm" else tfl,
                      "peak": float(peaks["hbm_gbs"]) if bound == "hbm" else float(peaks["bf16_tflops"]),
                      "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
@@ -504,11 +509,12 @@ def main(argv=None) -> int:
     ap.add_argument("--S", type=int, default=WORKLOAD["S"], help="residual steps")
     ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
     ap.add_argument("--kernel", default="fused",
-                    choices=["fused", "neumann", "fwdsub", "int8", "build_A", "wy", "forward",
-                             "decode"],
+                    choices=["fused", "neumann", "newton", "fwdsub", "int8", "build_A", "wy",
+                             "forward", "decode"],
                     help="time one component instead of the fused step (not the headline)")
     ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")
     ap.add_argument("--batch", type=int, default=64, help="sequences per --kernel decode step")
+    ap.add_argument("--M", type=int, default=3, help="sequential correction steps (--kernel newton)")
     ap.add_argument("--tokens", type=int, default=1, help="tokens per --kernel decode call")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="input/output sets cycled through the timed steps")

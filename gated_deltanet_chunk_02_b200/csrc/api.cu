@@ -128,6 +128,20 @@ int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask, i
     return launched(gdn::launch_neumann_simt(A, T, nc, s.k, N, mask, S, st), "neumann");
 }
 
+int gdn_invert_newton(const float* A, float* T, gdn_shape s, int N, int mask, int M,
+                      void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_NS(N, mask, 0, s.k));
+    if (M < 0 || M > 6) return fail(GDN_ERR_ARG, "correction steps M=%d outside [0, 6]", M);
+    if (s.k == 256) return fail(GDN_ERR_UNSUPPORTED, "sequential correction supports k <= 128");
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
+    return launched(gdn::launch_newton_tc(A, T, nc, s.k, N, mask, M, (cudaStream_t)stream),
+                    "newton (tcgen05)");
+}
+
 int gdn_invert_fwdsub(const float* A, float* T, gdn_shape s, void* stream) {
     int64_t nc;
     GDN_TRY(check_shape(s, &nc));

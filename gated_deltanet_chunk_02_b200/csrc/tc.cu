@@ -43,10 +43,12 @@ constexpr int kRows = 128;                       // rows per tile
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr int kStatusSmemAlign = 2;              // dynamic shared memory not 1024-aligned
 
-enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3 };
+enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3, kNewton = 4 };
 
 __host__ __device__ constexpr bool uses_K(int m) { return m == kFused || m == kBuildA || m == kWY; }
 __host__ __device__ constexpr bool uses_V(int m) { return m == kFused || m == kWY; }
+// the standalone inverses: A in by TMA (staged a tile ahead), T out by TMA
+__host__ __device__ constexpr bool inv_only(int m) { return m == kNeumann || m == kNewton; }
 __host__ __device__ constexpr int block_of(int kc) { return kc < 64 ? 64 : kc; }
 
 // Per-slot shared-memory layout (bytes).  The 1024-byte aligned operand
@@ -55,7 +57,7 @@ template <int KB, int MODE>
 struct SlotLayout {
     static constexpr int kK = uses_K(MODE) ? kRows * kD * 2 : 0;        // bf16 [2][128][64]
     static constexpr int kV = uses_V(MODE) ? kRows * kD * 2 : 0;
-    static constexpr int kAop = (MODE == kFused || MODE == kNeumann) ? kRows * KB * 2 : 0;
+    static constexpr int kAop = (MODE == kFused || inv_only(MODE)) ? kRows * KB * 2 : 0;
     static constexpr int kXY = (MODE == kBuildA) ? 0 : kRows * KB * 2;  // 16-bit [KB/64][128][64]
     static constexpr int offK = 0;
     static constexpr int offV = offK + kK;
@@ -64,7 +66,7 @@ struct SlotLayout {
     static constexpr int offY = offAop + kAop;
     // the standalone inverse stages the next tile's A (fp32, 128-byte swizzled
     // boxes of 32 columns x 128 rows) while it works on the current one
-    static constexpr int kStage = (MODE == kNeumann) ? kRows * KB * 4 : 0;
+    static constexpr int kStage = inv_only(MODE) ? kRows * KB * 4 : 0;
     static constexpr int offStage = offY + kXY;
     static constexpr int bytes = offStage + kStage;
     static constexpr int bg_bytes = uses_K(MODE) ? 2 * kRows * 4 : 0;  // beta[128], g[128]
@@ -392,10 +394,11 @@ struct Params {
     int64_t rows;        // B*H*T
     int ntiles;
     int N, mask, S, gated;
-    const float* Ain;    // kNeumann
+    const float* Ain;    // kNeumann, kNewton
     const float* Tin;    // kWY
     float* Aout;         // kBuildA
-    float* Tout;         // kFused (optional), kNeumann
+    float* Tout;         // kFused (optional), kNeumann, kNewton
+    int M;               // kNewton: sequential correction steps
     int* status;
 };
 
@@ -545,7 +548,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     // barrier and issuing thread, and their products are M = 128, N = 64 (the
     // other block's rows come out as unused values), so the two blocks' rounds
     // interleave on the SM instead of waiting for each other.
-    constexpr bool kSplit = (NCH == 2) && (MODE == kFused || MODE == kNeumann);
+    constexpr bool kSplit = (NCH == 2) && (MODE == kFused || inv_only(MODE));
     const int cg = kSplit ? blk : 0;
     const bool cleader = kSplit ? (lane == 0 && (warp % 8) == 2 * cg) : leader;
     const int cbar = kSplit ? 3 + 2 * s + cg : bar_id;
@@ -604,10 +607,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
     auto issue_k = [&](int n) {
         const int tile = blockIdx.x + n * gridDim.x;
-        if (!(uses_K(MODE) || MODE == kNeumann) || tile >= p.ntiles) return;
+        if (!(uses_K(MODE) || inv_only(MODE)) || tile >= p.ntiles) return;
         ++k_issued;
         const int y = tile * kRows;
-        if (MODE == kNeumann) {                        // A: KC / 32 boxes of 16 KB
+        if (inv_only(MODE)) {                          // A: KC / 32 boxes of 16 KB
             mbar_expect_tx(&ctrl->fullK[s], (KC / 32) * 16384);
 #pragma unroll 1
             for (int b = 0; b < KC / 32; ++b)
@@ -714,7 +717,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         const int64_t rin = grow % KC;                   // row inside the chunk
         float T0[kT0Tmem ? 1 : PPT * 32];                // this thread's part of row r of T0 / T
 
-        if ((uses_K(MODE) || MODE == kNeumann) && !mbar_wait(&ctrl->fullK[s], use_par))
+        if ((uses_K(MODE) || inv_only(MODE)) && !mbar_wait(&ctrl->fullK[s], use_par))
             fail_wait();
         bar_sync(bar_id, 256);
         if (*(volatile int*)&ctrl->abort) { ok = false; break; }
@@ -778,7 +781,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 if (leader) issue_k(n + NS);
                 continue;
             }
-        } else if (MODE == kNeumann) {
+        } else if (inv_only(MODE)) {
             // ---- A rows from the staged tile ----
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
@@ -842,7 +845,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         }
 
         if (MODE == kFused) release_staging(n);
-        if (MODE == kFused || MODE == kNeumann) {
+        if (MODE == kFused || inv_only(MODE)) {
             // ---- truncated Neumann series in Horner form ----
             // X_1 = I + M.A, X_n = I + M.(X_{n-1} A), T0 = X_N: inside the band
             // X_{n-1} A reads only in-band entries of X_{n-1}, so masking every
@@ -882,7 +885,54 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             // (fp16) goes to the Aop buffer, E = I - T0 + A + A (T0 - I) to X,
             // G - I to Y, and T = T0 + (G - I) + (T0 - I)(G - I); T0 stays in
             // registers.
-            if (p.S > 0) {
+            if constexpr (MODE == kNewton) {
+                // Sequential correction, the form the method's parallel residual
+                // replaces: R_m = I - (I - A) T_m = I - T_m + A T_m and
+                // T_{m+1} = T_m + T_m R_m, two dependent products per step.
+                // T_m stays fp32 (T0 columns / registers); its fp16 copy goes
+                // to Y (right operand of A T_m) and to TMEM (left operand of
+                // T_m R_m), and R_m to Y.
+                for (int it = 0; it < p.M; ++it) {
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        float t[32];
+                        t0_get(pp, t, T0);
+                        st_op32<false>(sY, r, pc0 + pp, t);                // T_m
+                    }
+                    cpublish(true);
+                    cchain(sX, sY);                                      // A T_m
+                    if (!cwait()) { ok = false; break; }
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
+                        float v[32], t[32];
+                        tmem_ld32(tD + pc * 32, v);
+                        t0_get(pp, t, T0);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int j = pc * 32 + jj;
+                            v[jj] = in_chunk(j) ? eye(j) - t[jj] + v[jj] : 0.f;   // R_m
+                        }
+                        st_op32<false>(sY, r, pc, v);
+                        tmem_st_h16(tA + pc * 16, t);                      // T_m, left operand
+                    }
+                    cpublish(true);
+                    cchain_t(sY);                                        // T_m R_m
+                    if (!cwait()) { ok = false; break; }
+#pragma unroll
+                    for (int pp = 0; pp < PPT; ++pp) {
+                        const int pc = pc0 + pp;
+                        float v[32], t[32];
+                        tmem_ld32(tD + pc * 32, v);
+                        t0_get(pp, t, T0);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];      // T_{m+1}
+                        t0_put(pp, t, T0);
+                    }
+                }
+                if (!ok) break;
+            } else if (p.S > 0) {
                 const int S = p.S;
                 int K2 = 0;
                 while ((2 << K2) <= S + 1) ++K2;
@@ -1224,7 +1274,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
             }
             // ---- T out ----
-            if (MODE == kNeumann) {
+            if (inv_only(MODE)) {
                 // through the Aop | Y buffers as fp32 128-byte swizzled boxes, TMA store
                 bar_sync(bar_id, 256);                 // this tile's Aop / Y operands are read
                 const uint32_t st0 = su32(sAop);
@@ -2235,7 +2285,7 @@ static cudaError_t launch(const IO& io, const Params& p0, cudaStream_t st) {
             !map_kd(&mU, io.U, p0.rows))
             return cudaErrorInvalidValue;
     }
-    if (MODE == kNeumann) {                        // A in through mK, T out through mW
+    if (inv_only(MODE)) {                          // A in through mK, T out through mW
         if (!map_f32(&mK, p0.Ain, p0.rows, KC) || !map_f32(&mW, p0.Tout, p0.rows, KC))
             return cudaErrorInvalidValue;
     }
@@ -2315,6 +2365,17 @@ cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N
     p.mask = mask;
     p.S = S;
     return tcg::dispatch<tcg::kNeumann, 1>(k, tcg::IO(), p, st);
+}
+
+cudaError_t launch_newton_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int M,
+                             cudaStream_t st) {
+    tcg::Params p = tcg::base_params(nc, k);
+    p.Ain = A;
+    p.Tout = T;
+    p.N = N;
+    p.mask = mask;
+    p.M = M;
+    return tcg::dispatch<tcg::kNewton, 1>(k, tcg::IO(), p, st);
 }
 
 cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const float* beta,

@@ -17,6 +17,9 @@ cudaError_t launch_build_A256_tc(const void* K, const float* beta, const float* 
                                  int64_t nc, cudaStream_t st);
 cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int S,
                               cudaStream_t st);
+// truncated series, then M sequential correction steps T <- T + T (I - (I - A) T)
+cudaError_t launch_newton_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int M,
+                             cudaStream_t st);
 // k = 256: truncated series (Horner, by 128 x 128 blocks) and residual, one chunk per CTA
 cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, int mask, int S,
                                 cudaStream_t st);

@@ -92,6 +92,19 @@ int gdn_invert_neumann(const float* A, float* T, gdn_shape s, int N, int mask,
                        int S, gdn_prec prec, void* stream);
 
 /*
+ * Sequential residual correction, the comparison point of "Méthodologie" §3
+ * (the iterative update the method replaces by its parallel sum): T_0 is the
+ * truncated series with the band mask as in gdn_invert_neumann, then M steps
+ *   R_m = I - (I - A) T_m,   T_{m+1} = T_m + T_m R_m,
+ * two dependent products per step.  In exact arithmetic T_M equals
+ * gdn_invert_neumann with S = 2^M - 1.  Tensor cores (fp16 operands, fp32
+ * accumulation), k in {32, 64, 128} (GDN_ERR_UNSUPPORTED at 256),
+ * 0 <= M <= 6.  In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.
+ */
+int gdn_invert_newton(const float* A, float* T, gdn_shape s, int N, int mask, int M,
+                      void* stream);
+
+/*
  * Exact T = (I - A)^{-1} by forward substitution ("Énoncé du Problème": the
  * k-1 sequential row steps the method replaces).  fp32 on CUDA cores.
  * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.

@@ -128,6 +128,15 @@ def test_empty_inputs_are_noops(lib):
     assert lib.gdn_launch_count() == n0
 
 
+def test_newton_limits(lib):
+    assert lib.gdn_invert_newton(P(FAKE), P(FAKE), sh(), 3, 1, 7, None) == gdn.GDN_ERR_ARG
+    assert lib.gdn_invert_newton(P(FAKE), P(FAKE), sh(), 0, 1, 2, None) == gdn.GDN_ERR_ARG
+    assert lib.gdn_invert_newton(P(FAKE), P(FAKE), sh(T=512, k=256), 3, 1, 2,
+                                 None) == gdn.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_invert_newton(P(FAKE), P(MISALIGNED), sh(), 3, 1, 2, None) == gdn.GDN_ERR_ALIGN
+    assert lib.gdn_invert_newton(None, None, sh(B=0), 3, 1, 2, None) == gdn.GDN_OK
+
+
 def test_decode_argument_checks(lib):
     n0 = lib.gdn_launch_count()
     args = [P(FAKE)] * 7

@@ -236,6 +236,38 @@ def test_neumann_tensor_cores(k, N, mask, S):
             assert np.all(Th[:, dist > N] == 0)
 
 
+@pytest.mark.parametrize("k", [32, 64, 128])
+@pytest.mark.parametrize("N,mask", [(1, 1), (3, 1), (3, 0)])
+@pytest.mark.parametrize("M", [0, 1, 2, 3, 4])
+def test_newton_tensor_cores(k, N, mask, M):
+    """The sequential correction T <- T + T (I - (I - A) T) on the tensor cores,
+    9 chunks (a ragged last tile), against the oracle's literal iteration."""
+    w = Workload(B=1, H=3, T=3 * k, k=k, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=12), w)
+    T = torch.full((w.B, w.H, w.T // k, k, k), float("nan"), device="cuda")
+    gdn.gdn_invert_newton(to_dev(A_tensor(A32, w)), T, N, mask, M)
+    check_status()
+    ref = O.invert_newton(A32.astype(np.float64), N, bool(mask), M)
+    assert torch.isfinite(T).all()
+    assert rel(T, ref) <= TOL_BF16
+    assert per_chunk_max_rel(T, ref) <= TOL_BF16
+    assert np.all(np.triu(T.cpu().numpy().reshape(ref.shape), 1) == 0)
+
+
+def test_newton_matches_parallel_residual_on_gpu():
+    """M = 3 sequential steps and the parallel residual with S = 7 compute the
+    same T (exactly so in exact arithmetic)."""
+    k = 64
+    w = Workload(B=1, H=4, T=8 * k, k=k, dtype="bf16")
+    A = to_dev(A_tensor(oracle_A32(make_inputs(w, seed=13), w), w))
+    T1 = torch.empty(w.B, w.H, w.T // k, k, k, device="cuda")
+    T2 = torch.empty_like(T1)
+    gdn.gdn_invert_newton(A, T1, 3, 1, 3)
+    gdn.gdn_invert_neumann(A, T2, 3, 1, 7, gdn.GDN_PREC_F16)
+    check_status()
+    assert rel(T1, T2.cpu().double().numpy()) <= 1e-3
+
+
 @pytest.mark.parametrize("N,mask,S", [(1, 1, 0), (2, 1, 0), (3, 1, 0), (4, 1, 0), (3, 0, 0),
                                       (8, 0, 0), (40, 1, 0), (255, 1, 0), (1, 1, 1), (3, 1, 1),
                                       (3, 1, 2), (3, 1, 8), (2, 0, 3), (40, 1, 8)])
