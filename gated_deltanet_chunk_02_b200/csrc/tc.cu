@@ -668,21 +668,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     auto eye = [&](int j) { return i == j ? 1.f : 0.f; };
     auto piece_in_chunk = [&](int pc) { return !SUB || (pc * 32 >= cl && pc * 32 < ch); };
 
-    // products of one residual round: D[0,128) = X X, D[128,256) = Y X
-    auto mma_pair = [&](bool sq, bool gp) {
-        if (leader) {
-            constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
-            const uint32_t xb = su32(sX), yb = su32(sY);
-#pragma unroll 1
-            for (int kk = 0; kk < KB / 16; ++kk) {
-                const uint32_t ko = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
-                const uint64_t bx = sdesc(xb + kk * 2048, KB * 128, 1024);
-                if (sq) mma_ss(tm, sdesc(xb + ko, 16, 1024), bx, id, kk > 0);
-                if (gp) mma_ss(tm + 128, sdesc(yb + ko, 16, 1024), bx, id, kk > 0);
-            }
-            mma_commit(&ctrl->mma[s]);
-        }
-    };
     // 8 fp16 values of row rr, columns 8q .. 8q + 7, of an operand buffer
     auto ld_h8 = [&](const uint8_t* buf, int rr, int q, float (&o)[8]) {
         uint4 u;
@@ -696,10 +681,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             o[2 * c] = f.x;
             o[2 * c + 1] = f.y;
         }
-    };
-    auto st_h8 = [&](uint8_t* buf, int rr, int q, const float (&v)[8]) {
-        sts128(su32(buf) + op_off(rr, q), make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]),
-                                                     pack_h2(v[4], v[5]), pack_h2(v[6], v[7])));
     };
     if (leader) {
         issue_k(s);
@@ -870,21 +851,15 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             }
             if (!ok) break;
             // ---- parallel residual correction: T = T0 G, G = sum_{s<=S} E^s ----
-            // Three schedules.  Horner keeps (I + Q_m) in TMEM as the left
-            // operand of Q_{m+1} = (I + Q_m) E (S - 1 products, one per round,
-            // in 64-row blocks that do not wait for each other) and T0 in fp32;
-            // it serves the fused step and every S the doubling forms do not.
-            // The standalone inverse doubles when S + 1 is 2^m or 2^m + 1:
-            // stacked at KB = 64 (below), with two products per round at KB =
-            // 128.  In the fused step the stacked form measured slower at S <= 8
-            // (its lockstep rounds and wider epilogues cost more than the two
-            // rounds it saves), so the fused step keeps Horner.
-            // Two-product doubling (KB = 128): with a = 2^r,
-            // G(2a) - I = (G(a) - I) + E^a + (G(a) - I) E^a and E^2a = E^a E^a,
-            // two products per round sharing the right operand E^a.  T0 - I
-            // (fp16) goes to the Aop buffer, E = I - T0 + A + A (T0 - I) to X,
-            // G - I to Y, and T = T0 + (G - I) + (T0 - I)(G - I); T0 stays in
-            // registers.
+            // Two schedules.  Horner keeps Q_m in TMEM as the left operand
+            // (stride 2 below: one product per round, in 64-row blocks that do
+            // not wait for each other) and T0 in fp32; it serves the fused step,
+            // k = 128 and every S the doubling does not.  The standalone inverse
+            // at KB = 64 doubles when S + 1 is 2^m or 2^m + 1 (stacked, below).
+            // In the fused step the stacked form measured slower at S <= 8 (its
+            // lockstep rounds and wider epilogues cost more than the two rounds
+            // it saves); at k = 128 a doubling with two products per round lost
+            // to Horner, its extra k^3 products outweighing the rounds.
             if constexpr (MODE == kNewton) {
                 // Sequential correction, the form the method's parallel residual
                 // replaces: R_m = I - (I - A) T_m = I - T_m + A T_m and
@@ -1036,7 +1011,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             t0_put(pp, v, T0);
                         }
                     }
-                } else if (!(MODE == kNeumann && dbl)) {
+                } else {
                     // Horner with stride 2: Q_1 = E, E^2 = E E, F = E + E^2,
                     // Q_{m+2} = F + Q_m E^2, and Q_{m+1} = E + Q_m E when one
                     // step is left; Q_m (no identity) is the left operand in
@@ -1165,110 +1140,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
                             if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];          // T = T0 + T0 Q
-                        t0_put(pp, t, T0);
-                    }
-                } else if constexpr (MODE == kNeumann && KB != 64) {
-#pragma unroll
-                    for (int pp = 0; pp < PPT; ++pp) {
-                        const int pc = pc0 + pp;
-                        float t[32];
-                        t0_get(pp, t, T0);
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) t[jj] -= eye(pc * 32 + jj);
-                        st_op32<false>(sAop, r, pc, t);                    // T0 - I
-                    }
-                    publish(true);
-                    mma_chain(sX, sAop);                                    // A (T0 - I)
-                    if (!wait_mma()) { ok = false; break; }
-                    const int rounds = K2;
-#pragma unroll
-                    for (int pp = 0; pp < PPT; ++pp) {
-                        const int pc = pc0 + pp;
-                        float v[32], t[32];
-                        tmem_ld32(tD + pc * 32, v);
-                        t0_get(pp, t, T0);
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            float a8[8], e8[8], z8[8];
-                            ld_h8(sX, r, 4 * pc + g, a8);                    // A
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const int jj = 8 * g + c, j = pc * 32 + jj;
-                                e8[c] = in_chunk(j) ? eye(j) - t[jj] + a8[c] + v[jj] : 0.f;
-                                z8[c] = 0.f;
-                            }
-                            st_h8(sX, r, 4 * pc + g, e8);                    // E^1
-                            st_h8(sY, r, 4 * pc + g, z8);                    // G(1) - I = 0
-                        }
-                    }
-                    for (int rd = 1; rd <= rounds; ++rd) {
-                        const bool sq = rd < K2 || p2p1;                   // E^a E^a
-                        const bool gp = rd > 1;                            // (G - I) E^a
-                        const bool add_sq = rd == K2 && p2p1;              // + E^(2^m)
-                        const bool ea_out = sq && rd < K2;
-                        if (sq || gp) {
-                            publish(true);
-                            mma_pair(sq, gp);
-                            if (!wait_mma()) { ok = false; break; }
-                        }
-#pragma unroll
-                        for (int pp = 0; pp < PPT; ++pp) {
-                            const int pc = pc0 + pp;
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                float da[16], db[16];
-                                const uint32_t c0 = tD + pc * 32 + 16 * hh;
-                                if (sq && gp) {
-                                    tmem_ld2x16(c0, da, c0 + 128, db);
-                                } else if (sq) {
-                                    tmem_ld2x16(c0, da, c0, db);
-                                } else if (gp) {
-                                    tmem_ld2x16(c0 + 128, db, c0 + 128, da);
-                                } else {
-#pragma unroll
-                                    for (int c = 0; c < 16; ++c) da[c] = db[c] = 0.f;
-                                }
-#pragma unroll
-                                for (int g2 = 0; g2 < 2; ++g2) {
-                                    const int q = 4 * pc + 2 * hh + g2;
-                                    float ea[8], gb[8], go[8], eo[8];
-                                    ld_h8(sX, r, q, ea);
-                                    ld_h8(sY, r, q, gb);
-#pragma unroll
-                                    for (int c = 0; c < 8; ++c) {
-                                        float x = ea[c];
-                                        x += gb[c];
-                                        if (gp) x += db[8 * g2 + c];
-                                        if (add_sq) x += da[8 * g2 + c];
-                                        go[c] = in_chunk(8 * q + c) ? x : 0.f;
-                                        eo[c] = in_chunk(8 * q + c) ? da[8 * g2 + c] : 0.f;
-                                    }
-                                    st_h8(sY, r, q, go);
-                                    if (ea_out) st_h8(sX, r, q, eo);
-                                }
-                            }
-                        }
-                    }
-                    if (!ok) break;
-                    publish(true);
-                    mma_chain(sAop, sY);                                    // (T0 - I)(G - I)
-                    if (!wait_mma()) { ok = false; break; }
-#pragma unroll
-                    for (int pp = 0; pp < PPT; ++pp) {
-                        const int pc = pc0 + pp;
-                        float v[32], t[32];
-                        tmem_ld32(tD + pc * 32, v);
-                        t0_get(pp, t, T0);
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            float g8[8];
-                            ld_h8(sY, r, 4 * pc + g, g8);                    // G - I
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const int jj = 8 * g + c;
-                                t[jj] = in_chunk(pc * 32 + jj) ? t[jj] + g8[c] + v[jj] : 0.f;
-                            }
-                        }
                         t0_put(pp, t, T0);
                     }
                 }
