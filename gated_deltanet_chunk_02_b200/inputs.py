@@ -58,19 +58,21 @@ def chunk_cumsum(loggate: torch.Tensor, k: int) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, seed: int = 0, with_q: bool = False,
-                gate_scale: float = 1.0) -> dict:
+                gate_scale: float = 1.0, raw_keys: bool = False) -> dict:
     """Draw one batch of inputs for workload ``w`` on the CPU.
 
     Returns a dict of CPU tensors: ``K``, ``V`` (``[B,H,T,d]`` in ``w.dtype``),
     ``beta``, ``loggate``, ``g`` (``[B,H,T]`` float32) and, if ``with_q``,
-    ``Q`` (``[B,H,T,d]`` in ``w.dtype``).
+    ``Q`` (``[B,H,T,d]`` in ``w.dtype``).  ``raw_keys`` leaves the key rows
+    un-normalised (same draws, for the kernels that normalise them).
     """
     if w.T % w.k:
         raise ValueError("T must be a multiple of the chunk size k")
     gen = torch.Generator().manual_seed(seed)
     shp = (w.B, w.H, w.T, w.d)
     K = torch.randn(shp, generator=gen, dtype=torch.float32)
-    K = K / K.norm(dim=-1, keepdim=True)
+    if not raw_keys:
+        K = K / K.norm(dim=-1, keepdim=True)
     V = torch.randn(shp, generator=gen, dtype=torch.float32)
     beta = torch.sigmoid(torch.randn(shp[:3], generator=gen, dtype=torch.float32))
     loggate = -torch.nn.functional.softplus(

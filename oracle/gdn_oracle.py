@@ -35,7 +35,8 @@ import math
 import numpy as np
 
 __all__ = [
-    "to_chunks", "from_chunks", "band_mask", "build_A", "invert_fwdsub",
+    "to_chunks", "from_chunks", "l2_normalize_rows", "chunk_cumsum", "band_mask", "build_A",
+    "invert_fwdsub",
     "neumann_powers_sum", "invert_neumann", "invert_newton", "residual_matrix", "wy",
     "int8_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
 ]
@@ -67,6 +68,25 @@ def snr_db(x: np.ndarray, ref: np.ndarray) -> float:
     """Signal-to-noise ratio 10 log10(||ref||^2 / ||x - ref||^2) in dB."""
     err = rel_fro(x, ref)
     return float("inf") if err == 0.0 else float(-20.0 * np.log10(err))
+
+
+# --------------------------------------------------------------------------- #
+# the prologue: key normalisation and chunk-local cumulative gates
+# --------------------------------------------------------------------------- #
+def l2_normalize_rows(K: np.ndarray) -> np.ndarray:
+    """k_i / ||k_i||_2 over the last axis; an all-zero row stays zero.  The
+    workloads' keys are unit rows ("K rows N(0,1) then L2-normalised")."""
+    K = np.asarray(K, np.float64)
+    n = np.sqrt(np.sum(K * K, axis=-1, keepdims=True))
+    return np.divide(K, n, out=np.zeros_like(K), where=n > 0)
+
+
+def chunk_cumsum(loggate: np.ndarray, k: int) -> np.ndarray:
+    """Inclusive cumulative sum of the per-token log-gates over the last axis,
+    restarted every ``k`` entries (the chunk-local g; g_i includes token i)."""
+    x = np.asarray(loggate, np.float64)
+    T = x.shape[-1]
+    return np.cumsum(x.reshape(*x.shape[:-1], T // k, k), axis=-1).reshape(x.shape)
 
 
 # --------------------------------------------------------------------------- #

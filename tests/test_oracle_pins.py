@@ -320,6 +320,30 @@ def test_I8_chunk_form_equals_token_recurrence(T_len, d):
 
 
 # --------------------------------------------------------------------------- #
+# prologue: normalised keys, chunk-local cumulative gates
+# --------------------------------------------------------------------------- #
+def test_l2_normalize_rows():
+    x = np.array([[3.0, 4.0], [0.0, 0.0], [-1.0, 0.0]])
+    assert np.array_equal(O.l2_normalize_rows(x), np.array([[0.6, 0.8], [0.0, 0.0], [-1.0, 0.0]]))
+    rng = np.random.default_rng(41)
+    K = rng.standard_normal((3, 5, 16)) * rng.uniform(0.1, 10.0, (3, 5, 1))
+    Kn = O.l2_normalize_rows(K)
+    assert np.allclose(np.linalg.norm(Kn, axis=-1), 1.0, rtol=0, atol=1e-15)
+    assert np.allclose(Kn * np.linalg.norm(K, axis=-1, keepdims=True), K, rtol=1e-14, atol=0)
+
+
+def test_chunk_cumsum_restarts_every_chunk():
+    lg = np.arange(1.0, 9.0)[None]                    # 1..8, chunks of 4
+    assert np.array_equal(O.chunk_cumsum(lg, 4), np.array([[1, 3, 6, 10, 5, 11, 18, 26.0]]))
+    rng = np.random.default_rng(42)
+    x = -rng.uniform(0, 1, (2, 3, 64))
+    g = O.chunk_cumsum(x, 16)
+    c = g.reshape(2, 3, 4, 16)
+    assert np.allclose(np.diff(c, axis=-1), x.reshape(2, 3, 4, 16)[..., 1:], rtol=0, atol=1e-15)
+    assert np.array_equal(c[..., 0], x.reshape(2, 3, 4, 16)[..., 0])
+
+
+# --------------------------------------------------------------------------- #
 # sequential correction (the comparison point of the parallel residual)
 # --------------------------------------------------------------------------- #
 @pytest.mark.parametrize("N,mask", [(1, True), (3, True), (3, False), (2, True)])
