@@ -291,6 +291,8 @@ def run_component(args, world, rank, local, dev) -> int:
     kern = args.kernel
     if kern == "forward":
         wl = Workload(B=1, H=16, T=65536, k=64, dtype="bf16")
+    elif kern == "fused_raw":                       # the headline step plus its prologue
+        wl = Workload(B=4, H=16, T=4096, k=args.k or 64, dtype="bf16")
     else:
         k = args.k or 64
         wl = Workload(B=1, H=32, T=16384, k=k, dtype="bf16")
@@ -298,7 +300,8 @@ def run_component(args, world, rank, local, dev) -> int:
     stream = torch.cuda.current_stream(dev)
     sets = []
     for r in range(args.rotate):
-        inp = make_inputs(wl, seed=shard_seed(rank, r), with_q=(kern == "forward"))
+        inp = make_inputs(wl, seed=shard_seed(rank, r), with_q=(kern == "forward"),
+                          raw_keys=(kern == "fused_raw"))
         st = {key: v.to(dev) for key, v in inp.items()}
         st["A"] = torch.empty(wl.B, wl.H, wl.T // k, k, k, device=dev)
         st["T"] = torch.empty_like(st["A"])
@@ -306,7 +309,7 @@ def run_component(args, world, rank, local, dev) -> int:
             gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
         if kern == "wy":
             gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
-        if kern in ("wy", "forward"):
+        if kern in ("wy", "forward", "fused_raw"):
             st["W"] = torch.empty_like(st["K"])
             st["U"] = torch.empty_like(st["V"])
         if kern == "forward":
@@ -321,6 +324,9 @@ def run_component(args, world, rank, local, dev) -> int:
         if kern == "neumann":
             gdn.gdn_invert_neumann(st["A"], st["T"], args.N, args.mask, args.S, gdn.GDN_PREC_F16,
                                    stream=stream)
+        elif kern == "fused_raw":
+            gdn.gdn_chunk_wy_fused_raw(st["K"], st["V"], st["beta"], st["loggate"], args.N,
+                                       args.mask, args.S, 0, st["W"], st["U"], k=k, stream=stream)
         elif kern == "newton":
             gdn.gdn_invert_newton(st["A"], st["T"], args.N, args.mask, args.M, stream=stream)
         elif kern == "fwdsub":
@@ -362,6 +368,8 @@ def run_component(args, world, rank, local, dev) -> int:
     per = {
         "neumann": (2 * kk2, chain),
         "newton": (2 * kk2, (args.N - 1 + 2 * args.M) * 2 * k ** 3),
+        "fused_raw": (algorithmic_bytes_per_chunk(k, d, 2),
+                      algorithmic_flops_per_chunk(k, d, args.N, args.S)),
         "fwdsub": (2 * kk2, 2 * k ** 3 // 6),
         "int8": (2 * kk2, (args.N - 1) * 2 * k ** 3),
         "build_A": (kd + 8 * k + kk2, 2 * k * k * d),
@@ -509,8 +517,8 @@ def main(argv=None) -> int:
     ap.add_argument("--S", type=int, default=WORKLOAD["S"], help="residual steps")
     ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
     ap.add_argument("--kernel", default="fused",
-                    choices=["fused", "neumann", "newton", "fwdsub", "int8", "build_A", "wy",
-                             "forward", "decode"],
+                    choices=["fused", "fused_raw", "neumann", "newton", "fwdsub", "int8",
+                             "build_A", "wy", "forward", "decode"],
                     help="time one component instead of the fused step (not the headline)")
     ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")
     ap.add_argument("--batch", type=int, default=64, help="sequences per --kernel decode step")

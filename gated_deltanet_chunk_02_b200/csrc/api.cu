@@ -210,6 +210,28 @@ int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta, const fl
                     "chunk_wy_fused");
 }
 
+int gdn_chunk_wy_fused_raw(const void* K_raw, const void* V, const float* beta,
+                           const float* loggate, int N, int mask, int S, int gated, void* W,
+                           void* U, float* T_out, void* K_out, float* g_out, gdn_shape s,
+                           gdn_dtype dtype, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_dtype(dtype));
+    GDN_TRY(check_NS(N, mask, S, s.k));
+    if (dtype != GDN_BF16) return fail(GDN_ERR_UNSUPPORTED, "the prologue is built for bf16 data");
+    if (s.k == 256) return fail(GDN_ERR_UNSUPPORTED, "the fused step supports k <= 128");
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{K_raw, "K_raw"}, {V, "V"}, {beta, "beta"}, {loggate, "loggate"},
+                        {W, "W"}, {U, "U"}}));
+    GDN_TRY(check_opt_ptr(T_out, "T_out"));
+    GDN_TRY(check_opt_ptr(K_out, "K_out"));
+    GDN_TRY(check_opt_ptr(g_out, "g_out"));
+    if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
+    return launched(gdn::launch_fused_raw_tc(K_raw, V, beta, loggate, N, mask, S, gated, W, U,
+                                             T_out, K_out, g_out, nc, s.k, (cudaStream_t)stream),
+                    "fused with prologue (tcgen05)");
+}
+
 int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype) {
     int64_t nc;
     if (check_shape(s, &nc) != GDN_OK) return -1;

@@ -43,10 +43,12 @@ constexpr int kRows = 128;                       // rows per tile
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr int kStatusSmemAlign = 2;              // dynamic shared memory not 1024-aligned
 
-enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3, kNewton = 4 };
+enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3, kNewton = 4, kFusedRaw = 5 };
 
-__host__ __device__ constexpr bool uses_K(int m) { return m == kFused || m == kBuildA || m == kWY; }
-__host__ __device__ constexpr bool uses_V(int m) { return m == kFused || m == kWY; }
+// the fused step, on prepared inputs or with the prologue (raw K, per-token log-gates)
+__host__ __device__ constexpr bool is_fused(int m) { return m == kFused || m == kFusedRaw; }
+__host__ __device__ constexpr bool uses_K(int m) { return is_fused(m) || m == kBuildA || m == kWY; }
+__host__ __device__ constexpr bool uses_V(int m) { return is_fused(m) || m == kWY; }
 // the standalone inverses: A in by TMA (staged a tile ahead), T out by TMA
 __host__ __device__ constexpr bool inv_only(int m) { return m == kNeumann || m == kNewton; }
 __host__ __device__ constexpr int block_of(int kc) { return kc < 64 ? 64 : kc; }
@@ -57,7 +59,7 @@ template <int KB, int MODE>
 struct SlotLayout {
     static constexpr int kK = uses_K(MODE) ? kRows * kD * 2 : 0;        // bf16 [2][128][64]
     static constexpr int kV = uses_V(MODE) ? kRows * kD * 2 : 0;
-    static constexpr int kAop = (MODE == kFused || inv_only(MODE)) ? kRows * KB * 2 : 0;
+    static constexpr int kAop = (is_fused(MODE) || inv_only(MODE)) ? kRows * KB * 2 : 0;
     static constexpr int kXY = (MODE == kBuildA) ? 0 : kRows * KB * 2;  // 16-bit [KB/64][128][64]
     static constexpr int offK = 0;
     static constexpr int offV = offK + kK;
@@ -254,6 +256,13 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 u) {
                  "r"(u.z), "r"(u.w)
                  : "memory");
 }
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 u;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+                 : "r"(addr));
+    return u;
+}
 __device__ __forceinline__ void sts16(uint32_t addr, uint16_t v) {
     asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -399,6 +408,8 @@ struct Params {
     float* Aout;         // kBuildA
     float* Tout;         // kFused (optional), kNeumann, kNewton
     int M;               // kNewton: sequential correction steps
+    __nv_bfloat16* Kout; // kFusedRaw (optional): the L2-normalised K
+    float* gout;         // kFusedRaw (optional): the chunk-local cumulative log-gates
     int* status;
 };
 
@@ -548,7 +559,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     // barrier and issuing thread, and their products are M = 128, N = 64 (the
     // other block's rows come out as unused values), so the two blocks' rounds
     // interleave on the SM instead of waiting for each other.
-    constexpr bool kSplit = (NCH == 2) && (MODE == kFused || inv_only(MODE));
+    constexpr bool kSplit = (NCH == 2) && (is_fused(MODE) || inv_only(MODE));
     const int cg = kSplit ? blk : 0;
     const bool cleader = kSplit ? (lane == 0 && (warp % 8) == 2 * cg) : leader;
     const int cbar = kSplit ? 3 + 2 * s + cg : bar_id;
@@ -703,7 +714,69 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         bar_sync(bar_id, 256);
         if (*(volatile int*)&ctrl->abort) { ok = false; break; }
 
-        if (MODE == kFused || MODE == kBuildA) {
+        if (is_fused(MODE) || MODE == kBuildA) {
+            if constexpr (MODE == kFusedRaw) {
+                // ---- prologue: K rows to unit L2 norm (in place, bf16) and the
+                // per-token log-gates to chunk-local cumulative sums ----
+                // Here lane l of the slot's warp w takes row 16 w + l / 2, panel
+                // (64 columns) l % 2: its 64 values stay in registers, the two
+                // halves' sums of squares (fp32) meet by one shuffle, and the
+                // panel is rescaled in place; an all-zero row (past the end of
+                // the data) stays zero.
+                {
+                    const int pr = 16 * (warp & 7) + (lane >> 1), pn = lane & 1;
+                    const uint32_t rb = su32(sK) + pn * (kRows * 128) + pr * 128;
+                    uint32_t w[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 u = lds128(rb + ((c ^ (pr & 7)) << 4));
+                        w[4 * c] = u.x; w[4 * c + 1] = u.y; w[4 * c + 2] = u.z; w[4 * c + 3] = u.w;
+                    }
+                    float ss = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {                 // bf16 pair -> two floats
+                        const float lo = __uint_as_float(w[e] << 16);
+                        const float hi = __uint_as_float(w[e] & 0xffff0000u);
+                        ss = fmaf(lo, lo, ss);
+                        ss = fmaf(hi, hi, ss);
+                    }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    const float inv = ss > 0.f ? rsqrtf(ss) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        w[e] = pack_b2(__uint_as_float(w[e] << 16) * inv,
+                                       __uint_as_float(w[e] & 0xffff0000u) * inv);
+                    const int64_t gr = row0 + pr;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 u = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+                        sts128(rb + ((c ^ (pr & 7)) << 4), u);
+                        if (p.Kout && gr < p.rows)
+                            *reinterpret_cast<uint4*>(p.Kout + gr * kD + pn * 64 + c * 8) = u;
+                    }
+                }
+                // warp 0 of the slot: inclusive sums of the log-gates, restarted
+                // every KC rows (lane l owns rows 4l .. 4l + 3)
+                if ((warp & 7) == 0) {
+                    const float4 x = *reinterpret_cast<const float4*>(sg + 4 * lane);
+                    float y0 = x.x, y1 = y0 + x.y, y2 = y1 + x.z, y3 = y2 + x.w;
+                    constexpr int seg = KC / 4;            // lanes per chunk
+                    float run = y3;
+#pragma unroll
+                    for (int o = 1; o < seg; o <<= 1) {
+                        const float up = __shfl_up_sync(0xffffffffu, run, o);
+                        if ((lane % seg) >= o) run += up;
+                    }
+                    const float before = run - y3;        // this chunk's lanes before lane
+                    y0 += before; y1 += before; y2 += before; y3 += before;
+                    *reinterpret_cast<float4*>(sg + 4 * lane) = make_float4(y0, y1, y2, y3);
+                    if (p.gout && row0 + 4 * lane < p.rows)
+                        *reinterpret_cast<float4*>(p.gout + row0 + 4 * lane) =
+                            make_float4(y0, y1, y2, y3);
+                }
+                fence_async_smem();                       // the rescaled K feeds the MMAs
+                bar_sync(bar_id, 256);
+            }
             // ---- G = K K^T over the tile, then A = -beta_i G_ij exp(g_i - g_j) ----
             if (leader) {
                 tc_fence_after();
@@ -825,8 +898,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             }
         }
 
-        if (MODE == kFused) release_staging(n);
-        if (MODE == kFused || inv_only(MODE)) {
+        if (is_fused(MODE)) release_staging(n);
+        if (is_fused(MODE) || inv_only(MODE)) {
             // ---- truncated Neumann series in Horner form ----
             // X_1 = I + M.A, X_n = I + M.(X_{n-1} A), T0 = X_N: inside the band
             // X_{n-1} A reads only in-band entries of X_{n-1}, so masking every
@@ -1190,7 +1263,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             }
         }
 
-        if (MODE == kFused || MODE == kWY) {
+        if (is_fused(MODE) || MODE == kWY) {
             // ---- WY: T diag(beta [exp g]) -> X (bf16), T diag(beta) -> Y ----
             release_staging(n);
             const float* bcol = sb + blk * KB;
@@ -2329,6 +2402,28 @@ cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, con
     io.W = W;
     io.U = U;
     return tcg::dispatch<tcg::kFused, 1>(k, io, p, st);
+}
+
+cudaError_t launch_fused_raw_tc(const void* K, const void* V, const float* beta,
+                                const float* loggate, int N, int mask, int S, int gated, void* W,
+                                void* U, float* Tout, void* Kout, float* gout, int64_t nc, int k,
+                                cudaStream_t st) {
+    tcg::Params p = tcg::base_params(nc, k);
+    p.N = N;
+    p.mask = mask;
+    p.S = S;
+    p.gated = gated;
+    p.Tout = Tout;
+    p.Kout = static_cast<__nv_bfloat16*>(Kout);
+    p.gout = gout;
+    tcg::IO io;
+    io.K = K;
+    io.V = V;
+    io.beta = beta;
+    io.g = loggate;
+    io.W = W;
+    io.U = U;
+    return tcg::dispatch<tcg::kFusedRaw, 1>(k, io, p, st);
 }
 
 }  // namespace gdn

@@ -24,7 +24,7 @@ GDN_OK, GDN_ERR_ARG, GDN_ERR_ALIGN, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_T
 
 EXPORTS = [
     "gdn_build_A", "gdn_invert_neumann", "gdn_invert_newton", "gdn_invert_fwdsub", "gdn_wy",
-    "gdn_invert_neumann_i8", "gdn_chunk_wy_fused", "gdn_forward",
+    "gdn_invert_neumann_i8", "gdn_chunk_wy_fused", "gdn_chunk_wy_fused_raw", "gdn_forward",
     "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_decode", "gdn_get_status",
     "gdn_last_error", "gdn_launch_count",
 ]
@@ -66,6 +66,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gdn_wy": [_P, _P, _P, _P, _P, _P, _P, S, _I, _P],
         "gdn_invert_neumann_i8": [_P, _P, _I, _I, _P, _P, _P, S, _P],
         "gdn_chunk_wy_fused": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, S, _I, _P],
+        "gdn_chunk_wy_fused_raw": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, S, _I,
+                                   _P],
         "gdn_forward": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I64, S, _I, _P],
         "gdn_forward_workspace_bytes": [S, _I],
         "gdn_forward_static": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, S, _I, _P],
@@ -166,6 +168,16 @@ def gdn_chunk_wy_fused(K, V, beta, g, N, mask, S, gated, W, U, T=None, k=64, str
     _check(load().gdn_chunk_wy_fused(_ptr(K), _ptr(V), _ptr(beta), _ptr(g), N, int(mask), S,
                                      int(gated), _ptr(W), _ptr(U), _ptr(T), shape_of(K, k),
                                      _dtype(K), _stream(stream)))
+
+
+def gdn_chunk_wy_fused_raw(K_raw, V, beta, loggate, N, mask, S, gated, W, U, T=None,
+                           K_out=None, g_out=None, k=64, stream=None):
+    """The fused step from raw keys (normalised in the kernel) and per-token
+    log-gates (summed chunk-locally in the kernel)."""
+    _check(load().gdn_chunk_wy_fused_raw(_ptr(K_raw), _ptr(V), _ptr(beta), _ptr(loggate), N,
+                                         int(mask), S, int(gated), _ptr(W), _ptr(U), _ptr(T),
+                                         _ptr(K_out), _ptr(g_out), shape_of(K_raw, k),
+                                         _dtype(K_raw), _stream(stream)))
 
 
 def gdn_forward_workspace_bytes(K, k):

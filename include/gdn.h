@@ -152,6 +152,21 @@ int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta,
                        gdn_dtype dtype, void* stream);
 
 /*
+ * gdn_chunk_wy_fused with its prologue fused in: the steps just before A in a
+ * layer.  K_raw rows are L2-normalised, k_i <- k_i / ||k_i|| (norm in fp32, the
+ * result rounded to bf16; an all-zero row stays zero), and loggate holds each
+ * token's own log-gate, summed chunk-locally into g (g_i includes token i),
+ * inside the kernel before K K^T.  Everything else is gdn_chunk_wy_fused.
+ * Optional outputs (NULL to skip): K_out [B,H,T,d] bf16, the normalised keys;
+ * g_out [B,H,T] f32, the cumulative log-gates (what a later scan reads).
+ * bf16 data, k in {32, 64, 128}.
+ */
+int gdn_chunk_wy_fused_raw(const void* K_raw, const void* V, const float* beta,
+                           const float* loggate, int N, int mask, int S, int gated, void* W,
+                           void* U, float* T_out, void* K_out, float* g_out, gdn_shape s,
+                           gdn_dtype dtype, void* stream);
+
+/*
  * Full chunk-wise Gated DeltaNet forward.  Per chunk: V~ = U - W_g S0^T,
  * O = diag(exp g) Q S0^T + (Q K^T . Gamma . L) V~,
  * S' = exp(g_last) S0 + V~^T diag(exp(g_last - g)) K, with

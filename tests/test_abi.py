@@ -128,6 +128,19 @@ def test_empty_inputs_are_noops(lib):
     assert lib.gdn_launch_count() == n0
 
 
+def test_prologue_limits(lib):
+    args = [P(FAKE)] * 4
+    outs = [P(FAKE), P(FAKE), None, None, None]
+    assert lib.gdn_chunk_wy_fused_raw(*args, 3, 1, 8, 0, *outs, sh(), 0, None) == \
+        gdn.GDN_ERR_UNSUPPORTED                                  # float32 data
+    assert lib.gdn_chunk_wy_fused_raw(*args, 3, 1, 8, 0, *outs, sh(T=512, k=256), 1, None) == \
+        gdn.GDN_ERR_UNSUPPORTED
+    bad = [P(FAKE), P(FAKE), None, P(MISALIGNED), None]
+    assert lib.gdn_chunk_wy_fused_raw(*args, 3, 1, 8, 0, *bad, sh(), 1, None) == gdn.GDN_ERR_ALIGN
+    assert lib.gdn_chunk_wy_fused_raw(*[None] * 4, 3, 1, 8, 0, *[None] * 5, sh(B=0), 1,
+                                      None) == gdn.GDN_OK
+
+
 def test_newton_limits(lib):
     assert lib.gdn_invert_newton(P(FAKE), P(FAKE), sh(), 3, 1, 7, None) == gdn.GDN_ERR_ARG
     assert lib.gdn_invert_newton(P(FAKE), P(FAKE), sh(), 0, 1, 2, None) == gdn.GDN_ERR_ARG
