@@ -38,7 +38,7 @@ __all__ = [
     "to_chunks", "from_chunks", "l2_normalize_rows", "chunk_cumsum", "band_mask", "build_A",
     "invert_fwdsub",
     "neumann_powers_sum", "invert_neumann", "invert_newton", "residual_matrix", "wy",
-    "int8_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
+    "int8_neumann", "int16_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
 ]
 
 
@@ -310,6 +310,65 @@ def int8_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:
     for n in range(N):
         T = (T + (scale[:, n, None, None] * q[:, n].astype(f32)).astype(f32)).astype(f32)
     return {"q": q, "acc": acc, "scale": scale, "T": T}
+
+
+def int16_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:
+    """INT16 truncated Neumann series with symmetric per-chunk scales.
+
+    "When Good Enough Is Optimal", Adaptation à la Quantification: the INT16
+    operating point beside INT8.  Same steps as ``int8_neumann`` with codes in
+    [-32767, 32767]; products of two code matrices reach 2^36, beyond float32's
+    exact integers, so the accumulators are int64 and every scale operation is
+    IEEE binary64 (round to nearest even, no fused multiply-add):
+
+      1. P_1 = M (.) A;  a = max |P_1|;  r = 32767 / double(a);
+         q_1 = clamp(rint(double(P_1) * r), -32767, 32767);  s_1 = double(a) / 32767;
+      2. for n = 2..N: acc_n = q_{n-1} q_1 (exact int64), masked;
+         m_n = max |acc_n|;  r_n = 32767 / double(m_n);
+         q_n = clamp(rint(double(acc_n) * r_n), -32767, 32767);
+         s_n = (s_{n-1} * s_1) * (double(m_n) / 32767);
+      3. a zero maximum gives q = 0 and s = 0;
+      4. T^(0) = I + sum_{n=1}^{N} s_n * double(q_n), summed in binary64 in the
+         order n = 1..N, then rounded once to float32.
+
+    ``A32`` float32 ``[nc, k, k]``.  Returns ``q`` (int16 ``[nc, N, k, k]``),
+    ``acc`` (int64, slot 0 zero), ``scale`` (float64 ``[nc, N]``) and ``T``
+    (float32).
+    """
+    if N < 1:
+        raise ValueError("the INT16 path needs N >= 1")
+    A32 = np.asarray(A32)
+    if A32.dtype != np.float32:
+        raise TypeError("A32 must be float32")
+    nc, k, _ = A32.shape
+    M = band_mask(k, N).astype(bool) if mask else np.ones((k, k), dtype=bool)
+
+    def quantise(x: np.ndarray, xmax: np.ndarray) -> np.ndarray:
+        # x float64 [nc,k,k], xmax float64 [nc] (> 0 where used)
+        safe = np.where(xmax > 0, xmax, 1.0)
+        r = 32767.0 / safe
+        q = np.clip(np.rint(x * r[:, None, None]), -32767, 32767).astype(np.int16)
+        return np.where((xmax > 0)[:, None, None], q, np.int16(0))
+
+    q = np.zeros((nc, N, k, k), np.int16)
+    acc = np.zeros((nc, N, k, k), np.int64)
+    scale = np.zeros((nc, N), np.float64)
+    A1 = np.where(M, A32, np.float32(0.0)).astype(np.float64)   # P_1 = M (.) A
+    amax = np.abs(A1).reshape(nc, -1).max(axis=1)
+    q[:, 0] = quantise(A1, amax)
+    scale[:, 0] = np.where(amax > 0, amax / 32767.0, 0.0)
+    q1 = q[:, 0].astype(np.int64)
+    for n in range(1, N):
+        prod = np.where(M, q[:, n - 1].astype(np.int64) @ q1, 0)     # exact
+        acc[:, n] = prod
+        m = np.abs(prod).reshape(nc, -1).max(axis=1)
+        mf = m.astype(np.float64)                                   # exact: m < 2^53
+        q[:, n] = quantise(prod.astype(np.float64), mf)
+        scale[:, n] = np.where(m > 0, (scale[:, n - 1] * scale[:, 0]) * (mf / 32767.0), 0.0)
+    T = np.broadcast_to(np.eye(k), (nc, k, k)).copy()
+    for n in range(N):
+        T = T + scale[:, n, None, None] * q[:, n].astype(np.float64)
+    return {"q": q, "acc": acc, "scale": scale, "T": T.astype(np.float32)}
 
 
 # --------------------------------------------------------------------------- #

@@ -528,6 +528,61 @@ def test_int8_scale_recursion_exact_integers():
     np.testing.assert_allclose(r["T"][0], np.eye(k) + A[0] + deq, rtol=1e-6, atol=1e-3)
 
 
+def test_int16_codes_and_int64_accumulators():
+    k, N = 16, 4
+    K, _, beta, g, _ = random_chunks(3, k, 16, seed=14, gate_scale=0.2)
+    A32 = O.build_A(K, beta, g).astype(np.float32)
+    dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+    for mask in (False, True):
+        r = O.int16_neumann(A32, N, mask)
+        q, acc = r["q"], r["acc"]
+        assert q.min() >= -32767 and q.max() <= 32767
+        assert np.any(np.abs(q[:, 0]) == 32767)
+        for n in range(1, N):
+            for c in range(3):
+                for i in range(k):
+                    for j in range(k):
+                        want = sum(int(q[c, n - 1, i, l]) * int(q[c, 0, l, j]) for l in range(k))
+                        if mask and dist[i, j] > N:
+                            want = 0
+                        assert int(acc[c, n, i, j]) == want
+                # the code of the largest accumulator is +-32767
+                assert np.abs(q[c, n]).max() in (0, 32767)
+        if mask:
+            assert np.all(q[:, :, dist > N] == 0)
+
+
+def test_int16_rounding_and_scale_by_hand():
+    A = np.zeros((1, 4, 4), np.float32)
+    A[0, 1, 0] = 32767.0                 # r = 1 exactly: the codes are rint of the entries
+    A[0, 2, 0] = 2.5
+    A[0, 2, 1] = -1.5
+    A[0, 3, 2] = 1000.5
+    r = O.int16_neumann(A, 2, False)
+    assert r["q"][0, 0, 1, 0] == 32767
+    assert r["q"][0, 0, 2, 0] == 2 and r["q"][0, 0, 2, 1] == -2 and r["q"][0, 0, 3, 2] == 1000
+    assert r["scale"][0, 0] == 1.0
+    # A^2 by hand: (2,0) += 0, (3,1) = 1000 * -2, (3,0) = 1000 * 2, (2,0) = -2 * 32767
+    A2 = np.zeros((4, 4), np.int64)
+    A2[2, 0] = -2 * 32767
+    A2[3, 0] = 1000 * 2
+    A2[3, 1] = 1000 * -2
+    assert np.array_equal(r["acc"][0, 1], A2)
+    assert r["scale"][0, 1] == 1.0 * 1.0 * (2 * 32767 / 32767.0)
+    assert r["q"][0, 1, 2, 0] == -32767 and r["q"][0, 1, 3, 0] == 1000
+
+
+def test_int16_dequantised_much_closer_than_int8():
+    k, N = 64, 3
+    K, _, beta, g, _ = random_chunks(6, k, 128, seed=15)
+    A32 = O.build_A(K, beta, g).astype(np.float32)
+    for mask in (False, True):
+        ref = O.invert_neumann(A32.astype(np.float64), N, mask, 0)
+        e16 = O.rel_fro(O.int16_neumann(A32, N, mask)["T"], ref)
+        e8 = O.rel_fro(O.int8_neumann(A32, N, mask)["T"], ref)
+        assert e16 <= 1e-4 and e16 < e8 / 50
+
+
 def test_int8_dequantised_close_to_float64():
     k, N = 64, 3
     K, _, beta, g, _ = random_chunks(8, k, 128, seed=13)
