@@ -186,6 +186,24 @@ int gdn_invert_neumann_i8(const float* A, float* T, int N, int mask, int8_t* q_d
                     "neumann_i8");
 }
 
+int gdn_invert_neumann_i16(const float* A, float* T, int N, int mask, int16_t* q_dbg,
+                           int64_t* acc_dbg, double* scale_dbg, gdn_shape s, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    if (s.k != 64) return fail(GDN_ERR_UNSUPPORTED, "the INT16 path is built for k = 64");
+    if (N < 1 || N > 8) return fail(GDN_ERR_ARG, "INT16 Neumann order N=%d outside [1, 8]", N);
+    if (mask != 0 && mask != 1) return fail(GDN_ERR_ARG, "mask must be 0 or 1");
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    GDN_TRY(check_opt_ptr(q_dbg, "q"));
+    GDN_TRY(check_opt_ptr(acc_dbg, "acc"));
+    GDN_TRY(check_opt_ptr(scale_dbg, "scale"));
+    if (!gdn::tc_i8_available()) return fail(GDN_ERR_UNSUPPORTED, "integer tensor-core path not built");
+    return launched(gdn::launch_neumann_i16_tc(A, T, N, mask, q_dbg, acc_dbg, scale_dbg, nc,
+                                               (cudaStream_t)stream),
+                    "neumann int16 (tcgen05)");
+}
+
 int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta, const float* g, int N,
                        int mask, int S, int gated, void* W, void* U, float* T_out, gdn_shape s,
                        gdn_dtype dtype, void* stream) {

@@ -1692,6 +1692,341 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
 }
 
 // ------------------------------------------------------------------------- //
+// INT16 truncated Neumann series (k = 64): int16 codes through 8-bit products
+// ------------------------------------------------------------------------- //
+// The INT16 scheme of gdn.h: codes in [-32767, 32767], accumulators exact in
+// int64, every scale operation in IEEE binary64.  The tensor cores multiply
+// 8-bit codes, so each product of two code matrices is assembled from bytes.
+// With the offset code q' = q + 32768 = 256 h + l (h, l unsigned bytes),
+//   sum_l q'_a q'_b = 65536 HH + 256 (HL + LH) + LL
+// takes three accumulators of unsigned x unsigned kind::i8 products (HL and
+// LH share one), and
+//   sum_l q_a q_b = sum_l q'_a q'_b - 32768 (R_a + C_b) + 64 * 32768^2
+// with R_a the row sums of q'_a and C_b the column sums of q'_b (64 terms per
+// chunk).  Every intermediate is an exact integer, so codes, accumulators,
+// scales and T match the oracle bit for bit.  One slot of 8 warps per CTA
+// (the three accumulators take 384 of the SM's 512 TMEM columns), A staged
+// by TMA one tile ahead.
+struct ParamsI16 {
+    int64_t rows;
+    int ntiles;
+    int N, mask;
+    const float* A;
+    float* T;
+    int16_t* q;
+    int64_t* acc;
+    double* scale;
+    int* status;
+};
+
+constexpr int kI16Op = kRows * 128;                  // 16 KB: 128 rows x 64 byte codes
+constexpr int kI16B = 64 * 128;                      // 8 KB: 64 rows x 128 byte codes
+constexpr int kI16Stage = kRows * 64 * 4;            // 32 KB: the next tile's A
+constexpr int kI16Smem = 2 * kI16Op + 2 * kI16B + kI16Stage;
+
+// 32 byte codes -> two 16-byte groups of a 128-byte swizzled row
+__device__ __forceinline__ void st_u8x32(uint8_t* buf, int row, int q0, const uint32_t (&b)[32]) {
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int e = 16 * g + 4 * k;
+            w[k] = b[e] | (b[e + 1] << 8) | (b[e + 2] << 16) | (b[e + 3] << 24);
+        }
+        const int q = q0 + g;
+        *reinterpret_cast<uint4*>(buf + row * 128 + (((q & 7) ^ (row & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+__device__ __forceinline__ int quant_i16(double x, double r) {
+    double y = rint(__dmul_rn(x, r));
+    y = fmin(fmax(y, -32767.0), 32767.0);
+    return (int)y;
+}
+
+__global__ void __launch_bounds__(256, 1)
+k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
+    constexpr int KC = 64;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((su32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    struct __align__(8) CtrlI16 {
+        uint64_t mma;
+        uint64_t full;                             // the staged A landed
+        uint32_t tmem;
+        int abort;
+        float red_f[2][4];
+        long long red_l[2][4];
+        int rsum[kRows][2];                        // row sums of the left operand's q'
+        int csum[2][64];                           // column sums of q'_1, per chunk
+    };
+    uint8_t* sAh = smem;
+    uint8_t* sAl = sAh + kI16Op;
+    uint8_t* sBh = sAl + kI16Op;
+    uint8_t* sBl = sBh + kI16B;
+    uint8_t* sStage = sBl + kI16B;
+    CtrlI16* ctrl = reinterpret_cast<CtrlI16*>(smem + kI16Smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&ctrl->mma, 1);
+        mbar_init(&ctrl->full, 1);
+        ctrl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tmem_alloc(&ctrl->tmem, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = ctrl->tmem;
+
+    const int h = warp / 4;
+    const int r = ((warp & 3) << 5) | lane;
+    const int c = r / KC;                          // chunk of this row in the tile
+    const int i = r % KC;
+    const int wq = ((warp & 3) & 1) * 2 + h;       // this warp's slot among its chunk's 4 warps
+    const int jmin = p.mask ? i - p.N : -KC;
+    const uint32_t tD = tm + ((uint32_t)((warp & 3) * 32) << 16) + c * KC + 32 * h;
+    const bool leader = warp == 0 && lane == 0;
+    uint32_t mma_phase = 0;
+    bool ok = true;
+
+    auto chunk_max_f = [&](float v) {
+        for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) ctrl->red_f[c][wq] = v;
+        __syncthreads();
+        return fmaxf(fmaxf(ctrl->red_f[c][0], ctrl->red_f[c][1]),
+                     fmaxf(ctrl->red_f[c][2], ctrl->red_f[c][3]));
+    };
+    auto chunk_max_l = [&](long long v) {
+        for (int o = 16; o; o >>= 1) {
+            const long long w = __shfl_xor_sync(0xffffffffu, v, o);
+            v = v > w ? v : w;
+        }
+        if (lane == 0) ctrl->red_l[c][wq] = v;
+        __syncthreads();
+        long long m = ctrl->red_l[c][0];
+#pragma unroll
+        for (int k = 1; k < 4; ++k) m = m > ctrl->red_l[c][k] ? m : ctrl->red_l[c][k];
+        return m;
+    };
+    // offset codes q' = q + 32768 as high and low bytes; row sum of this half-row
+    auto split = [&](const int (&q)[32], uint32_t (&hb)[32], uint32_t (&lb)[32]) {
+        int sum = 0;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            const uint32_t o = (uint32_t)(q[jj] + 32768);
+            hb[jj] = o >> 8;
+            lb[jj] = o & 0xffu;
+            sum += (int)o;
+        }
+        return sum;
+    };
+    int a_issued = 0;
+    auto issue_a = [&](int n) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (tile >= p.ntiles) return;
+        ++a_issued;
+        mbar_expect_tx(&ctrl->full, kI16Stage);
+        tma_load_2d(sStage, &mA, 0, tile * kRows, &ctrl->full);
+        tma_load_2d(sStage + 16384, &mA, 32, tile * kRows, &ctrl->full);
+    };
+    if (leader) issue_a(0);
+
+    for (int n = 0;; ++n) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (tile >= p.ntiles) break;
+        const int64_t grow = (int64_t)tile * kRows + r;
+        const bool valid = grow < p.rows;
+        const int64_t cidx = grow / KC, rin = grow % KC;
+        if (!mbar_wait(&ctrl->full, (uint32_t)(n & 1))) {
+            atomicExch(&ctrl->abort, 1);
+            raise_status(p.status, kStatusTimeout);
+        }
+        float a[32];                                // rows past the end were zero-filled
+        {
+            const uint32_t rb = su32(sStage) + (uint32_t)(h * 16384 + r * 128);
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4) {
+                const uint4 u = lds128(rb + ((c4 ^ (r & 7)) << 4));
+                a[4 * c4] = __uint_as_float(u.x);
+                a[4 * c4 + 1] = __uint_as_float(u.y);
+                a[4 * c4 + 2] = __uint_as_float(u.z);
+                a[4 * c4 + 3] = __uint_as_float(u.w);
+            }
+        }
+        fence_async_smem();
+        __syncthreads();                           // the previous tile's operand reads are done
+        if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+        if (leader) issue_a(n + 1);
+        float amax = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            if (32 * h + jj < jmin) a[jj] = 0.f;   // P_1 = M . A
+            amax = fmaxf(amax, fabsf(a[jj]));
+        }
+        amax = chunk_max_f(amax);
+        const double r1 = amax > 0.f ? __ddiv_rn(32767.0, (double)amax) : 0.0;
+        const double s1 = amax > 0.f ? __ddiv_rn((double)amax, 32767.0) : 0.0;
+        int q[32];
+        double t[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+            q[jj] = amax > 0.f ? quant_i16((double)a[jj], r1) : 0;
+            t[jj] = __dadd_rn(i == 32 * h + jj ? 1.0 : 0.0, __dmul_rn(s1, (double)q[jj]));
+        }
+        {
+            uint32_t hb[32], lb[32];
+            ctrl->rsum[r][h] = split(q, hb, lb);
+            st_u8x32(sAh, r, 2 * h, hb);           // q'_1 as the left operand
+            st_u8x32(sAl, r, 2 * h, lb);
+            st_u8x32(sBh, i, 4 * c + 2 * h, hb);   // and as the right operand
+            st_u8x32(sBl, i, 4 * c + 2 * h, lb);
+            // column sums of q'_1 over the chunk's 64 rows: the two warps of
+            // this chunk and half reduce 32 columns each by recursive halving
+            int v[32];
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) v[jj] = q[jj] + 32768;
+#pragma unroll
+            for (int sh = 16; sh >= 1; sh >>= 1) {
+                const bool up = (lane & sh) != 0;
+#pragma unroll
+                for (int k = 0; k < sh; ++k) {
+                    const int send = up ? v[k] : v[k + sh];
+                    const int keep = up ? v[k + sh] : v[k];
+                    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+                }
+            }
+            // lane holds column 32 h + lane summed over this warp's 32 rows
+            if ((warp & 1) == 0) ctrl->csum[c][32 * h + lane] = v[0];
+            __syncthreads();
+            if ((warp & 1) == 1) ctrl->csum[c][32 * h + lane] += v[0];
+        }
+        if (valid) {
+            const int64_t base = (cidx * p.N * KC + rin) * KC + 32 * h;
+            if (p.q) {
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 4)
+                    *reinterpret_cast<short4*>(p.q + base + jj) =
+                        make_short4((short)q[jj], (short)q[jj + 1], (short)q[jj + 2], (short)q[jj + 3]);
+            }
+            if (p.acc) {
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 2)
+                    *reinterpret_cast<longlong2*>(p.acc + base + jj) = make_longlong2(0, 0);
+            }
+            if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N] = s1;
+        }
+        double sprev = s1;
+        for (int pw = 1; pw < p.N; ++pw) {
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();                       // operands, row and column sums written
+            tc_fence_after();
+            if (leader) {
+                constexpr uint32_t id = (2u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) |
+                                        ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+#pragma unroll
+                for (int kk = 0; kk < KC / 32; ++kk) {
+                    const uint64_t ah = sdesc(su32(sAh) + kk * 32, 16, 1024);
+                    const uint64_t al = sdesc(su32(sAl) + kk * 32, 16, 1024);
+                    const uint64_t bh = sdesc(su32(sBh) + kk * 32 * 128, 16, 1024);
+                    const uint64_t bl = sdesc(su32(sBl) + kk * 32 * 128, 16, 1024);
+                    mma_i8(tm, ah, bh, id, kk > 0);                 // HH
+                    mma_i8(tm + 128, ah, bl, id, kk > 0);           // HL
+                    mma_i8(tm + 128, al, bh, id, 1);                // + LH
+                    mma_i8(tm + 256, al, bl, id, kk > 0);           // LL
+                }
+                mma_commit(&ctrl->mma);
+            }
+            bool good = mbar_wait(&ctrl->mma, mma_phase);
+            mma_phase ^= 1;
+            if (!good) {
+                atomicExch(&ctrl->abort, 1);
+                raise_status(p.status, kStatusTimeout);
+            }
+            tc_fence_after();
+            uint32_t hh[32], mm[32], ll[32];
+            tmem_ld32_async(tD, hh);
+            tmem_ld32_async(tD + 128, mm);
+            tmem_ld32_async(tD + 256, ll);
+            tmem_wait_ld();
+            const long long ra = (long long)ctrl->rsum[r][0] + ctrl->rsum[r][1];
+            long long accv[32];
+            long long m = 0;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                const long long full = 65536LL * (int)hh[jj] + 256LL * (int)mm[jj] + (long long)(int)ll[jj]
+                                       - 32768LL * (ra + ctrl->csum[c][32 * h + jj]) +
+                                       (long long)KC * 32768LL * 32768LL;
+                accv[jj] = (32 * h + jj < jmin) ? 0 : full;
+                const long long ab = accv[jj] < 0 ? -accv[jj] : accv[jj];
+                m = m > ab ? m : ab;
+            }
+            m = chunk_max_l(m);
+            if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+            const double mf = (double)m;
+            const double rn = m > 0 ? __ddiv_rn(32767.0, mf) : 0.0;
+            const double sn = m > 0 ? __dmul_rn(__dmul_rn(sprev, s1), __ddiv_rn(mf, 32767.0)) : 0.0;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                q[jj] = m > 0 ? quant_i16((double)accv[jj], rn) : 0;
+                t[jj] = __dadd_rn(t[jj], __dmul_rn(sn, (double)q[jj]));
+            }
+            if (pw + 1 < p.N) {
+                uint32_t hb[32], lb[32];
+                const int sum = split(q, hb, lb);
+                tc_fence_before();
+                __syncthreads();                   // every row sum of q'_{n-1} has been read
+                ctrl->rsum[r][h] = sum;
+                st_u8x32(sAh, r, 2 * h, hb);
+                st_u8x32(sAl, r, 2 * h, lb);
+            }
+            if (valid) {
+                const int64_t base = ((cidx * p.N + pw) * KC + rin) * KC + 32 * h;
+                if (p.q) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 4)
+                        *reinterpret_cast<short4*>(p.q + base + jj) =
+                            make_short4((short)q[jj], (short)q[jj + 1], (short)q[jj + 2], (short)q[jj + 3]);
+                }
+                if (p.acc) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; jj += 2)
+                        *reinterpret_cast<longlong2*>(p.acc + base + jj) =
+                            make_longlong2(accv[jj], accv[jj + 1]);
+                }
+                if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N + pw] = sn;
+            }
+            sprev = sn;
+        }
+        if (!ok) break;
+        if (valid) {
+            float* dst = p.T + cidx * KC * KC + rin * KC + 32 * h;
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+                reinterpret_cast<float4*>(dst)[q4] =
+                    make_float4(__double2float_rn(t[4 * q4]), __double2float_rn(t[4 * q4 + 1]),
+                                __double2float_rn(t[4 * q4 + 2]), __double2float_rn(t[4 * q4 + 3]));
+        }
+        tc_fence_before();
+    }
+    if (!ok) {
+        mbar_wait(&ctrl->mma, mma_phase);
+        if (leader && a_issued > 0) mbar_wait(&ctrl->full, (uint32_t)((a_issued - 1) & 1));
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+// ------------------------------------------------------------------------- //
 // k = 256: the truncated Neumann series on the tensor cores, S = 0
 // ------------------------------------------------------------------------- //
 // The chunk is a 2 x 2 block matrix of 128 x 128 blocks (the upper-right block
@@ -2362,6 +2697,36 @@ cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8
     const int cap = 2 * tcg::num_sms();
     const int grid = p.ntiles < cap ? p.ntiles : cap;
     tcg::k_neumann_i8_tc<<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int16_t* q,
+                                  int64_t* acc, double* sc, int64_t nc, cudaStream_t st) {
+    tcg::ParamsI16 p;
+    memset(&p, 0, sizeof p);
+    p.rows = nc * 64;
+    p.ntiles = (int)((p.rows + tcg::kRows - 1) / tcg::kRows);
+    p.N = N;
+    p.mask = mask;
+    p.A = A;
+    p.T = T;
+    p.q = q;
+    p.acc = acc;
+    p.scale = sc;
+    p.status = status_ptr();
+    CUtensorMap mA;
+    memset(&mA, 0, sizeof mA);
+    if (!tcg::map_f32(&mA, A, p.rows, 64)) return cudaErrorInvalidValue;
+    // one CTA per SM: it takes all 512 TMEM columns (the shared-memory request
+    // keeps a second CTA off the SM)
+    size_t smem = tcg::kI16Smem + 2048;
+    if (smem < 120 * 1024) smem = 120 * 1024;
+    cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i16_tc,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int sms = tcg::num_sms();
+    const int grid = p.ntiles < sms ? p.ntiles : sms;
+    tcg::k_neumann_i16_tc<<<grid, 256, smem, st>>>(mA, p);
     return cudaGetLastError();
 }
 

@@ -141,6 +141,24 @@ int gdn_invert_neumann_i8(const float* A, float* T, int N, int mask,
                           gdn_shape s, void* stream);
 
 /*
+ * INT16 truncated Neumann series ("Adaptation à la Quantification", the INT16
+ * operating point): as gdn_invert_neumann_i8 with codes in [-32767, 32767].
+ * Products of two code matrices reach 2^36, so accumulators are exact int64
+ * and every scale operation is IEEE binary64 (round to nearest even, no FMA):
+ *   P1 = M.A; a = max|P1|; q1 = clamp(rint(double(P1) * (32767/double(a))), +-32767);
+ *   s1 = double(a)/32767; acc_n = q_{n-1} q1 (masked); m = max|acc_n|;
+ *   q_n = clamp(rint(double(acc_n) * (32767/double(m))), +-32767);
+ *   s_n = (s_{n-1} * s1) * (double(m)/32767); zero maxima give q = 0, s = 0;
+ *   T0 = I + s_1 q_1 + ... + s_N q_N summed left to right in binary64, then
+ *   rounded once to float32.
+ * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.  Optional debug outputs (NULL to
+ * skip): q [nc,N,k,k] int16, acc [nc,N,k,k] int64 (slot 0 zero), scale
+ * [nc,N] f64.  k = 64, 1 <= N <= 8.
+ */
+int gdn_invert_neumann_i16(const float* A, float* T, int N, int mask, int16_t* q_dbg,
+                           int64_t* acc_dbg, double* scale_dbg, gdn_shape s, void* stream);
+
+/*
  * Fused per-chunk pipeline: A from K, beta, g; T by the Neumann + mask +
  * residual method (as gdn_invert_neumann); then W, U (gated W if gated != 0).
  * Only K, V, beta, g are read and only W, U (and T when T_out is non-NULL)

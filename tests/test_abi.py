@@ -128,6 +128,17 @@ def test_empty_inputs_are_noops(lib):
     assert lib.gdn_launch_count() == n0
 
 
+def test_int16_limits(lib):
+    assert lib.gdn_invert_neumann_i16(P(FAKE), P(FAKE), 3, 1, None, None, None, sh(k=128),
+                                      None) == gdn.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_invert_neumann_i16(P(FAKE), P(FAKE), 9, 1, None, None, None, sh(),
+                                      None) == gdn.GDN_ERR_ARG
+    assert lib.gdn_invert_neumann_i16(P(FAKE), P(FAKE), 3, 1, None, P(MISALIGNED), None, sh(),
+                                      None) == gdn.GDN_ERR_ALIGN
+    assert lib.gdn_invert_neumann_i16(None, None, 3, 1, None, None, None, sh(B=0),
+                                      None) == gdn.GDN_OK
+
+
 def test_prologue_limits(lib):
     args = [P(FAKE)] * 4
     outs = [P(FAKE), P(FAKE), None, None, None]

@@ -188,6 +188,54 @@ def test_fused_without_T_output_matches():
 # --------------------------------------------------------------------------- #
 # INT8
 # --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("N", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("mask", [0, 1])
+def test_int16_bit_exact(N, mask):
+    """INT16 codes (byte-split products), int64 accumulators, binary64 scales
+    and T, bit for bit against the oracle; 67 chunks (a ragged last tile)."""
+    w = Workload(B=1, H=1, T=67 * 64, k=64, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=17), w)
+    nc = A32.shape[0]
+    Ad = to_dev(A_tensor(A32, w))
+    T = torch.empty_like(Ad)
+    q = torch.empty(nc, N, 64, 64, dtype=torch.int16, device="cuda")
+    acc = torch.empty(nc, N, 64, 64, dtype=torch.int64, device="cuda")
+    sc = torch.empty(nc, N, dtype=torch.float64, device="cuda")
+    gdn.gdn_invert_neumann_i16(Ad, T, N, mask, q, acc, sc)
+    check_status()
+    r = O.int16_neumann(A32, N, bool(mask))
+    np.testing.assert_array_equal(q.cpu().numpy(), r["q"])
+    np.testing.assert_array_equal(acc.cpu().numpy(), r["acc"])
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint64), r["scale"].view(np.uint64))
+    np.testing.assert_array_equal(T.cpu().numpy().reshape(nc, 64, 64).view(np.uint32),
+                                  r["T"].view(np.uint32))
+    T2 = torch.empty_like(Ad)
+    gdn.gdn_invert_neumann_i16(Ad, T2, N, mask)
+    check_status()
+    assert torch.equal(T, T2)
+
+
+def test_int16_extreme_codes():
+    """Entries at +-amax and sign flips: the byte split must carry codes of
+    +-32767 and the int64 accumulators reach ~2^36."""
+    rng = np.random.default_rng(19)
+    nc = 6
+    A32 = np.tril(rng.choice([-1.0, 1.0], (nc, 64, 64)), -1).astype(np.float32)
+    A32[:, 1:, 0] = 1.0                                      # a full column at the maximum
+    Ad = torch.from_numpy(A32).reshape(1, 1, nc, 64, 64).cuda()
+    for N, mask in [(2, 0), (3, 0), (3, 1)]:
+        T = torch.empty_like(Ad)
+        acc = torch.empty(nc, N, 64, 64, dtype=torch.int64, device="cuda")
+        gdn.gdn_invert_neumann_i16(Ad, T, N, mask, None, acc, None)
+        check_status()
+        r = O.int16_neumann(A32, N, bool(mask))
+        np.testing.assert_array_equal(acc.cpu().numpy(), r["acc"])
+        np.testing.assert_array_equal(T.cpu().numpy().reshape(nc, 64, 64).view(np.uint32),
+                                      r["T"].view(np.uint32))
+        if not mask:
+            assert np.abs(r["acc"]).max() > 2 ** 31        # beyond int32
+
+
 @pytest.mark.parametrize("N", [1, 2, 3, 4])
 @pytest.mark.parametrize("mask", [0, 1])
 def test_int8_bit_exact(N, mask):
