@@ -1085,10 +1085,12 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         }
                     }
                 } else {
-                    // Horner with stride 2: Q_1 = E, E^2 = E E, F = E + E^2,
-                    // Q_{m+2} = F + Q_m E^2, and Q_{m+1} = E + Q_m E when one
-                    // step is left; Q_m (no identity) is the left operand in
-                    // TMEM, E in X, E^2 then Q_S in Y, F in TMEM as fp16.
+                    // Horner with stride 2: Q_1 = E, E^2 = E E, F = E + E^2 = Q_2,
+                    // Q_{m+2} = F + Q_m E^2, from Q_2 when S is even and from Q_1
+                    // when it is odd, so no single step is left over (S = 8
+                    // takes E^2, Q_4, Q_6, Q_8); Q_m (no identity) is the left
+                    // operand in TMEM, E in X, E^2 then Q_S in Y, F in TMEM as
+                    // fp16.
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         float t[32];
@@ -1155,14 +1157,17 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             } else {
 #pragma unroll
                                 for (int jj = 0; jj < 32; ++jj)
-                                    if (!in_chunk(pc * 32 + jj)) v[jj] = 0.f;
+                                    if (!in_chunk(pc * 32 + jj)) v[jj] = e[jj] = 0.f;
                                 st_op32<false>(sY, r, pc, v);               // E^2
                                 tmem_st_h16(tF + pc * 16, e);             // F
+                                if (p.S % 2 == 0) tmem_st_h16(tA + pc * 16, e);   // Q_2
                             }
                         }
-                        int m = 1;
+                        int m = p.S % 2 == 0 ? 2 : 1;
+                        bool first = true;
                         while (p.S >= 3 && m + 2 <= p.S) {
-                            cpublish(m == 1);
+                            cpublish(first);
+                            first = false;
                             cchain_t(sY);                                // Q_m E^2
                             if (!cwait()) { ok = false; break; }
                             m += 2;
@@ -1185,21 +1190,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             }
                         }
                         if (!ok) break;
-                        if (p.S >= 3 && m < p.S) {                          // one step left
-                            cpublish(false);
-                            cchain_t(sX);                                // Q_m E
-                            if (!cwait()) { ok = false; break; }
-#pragma unroll
-                            for (int pp = 0; pp < PPT; ++pp) {
-                                const int pc = pc0 + pp;
-                                float v[32], e[32];
-                                tmem_ld32(tD + pc * 32, v);
-                                e_row(pc, e);
-#pragma unroll
-                                for (int jj = 0; jj < 32; ++jj) v[jj] += e[jj];     // Q_S
-                                finish_q(pp, v);
-                            }
-                        }
                     }
                     cpublish(true);
                     cchain_t(sY);                                        // T0 Q_S
