@@ -344,6 +344,33 @@ def test_chunk_cumsum_restarts_every_chunk():
 
 
 # --------------------------------------------------------------------------- #
+# block-decomposition inverse (the other comparison point)
+# --------------------------------------------------------------------------- #
+def test_blocked_inverse_is_exact():
+    K, _, beta, g, _ = random_chunks(3, 64, 32, seed=34)
+    A = O.build_A(K, beta, g)
+    for base in (16, 8, 4):
+        T = O.invert_blocked(A, base)
+        assert np.allclose((np.eye(64) - A) @ T, np.eye(64), rtol=0, atol=1e-13)
+        assert np.allclose(T, O.invert_fwdsub(A), rtol=0, atol=1e-13)
+
+
+def test_blocked_inverse_exact_rationals_4x4():
+    """base 1 on a 4 x 4 chunk: every step is the 2 x 2 block formula; checked
+    against the exact rational inverse."""
+    rng = np.random.default_rng(35)
+    A = np.tril(rng.integers(-4, 5, (4, 4)), -1).astype(np.float64) / 4.0
+    T = O.invert_blocked(A[None], 1)[0]
+    L = frac_matrix(np.eye(4) - A)
+    # exact inverse of the unit lower-triangular L by forward substitution in rationals
+    Tq = [[Fraction(int(i == j)) for j in range(4)] for i in range(4)]
+    for i in range(4):
+        for j in range(i):
+            Tq[i][j] = -sum((L[i][l] * Tq[l][j] for l in range(j, i)), Fraction(0))
+    assert all(Fraction(float(T[i][j])) == Tq[i][j] for i in range(4) for j in range(4))
+
+
+# --------------------------------------------------------------------------- #
 # sequential correction (the comparison point of the parallel residual)
 # --------------------------------------------------------------------------- #
 @pytest.mark.parametrize("N,mask", [(1, True), (3, True), (3, False), (2, True)])
