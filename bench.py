@@ -305,7 +305,7 @@ def run_component(args, world, rank, local, dev) -> int:
         st = {key: v.to(dev) for key, v in inp.items()}
         st["A"] = torch.empty(wl.B, wl.H, wl.T // k, k, k, device=dev)
         st["T"] = torch.empty_like(st["A"])
-        if kern in ("neumann", "newton", "fwdsub", "int8", "int16", "wy"):
+        if kern in ("neumann", "newton", "blocked", "fwdsub", "int8", "int16", "wy"):
             gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
         if kern == "wy":
             gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
@@ -331,6 +331,8 @@ def run_component(args, world, rank, local, dev) -> int:
             gdn.gdn_invert_newton(st["A"], st["T"], args.N, args.mask, args.M, stream=stream)
         elif kern == "fwdsub":
             gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
+        elif kern == "blocked":
+            gdn.gdn_invert_blocked(st["A"], st["T"], stream=stream)
         elif kern == "int8":
             gdn.gdn_invert_neumann_i8(st["A"], st["T"], args.N, args.mask, stream=stream)
         elif kern == "int16":
@@ -373,6 +375,7 @@ def run_component(args, world, rank, local, dev) -> int:
         "fused_raw": (algorithmic_bytes_per_chunk(k, d, 2),
                       algorithmic_flops_per_chunk(k, d, args.N, args.S)),
         "fwdsub": (2 * kk2, 2 * k ** 3 // 6),
+        "blocked": (2 * kk2, 4 * 2 * k ** 3),
         "int8": (2 * kk2, (args.N - 1) * 2 * k ** 3),
         "int16": (2 * kk2, (args.N - 1) * 2 * k ** 3),
         "build_A": (kd + 8 * k + kk2, 2 * k * k * d),
@@ -520,7 +523,8 @@ def main(argv=None) -> int:
     ap.add_argument("--S", type=int, default=WORKLOAD["S"], help="residual steps")
     ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
     ap.add_argument("--kernel", default="fused",
-                    choices=["fused", "fused_raw", "neumann", "newton", "fwdsub", "int8", "int16",
+                    choices=["fused", "fused_raw", "neumann", "newton", "blocked", "fwdsub", "int8",
+                             "int16",
                              "build_A", "wy", "forward", "decode"],
                     help="time one component instead of the fused step (not the headline)")
     ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")

@@ -142,6 +142,17 @@ int gdn_invert_newton(const float* A, float* T, gdn_shape s, int N, int mask, in
                     "newton (tcgen05)");
 }
 
+int gdn_invert_blocked(const float* A, float* T, gdn_shape s, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    if (s.k > 64) return fail(GDN_ERR_UNSUPPORTED, "the block-decomposition inverse supports k <= 64");
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
+    return launched(gdn::launch_blockinv_tc(A, T, nc, s.k, (cudaStream_t)stream),
+                    "blocked inverse (tcgen05)");
+}
+
 int gdn_invert_fwdsub(const float* A, float* T, gdn_shape s, void* stream) {
     int64_t nc;
     GDN_TRY(check_shape(s, &nc));

@@ -43,14 +43,17 @@ constexpr int kRows = 128;                       // rows per tile
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr int kStatusSmemAlign = 2;              // dynamic shared memory not 1024-aligned
 
-enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3, kNewton = 4, kFusedRaw = 5 };
+enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3, kNewton = 4, kFusedRaw = 5,
+            kBlockInv = 6 };
 
 // the fused step, on prepared inputs or with the prologue (raw K, per-token log-gates)
 __host__ __device__ constexpr bool is_fused(int m) { return m == kFused || m == kFusedRaw; }
 __host__ __device__ constexpr bool uses_K(int m) { return is_fused(m) || m == kBuildA || m == kWY; }
 __host__ __device__ constexpr bool uses_V(int m) { return is_fused(m) || m == kWY; }
 // the standalone inverses: A in by TMA (staged a tile ahead), T out by TMA
-__host__ __device__ constexpr bool inv_only(int m) { return m == kNeumann || m == kNewton; }
+__host__ __device__ constexpr bool inv_only(int m) {
+    return m == kNeumann || m == kNewton || m == kBlockInv;
+}
 __host__ __device__ constexpr int block_of(int kc) { return kc < 64 ? 64 : kc; }
 
 // Per-slot shared-memory layout (bytes).  The 1024-byte aligned operand
@@ -837,6 +840,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             }
         } else if (inv_only(MODE)) {
             // ---- A rows from the staged tile ----
+            float av[32];                                  // kBlockInv: this thread's A piece
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
@@ -859,15 +863,20 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
                 }
-                st_op32<false>(sX, r, pc, v);
-                float t[32];
+                if constexpr (MODE == kBlockInv) {
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int j = pc * 32 + jj;
-                    t[jj] = eye(j) + (j >= jmin ? v[jj] : 0.f);       // X_1 = I + M.A
+                    for (int jj = 0; jj < 32; ++jj) av[jj] = v[jj];
+                } else {
+                    st_op32<false>(sX, r, pc, v);
+                    float t[32];
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = pc * 32 + jj;
+                        t[jj] = eye(j) + (j >= jmin ? v[jj] : 0.f);       // X_1 = I + M.A
+                    }
+                    if (p.N == 1) t0_put(pp, t, T0);
+                    else tmem_st_h16(tA + pc * 16, t);
                 }
-                if (p.N == 1) t0_put(pp, t, T0);
-                else tmem_st_h16(tA + pc * 16, t);
             }
             // the stage is read: it takes the slot's next tile; the previous
             // tile's T store has read the Aop / Y staging before it is reused
@@ -875,6 +884,42 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             if (leader) bulk_wait_read();
             bar_sync(bar_id, 256);
             if (leader) issue_k(n + NS);
+            if constexpr (MODE == kBlockInv && KB == 64) {
+                // ---- exact inverse by 2 x 2 block decomposition: the 16 x 16
+                // diagonal blocks by substitution, then per doubling level
+                // T <- T + T (A_L T), A_L = A on that level's off-diagonal
+                // blocks.  Row i's diagonal block b = i / 16 lies in piece
+                // b / 2 (warp-uniform); its 16 rows are 16 lanes of one warp.
+                const int b16 = i >> 4;
+                const bool diag = (b16 >> 1) == h;
+                float d[16];
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) d[cc] = cc == (i & 15) ? 1.f : 0.f;
+                if (diag) {
+                    // T = I + A T inside the block, row j final before it is used;
+                    // rows l <= j add A[l][j] = 0
+                    const int base = lane & 16;
+#pragma unroll
+                    for (int j = 0; j < 15; ++j) {
+                        const float aij = (b16 & 1) ? av[16 + j] : av[j];
+#pragma unroll
+                        for (int cc = 0; cc < 16; ++cc)
+                            d[cc] = fmaf(aij, __shfl_sync(0xffffffffu, d[cc], base + j), d[cc]);
+                    }
+                }
+                float b1[32], a1[32], a2[32];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const float dj = (b16 & 1) ? (jj >= 16 ? d[jj & 15] : 0.f) : (jj < 16 ? d[jj & 15] : 0.f);
+                    b1[jj] = diag ? dj : 0.f;
+                    a1[jj] = (diag && (b16 & 1) && jj < 16) ? av[jj] : 0.f;   // block (2p+1, 2p)
+                    a2[jj] = (KC == 64 && i >= 32 && h == 0) ? av[jj] : 0.f;  // block (1, 0) of 32s
+                }
+                st_op32<false>(sX, r, pc0, a1);
+                st_op32<false>(sY, r, pc0, b1);
+                st_op32<false>(sAop, r, pc0, a2);
+                t0_put(0, b1, T0);
+            }
         } else {
             // ---- kWY: T row from global memory ----
             release_staging(n);
@@ -933,7 +978,32 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             // lockstep rounds and wider epilogues cost more than the two rounds
             // it saves); at k = 128 a doubling with two products per round lost
             // to Horner, its extra k^3 products outweighing the rounds.
-            if constexpr (MODE == kNewton) {
+            if constexpr (MODE == kBlockInv && KB == 64) {
+                // level 1 (16 -> 32): A1 in X, T in Y; level 2 (32 -> 64): A2 in Aop
+                for (int lv = 0; lv < (KC == 64 ? 2 : 1); ++lv) {
+                    cpublish(true);
+                    cchain(lv == 0 ? sX : sAop, sY);                     // P = A_L T
+                    if (!cwait()) { ok = false; break; }
+                    {
+                        float v[32];
+                        tmem_ld32(tD + pc0 * 32, v);
+                        st_op32<false>(sX, r, pc0, v);
+                    }
+                    cpublish(true);
+                    cchain(sY, sX);                                      // T P
+                    if (!cwait()) { ok = false; break; }
+                    {
+                        float v[32], t[32];
+                        tmem_ld32(tD + pc0 * 32, v);
+                        t0_get(0, t, T0);
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) t[jj] += v[jj];
+                        t0_put(0, t, T0);
+                        if (lv == 0) st_op32<false>(sY, r, pc0, t);
+                    }
+                }
+                if (!ok) break;
+            } else if constexpr (MODE == kNewton) {
                 // Sequential correction, the form the method's parallel residual
                 // replaces: R_m = I - (I - A) T_m = I - T_m + A T_m and
                 // T_{m+1} = T_m + T_m R_m, two dependent products per step.
@@ -2634,6 +2704,18 @@ cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N
     p.mask = mask;
     p.S = S;
     return tcg::dispatch<tcg::kNeumann, 1>(k, tcg::IO(), p, st);
+}
+
+cudaError_t launch_blockinv_tc(const float* A, float* T, int64_t nc, int k, cudaStream_t st) {
+    tcg::Params p = tcg::base_params(nc, k);
+    p.Ain = A;
+    p.Tout = T;
+    p.N = 1;
+    switch (k) {
+        case 32: return tcg::launch<32, tcg::kBlockInv, 2>(tcg::IO(), p, st);
+        case 64: return tcg::launch<64, tcg::kBlockInv, 2>(tcg::IO(), p, st);
+        default: return cudaErrorNotSupported;
+    }
 }
 
 cudaError_t launch_newton_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int M,

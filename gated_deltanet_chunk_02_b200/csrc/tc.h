@@ -17,6 +17,9 @@ cudaError_t launch_build_A256_tc(const void* K, const float* beta, const float* 
                                  int64_t nc, cudaStream_t st);
 cudaError_t launch_neumann_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int S,
                               cudaStream_t st);
+// exact inverse by 2 x 2 block decomposition (16 x 16 diagonal blocks by
+// substitution, then T <- T + T (A_L T) per doubling level); k in {32, 64}
+cudaError_t launch_blockinv_tc(const float* A, float* T, int64_t nc, int k, cudaStream_t st);
 // truncated series, then M sequential correction steps T <- T + T (I - (I - A) T)
 cudaError_t launch_newton_tc(const float* A, float* T, int64_t nc, int k, int N, int mask, int M,
                              cudaStream_t st);

@@ -23,7 +23,8 @@ GDN_OK, GDN_ERR_ARG, GDN_ERR_ALIGN, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_T
     0, -1, -2, -3, -4, -5
 
 EXPORTS = [
-    "gdn_build_A", "gdn_invert_neumann", "gdn_invert_newton", "gdn_invert_fwdsub", "gdn_wy",
+    "gdn_build_A", "gdn_invert_neumann", "gdn_invert_newton", "gdn_invert_blocked",
+    "gdn_invert_fwdsub", "gdn_wy",
     "gdn_invert_neumann_i8", "gdn_invert_neumann_i16", "gdn_chunk_wy_fused", "gdn_chunk_wy_fused_raw", "gdn_forward",
     "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_decode", "gdn_get_status",
     "gdn_last_error", "gdn_launch_count",
@@ -62,6 +63,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gdn_build_A": [_P, _P, _P, _P, S, _I, _P],
         "gdn_invert_neumann": [_P, _P, S, _I, _I, _I, _I, _P],
         "gdn_invert_newton": [_P, _P, S, _I, _I, _I, _P],
+        "gdn_invert_blocked": [_P, _P, S, _P],
         "gdn_invert_fwdsub": [_P, _P, S, _P],
         "gdn_wy": [_P, _P, _P, _P, _P, _P, _P, S, _I, _P],
         "gdn_invert_neumann_i8": [_P, _P, _I, _I, _P, _P, _P, S, _P],
@@ -148,6 +150,10 @@ def gdn_invert_neumann(A, T, N, mask, S, prec=GDN_PREC_F32, stream=None):
 def gdn_invert_newton(A, T, N, mask, M, stream=None):
     _check(load().gdn_invert_newton(_ptr(A), _ptr(T), shape_of_chunks(A), N, int(mask), M,
                                     _stream(stream)))
+
+
+def gdn_invert_blocked(A, T, stream=None):
+    _check(load().gdn_invert_blocked(_ptr(A), _ptr(T), shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_invert_fwdsub(A, T, stream=None):

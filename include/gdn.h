@@ -105,6 +105,16 @@ int gdn_invert_newton(const float* A, float* T, gdn_shape s, int N, int mask, in
                       void* stream);
 
 /*
+ * Exact T = (I - A)^{-1} by 2 x 2 block decomposition, the other comparison
+ * point of "Énoncé du Problème" (block inversion): the 16 x 16 diagonal
+ * blocks by substitution, then per doubling level T <- T + T (A_L T) with
+ * A_L = A on that level's off-diagonal blocks (T10 = T11 A10 T00).  Tensor
+ * cores with fp16 operands and fp32 accumulation, like GDN_PREC_F16.
+ * k in {32, 64} (GDN_ERR_UNSUPPORTED above).  In: A [nc,k,k] f32.  Out: T f32.
+ */
+int gdn_invert_blocked(const float* A, float* T, gdn_shape s, void* stream);
+
+/*
  * Exact T = (I - A)^{-1} by forward substitution ("Énoncé du Problème": the
  * k-1 sequential row steps the method replaces).  fp32 on CUDA cores.
  * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.

@@ -152,6 +152,12 @@ def test_prologue_limits(lib):
                                       None) == gdn.GDN_OK
 
 
+def test_blocked_limits(lib):
+    assert lib.gdn_invert_blocked(P(FAKE), P(FAKE), sh(k=128), None) == gdn.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_invert_blocked(P(FAKE), P(MISALIGNED), sh(), None) == gdn.GDN_ERR_ALIGN
+    assert lib.gdn_invert_blocked(None, None, sh(B=0), None) == gdn.GDN_OK
+
+
 def test_newton_limits(lib):
     assert lib.gdn_invert_newton(P(FAKE), P(FAKE), sh(), 3, 1, 7, None) == gdn.GDN_ERR_ARG
     assert lib.gdn_invert_newton(P(FAKE), P(FAKE), sh(), 0, 1, 2, None) == gdn.GDN_ERR_ARG

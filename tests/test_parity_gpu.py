@@ -302,6 +302,26 @@ def test_newton_tensor_cores(k, N, mask, M):
     assert np.all(np.triu(T.cpu().numpy().reshape(ref.shape), 1) == 0)
 
 
+@pytest.mark.parametrize("k", [32, 64])
+@pytest.mark.parametrize("gate_scale", [1.0, 0.05])
+def test_blocked_inverse_tensor_cores(k, gate_scale):
+    """The exact block-decomposition inverse (fp16 operands) against the oracle
+    on 9 chunks (a ragged last tile); slow gates keep far entries large."""
+    w = Workload(B=1, H=3, T=3 * k, k=k, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=14, gate_scale=gate_scale), w)
+    T = torch.full((w.B, w.H, w.T // k, k, k), float("nan"), device="cuda")
+    gdn.gdn_invert_blocked(to_dev(A_tensor(A32, w)), T)
+    check_status()
+    A64 = A32.astype(np.float64)
+    ref = O.invert_blocked(A64)
+    assert np.allclose(ref, O.invert_fwdsub(A64), rtol=0, atol=1e-12)
+    assert torch.isfinite(T).all()
+    assert rel(T, ref) <= TOL_BF16
+    assert per_chunk_max_rel(T, ref) <= TOL_BF16
+    Th = T.cpu().numpy().reshape(ref.shape)
+    assert np.all(np.triu(Th, 1) == 0) and np.all(np.diagonal(Th, axis1=1, axis2=2) == 1)
+
+
 def test_newton_matches_parallel_residual_on_gpu():
     """M = 3 sequential steps and the parallel residual with S = 7 compute the
     same T (exactly so in exact arithmetic)."""
