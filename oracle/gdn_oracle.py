@@ -39,7 +39,7 @@ __all__ = [
     "invert_fwdsub",
     "neumann_powers_sum", "invert_neumann", "invert_newton", "invert_blocked", "residual_matrix",
     "wy",
-    "int8_neumann", "int16_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
+    "int8_neumann", "int8_residual", "int16_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
 ]
 
 
@@ -335,6 +335,74 @@ def int8_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:
     for n in range(N):
         T = (T + (scale[:, n, None, None] * q[:, n].astype(f32)).astype(f32)).astype(f32)
     return {"q": q, "acc": acc, "scale": scale, "T": T}
+
+
+def int8_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
+    """INT8 series followed by the parallel residual correction, every product
+    an int8 product ("When Good Enough Is Optimal", Adaptation à la
+    Quantification: N = 3 compensated by S = 8 residual steps; Méthodologie
+    §3 for E and T = T^(0) sum E^s).  The pages fix neither how E is formed
+    nor the precision of the last product; this reading keeps every matrix
+    product in int8 codes with the rules of ``int8_neumann`` (per-chunk
+    symmetric scales, int32 accumulators, IEEE float32 without FMA, round to
+    nearest even, zero maxima give zero codes and scales):
+
+      1. T^(0) from ``int8_neumann``; X = T^(0) - I (exact: T^(0)_ii = 1);
+      2. codes of the whole A (no mask) and of X: (q_A, s_A), (q_X, s_X);
+         E = (A - X) + (s_A * s_X) * float(q_A q_X)   [= I - (I - A) T^(0)];
+      3. codes of E: (q_E1, s_E1); for s = 2..S: acc = q_E,s-1 q_E1,
+         q_E,s and s_E,s requantised as the powers of A (E is not masked);
+         Gm = sum_{s=1}^{S} s_E,s * float(q_E,s), left to right from s = 1;
+      4. codes of Gm: (q_G, s_G);
+         T = (T^(0) + Gm) + (s_X * s_G) * float(q_X q_G)   [= T^(0) (I + Gm)].
+
+    ``A32`` float32 ``[nc, k, k]``; returns T float32 ``[nc, k, k]``.
+    """
+    if S < 1:
+        raise ValueError("the residual needs S >= 1")
+    f32 = np.float32
+    A32 = np.asarray(A32)
+    if A32.dtype != np.float32:
+        raise TypeError("A32 must be float32")
+    nc, k, _ = A32.shape
+
+    def codes(x):
+        # (int64 codes, float32 scale per chunk) of a float32 [nc, k, k] array
+        amax = np.abs(x).reshape(nc, -1).max(axis=1).astype(f32)
+        safe = np.where(amax > 0, amax, f32(1.0)).astype(f32)
+        r = (f32(127.0) / safe).astype(f32)
+        q = np.clip(np.rint((x * r[:, None, None]).astype(f32)), -127, 127).astype(np.int64)
+        q = np.where((amax > 0)[:, None, None], q, 0)
+        sc = np.where(amax > 0, (amax / f32(127.0)).astype(f32), f32(0.0)).astype(f32)
+        return q, sc
+
+    def deq(sa, sb, acc):
+        # (s_a * s_b) * float(acc), float32 (|acc| < 2^24: exact in float32)
+        assert np.abs(acc).max(initial=0) < 2 ** 24
+        return ((sa * sb).astype(f32)[:, None, None] * acc.astype(f32)).astype(f32)
+
+    T0 = int8_neumann(A32, N, mask)["T"]
+    X = (T0 - np.eye(k, dtype=f32)).astype(f32)
+    qA, sA = codes(A32)
+    qX, sX = codes(X)
+    E = ((A32 - X).astype(f32) + deq(sA, sX, qA @ qX)).astype(f32)
+    qE, sE = codes(E)
+    qs, ss = qE, sE
+    Gm = (ss[:, None, None] * qs.astype(f32)).astype(f32)
+    for _ in range(2, S + 1):
+        acc = qs @ qE
+        assert np.abs(acc).max(initial=0) < 2 ** 31
+        m = np.abs(acc).reshape(nc, -1).max(axis=1)
+        mf = m.astype(f32)
+        safe = np.where(m > 0, mf, f32(1.0)).astype(f32)
+        r = (f32(127.0) / safe).astype(f32)
+        q = np.clip(np.rint((acc.astype(f32) * r[:, None, None]).astype(f32)), -127, 127)
+        qs = np.where((m > 0)[:, None, None], q.astype(np.int64), 0)
+        ss = np.where(m > 0, ((ss * sE).astype(f32) * (mf / f32(127.0)).astype(f32)).astype(f32),
+                      f32(0.0)).astype(f32)
+        Gm = (Gm + (ss[:, None, None] * qs.astype(f32)).astype(f32)).astype(f32)
+    qG, sG = codes(Gm)
+    return ((T0 + Gm).astype(f32) + deq(sX, sG, qX @ qG)).astype(f32)
 
 
 def int16_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:

@@ -555,6 +555,30 @@ def test_int8_scale_recursion_exact_integers():
     np.testing.assert_allclose(r["T"][0], np.eye(k) + A[0] + deq, rtol=1e-6, atol=1e-3)
 
 
+def test_int8_residual_tracks_the_float_formula_and_repairs_t0():
+    """The int8 residual against the same correction in float64 on the same
+    int8 T0 (E = I - (I - A) T0 and T0 sum E^s, literal powers): they differ
+    only by the quantisation of A X, E and its powers, and X Gm.  Both beat
+    the INT8 series alone by far (the pages' claim for N = 3, S = 8)."""
+    K, _, beta, g, _ = random_chunks(8, 64, 128, seed=16)
+    A32 = O.build_A(K, beta, g).astype(np.float32)
+    A64 = A32.astype(np.float64)
+    exact = O.invert_fwdsub(A64)
+    T0 = O.int8_neumann(A32, 3, True)["T"].astype(np.float64)
+    E = np.eye(64) - (np.eye(64) - A64) @ T0
+    for S in (1, 2, 8):
+        acc = np.broadcast_to(np.eye(64), E.shape).copy()
+        P = acc.copy()
+        for _ in range(S):
+            P = P @ E
+            acc = acc + P
+        Tf = T0 @ acc
+        Tq = O.int8_residual(A32, 3, True, S)
+        assert O.rel_fro(Tq, Tf) <= 5e-4
+        assert O.rel_fro(Tq, exact) <= O.rel_fro(T0, exact) / 10
+        assert np.all(np.triu(Tq, 1) == 0) and np.all(np.diagonal(Tq, axis1=1, axis2=2) == 1)
+
+
 def test_int16_codes_and_int64_accumulators():
     k, N = 16, 4
     K, _, beta, g, _ = random_chunks(3, k, 16, seed=14, gate_scale=0.2)
