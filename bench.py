@@ -305,7 +305,8 @@ def run_component(args, world, rank, local, dev) -> int:
         st = {key: v.to(dev) for key, v in inp.items()}
         st["A"] = torch.empty(wl.B, wl.H, wl.T // k, k, k, device=dev)
         st["T"] = torch.empty_like(st["A"])
-        if kern in ("neumann", "newton", "blocked", "fwdsub", "int8", "int16", "wy"):
+        if kern in ("neumann", "newton", "blocked", "fwdsub", "int8", "int8_residual", "int16",
+                    "wy"):
             gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
         if kern == "wy":
             gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
@@ -335,6 +336,9 @@ def run_component(args, world, rank, local, dev) -> int:
             gdn.gdn_invert_blocked(st["A"], st["T"], stream=stream)
         elif kern == "int8":
             gdn.gdn_invert_neumann_i8(st["A"], st["T"], args.N, args.mask, stream=stream)
+        elif kern == "int8_residual":
+            gdn.gdn_invert_neumann_i8_residual(st["A"], st["T"], args.N, args.mask, args.S,
+                                               stream=stream)
         elif kern == "int16":
             gdn.gdn_invert_neumann_i16(st["A"], st["T"], args.N, args.mask, stream=stream)
         elif kern == "build_A":
@@ -378,6 +382,7 @@ def run_component(args, world, rank, local, dev) -> int:
         "blocked": (2 * kk2, 4 * 2 * k ** 3),
         "int8": (2 * kk2, (args.N - 1) * 2 * k ** 3),
         "int16": (2 * kk2, (args.N - 1) * 2 * k ** 3),
+        "int8_residual": (2 * kk2, (args.N - 1 + args.S + 1) * 2 * k ** 3),
         "build_A": (kd + 8 * k + kk2, 2 * k * k * d),
         "wy": (kk2 + 2 * kd + 4 * k + 2 * kd, 4 * k * k * d),
         "forward": (4 * kd + 8 * k, algorithmic_flops_per_chunk(k, d, args.N, args.S)
@@ -524,7 +529,7 @@ def main(argv=None) -> int:
     ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
     ap.add_argument("--kernel", default="fused",
                     choices=["fused", "fused_raw", "neumann", "newton", "blocked", "fwdsub", "int8",
-                             "int16",
+                             "int8_residual", "int16",
                              "build_A", "wy", "forward", "decode"],
                     help="time one component instead of the fused step (not the headline)")
     ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")

@@ -197,6 +197,22 @@ int gdn_invert_neumann_i8(const float* A, float* T, int N, int mask, int8_t* q_d
                     "neumann_i8");
 }
 
+int gdn_invert_neumann_i8_residual(const float* A, float* T, int N, int mask, int S,
+                                   gdn_shape s, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    if (s.k != 64) return fail(GDN_ERR_UNSUPPORTED, "INT8 path is built for k=64");
+    if (N < 1 || N > 8) return fail(GDN_ERR_ARG, "INT8 path: N=%d outside [1, 8]", N);
+    if (mask != 0 && mask != 1) return fail(GDN_ERR_ARG, "mask must be 0 or 1");
+    if (S < 1 || S > 64) return fail(GDN_ERR_ARG, "residual steps S=%d outside [1, 64]", S);
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    if (!gdn::tc_i8_available()) return fail(GDN_ERR_UNSUPPORTED, "integer tensor-core path not built");
+    return launched(gdn::launch_neumann_i8_tc(A, T, N, mask, nullptr, nullptr, nullptr, nc,
+                                              (cudaStream_t)stream, S),
+                    "neumann_i8 with residual (tcgen05)");
+}
+
 int gdn_invert_neumann_i16(const float* A, float* T, int N, int mask, int16_t* q_dbg,
                            int64_t* acc_dbg, double* scale_dbg, gdn_shape s, void* stream) {
     int64_t nc;

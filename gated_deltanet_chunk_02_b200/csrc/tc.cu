@@ -1507,6 +1507,7 @@ struct ParamsI8 {
     int64_t rows;
     int ntiles;
     int N, mask;
+    int S;               // residual steps (the RES instance)
     const float* A;
     float* T;
     int8_t* q;
@@ -1521,6 +1522,8 @@ constexpr int kI8BBytes = 64 * 128;                // 8 KB: K = 64 rows of 128 c
 constexpr int kI8Stage = kRows * 64 * 4;           // 32 KB: the next tile's A (fp32, swizzled)
 constexpr int kI8SlotBytes = kI8OpBytes + kI8BBytes + kI8Stage;
 
+// RES: the residual correction in int8 products follows the series (S >= 1)
+template <bool RES>
 __global__ void __launch_bounds__(256 * kI8Slots, 1)
 k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
     constexpr int KC = 64;
@@ -1633,8 +1636,10 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
             const int j = 32 * h + jj;
-            if (j < jmin) a[jj] = 0.f;                 // P_1 = M . A
-            amax = fmaxf(amax, fabsf(a[jj]));
+            if constexpr (!RES) {
+                if (j < jmin) a[jj] = 0.f;             // P_1 = M . A
+            }
+            amax = fmaxf(amax, fabsf(j < jmin ? 0.f : a[jj]));
         }
         amax = chunk_max_f(amax);
         const float r1 = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
@@ -1644,7 +1649,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
             const int j = 32 * h + jj;
-            q[jj] = amax > 0.f ? quant_i8(a[jj], r1) : 0;
+            q[jj] = amax > 0.f ? quant_i8(j < jmin ? 0.f : a[jj], r1) : 0;
             t[jj] = __fadd_rn(i == j ? 1.f : 0.f, __fmul_rn(s1, (float)q[jj]));
         }
         st_i8x32(sA, r, 2 * h, q);                     // q_1 as the left operand
@@ -1730,6 +1735,121 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             sprev = sn;
         }
         if (!ok) break;
+        if constexpr (RES) {
+            // ---- residual correction, every product in int8 codes ----
+            // X = T0 - I; E = (A - X) + s_A s_X (q_A q_X); E's powers as A's;
+            // Gm = sum s_E,s q_E,s; T = (T0 + Gm) + s_X s_G (q_X q_G).
+            auto product = [&](uint32_t (&raw)[32]) -> bool {   // codes in sA, sB -> TMEM
+                fence_async_smem();
+                tc_fence_before();
+                bar_sync(bar_id, 256);
+                tc_fence_after();
+                if (leader) {
+                    constexpr uint32_t id = idesc_i8(128, 128);
+#pragma unroll
+                    for (int kk = 0; kk < KC / 32; ++kk)
+                        mma_i8(tm, sdesc(su32(sA) + kk * 32, 16, 1024),
+                               sdesc(su32(sB) + kk * 32 * 128, 16, 1024), id, kk > 0);
+                    mma_commit(&ctrl->mma[s]);
+                }
+                const bool good = mbar_wait(&ctrl->mma[s], mma_phase);
+                mma_phase ^= 1;
+                if (!good) {
+                    atomicExch(&ctrl->abort, 1);
+                    raise_status(p.status, kStatusTimeout);
+                }
+                tc_fence_after();
+                tmem_ld32_async(tD, raw);
+                tmem_wait_ld();
+                return !*(volatile int*)&ctrl->abort;
+            };
+            auto eye_f = [&](int jj) { return i == 32 * h + jj ? 1.f : 0.f; };
+            // codes of the whole A and of X
+            float ma = 0.f, mx = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                ma = fmaxf(ma, fabsf(a[jj]));
+                mx = fmaxf(mx, fabsf(__fsub_rn(t[jj], eye_f(jj))));
+            }
+            ma = chunk_max_f(ma);
+            bar_sync(bar_id, 256);                       // every warp has read ma's partials
+            mx = chunk_max_f(mx);
+            const float rA = ma > 0.f ? __fdiv_rn(127.f, ma) : 0.f;
+            const float sA_ = ma > 0.f ? __fdiv_rn(ma, 127.f) : 0.f;
+            const float rX = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
+            const float sX_ = mx > 0.f ? __fdiv_rn(mx, 127.f) : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) q[jj] = ma > 0.f ? quant_i8(a[jj], rA) : 0;
+            st_i8x32(sA, r, 2 * h, q);                              // q_A (left)
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+                q[jj] = mx > 0.f ? quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX) : 0;
+            st_i8x32(sB, i, 4 * c + 2 * h, q);                      // q_X (right)
+            uint32_t raw[32];
+            if (!product(raw)) { ok = false; break; }
+            // E, then its codes
+            const float sAX = __fmul_rn(sA_, sX_);
+            float me = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                a[jj] = __fadd_rn(__fsub_rn(a[jj], __fsub_rn(t[jj], eye_f(jj))),
+                                  __fmul_rn(sAX, (float)(int)raw[jj]));      // E over A
+                me = fmaxf(me, fabsf(a[jj]));
+            }
+            me = chunk_max_f(me);
+            const float rE = me > 0.f ? __fdiv_rn(127.f, me) : 0.f;
+            const float sE1 = me > 0.f ? __fdiv_rn(me, 127.f) : 0.f;
+            float gm[32];
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                q[jj] = me > 0.f ? quant_i8(a[jj], rE) : 0;
+                gm[jj] = __fmul_rn(sE1, (float)q[jj]);
+            }
+            float sprevE = sE1;
+            for (int sp = 2; sp <= p.S; ++sp) {
+                tc_fence_before();
+                bar_sync(bar_id, 256);                              // the last product's reads
+                st_i8x32(sA, r, 2 * h, q);                          // q_E,s-1 (left)
+                if (sp == 2) st_i8x32(sB, i, 4 * c + 2 * h, q);     // q_E1 (right)
+                if (!product(raw)) { ok = false; break; }
+                int m = 0;
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) m = max(m, abs((int)raw[jj]));
+                m = chunk_max_i(m);
+                const float mf = (float)m;
+                const float rn = m > 0 ? __fdiv_rn(127.f, mf) : 0.f;
+                const float sn = m > 0 ? __fmul_rn(__fmul_rn(sprevE, sE1), __fdiv_rn(mf, 127.f)) : 0.f;
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    q[jj] = m > 0 ? quant_i8((float)(int)raw[jj], rn) : 0;
+                    gm[jj] = __fadd_rn(gm[jj], __fmul_rn(sn, (float)q[jj]));
+                }
+                sprevE = sn;
+            }
+            if (!ok) break;
+            // codes of Gm; T = (T0 + Gm) + s_X s_G (q_X q_G)
+            float mg = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) mg = fmaxf(mg, fabsf(gm[jj]));
+            bar_sync(bar_id, 256);                       // every warp has read me's partials
+            mg = chunk_max_f(mg);
+            const float rG = mg > 0.f ? __fdiv_rn(127.f, mg) : 0.f;
+            const float sG = mg > 0.f ? __fdiv_rn(mg, 127.f) : 0.f;
+            tc_fence_before();
+            bar_sync(bar_id, 256);                                  // the last product's reads
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+                q[jj] = mx > 0.f ? quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX) : 0;
+            st_i8x32(sA, r, 2 * h, q);                              // q_X (left)
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) q[jj] = mg > 0.f ? quant_i8(gm[jj], rG) : 0;
+            st_i8x32(sB, i, 4 * c + 2 * h, q);                      // q_G (right)
+            if (!product(raw)) { ok = false; break; }
+            const float sXG = __fmul_rn(sX_, sG);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+                t[jj] = __fadd_rn(__fadd_rn(t[jj], gm[jj]), __fmul_rn(sXG, (float)(int)raw[jj]));
+        }
         if (valid) {
             float* dst = p.T + cidx * KC * KC + rin * KC + 32 * h;
 #pragma unroll
@@ -2745,9 +2865,10 @@ cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const flo
 }
 
 cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8_t* q,
-                                 int32_t* acc, float* sc, int64_t nc, cudaStream_t st) {
+                                 int32_t* acc, float* sc, int64_t nc, cudaStream_t st, int S) {
     tcg::ParamsI8 p;
     memset(&p, 0, sizeof p);
+    p.S = S;
     p.rows = nc * 64;
     p.ntiles = (int)((p.rows + tcg::kRows - 1) / tcg::kRows);
     p.N = N;
@@ -2763,12 +2884,19 @@ cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8
     if (!tcg::map_f32(&mA, A, p.rows, 64)) return cudaErrorInvalidValue;
     // two CTAs per SM at most: each holds 256 of the SM's 512 TMEM columns
     const size_t smem = tcg::kI8Slots * tcg::kI8SlotBytes + 512;
-    cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const int cap = 2 * tcg::num_sms();
     const int grid = p.ntiles < cap ? p.ntiles : cap;
-    tcg::k_neumann_i8_tc<<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
+    if (p.S > 0) {
+        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        tcg::k_neumann_i8_tc<true><<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
+    } else {
+        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        tcg::k_neumann_i8_tc<false><<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
+    }
     return cudaGetLastError();
 }
 

@@ -28,8 +28,10 @@ cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, in
                                 cudaStream_t st);
 cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const float* beta,
                          const float* g, void* W, void* U, int64_t nc, int k, cudaStream_t st);
+// S > 0: the residual correction in int8 products follows (debug outputs still
+// describe the series)
 cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8_t* q,
-                                 int32_t* acc, float* sc, int64_t nc, cudaStream_t st);
+                                 int32_t* acc, float* sc, int64_t nc, cudaStream_t st, int S = 0);
 // the fused step with its prologue: K rows L2-normalised in shared memory and
 // the per-token log-gates summed chunk-locally; optional outputs of both
 cudaError_t launch_fused_raw_tc(const void* K, const void* V, const float* beta,

@@ -25,7 +25,8 @@ GDN_OK, GDN_ERR_ARG, GDN_ERR_ALIGN, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_T
 EXPORTS = [
     "gdn_build_A", "gdn_invert_neumann", "gdn_invert_newton", "gdn_invert_blocked",
     "gdn_invert_fwdsub", "gdn_wy",
-    "gdn_invert_neumann_i8", "gdn_invert_neumann_i16", "gdn_chunk_wy_fused", "gdn_chunk_wy_fused_raw", "gdn_forward",
+    "gdn_invert_neumann_i8", "gdn_invert_neumann_i8_residual", "gdn_invert_neumann_i16",
+    "gdn_chunk_wy_fused", "gdn_chunk_wy_fused_raw", "gdn_forward",
     "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_decode", "gdn_get_status",
     "gdn_last_error", "gdn_launch_count",
 ]
@@ -68,6 +69,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gdn_wy": [_P, _P, _P, _P, _P, _P, _P, S, _I, _P],
         "gdn_invert_neumann_i8": [_P, _P, _I, _I, _P, _P, _P, S, _P],
         "gdn_invert_neumann_i16": [_P, _P, _I, _I, _P, _P, _P, S, _P],
+        "gdn_invert_neumann_i8_residual": [_P, _P, _I, _I, _I, S, _P],
         "gdn_chunk_wy_fused": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, S, _I, _P],
         "gdn_chunk_wy_fused_raw": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, S, _I,
                                    _P],
@@ -169,6 +171,11 @@ def gdn_wy(T, K, V, beta, g, W, U, stream=None):
 def gdn_invert_neumann_i8(A, T, N, mask, q=None, acc=None, scale=None, stream=None):
     _check(load().gdn_invert_neumann_i8(_ptr(A), _ptr(T), N, int(mask), _ptr(q), _ptr(acc),
                                         _ptr(scale), shape_of_chunks(A), _stream(stream)))
+
+
+def gdn_invert_neumann_i8_residual(A, T, N, mask, S, stream=None):
+    _check(load().gdn_invert_neumann_i8_residual(_ptr(A), _ptr(T), N, int(mask), S,
+                                                 shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_invert_neumann_i16(A, T, N, mask, q=None, acc=None, scale=None, stream=None):

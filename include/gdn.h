@@ -151,6 +151,21 @@ int gdn_invert_neumann_i8(const float* A, float* T, int N, int mask,
                           gdn_shape s, void* stream);
 
 /*
+ * INT8 series followed by the parallel residual correction with every product
+ * in int8 codes ("Adaptation à la Quantification": N = 3 compensated by S = 8;
+ * "Méthodologie" §3 for E and T = T0 sum_{s<=S} E^s).  After the series of
+ * gdn_invert_neumann_i8, with the same quantisation rules (codes(x): per-chunk
+ * a = max|x|, q = clamp(rint(x * (127/a)), +-127), s = a/127; float32, no FMA):
+ *   X = T0 - I;  E = (A - X) + (s_A * s_X) * float(q_A q_X)   (whole A, no mask);
+ *   q_E1 = codes(E); q_E,s, s_E,s for s = 2..S requantised as the powers of A;
+ *   Gm = s_E1 q_E1 + ... + s_E,S q_E,S (left to right);
+ *   T = (T0 + Gm) + (s_X * s_G) * float(q_X q_G),  q_G = codes(Gm).
+ * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.  k = 64, 1 <= N <= 8, 1 <= S <= 64.
+ */
+int gdn_invert_neumann_i8_residual(const float* A, float* T, int N, int mask, int S,
+                                   gdn_shape s, void* stream);
+
+/*
  * INT16 truncated Neumann series ("Adaptation à la Quantification", the INT16
  * operating point): as gdn_invert_neumann_i8 with codes in [-32767, 32767].
  * Products of two code matrices reach 2^36, so accumulators are exact int64

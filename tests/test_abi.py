@@ -128,6 +128,13 @@ def test_empty_inputs_are_noops(lib):
     assert lib.gdn_launch_count() == n0
 
 
+def test_int8_residual_limits(lib):
+    assert lib.gdn_invert_neumann_i8_residual(P(FAKE), P(FAKE), 3, 1, 0, sh(), None) == gdn.GDN_ERR_ARG
+    assert lib.gdn_invert_neumann_i8_residual(P(FAKE), P(FAKE), 3, 1, 8, sh(k=128),
+                                              None) == gdn.GDN_ERR_UNSUPPORTED
+    assert lib.gdn_invert_neumann_i8_residual(None, None, 3, 1, 8, sh(B=0), None) == gdn.GDN_OK
+
+
 def test_int16_limits(lib):
     assert lib.gdn_invert_neumann_i16(P(FAKE), P(FAKE), 3, 1, None, None, None, sh(k=128),
                                       None) == gdn.GDN_ERR_UNSUPPORTED

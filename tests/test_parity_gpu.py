@@ -188,6 +188,27 @@ def test_fused_without_T_output_matches():
 # --------------------------------------------------------------------------- #
 # INT8
 # --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("N,mask", [(3, 1), (1, 1), (3, 0), (4, 1)])
+@pytest.mark.parametrize("S", [1, 2, 3, 8])
+def test_int8_residual_bit_exact(N, mask, S):
+    """INT8 series plus the residual in int8 products: T bit for bit against
+    the oracle on 67 chunks (a ragged last tile), and far closer to the exact
+    inverse than the series alone."""
+    w = Workload(B=1, H=1, T=67 * 64, k=64, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=18 + S), w)
+    nc = A32.shape[0]
+    Ad = to_dev(A_tensor(A32, w))
+    T = torch.empty_like(Ad)
+    gdn.gdn_invert_neumann_i8_residual(Ad, T, N, mask, S)
+    check_status()
+    ref = O.int8_residual(A32, N, bool(mask), S)
+    np.testing.assert_array_equal(T.cpu().numpy().reshape(nc, 64, 64).view(np.uint32),
+                                  ref.view(np.uint32))
+    if N == 3 and mask:
+        exact = O.invert_fwdsub(A32.astype(np.float64))
+        assert O.rel_fro(ref, exact) < O.rel_fro(O.int8_neumann(A32, N, True)["T"], exact) / 10
+
+
 @pytest.mark.parametrize("N", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("mask", [0, 1])
 def test_int16_bit_exact(N, mask):
