@@ -14,13 +14,18 @@
 // slice of S.
 //
 // bf16 data: only V~ and S' are on the serial path.  k_state_tc runs them
-// alone (tiles prefetched two chunks ahead with cp.async, the state slice
-// held as fp32 mma.sync accumulator fragments), writing V~ over U and each
+// alone (tiles fetched two chunks ahead by TMA, which one thread issues while
+// the others compute, the state slice held as fp32 mma.sync accumulator
+// fragments), writing V~ over U and each
 // chunk's start state S_c to the workspace; k_out_tc then forms O for every
 // chunk in parallel.  fp32 data: k_scan does the whole recurrence and O in
 // one pass with fp32 FMA loops.
+#include <cuda.h>
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.h"
 
 namespace gdn {
 
@@ -275,47 +280,99 @@ __device__ __forceinline__ uint32_t pack_h2f(float a, float b) {
 constexpr int kStThreads = 128;
 constexpr int kStStages = 3;
 
+// One stage: the chunk's K and W_g tiles as two 64-column panels each with the
+// 128-byte swizzle (the TMA layout), the U slice [64][16] and g [64], dense.
 struct StTile {
-    static constexpr int kPitch = kSD + 8;                     // staged bf16 row, elements
-    static constexpr int kTile = kSK * kPitch * 2;
+    static constexpr int kTile = kSK * kSD * 2;                // 16 KB, 1024-byte aligned
     static constexpr int kU = kSK * kDV * 2;
-    static constexpr int kStage = 2 * kTile + kU + kSK * 4;    // K, W_g, U slice, g
+    static constexpr int kTx = 2 * kTile + kU + kSK * 4;       // bytes the TMA brings
+    static constexpr int kStage = (kTx + 1023) / 1024 * 1024;  // K, W_g, U slice, g
 };
+// byte offset of element (row, col) of a staged [64][128] bf16 tile
+__device__ __forceinline__ uint32_t sw128(int row, int col) {
+    return (uint32_t)(((col >> 6) << 13) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) +
+                      ((col & 7) << 1));
+}
+__device__ __forceinline__ uint32_t sh32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sbar_init(uint64_t* b) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(sh32(b)) : "memory");
+}
+__device__ __forceinline__ void sbar_expect(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sh32(b)),
+                 "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool sbar_try(uint64_t* b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(sh32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// bounded (2 s of %globaltimer): false when the tiles never landed
+__device__ __forceinline__ bool sbar_wait(uint64_t* b, uint32_t parity) {
+    if (sbar_try(b, parity)) return true;
+    unsigned long long t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (sbar_try(b, parity)) return true;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > 2000000000ull) return false;
+    }
+}
+__device__ __forceinline__ void tma2d(void* dst, const CUtensorMap* m, int x, int y, uint64_t* b) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(sh32(dst)), "l"(m), "r"(x), "r"(y), "r"(sh32(b))
+        : "memory");
+}
+__device__ __forceinline__ void tma1d(void* dst, const CUtensorMap* m, int x, uint64_t* b) {
+    asm volatile(
+        "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2}], [%3];" ::"r"(sh32(dst)), "l"(m), "r"(x), "r"(sh32(b))
+        : "memory");
+}
 
-__device__ __forceinline__ void fetch_state(uint8_t* st, const __nv_bfloat16* K,
-                                            const __nv_bfloat16* Wg, const __nv_bfloat16* U,
-                                            const float* g, int64_t row0, int v0) {
-    constexpr int kPerRow = kSD / 8;
-    const __nv_bfloat16* src[2] = {K + row0 * kSD, Wg + row0 * kSD};
-#pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(st + m * StTile::kTile);
-        for (int e = threadIdx.x; e < kSK * kPerRow; e += kStThreads) {
-            const int r = e / kPerRow, c = (e % kPerRow) * 8;
-            cp_async16(dst + r * StTile::kPitch + c, src[m] + r * kSD + c);
-        }
-    }
-    __nv_bfloat16* ud = reinterpret_cast<__nv_bfloat16*>(st + 2 * StTile::kTile);
-    if (threadIdx.x < kSK * 2) {
-        const int r = threadIdx.x >> 1, c = (threadIdx.x & 1) * 8;
-        cp_async16(ud + r * kDV + c, U + (row0 + r) * kSD + v0 + c);
-    }
-    float* gd = reinterpret_cast<float*>(st + 2 * StTile::kTile + StTile::kU);
-    if (threadIdx.x < kSK / 4) cp_async16(gd + threadIdx.x * 4, g + row0 + threadIdx.x * 4);
+// thread 0: the TMA copies of one stage (chunk rows row0 .. row0 + 63)
+__device__ __forceinline__ void fetch_state(uint8_t* st, uint64_t* bar, const CUtensorMap* mK,
+                                            const CUtensorMap* mW, const CUtensorMap* mU,
+                                            const CUtensorMap* mG, int row0, int v0) {
+    // the stage's previous reads were generic; its new writes come from the async proxy
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    sbar_expect(bar, StTile::kTx);
+    tma2d(st, mK, 0, row0, bar);
+    tma2d(st + StTile::kTile / 2, mK, 64, row0, bar);
+    tma2d(st + StTile::kTile, mW, 0, row0, bar);
+    tma2d(st + StTile::kTile + StTile::kTile / 2, mW, 64, row0, bar);
+    tma2d(st + 2 * StTile::kTile, mU, v0, row0, bar);
+    tma1d(st + 2 * StTile::kTile + StTile::kU, mG, row0, bar);
 }
 
 __global__ void __launch_bounds__(kStThreads)
-k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ Wg,
-           __nv_bfloat16* __restrict__ U, const float* __restrict__ g, const float* __restrict__ S0,
-           __half* __restrict__ Sst, float* __restrict__ Sfin, int64_t nchunk) {
-    constexpr int P = StTile::kPitch;
+k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mW,
+           const __grid_constant__ CUtensorMap mU, const __grid_constant__ CUtensorMap mG,
+           __nv_bfloat16* __restrict__ U, const float* __restrict__ S0,
+           __half* __restrict__ Sst, float* __restrict__ Sfin, int64_t nchunk, int* status) {
     constexpr int P16 = ScanMma::kP16;
     constexpr int PS = ScanMma::kPS;
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((sh32(smem) & 1023u) != 0) {                // the swizzled tiles need 1024-byte alignment
+        if (threadIdx.x == 0) raise_status(status, 2);
+        return;
+    }
     // kStStages stages: the tiles of chunks ci + 1 .. ci + kStStages - 1 stream
     // in while chunk ci is used
     __half* sSh = reinterpret_cast<__half*>(smem + kStStages * StTile::kStage); // [16][136] S
     __nv_bfloat16* sVd = reinterpret_cast<__nv_bfloat16*>(sSh + kDV * PS);      // [16][72]
+    uint64_t* sbar = reinterpret_cast<uint64_t*>(sVd + kDV * P16);                // [kStStages]
     const int64_t bh = blockIdx.x;
     const int v0 = blockIdx.y * kDV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -336,11 +393,13 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
             *reinterpret_cast<uint32_t*>(sSh + v * PS + c) = pack_h2f(s0, s1);
         }
     }
-#pragma unroll
-    for (int q = 0; q < kStStages - 1; ++q) {
-        if (q < nchunk)
-            fetch_state(smem + q * StTile::kStage, K, Wg, U, g, (bh * nchunk + q) * kSK, v0);
-        cp_async_commit();
+    if (tid == 0) {
+        for (int q = 0; q < kStStages; ++q) sbar_init(&sbar[q]);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int q = 0; q < kStStages - 1; ++q)
+            if (q < nchunk)
+                fetch_state(smem + q * StTile::kStage, &sbar[q], &mK, &mW, &mU, &mG,
+                            (int)((bh * nchunk + q) * kSK), v0);
     }
 
     // Two barriers per chunk: the first makes this chunk's tiles and the
@@ -350,15 +409,18 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
     for (int64_t ci = 0; ci < nchunk; ++ci) {
         const int64_t row0 = (bh * nchunk + ci) * kSK;
         uint8_t* cur = smem + (ci % kStStages) * StTile::kStage;
-        // this chunk's group is complete; the later ones may be in flight
-        asm volatile("cp.async.wait_group %0;" ::"n"(kStStages - 2) : "memory");
+        // this chunk's stage has landed; the later ones may be in flight
+        if (!sbar_wait(&sbar[ci % kStStages], (uint32_t)((ci / kStStages) & 1))) {
+            if (tid == 0) raise_status(status, kStatusTimeout);
+            return;                                // the state is not written
+        }
         __syncthreads();
-        if (ci + kStStages - 1 < nchunk)
-            fetch_state(smem + ((ci + kStStages - 1) % kStStages) * StTile::kStage, K, Wg, U, g,
-                        row0 + (kStStages - 1) * kSK, v0);
-        cp_async_commit();                         // (possibly empty) keeps the group count
-        const __nv_bfloat16* Ks = reinterpret_cast<const __nv_bfloat16*>(cur);
-        const __nv_bfloat16* Ws = reinterpret_cast<const __nv_bfloat16*>(cur + StTile::kTile);
+        if (tid == 0 && ci + kStStages - 1 < nchunk) {
+            const int nx = (int)((ci + kStStages - 1) % kStStages);
+            fetch_state(smem + nx * StTile::kStage, &sbar[nx], &mK, &mW, &mU, &mG,
+                        (int)(row0 + (kStStages - 1) * kSK), v0);
+        }
+        const uint32_t Ksa = sh32(cur), Wsa = sh32(cur + StTile::kTile);
         const __nv_bfloat16* Us = reinterpret_cast<const __nv_bfloat16*>(cur + 2 * StTile::kTile);
         const float* gs = reinterpret_cast<const float*>(cur + 2 * StTile::kTile + StTile::kU);
         // the chunk's start state, for the output pass
@@ -381,10 +443,10 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
                 for (int i = 0; i < 4; ++i) acc[n][i] = acc2[n][i] = 0.f;
 #pragma unroll
             for (int k0 = 0; k0 < kSD; k0 += 16) {
-                const uint32_t a0 = bf2_to_h2(ld32(Ws + (mt + gr) * P + k0 + gc));
-                const uint32_t a1 = bf2_to_h2(ld32(Ws + (mt + gr + 8) * P + k0 + gc));
-                const uint32_t a2 = bf2_to_h2(ld32(Ws + (mt + gr) * P + k0 + gc + 8));
-                const uint32_t a3 = bf2_to_h2(ld32(Ws + (mt + gr + 8) * P + k0 + gc + 8));
+                const uint32_t a0 = bf2_to_h2(lds32(Wsa + sw128(mt + gr, k0 + gc)));
+                const uint32_t a1 = bf2_to_h2(lds32(Wsa + sw128(mt + gr + 8, k0 + gc)));
+                const uint32_t a2 = bf2_to_h2(lds32(Wsa + sw128(mt + gr, k0 + gc + 8)));
+                const uint32_t a3 = bf2_to_h2(lds32(Wsa + sw128(mt + gr + 8, k0 + gc + 8)));
 #pragma unroll
                 for (int n = 0; n < 2; ++n)
                     mma_f16(k0 < kSD / 2 ? acc[n] : acc2[n], a0, a1, a2, a3,
@@ -430,7 +492,7 @@ k_state_tc(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict_
                 for (int nt = 0; nt < 4; ++nt) {
                     const int n0 = 32 * warp + 8 * nt;
                     const int krow = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const uint32_t addr = (uint32_t)__cvta_generic_to_shared(Ks + krow * P + n0);
+                    const uint32_t addr = Ksa + sw128(krow, n0);
                     uint32_t b0, b1;
                     asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
                                  : "=r"(b0), "=r"(b1) : "r"(addr));
@@ -585,19 +647,70 @@ k_out_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ 
     }
 }
 
+// tensor maps of the recurrence's stages
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)ptr;
+    }
+    return fn;
+}
+// [rows, 128] bf16, box box_cols x box_rows
+static bool map_bf16_2d(CUtensorMap* m, const void* base, int64_t rows, int box_cols,
+                        int box_rows, CUtensorMapSwizzle sw) {
+    EncodeTiledFn f = encode_tiled();
+    if (!f) return false;
+    memset(m, 0, sizeof *m);
+    cuuint64_t dims[2] = {(cuuint64_t)kSD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kSD * 2};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// [rows] fp32, box box_rows
+static bool map_f32_1d(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+    EncodeTiledFn f = encode_tiled();
+    if (!f) return false;
+    memset(m, 0, sizeof *m);
+    cuuint64_t dims[1] = {(cuuint64_t)rows};
+    cuuint64_t strides[1] = {4};
+    cuuint32_t box[1] = {(cuuint32_t)box_rows};
+    cuuint32_t es[1] = {1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, const float* g,
                         const float* S0, void* O, float* Sfin, void* Sstates, int64_t BH,
                         int64_t nchunk, bool bf16, cudaStream_t st) {
     dim3 grid((unsigned)BH, kSD / kDV);
     if (bf16) {
         const size_t s1 = kStStages * StTile::kStage + (size_t)kDV * ScanMma::kPS * 2 +
-                          (size_t)kDV * ScanMma::kP16 * 2;
+                          (size_t)kDV * ScanMma::kP16 * 2 + kStStages * sizeof(uint64_t);
+        const int64_t rows = BH * nchunk * kSK;
+        CUtensorMap mK, mW, mU, mG;
+        if (!map_bf16_2d(&mK, K, rows, 64, kSK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !map_bf16_2d(&mW, Wg, rows, 64, kSK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !map_bf16_2d(&mU, U, rows, kDV, kSK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !map_f32_1d(&mG, g, rows, kSK))
+            return cudaErrorInvalidValue;
         cudaError_t e = cudaFuncSetAttribute(k_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)s1);
         if (e != cudaSuccess) return e;
-        k_state_tc<<<grid, kStThreads, s1, st>>>((const __nv_bfloat16*)K, (const __nv_bfloat16*)Wg,
-                                                 (__nv_bfloat16*)U, g, S0, (__half*)Sstates, Sfin,
-                                                 nchunk);
+        k_state_tc<<<grid, kStThreads, s1, st>>>(mK, mW, mU, mG, (__nv_bfloat16*)U, S0,
+                                                 (__half*)Sstates, Sfin, nchunk, status_ptr());
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(k_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
