@@ -341,7 +341,8 @@ __device__ __forceinline__ void tma1d(void* dst, const CUtensorMap* m, int x, ui
         : "memory");
 }
 
-// thread 0: the TMA copies of one stage (chunk rows row0 .. row0 + 63)
+// the producer warp's lane 0: the TMA copies of one stage (chunk rows row0 ..
+// row0 + 63)
 __device__ __forceinline__ void fetch_state(uint8_t* st, uint64_t* bar, const CUtensorMap* mK,
                                             const CUtensorMap* mW, const CUtensorMap* mU,
                                             const CUtensorMap* mG, int row0, int v0) {
@@ -356,7 +357,9 @@ __device__ __forceinline__ void fetch_state(uint8_t* st, uint64_t* bar, const CU
     tma1d(st + 2 * StTile::kTile + StTile::kU, mG, row0, bar);
 }
 
-__global__ void __launch_bounds__(kStThreads)
+// kStThreads compute threads (4 warps) plus one producer warp that only issues
+// the stages' TMA copies between the two barriers of each chunk step
+__global__ void __launch_bounds__(kStThreads + 32)
 k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mW,
            const __grid_constant__ CUtensorMap mU, const __grid_constant__ CUtensorMap mG,
            __nv_bfloat16* __restrict__ U, const float* __restrict__ S0,
@@ -379,6 +382,30 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     const int gr = lane >> 2, gc = (lane & 3) * 2;
     const int mt = 16 * warp;                      // token rows of this warp (V~)
 
+    if (tid == kStThreads) {
+        for (int q = 0; q < kStStages; ++q) sbar_init(&sbar[q]);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int q = 0; q < kStStages - 1; ++q)
+            if (q < nchunk)
+                fetch_state(smem + q * StTile::kStage, &sbar[q], &mK, &mW, &mU, &mG,
+                            (int)((bh * nchunk + q) * kSK), v0);
+    }
+    if (warp == kStThreads / 32) {                 // the producer warp
+        __syncthreads();                           // the barriers exist
+        for (int64_t ci = 0; ci < nchunk; ++ci) {
+            if (!sbar_wait(&sbar[ci % kStStages], (uint32_t)((ci / kStStages) & 1))) return;
+            __syncthreads();                       // stage of chunk ci - 1 is free
+            if (lane == 0 && ci + kStStages - 1 < nchunk) {
+                const int nx = (int)((ci + kStStages - 1) % kStStages);
+                fetch_state(smem + nx * StTile::kStage, &sbar[nx], &mK, &mW, &mU, &mG,
+                            (int)((bh * nchunk + ci + kStStages - 1) * kSK), v0);
+            }
+            __syncthreads();
+        }
+        return;
+    }
+    __syncthreads();                               // the barriers exist
+
     float Sacc[4][4];                              // columns 32w + 8nt + gc, rows gr, gr + 8
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
@@ -392,14 +419,6 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             Sacc[nt][2 * hh + 1] = s1;
             *reinterpret_cast<uint32_t*>(sSh + v * PS + c) = pack_h2f(s0, s1);
         }
-    }
-    if (tid == 0) {
-        for (int q = 0; q < kStStages; ++q) sbar_init(&sbar[q]);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        for (int q = 0; q < kStStages - 1; ++q)
-            if (q < nchunk)
-                fetch_state(smem + q * StTile::kStage, &sbar[q], &mK, &mW, &mU, &mG,
-                            (int)((bh * nchunk + q) * kSK), v0);
     }
 
     // Two barriers per chunk: the first makes this chunk's tiles and the
@@ -415,11 +434,6 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             return;                                // the state is not written
         }
         __syncthreads();
-        if (tid == 0 && ci + kStStages - 1 < nchunk) {
-            const int nx = (int)((ci + kStStages - 1) % kStStages);
-            fetch_state(smem + nx * StTile::kStage, &sbar[nx], &mK, &mW, &mU, &mG,
-                        (int)(row0 + (kStStages - 1) * kSK), v0);
-        }
         const uint32_t Ksa = sh32(cur), Wsa = sh32(cur + StTile::kTile);
         const __nv_bfloat16* Us = reinterpret_cast<const __nv_bfloat16*>(cur + 2 * StTile::kTile);
         const float* gs = reinterpret_cast<const float*>(cur + 2 * StTile::kTile + StTile::kU);
@@ -709,7 +723,7 @@ cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, c
         cudaError_t e = cudaFuncSetAttribute(k_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)s1);
         if (e != cudaSuccess) return e;
-        k_state_tc<<<grid, kStThreads, s1, st>>>(mK, mW, mU, mG, (__nv_bfloat16*)U, S0,
+        k_state_tc<<<grid, kStThreads + 32, s1, st>>>(mK, mW, mU, mG, (__nv_bfloat16*)U, S0,
                                                  (__half*)Sstates, Sfin, nchunk, status_ptr());
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
