@@ -296,6 +296,17 @@ __device__ __forceinline__ uint32_t sw128(int row, int col) {
 __device__ __forceinline__ uint32_t sh32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
+// four 8 x 8 b16 matrices: lanes 8j .. 8j + 7 give the row addresses of matrix j
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x4t(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                         uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
+}
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -455,17 +466,22 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             for (int n = 0; n < 2; ++n)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[n][i] = acc2[n][i] = 0.f;
+            // fragments by ldmatrix: A rows lane % 16, columns + 8 (lane / 16);
+            // B (rows of S) rows (lane % 8) + 8 (lane / 16), columns + 8 ((lane / 8) % 2)
+            const int lr = lane & 15, lc = (lane >> 4) * 8;
+            const uint32_t sbase = sh32(sSh) + (uint32_t)((((lane & 7) + ((lane >> 4) << 3)) * PS +
+                                                           ((lane >> 3) & 1) * 8) * 2);
 #pragma unroll
             for (int k0 = 0; k0 < kSD; k0 += 16) {
-                const uint32_t a0 = bf2_to_h2(lds32(Wsa + sw128(mt + gr, k0 + gc)));
-                const uint32_t a1 = bf2_to_h2(lds32(Wsa + sw128(mt + gr + 8, k0 + gc)));
-                const uint32_t a2 = bf2_to_h2(lds32(Wsa + sw128(mt + gr, k0 + gc + 8)));
-                const uint32_t a3 = bf2_to_h2(lds32(Wsa + sw128(mt + gr + 8, k0 + gc + 8)));
-#pragma unroll
-                for (int n = 0; n < 2; ++n)
-                    mma_f16(k0 < kSD / 2 ? acc[n] : acc2[n], a0, a1, a2, a3,
-                            ld32(sSh + (8 * n + gr) * PS + k0 + gc),
-                            ld32(sSh + (8 * n + gr) * PS + k0 + gc + 8));
+                uint32_t a0, a1, a2, a3, b00, b01, b10, b11;
+                ldsm_x4(Wsa + sw128(mt + lr, k0 + lc), a0, a1, a2, a3);
+                ldsm_x4(sbase + k0 * 2, b00, b01, b10, b11);
+                a0 = bf2_to_h2(a0);
+                a1 = bf2_to_h2(a1);
+                a2 = bf2_to_h2(a2);
+                a3 = bf2_to_h2(a3);
+                mma_f16(k0 < kSD / 2 ? acc[0] : acc2[0], a0, a1, a2, a3, b00, b01);
+                mma_f16(k0 < kSD / 2 ? acc[1] : acc2[1], a0, a1, a2, a3, b10, b11);
             }
 #pragma unroll
             for (int n = 0; n < 2; ++n)
@@ -496,21 +512,18 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) Sacc[nt][i] *= gl;
+            const uint32_t vbase = sh32(sVd) + (uint32_t)(((lane & 15) * P16 + (lane >> 4) * 8) * 2);
 #pragma unroll
             for (int k0 = 0; k0 < kSK; k0 += 16) {
-                const uint32_t a0 = ld32(sVd + gr * P16 + k0 + gc);
-                const uint32_t a1 = ld32(sVd + (gr + 8) * P16 + k0 + gc);
-                const uint32_t a2 = ld32(sVd + gr * P16 + k0 + gc + 8);
-                const uint32_t a3 = ld32(sVd + (gr + 8) * P16 + k0 + gc + 8);
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(vbase + k0 * 2, a0, a1, a2, a3);
+                const int krow = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int n0 = 32 * warp + 8 * nt;
-                    const int krow = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const uint32_t addr = Ksa + sw128(krow, n0);
-                    uint32_t b0, b1;
-                    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-                                 : "=r"(b0), "=r"(b1) : "r"(addr));
+                for (int nt = 0; nt < 4; nt += 2) {
+                    uint32_t b0, b1, b2, b3;             // columns n0 and n0 + 8
+                    ldsm_x4t(Ksa + sw128(krow, 32 * warp + 8 * nt + (lane >> 4) * 8), b0, b1, b2, b3);
                     mma_bf16(Sacc[nt], a0, a1, a2, a3, b0, b1);
+                    mma_bf16(Sacc[nt + 1], a0, a1, a2, a3, b2, b3);
                 }
             }
 #pragma unroll
