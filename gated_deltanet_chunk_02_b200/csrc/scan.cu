@@ -269,6 +269,10 @@ __device__ __forceinline__ uint32_t pack_h2f(float a, float b) {
     const __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t pack_b2f(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 // ---------------------------------------------------------------------------
 // bf16 forward in two kernels.  The recurrence is the only serial part, so it
@@ -384,7 +388,9 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     }
     // kStStages stages: the tiles of chunks ci + 1 .. ci + kStStages - 1 stream
     // in while chunk ci is used
-    __half* sSh = reinterpret_cast<__half*>(smem + kStStages * StTile::kStage); // [16][136] S
+    // S as bf16 (the right operand of W_g S^T, bf16 like W_g; the state itself
+    // stays fp32 in the accumulator fragments)
+    __nv_bfloat16* sSh = reinterpret_cast<__nv_bfloat16*>(smem + kStStages * StTile::kStage);
     __nv_bfloat16* sVd = reinterpret_cast<__nv_bfloat16*>(sSh + kDV * PS);      // [16][72]
     uint64_t* sbar = reinterpret_cast<uint64_t*>(sVd + kDV * P16);                // [kStStages]
     const int64_t bh = blockIdx.x;
@@ -428,7 +434,7 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             const float s1 = S0 ? S0[(bh * kSD + v0 + v) * kSD + c + 1] : 0.f;
             Sacc[nt][2 * hh] = s0;
             Sacc[nt][2 * hh + 1] = s1;
-            *reinterpret_cast<uint32_t*>(sSh + v * PS + c) = pack_h2f(s0, s1);
+            *reinterpret_cast<uint32_t*>(sSh + v * PS + c) = pack_b2f(s0, s1);
         }
     }
 
@@ -476,12 +482,8 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 uint32_t a0, a1, a2, a3, b00, b01, b10, b11;
                 ldsm_x4(Wsa + sw128(mt + lr, k0 + lc), a0, a1, a2, a3);
                 ldsm_x4(sbase + k0 * 2, b00, b01, b10, b11);
-                a0 = bf2_to_h2(a0);
-                a1 = bf2_to_h2(a1);
-                a2 = bf2_to_h2(a2);
-                a3 = bf2_to_h2(a3);
-                mma_f16(k0 < kSD / 2 ? acc[0] : acc2[0], a0, a1, a2, a3, b00, b01);
-                mma_f16(k0 < kSD / 2 ? acc[1] : acc2[1], a0, a1, a2, a3, b10, b11);
+                mma_bf16(k0 < kSD / 2 ? acc[0] : acc2[0], a0, a1, a2, a3, b00, b01);
+                mma_bf16(k0 < kSD / 2 ? acc[1] : acc2[1], a0, a1, a2, a3, b10, b11);
             }
 #pragma unroll
             for (int n = 0; n < 2; ++n)
@@ -529,9 +531,9 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int c = 32 * warp + 8 * nt + gc;
-                *reinterpret_cast<uint32_t*>(sSh + gr * PS + c) = pack_h2f(Sacc[nt][0], Sacc[nt][1]);
+                *reinterpret_cast<uint32_t*>(sSh + gr * PS + c) = pack_b2f(Sacc[nt][0], Sacc[nt][1]);
                 *reinterpret_cast<uint32_t*>(sSh + (gr + 8) * PS + c) =
-                    pack_h2f(Sacc[nt][2], Sacc[nt][3]);
+                    pack_b2f(Sacc[nt][2], Sacc[nt][3]);
             }
         }
     }
