@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import sys
 import threading
@@ -513,6 +514,60 @@ def run_decode(args, world, rank, local, dev) -> int:
     return 0
 
 
+def run_error(args, world, rank, local, dev) -> int:
+    """Approximation error of the fused step against the exact inverse on the
+    whole B=4, H=16, T=4096, k=64 bf16 workload, per Neumann order N, band mask
+    and residual order S: T from the fused kernel against forward substitution
+    (fp32), W and U against the WY factors of that exact T.  Not timed; one
+    JSON line with the table."""
+    import torch
+    from gated_deltanet_chunk_02_b200 import gdn
+    from gated_deltanet_chunk_02_b200.inputs import Workload, make_inputs
+
+    w = Workload(B=4, H=16, T=4096, k=64, d=128, dtype="bf16")
+    inp = make_inputs(w, seed=shard_seed(rank, 0), gate_scale=args.gate_scale)
+    s = {key: inp[key].to(dev) for key in ("K", "V", "beta", "g")}
+    k = w.k
+    stream = torch.cuda.current_stream(dev)
+    A = torch.empty(w.B, w.H, w.T // k, k, k, device=dev)
+    T_ex = torch.empty_like(A)
+    gdn.gdn_build_A(s["K"], s["beta"], s["g"], A, k, stream=stream)
+    gdn.gdn_invert_fwdsub(A, T_ex, stream=stream)
+    W_ex, U_ex = torch.empty_like(s["K"]), torch.empty_like(s["V"])
+    gdn.gdn_wy(T_ex, s["K"], s["V"], s["beta"], None, W_ex, U_ex, stream=stream)
+    T = torch.empty_like(A)
+    W, U = torch.empty_like(W_ex), torch.empty_like(U_ex)
+
+    def rel(x, ref):
+        x, ref = x.double(), ref.double()
+        return float((x - ref).norm() / ref.norm())
+
+    def snr(e):
+        return None if e == 0.0 else -20.0 * math.log10(e)
+
+    rows = []
+    for N in (1, 2, 3, 4):
+        for mask in (1, 0):
+            for S in (0, 8):
+                gdn.gdn_chunk_wy_fused(s["K"], s["V"], s["beta"], s["g"], N, mask, S, 0, W, U, T,
+                                       k=k, stream=stream)
+                torch.cuda.synchronize(dev)
+                et, ew, eu = rel(T, T_ex), rel(W, W_ex), rel(U, U_ex)
+                worst = float(((T - T_ex).double().flatten(3).norm(dim=-1)
+                               / T_ex.double().flatten(3).norm(dim=-1)).max())
+                rows.append({"N": N, "mask": mask, "S": S, "T_rel_fro": et, "T_snr_db": snr(et),
+                             "T_worst_chunk": worst, "W_rel_fro": ew, "U_rel_fro": eu})
+    assert gdn.gdn_get_status(stream) == gdn.GDN_OK
+    if rank == 0:
+        print(json.dumps({"metric": "fused step: error against the exact inverse",
+                          "config": {"workload": f"B={w.B} H={w.H} T={w.T} k={k} d={w.d} bf16, "
+                                                 f"log-gate scale {args.gate_scale}",
+                                     "chunks": w.n_chunks},
+                          "reference": "forward substitution (fp32) and its WY factors",
+                          "table": rows}), flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -530,12 +585,14 @@ def main(argv=None) -> int:
     ap.add_argument("--kernel", default="fused",
                     choices=["fused", "fused_raw", "neumann", "newton", "blocked", "fwdsub", "int8",
                              "int8_residual", "int16",
-                             "build_A", "wy", "forward", "decode"],
+                             "build_A", "wy", "forward", "decode", "error"],
                     help="time one component instead of the fused step (not the headline)")
     ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")
     ap.add_argument("--batch", type=int, default=64, help="sequences per --kernel decode step")
     ap.add_argument("--M", type=int, default=3, help="sequential correction steps (--kernel newton)")
     ap.add_argument("--tokens", type=int, default=1, help="tokens per --kernel decode call")
+    ap.add_argument("--gate-scale", type=float, default=1.0,
+                    help="log-gate scale of the --kernel error inputs (0.05: slow decay)")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="input/output sets cycled through the timed steps")
     args = ap.parse_args(argv)
@@ -558,6 +615,8 @@ def main(argv=None) -> int:
     dev = torch.device("cuda", local)
     if args.kernel == "decode":
         return run_decode(args, world, rank, local, dev)
+    if args.kernel == "error":
+        return run_error(args, world, rank, local, dev)
     if args.kernel != "fused":
         return run_component(args, world, rank, local, dev)
     w = dict(WORKLOAD, N=args.N, S=args.S, mask=args.mask)
@@ -601,6 +660,29 @@ def main(argv=None) -> int:
     ms = max_over_ranks(ms_local, world, dev)
     status = gdn.gdn_get_status(stream)
     assert status == gdn.GDN_OK, status
+
+    # The same step without the residual (S = 0), timed the same way after the
+    # headline, reported beside it: the series + mask + WY alone.
+    s0 = None
+    if w["S"] != 0 and args.steps > 0:
+        def step0(i):
+            s = sets[i % len(sets)]
+            gdn.gdn_chunk_wy_fused(s["K"], s["V"], s["beta"], s["g"], w["N"], w["mask"], 0,
+                                   w["gated"], s["W"], s["U"], None, k=k, stream=stream)
+        for i in range(args.warmup):
+            step0(i)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(args.steps):
+            step0(i)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        s0 = max_over_ranks(f0.elapsed_time(f1), world, dev) / args.steps
+        assert gdn.gdn_get_status(stream) == gdn.GDN_OK
 
     # End to end through the public API: every step copies its inputs from
     # pinned host memory, runs the fused step and copies W and U back to pinned
@@ -704,6 +786,11 @@ def main(argv=None) -> int:
                 if args.e2e_steps else None),
         "gpu_launches": launches,
     }
+    if s0 is not None:
+        line["s0"] = {"ms_per_step": s0,
+                      "value": nc * world / (s0 * 1e-3),
+                      "frac": bytes_per_launch / (s0 * 1e-3) / 1e9 / peak_gbs,
+                      "note": "same step with S=0 (no residual), timed after the headline"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, threads, _ = cpu_oracle_sample(w, args.sample_chunks)
         line["cpu_baseline"] = {"value": args.sample_chunks / dt, "unit": "chunks/s",

@@ -644,3 +644,28 @@ def test_int8_dequantised_close_to_float64():
         ref = O.invert_neumann(A32.astype(np.float64), N, mask, 0)
         # each power carries at most half a code step (1/254 of its max) of error
         assert O.rel_fro(r["T"], ref) <= 1e-2
+
+
+def test_error_table_follows_the_truncation_laws():
+    """The reported error table (``oracle/error_table.py``) on a few chunks of
+    the B=4, H=16, T=4096 workload: without the mask and residual the error of
+    T falls with every added power; the masked series is exact on its band but
+    loses the entries below it, so its error is the larger one at S = 0; the
+    residual (S = 8) leaves only rounding; W inherits T's error (W = T diag(b) K)."""
+    from oracle.error_table import error_table
+
+    res = error_table(n_chunks=6, Ns=(1, 2, 3), Ss=(0, 8))
+    err = {(r["N"], r["mask"], r["S"]): r for r in res["rows"]}
+    unmasked = [err[(N, 0, 0)]["T_rel_fro"] for N in (1, 2, 3)]
+    assert unmasked[0] > unmasked[1] > unmasked[2] > 0
+    for N in (1, 2, 3):
+        assert err[(N, 1, 0)]["T_rel_fro"] > err[(N, 0, 0)]["T_rel_fro"]
+        assert err[(N, 1, 8)]["T_rel_fro"] < 1e-12
+        assert err[(N, 0, 8)]["T_rel_fro"] < 1e-12
+        r = err[(N, 1, 0)]
+        assert 0.5 * r["T_rel_fro"] < r["W_rel_fro"] < 2.0 * r["T_rel_fro"]
+        assert r["T_worst_chunk"] >= r["T_rel_fro"] * 0.999
+        assert math.isclose(r["T_snr_db"], -20 * math.log10(r["T_rel_fro"]))
+    # the masked powers shrink with n on these fast-decaying gates
+    amax = res["amax_masked_powers"][3]
+    assert amax[0] > amax[1] > amax[2] > 0
