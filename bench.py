@@ -283,6 +283,11 @@ def workload_config(w: dict, nc: int, rotate: int = ROTATE) -> dict:
 
 
 
+# component kernels that take the series order / mask, and the residual order
+SERIES_KERNELS = ("neumann", "newton", "fused_raw", "int8", "int8_residual", "int16", "forward")
+RESIDUAL_KERNELS = ("neumann", "fused_raw", "int8_residual", "forward")
+
+
 def run_component(args, world, rank, local, dev) -> int:
     """Device-timed run of one component kernel (A, Neumann, fwdsub, INT8, WY
     or the full forward) on its own workload; same JSON keys as the headline."""
@@ -403,9 +408,10 @@ def run_component(args, world, rank, local, dev) -> int:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{kern}, B={wl.B} H={wl.H} T={wl.T} k={k} d={d} N={args.N} "
-                               f"mask={args.mask} "
-                               + (f"M={args.M}" if kern == "newton" else f"S={args.S}"),
+        "config": {"workload": f"{kern}, B={wl.B} H={wl.H} T={wl.T} k={k} d={d}"
+                               + (f" N={args.N} mask={args.mask}" if kern in SERIES_KERNELS else "")
+                               + (f" S={args.S}" if kern in RESIDUAL_KERNELS else "")
+                               + (f" M={args.M}" if kern == "newton" else ""),
                    "chunks": nc},
         "roofline": {"bound": bound, "achieved": gbs if bound == "hbm" else tfl,
                      "peak": float(peaks["hbm_gbs"]) if bound == "hbm" else float(peaks["bf16_tflops"]),
