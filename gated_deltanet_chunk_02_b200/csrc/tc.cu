@@ -1771,6 +1771,9 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
                 ma = fmaxf(ma, fabsf(a[jj]));
                 mx = fmaxf(mx, fabsf(__fsub_rn(t[jj], eye_f(jj))));
             }
+            // with N = 1 no product separates A's maximum from this one: every
+            // warp must have read A's partials before they are overwritten
+            if (p.N == 1) bar_sync(bar_id, 256);
             ma = chunk_max_f(ma);
             bar_sync(bar_id, 256);                       // every warp has read ma's partials
             mx = chunk_max_f(mx);
