@@ -6,9 +6,9 @@ K and V, as stored) it reports, per Neumann order N, band mask and residual
 order S, the relative Frobenius error and the SNR of T and of W = T diag(b) K
 against the exact inverse (forward substitution), the worst chunk, and the
 largest entry of each masked power (the dynamic range the INT8 / INT16 codes
-must cover).  "When Good Enough Is Optimal", Études d'Ablation, reports these
-quantities per N and mask on its own models; here they are measured on the
-synthetic inputs.
+must cover), and the same errors for the INT8 and INT16 series.  "When Good
+Enough Is Optimal", Études d'Ablation, reports these quantities per N and
+mask on its own models; here they are measured on the synthetic inputs.
 
     python -m oracle.error_table [--chunks 256] [--gate-scale 1.0]
 """
@@ -55,6 +55,21 @@ def error_table(n_chunks: int = 256, gate_scale: float = 1.0, Ns=(1, 2, 3, 4), S
                              "T_rel_fro": o.rel_fro(T, T_ex), "T_snr_db": o.snr_db(T, T_ex),
                              "T_worst_chunk": max(per_chunk),
                              "W_rel_fro": o.rel_fro(W, W_ex), "W_snr_db": o.snr_db(W, W_ex)})
+    # the quantised series (S = 0): INT8 and INT16 codes with per-chunk scales,
+    # from the float32 A both integer schemes start from
+    A32 = A.astype(np.float32)
+    quant = []
+    for N in Ns:
+        for mask in (True, False):
+            T8 = o.int8_neumann(A32, N, mask)["T"]
+            T16 = o.int16_neumann(A32, N, mask)["T"]
+            Tf = o.invert_neumann(A, N, mask, 0)
+            quant.append({"N": N, "mask": int(mask),
+                          "float_rel_fro": o.rel_fro(Tf, T_ex),
+                          "int8_rel_fro": o.rel_fro(T8, T_ex),
+                          "int16_rel_fro": o.rel_fro(T16, T_ex),
+                          "int8_vs_float": o.rel_fro(T8, Tf),
+                          "int16_vs_float": o.rel_fro(T16, Tf)})
     # largest entry of the masked powers P_n = M (.) (P_{n-1} A), mean over chunks
     amax = {}
     k = A.shape[-1]
@@ -66,7 +81,8 @@ def error_table(n_chunks: int = 256, gate_scale: float = 1.0, Ns=(1, 2, 3, 4), S
             P = (P @ A) * Mb
             vals.append(float(np.mean(np.max(np.abs(P), axis=(1, 2)))))
         amax[N] = vals
-    return {"chunks": n_chunks, "gate_scale": gate_scale, "rows": rows, "amax_masked_powers": amax}
+    return {"chunks": n_chunks, "gate_scale": gate_scale, "rows": rows, "quantised": quant,
+            "amax_masked_powers": amax}
 
 
 def main(argv=None) -> int:
@@ -86,6 +102,13 @@ def main(argv=None) -> int:
         print(f"| {r['N']} | {'on' if r['mask'] else 'off'} | {r['S']} | {r['T_rel_fro']:.3e} | "
               f"{r['T_snr_db']:.1f} | {r['T_worst_chunk']:.3e} | {r['W_rel_fro']:.3e} | "
               f"{r['W_snr_db']:.1f} |")
+    print()
+    print("| N | mask | float64 series | INT8 | INT16 | INT8 vs float64 series | INT16 vs float64 series |")
+    print("|---|---|---|---|---|---|---|")
+    for r in res["quantised"]:
+        print(f"| {r['N']} | {'on' if r['mask'] else 'off'} | {r['float_rel_fro']:.3e} | "
+              f"{r['int8_rel_fro']:.3e} | {r['int16_rel_fro']:.3e} | {r['int8_vs_float']:.3e} | "
+              f"{r['int16_vs_float']:.3e} |")
     print("max |P_n| (masked powers, mean over chunks):",
           {N: [f"{v:.3g}" for v in vals] for N, vals in res["amax_masked_powers"].items()})
     return 0

@@ -669,3 +669,8 @@ def test_error_table_follows_the_truncation_laws():
     # the masked powers shrink with n on these fast-decaying gates
     amax = res["amax_masked_powers"][3]
     assert amax[0] > amax[1] > amax[2] > 0
+    # the quantised series: INT16 stays orders of magnitude closer to the
+    # float64 series than INT8; the float64 row repeats the S = 0 error above
+    for q in res["quantised"]:
+        assert 0 < q["int16_vs_float"] < q["int8_vs_float"] / 30
+        assert math.isclose(q["float_rel_fro"], err[(q["N"], q["mask"], 0)]["T_rel_fro"])
