@@ -264,6 +264,12 @@ def cpu_oracle_step(w: dict, data: OracleInputs, first: int, n: int) -> tuple[fl
 REFERENCE_CHUNK_BUDGET = 32768
 
 
+def reference_window(steps: int, warmup: int, sample_chunks: int) -> int:
+    """Chunks per step of the reference arm: at most ``sample_chunks``, and
+    few enough that all steps together stay within the budget (at least 1)."""
+    return max(1, min(sample_chunks, REFERENCE_CHUNK_BUDGET // max(1, steps + warmup)))
+
+
 def run_reference(args, world, rank):
     """Reference arm: the CPU oracle, each step a bounded window of the workload
     (rank 0 only)."""
@@ -272,8 +278,7 @@ def run_reference(args, world, rank):
     w = dict(WORKLOAD)
     data = OracleInputs(w)
     nc = data.nc
-    n_sample = max(1, min(args.sample_chunks,
-                          REFERENCE_CHUNK_BUDGET // max(1, args.steps + args.warmup)))
+    n_sample = reference_window(args.steps, args.warmup, args.sample_chunks)
     pos = 0
     for _ in range(args.warmup):
         cpu_oracle_step(w, data, pos, n_sample)

@@ -88,3 +88,20 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["impl"] == "reference" and d["n_gpus"] == 2
     assert d["unit"] == "chunks/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_bounds_its_work():
+    """However many steps are asked for, the reference arm's windows shrink so
+    that warm-up and timed steps together stay within its chunk budget."""
+    import bench
+
+    for steps in (1, 10, 100, 500, 5000, 100000):
+        n = bench.reference_window(steps, 5, 512)
+        assert 1 <= n <= 512
+        assert n * (steps + 5) <= max(bench.REFERENCE_CHUNK_BUDGET, steps + 5)
+    assert bench.reference_window(1, 3, 512) == 512
+    # the windows wrap around the workload's chunks
+    w = dict(bench.WORKLOAD)
+    data = bench.OracleInputs(w)
+    K, V, b, g = data.window(data.nc - 2, 5)
+    assert K.shape[0] == 5 and (K[2] == data.K[0]).all() and (g[4] == data.g[2]).all()
