@@ -674,3 +674,38 @@ def test_error_table_follows_the_truncation_laws():
     for q in res["quantised"]:
         assert 0 < q["int16_vs_float"] < q["int8_vs_float"] / 30
         assert math.isclose(q["float_rel_fro"], err[(q["N"], q["mask"], 0)]["T_rel_fro"])
+
+
+def test_series_and_residual_band_laws_on_random_shapes():
+    """Property check over random chunk sizes, orders, masks and strictly
+    lower-triangular A (entries up to 0.9 in size, so far entries stay large):
+    the truncated series equals the exact inverse on sub-diagonals 0..N (and,
+    masked, is zero below); with the residual it is exact on sub-diagonals
+    0..(S+1)(N+1)-1 and differs on the next one; a sum long enough to cover
+    the chunk is the exact inverse."""
+    hyp = pytest.importorskip("hypothesis")
+    st = hyp.strategies
+
+    @hyp.settings(max_examples=60, deadline=None, derandomize=True)
+    @hyp.given(k=st.integers(2, 24), N=st.integers(1, 6), S=st.integers(0, 4),
+               mask=st.booleans(), seed=st.integers(0, 2 ** 31 - 1))
+    def check(k, N, S, mask, seed):
+        rng = np.random.default_rng(seed)
+        A = np.tril(rng.uniform(-0.9, 0.9, size=(1, k, k)), -1)
+        T = O.invert_fwdsub(A)
+        dist = np.arange(k)[:, None] - np.arange(k)[None, :]
+        scale = max(1.0, float(np.abs(T).max()))
+        T0 = O.invert_neumann(A, N, mask, 0)
+        assert np.abs(T0 - T)[:, (dist >= 0) & (dist <= N)].max() <= 1e-12 * scale
+        if mask:
+            assert not T0[:, dist > N].any()
+        L = (S + 1) * (N + 1)
+        Tr = O.invert_neumann(A, N, mask, S)
+        err = np.abs(Tr - T)
+        assert err[:, (dist >= 0) & (dist <= min(L, k) - 1)].max() <= 1e-10 * scale ** (S + 2)
+        if L >= k:
+            assert O.rel_fro(Tr, T) <= 1e-10 * scale ** (S + 2)
+        else:
+            assert err[:, dist == L].max() > 0          # the first sub-diagonal left out
+
+    check()
