@@ -1,8 +1,10 @@
 // tc.cu — tcgen05 tensor-core kernels of libgdn (sm_100a).
 //
-// One persistent kernel template serves the bf16 chunk pipeline in four
-// modes: the fused inverse + WY step, A alone, the Neumann inverse alone and
-// WY alone.  Design:
+// One persistent kernel template serves the bf16 chunk pipeline in seven
+// modes: the fused inverse + WY step (on prepared inputs, or with the key
+// normalisation and gate sums in front), A alone, WY alone, and three
+// standalone inverses (the Neumann series with its residual, the sequential
+// correction, the block decomposition).  Design:
 //
 // * A "tile" is 128 consecutive rows of the flattened [B*H*T, d] arrays, i.e.
 //   128/KB blocks of KB tokens (KB = 64 or 128; chunks of k = 32 run as 64-token
