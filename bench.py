@@ -833,11 +833,19 @@ def main(argv=None) -> int:
                       "note": "same step with S=0 (no residual), timed after the headline"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_cpu = min(nc, args.cpu_chunks)
-        dt, threads = cpu_oracle_step(w, OracleInputs(w), 0, n_cpu)
+        data = OracleInputs(w)
+        dt, threads = cpu_oracle_step(w, data, 0, n_cpu)
+        # the same oracle held to one thread, on the first 256 chunks
+        from threadpoolctl import threadpool_limits
+        n_one = min(nc, 256)
+        with threadpool_limits(limits=1):
+            dt1, _ = cpu_oracle_step(w, data, 0, n_one)
         line["cpu_baseline"] = {"value": n_cpu / dt, "unit": "chunks/s",
                                 "cores": threads, "kind": "oracle",
                                 "sample": f"first {n_cpu} of {nc} chunks "
-                                          f"({'one whole step' if n_cpu == nc else 'part of a step'}), fp64"}
+                                          f"({'one whole step' if n_cpu == nc else 'part of a step'}), fp64",
+                                "one_core": {"value": n_one / dt1, "unit": "chunks/s", "cores": 1,
+                                             "sample": f"first {n_one} of {nc} chunks"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
