@@ -39,7 +39,7 @@ __all__ = [
     "invert_fwdsub",
     "neumann_powers_sum", "invert_neumann", "invert_newton", "invert_blocked", "residual_matrix",
     "wy",
-    "int8_neumann", "int8_residual", "int16_neumann", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
+    "int8_neumann", "int8_residual", "int16_neumann", "int16_residual", "chunk_forward", "token_recurrence", "decode", "rel_fro", "snr_db",
 ]
 
 
@@ -462,6 +462,75 @@ def int16_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:
     for n in range(N):
         T = T + scale[:, n, None, None] * q[:, n].astype(np.float64)
     return {"q": q, "acc": acc, "scale": scale, "T": T.astype(np.float32)}
+
+
+def int16_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
+    """INT16 series followed by the parallel residual correction, every
+    product an int16 code product ("When Good Enough Is Optimal", Adaptation
+    à la Quantification: the INT16 operating point with N = 3 and S = 8;
+    Méthodologie §3 for E and T = T^(0) sum E^s).  The steps of
+    ``int8_residual`` under the rules of ``int16_neumann``: codes in
+    [-32767, 32767], int64 accumulators (exact), every scale and sum in IEEE
+    binary64, zero maxima give zero codes and scales, and T rounded once to
+    float32 at the end:
+
+      1. T^(0) = I + sum_n s_n q_n in binary64 (``int16_neumann``'s sum before
+         its rounding); X = T^(0) - I;
+      2. codes of the whole A (no mask) and of X: (q_A, s_A), (q_X, s_X);
+         E = (A - X) + (s_A * s_X) * double(q_A q_X);
+      3. codes of E: (q_E1, s_E1); for s = 2..S: acc = q_E,s-1 q_E1,
+         m = max |acc|, q_E,s = clamp(rint(double(acc) * (32767 / m))),
+         s_E,s = (s_E,s-1 * s_E1) * (m / 32767) (E is not masked);
+         Gm = sum_{s=1}^{S} s_E,s * double(q_E,s), left to right;
+      4. codes of Gm: (q_G, s_G);
+         T = (T^(0) + Gm) + (s_X * s_G) * double(q_X q_G), then float32.
+
+    ``A32`` float32 ``[nc, k, k]``; returns T float32 ``[nc, k, k]``.
+    """
+    if S < 1:
+        raise ValueError("the residual needs S >= 1")
+    A32 = np.asarray(A32)
+    if A32.dtype != np.float32:
+        raise TypeError("A32 must be float32")
+    nc, k, _ = A32.shape
+
+    def codes(x):
+        # (int64 codes, binary64 scale per chunk) of a binary64 [nc, k, k] array
+        amax = np.abs(x).reshape(nc, -1).max(axis=1)
+        safe = np.where(amax > 0, amax, 1.0)
+        q = np.clip(np.rint(x * (32767.0 / safe)[:, None, None]), -32767, 32767).astype(np.int64)
+        q = np.where((amax > 0)[:, None, None], q, 0)
+        return q, np.where(amax > 0, amax / 32767.0, 0.0)
+
+    def deq(sa, sb, acc):
+        # (s_a * s_b) * double(acc); |acc| <= k 32767^2 < 2^53, exact in binary64
+        assert np.abs(acc).max(initial=0) < 2 ** 53
+        return (sa * sb)[:, None, None] * acc.astype(np.float64)
+
+    r16 = int16_neumann(A32, N, mask)
+    T0 = np.broadcast_to(np.eye(k), (nc, k, k)).copy()
+    for n in range(N):
+        T0 = T0 + r16["scale"][:, n, None, None] * r16["q"][:, n].astype(np.float64)
+    X = T0 - np.eye(k)
+    A = A32.astype(np.float64)
+    qA, sA = codes(A)
+    qX, sX = codes(X)
+    E = (A - X) + deq(sA, sX, qA @ qX)
+    qE, sE = codes(E)
+    qs, ss = qE, sE
+    Gm = ss[:, None, None] * qs.astype(np.float64)
+    for _ in range(2, S + 1):
+        acc = qs @ qE
+        m = np.abs(acc).reshape(nc, -1).max(axis=1)
+        mf = m.astype(np.float64)
+        safe = np.where(m > 0, mf, 1.0)
+        q = np.clip(np.rint(acc.astype(np.float64) * (32767.0 / safe)[:, None, None]),
+                    -32767, 32767)
+        qs = np.where((m > 0)[:, None, None], q.astype(np.int64), 0)
+        ss = np.where(m > 0, (ss * sE) * (mf / 32767.0), 0.0)
+        Gm = Gm + ss[:, None, None] * qs.astype(np.float64)
+    qG, sG = codes(Gm)
+    return ((T0 + Gm) + deq(sX, sG, qX @ qG)).astype(np.float32)
 
 
 # --------------------------------------------------------------------------- #

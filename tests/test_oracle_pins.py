@@ -579,6 +579,40 @@ def test_int8_residual_tracks_the_float_formula_and_repairs_t0():
         assert np.all(np.triu(Tq, 1) == 0) and np.all(np.diagonal(Tq, axis1=1, axis2=2) == 1)
 
 
+def test_int16_residual_tracks_the_float_formula_and_repairs_t0():
+    """The int16 residual against the same correction in float64 on the same
+    int16 T0 (literal powers of E = I - (I - A) T0): they differ only by the
+    16-bit quantisation of A X, E and its powers, and X Gm.  It repairs the
+    INT16 series by orders of magnitude, reaches the exact inverse within the
+    codes' resolution, and stays far closer than the INT8 residual."""
+    K, _, beta, g, _ = random_chunks(8, 64, 128, seed=16)
+    A32 = O.build_A(K, beta, g).astype(np.float32)
+    A64 = A32.astype(np.float64)
+    exact = O.invert_fwdsub(A64)
+    r16 = O.int16_neumann(A32, 3, True)
+    T0 = np.broadcast_to(np.eye(64), exact.shape).copy()
+    for n in range(3):
+        T0 = T0 + r16["scale"][:, n, None, None] * r16["q"][:, n].astype(np.float64)
+    E = np.eye(64) - (np.eye(64) - A64) @ T0
+    for S in (1, 2, 8):
+        acc = np.broadcast_to(np.eye(64), E.shape).copy()
+        P = acc.copy()
+        for _ in range(S):
+            P = P @ E
+            acc = acc + P
+        Tf = T0 @ acc
+        Tq = O.int16_residual(A32, 3, True, S)
+        assert Tq.dtype == np.float32
+        assert O.rel_fro(Tq, Tf) <= 1e-5
+        assert O.rel_fro(Tq, exact) <= O.rel_fro(r16["T"], exact) / 100
+        if S == 8:          # truncation gone: only the codes' resolution is left
+            assert O.rel_fro(Tq, exact) <= O.rel_fro(O.int8_residual(A32, 3, True, S), exact) / 20
+        assert np.all(np.triu(Tq, 1) == 0) and np.all(np.diagonal(Tq, axis1=1, axis2=2) == 1)
+    # a zero chunk: zero codes and scales everywhere, T = I exactly
+    z = np.zeros((2, 8, 8), np.float32)
+    assert np.array_equal(O.int16_residual(z, 3, True, 4), np.broadcast_to(np.eye(8, dtype=np.float32), z.shape))
+
+
 def test_int16_codes_and_int64_accumulators():
     k, N = 16, 4
     K, _, beta, g, _ = random_chunks(3, k, 16, seed=14, gate_scale=0.2)
