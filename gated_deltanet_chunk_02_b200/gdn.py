@@ -140,50 +140,68 @@ def shape_of_chunks(A: torch.Tensor, d: int = 128) -> GdnShape:
 
 
 def gdn_build_A(K, beta, g, A, k, stream=None):
+    """A = -b_i (k_i . k_j) e^(g_i - g_j) below the diagonal of every chunk: K
+    ``[B, H, T, d]`` (bf16 or float32), beta, g ``[B, H, T]`` float32 -> A
+    ``[B, H, T/k, k, k]`` float32."""
     _check(load().gdn_build_A(_ptr(K), _ptr(beta), _ptr(g), _ptr(A), shape_of(K, k), _dtype(K),
                               _stream(stream)))
 
 
 def gdn_invert_neumann(A, T, N, mask, S, prec=GDN_PREC_F32, stream=None):
+    """T = truncated series of order N (band mask if ``mask``) corrected by S
+    residual powers; A, T ``[B, H, T/k, k, k]`` float32; ``prec`` selects the
+    fp16-operand tensor-core chain or the float32 CUDA-core one."""
     _check(load().gdn_invert_neumann(_ptr(A), _ptr(T), shape_of_chunks(A), N, int(mask), S, prec,
                                      _stream(stream)))
 
 
 def gdn_invert_newton(A, T, N, mask, M, stream=None):
+    """The series of order N, then M sequential corrections T <- T + T(I - (I - A)T)."""
     _check(load().gdn_invert_newton(_ptr(A), _ptr(T), shape_of_chunks(A), N, int(mask), M,
                                     _stream(stream)))
 
 
 def gdn_invert_blocked(A, T, stream=None):
+    """Exact T by 2 x 2 block decomposition on the tensor cores (k <= 64)."""
     _check(load().gdn_invert_blocked(_ptr(A), _ptr(T), shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_invert_fwdsub(A, T, stream=None):
+    """Exact T by forward substitution (float32)."""
     _check(load().gdn_invert_fwdsub(_ptr(A), _ptr(T), shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_wy(T, K, V, beta, g, W, U, stream=None):
+    """W = T diag(beta) K (W_g = T diag(beta e^g) K when ``g`` is given) and
+    U = T diag(beta) V; W, U ``[B, H, T, d]`` in the dtype of K."""
     k = T.shape[-1]
     _check(load().gdn_wy(_ptr(T), _ptr(K), _ptr(V), _ptr(beta), _ptr(g), _ptr(W), _ptr(U),
                          shape_of(K, k), _dtype(K), _stream(stream)))
 
 
 def gdn_invert_neumann_i8(A, T, N, mask, q=None, acc=None, scale=None, stream=None):
+    """INT8 series (bit-exact scheme of gdn.h); optional dumps: codes ``q``
+    int8 ``[nc, N, k, k]``, accumulators ``acc`` int32, scales float32 ``[nc, N]``."""
     _check(load().gdn_invert_neumann_i8(_ptr(A), _ptr(T), N, int(mask), _ptr(q), _ptr(acc),
                                         _ptr(scale), shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_invert_neumann_i8_residual(A, T, N, mask, S, stream=None):
+    """INT8 series followed by S residual powers, every product in int8 codes."""
     _check(load().gdn_invert_neumann_i8_residual(_ptr(A), _ptr(T), N, int(mask), S,
                                                  shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_invert_neumann_i16(A, T, N, mask, q=None, acc=None, scale=None, stream=None):
+    """INT16 series (int64 accumulators, binary64 scales); optional dumps: codes
+    int16, accumulators int64, scales float64."""
     _check(load().gdn_invert_neumann_i16(_ptr(A), _ptr(T), N, int(mask), _ptr(q), _ptr(acc),
                                          _ptr(scale), shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_chunk_wy_fused(K, V, beta, g, N, mask, S, gated, W, U, T=None, k=64, stream=None):
+    """A, the series + mask + residual and W, U in one kernel; T is written
+    only when a ``T`` tensor is given."""
     _check(load().gdn_chunk_wy_fused(_ptr(K), _ptr(V), _ptr(beta), _ptr(g), N, int(mask), S,
                                      int(gated), _ptr(W), _ptr(U), _ptr(T), shape_of(K, k),
                                      _dtype(K), _stream(stream)))
@@ -200,11 +218,15 @@ def gdn_chunk_wy_fused_raw(K_raw, V, beta, loggate, N, mask, S, gated, W, U, T=N
 
 
 def gdn_forward_workspace_bytes(K, k):
+    """Scratch bytes ``gdn_forward`` needs for K's shape and dtype."""
     return int(load().gdn_forward_workspace_bytes(shape_of(K, k), _dtype(K)))
 
 
 def gdn_forward(Q, K, V, beta, g, S0, N, mask, S, exact, O, S_final, workspace, k=64,
                 stream=None):
+    """Chunk-wise forward: O ``[B, H, T, d]`` and the final state ``S_final``
+    ``[B, H, d, d]`` float32 from the start state ``S0`` (None = zero);
+    ``exact`` inverts by forward substitution instead of the series."""
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(load().gdn_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(g), _ptr(S0), N,
                               int(mask), S, int(exact), _ptr(O), _ptr(S_final), _ptr(workspace),
