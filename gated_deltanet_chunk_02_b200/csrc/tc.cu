@@ -44,12 +44,19 @@ constexpr int kD = 128;
 constexpr int kRows = 128;                       // rows per tile
 constexpr unsigned long long kTimeoutNs = 2000000000ull;
 constexpr int kStatusSmemAlign = 2;              // dynamic shared memory not 1024-aligned
+constexpr int kBandMax = 4;                      // widest band the fused step's band path takes
 
 enum Mode { kFused = 0, kBuildA = 1, kNeumann = 2, kWY = 3, kNewton = 4, kFusedRaw = 5,
-            kBlockInv = 6 };
+            kBlockInv = 6, kFusedBand = 7, kFusedRawBand = 8 };
 
 // the fused step, on prepared inputs or with the prologue (raw K, per-token log-gates)
-__host__ __device__ constexpr bool is_fused(int m) { return m == kFused || m == kFusedRaw; }
+__host__ __device__ constexpr bool is_fused(int m) {
+    return m == kFused || m == kFusedRaw || m == kFusedBand || m == kFusedRawBand;
+}
+// the fused step with the prologue in front
+__host__ __device__ constexpr bool is_raw(int m) { return m == kFusedRaw || m == kFusedRawBand; }
+// the fused step's band path (k = 64, mask on, N <= kBandMax; chosen at launch)
+__host__ __device__ constexpr bool is_band(int m) { return m == kFusedBand || m == kFusedRawBand; }
 __host__ __device__ constexpr bool uses_K(int m) { return is_fused(m) || m == kBuildA || m == kWY; }
 __host__ __device__ constexpr bool uses_V(int m) { return is_fused(m) || m == kWY; }
 // the standalone inverses: A in by TMA (staged a tile ahead), T out by TMA
@@ -220,6 +227,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
         "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
         : "memory");
+}
+
+// 4 consecutive TMEM columns of this thread's lane -> 4 floats.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // e^x = 2^(x log2 e), with the PTX base-2 exponential ex2.approx.ftz (relative
@@ -619,6 +637,29 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     constexpr bool kT0Tmem = (KB == 64);
     const uint32_t tT = tl + 160;
     const uint32_t tF = tl + (KB == 64 ? 224 : 192);  // F = E + E^2 of the residual (fp16 pairs)
+    // Band path of the fused step (k = 64, mask on, N <= kBandMax).  With the
+    // mask, T0 = M.(sum_{n<=N} A^n) is zero below its N-th sub-diagonal, so the
+    // series' products are needed only on the N + 1 diagonals the mask keeps,
+    // and the two products with T0 as a factor, A T0 (for the residual E) and
+    // T0 Q_S (for T), take at most N + 1 terms per entry.  These run on the
+    // CUDA cores; the dense products (K K^T, the powers of E, WY) stay on the
+    // tensor cores.  Storage:
+    //   X (fp16)       A - I, for the band entries other rows read;
+    //   TMEM           A - I in fp32, then T, in the block's own accumulator
+    //                  columns (no other block's product writes them);
+    //   Aop            bT[d-1][c] = T0[c+d][c], T0's band by column (zero past
+    //                  the chunk);
+    //   Y (fp16)       I + Q_S, whose rows the T0 (I + Q_S) product reads.
+    constexpr bool kBandable = is_band(MODE) && KC == 64;
+    constexpr bool band = kBandable;
+    float* const bT = reinterpret_cast<float*>(sAop);
+    float tb[kBandMax + 1];                        // tb[d] = T0[i][i-d], zero past N
+    auto band_row = [&]() {                        // row i's band of T0 back from bT
+        tb[0] = 1.f;
+#pragma unroll
+        for (int d = 1; d <= kBandMax; ++d)
+            tb[d] = (d <= p.N && i - d >= 0) ? bT[(d - 1) * kRows + blk * KB + i - d] : 0.f;
+    };
     // the slot's leader loads its own tiles: K, beta, g on fullK, V on fullV
     int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
     auto issue_k = [&](int n) {
@@ -667,7 +708,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     // read / write this thread's 32-column piece pp of T0
     auto t0_get = [&](int pp, float (&t)[32], float* T0r) {
         if (kT0Tmem) {
-            tmem_ld32(tT + (pc0 + pp) * 32, t);
+            tmem_ld32((band ? tD : tT) + (pc0 + pp) * 32, t);
         } else {
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) t[jj] = T0r[pp * 32 + jj];
@@ -675,7 +716,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     };
     auto t0_put = [&](int pp, const float (&t)[32], float* T0r) {
         if (kT0Tmem) {
-            tmem_st32(tT + (pc0 + pp) * 32, t);
+            tmem_st32((band ? tD : tT) + (pc0 + pp) * 32, t);
         } else {
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) T0r[pp * 32 + jj] = t[jj];
@@ -720,7 +761,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         if (*(volatile int*)&ctrl->abort) { ok = false; break; }
 
         if (is_fused(MODE) || MODE == kBuildA) {
-            if constexpr (MODE == kFusedRaw) {
+            if constexpr (is_raw(MODE)) {
                 // ---- prologue: K rows to unit L2 norm (in place, bf16) and the
                 // per-token log-gates to chunk-local cumulative sums ----
                 // Here lane l of the slot's warp w takes row 16 w + l / 2, panel
@@ -795,6 +836,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 mma_commit(&ctrl->mma[s]);
             }
             if (!wait_mma()) { ok = false; break; }
+            if (band) release_staging(n);             // the band tables take Aop
             const float bi = sb[r], gi = sg[r];
             const float* gcol = sg + blk * KB;
 #pragma unroll
@@ -822,6 +864,15 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             reinterpret_cast<float4*>(dst)[q] =
                                 make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                     }
+                } else if (kBandable && band) {
+                    // A - I: fp16 to X, fp32 to the T0 columns of TMEM
+                    if (pc == (i >> 5)) {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj)
+                            if (pc * 32 + jj == i) v[jj] = -1.f;
+                    }
+                    st_op32<false>(sX, r, pc, v);
+                    tmem_st32(tD + pc * 32, v);
                 } else {
                     st_op32<false>(sX, r, pc, v);             // A (chain's right operand)
                     float t[32];
@@ -951,7 +1002,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             // X_1 = I + M.A, X_n = I + M.(X_{n-1} A), T0 = X_N: inside the band
             // X_{n-1} A reads only in-band entries of X_{n-1}, so masking every
             // step gives M.(sum_{n<=N} A^n) exactly.
-            for (int pw = 2; pw <= p.N; ++pw) {
+            for (int pw = 2; !band && pw <= p.N; ++pw) {
                 cpublish(pw == 2);
                 cchain_t(sX);                                           // X_{n-1} A
                 if (!cwait()) { ok = false; break; }
@@ -970,6 +1021,67 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
             }
             if (!ok) break;
+            if (kBandable && band) {
+                // ---- the series on its band: X_1 = I + M.A, X_n = I + M.(X_{n-1} A)
+                // evaluated on the N + 1 diagonals the mask keeps, row by row:
+                // X_n[i][i-d] = [d = 0] + sum_{m<d} X_{n-1}[i][i-m] A[i-m][i-d].
+                // Entries before the chunk's first column do not exist (zero).
+                tmem_wait_st();
+                tc_fence_before();
+                bar_sync(cbar, 128);                              // A - I in X and TMEM
+                tc_fence_after();
+                // A[i-m][i-d] (m < d) from X, zero where the entry is not in the chunk
+                auto wA = [&](int m, int d) {
+                    const bool in = d <= p.N && i - d >= 0;
+                    const int row = in ? r - m : r, col = in ? i - d : 0;
+                    uint16_t u;
+                    asm volatile("ld.shared.u16 %0, [%1];"
+                                 : "=h"(u)
+                                 : "r"(su32(sX) + op_off(row, col >> 3) + 2 * (col & 7)));
+                    return in ? __half2float(__ushort_as_half(u)) : 0.f;
+                };
+                tb[0] = 1.f;
+#pragma unroll
+                for (int d = 1; d <= kBandMax; ++d) tb[d] = wA(0, d);
+#pragma unroll
+                for (int nn = 2; nn <= kBandMax; ++nn) {
+                    if (nn > p.N) break;
+                    float y[kBandMax + 1];
+#pragma unroll
+                    for (int d = 1; d <= kBandMax; ++d) {
+                        float acc = wA(0, d);
+#pragma unroll
+                        for (int m = 1; m < d; ++m) acc = fmaf(tb[m], wA(m, d), acc);
+                        y[d] = acc;
+                    }
+#pragma unroll
+                    for (int d = 1; d <= kBandMax; ++d) tb[d] = y[d];
+                }
+                if (p.S == 0) {
+                    // T = T0: the band, zero elsewhere
+                    float t[32];
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int dd = i - (pc0 * 32 + jj);
+                        float x = 0.f;
+#pragma unroll
+                        for (int d = 0; d <= kBandMax; ++d) x = dd == d ? tb[d] : x;
+                        t[jj] = x;
+                    }
+                    t0_put(0, t, T0);
+                } else {
+                    // T0 by column for A T0: column c of row c + d, zero past the chunk
+                    if (h == 0) {
+#pragma unroll
+                        for (int d = 1; d <= kBandMax; ++d) {
+                            if (d > p.N) break;
+                            if (i - d >= 0) bT[(d - 1) * kRows + blk * KB + i - d] = tb[d];
+                            if (i + d >= KB) bT[(d - 1) * kRows + blk * KB + i] = 0.f;
+                        }
+                    }
+                    bar_sync(cbar, 128);                          // bT written
+                }
+            }
             // ---- parallel residual correction: T = T0 G, G = sum_{s<=S} E^s ----
             // Two schedules.  Horner keeps Q_m in TMEM as the left operand
             // (stride 2 below: one product per round, in 64-row blocks that do
@@ -1163,6 +1275,50 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     // takes E^2, Q_4, Q_6, Q_8); Q_m (no identity) is the left
                     // operand in TMEM, E in X, E^2 then Q_S in Y, F in TMEM as
                     // fp16.
+                    if (kBandable && band) {
+                        // E = I + (A - I) T0 on this thread's columns j:
+                        // (A - I) T0 [i][j] = sum_{d<=N} (A - I)[i][j+d] T0[j+d][j]
+                        // (T0[j][j] = 1); the -I term takes T0's band off
+                        float a[32], ed[4], v[32];
+                        tmem_ld32(tD + pc0 * 32, a);
+                        if (h == 0) {
+                            tmem_ld4(tD + 32, ed);                  // the partner's first columns
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) ed[e] = 0.f;   // past the chunk
+                        }
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) v[jj] = a[jj];              // d = 0
+#pragma unroll
+                        for (int d = 1; d <= kBandMax; ++d) {
+                            if (d > p.N) break;
+                            const float* tc = bT + (d - 1) * kRows + blk * KB + pc0 * 32;
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 t4 = *reinterpret_cast<const float4*>(tc + 4 * q);
+                                const float tt[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                                for (int c = 0; c < 4; ++c) {
+                                    const int jj = 4 * q + c;
+                                    const float ad = jj + d < 32 ? a[(jj + d) & 31] : ed[(jj + d) & 3];
+                                    v[jj] = fmaf(ad, tt[c], v[jj]);
+                                }
+                            }
+                        }
+                        // the diagonal of the sum is -1 exactly: E[i][i] = 0, and
+                        // (I + E)[i][i] = 1 for S = 1, where Q_1 = E is final
+                        if (pc0 == (i >> 5)) {
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj)
+                                if (pc0 * 32 + jj == i) v[jj] = p.S == 1 ? 1.f : 0.f;
+                        }
+                        if (p.S == 1) {
+                            st_op32<false>(sY, r, pc0, v);                // I + Q_1
+                        } else {
+                            st_op32<false>(sX, r, pc0, v);                  // E
+                            tmem_st_h16(tA + pc0 * 16, v);                // Q_1 = E
+                        }
+                    } else {
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         float t[32];
@@ -1191,6 +1347,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             tmem_st_h16(tA + pc * 16, v);                 // Q_1 = E
                         }
                     }
+                    }
                     // this row's E from X, 8 columns at a time
                     auto e_row = [&](int pc, float (&e)[32]) {
 #pragma unroll
@@ -1201,12 +1358,22 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             for (int c = 0; c < 8; ++c) e[8 * g + c] = h8[c];
                         }
                     };
-                    // Q_S is final: Q_S -> Y (right operand), T0 -> TMEM (left)
+                    // Q_S is final: Q_S -> Y (right operand), T0 -> TMEM (left;
+                    // the band path reads Q_S's rows from Y instead)
                     auto finish_q = [&](int pp, float (&q)[32]) {
                         const int pc = pc0 + pp;
 #pragma unroll
                         for (int jj = 0; jj < 32; ++jj)
                             if (!in_chunk(pc * 32 + jj)) q[jj] = 0.f;
+                        if (kBandable && band) {
+                            if (pc == (i >> 5)) {
+#pragma unroll
+                                for (int jj = 0; jj < 32; ++jj)
+                                    if (pc * 32 + jj == i) q[jj] = 1.f;        // I + Q_S
+                            }
+                            st_op32<false>(sY, r, pc, q);
+                            return;
+                        }
                         st_op32<false>(sY, r, pc, q);
                         float t[32];
                         t0_get(pp, t, T0);
@@ -1263,6 +1430,29 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         }
                         if (!ok) break;
                     }
+                    if (kBandable && band) {
+                        // T = T0 (I + Q_S): T[i][j] = sum_{e<=N} T0[i][i-e] (I + Q_S)[i-e][j],
+                        // the rows of I + Q_S (fp16) from Y and row
+                        // i's band of T0 back from bT
+                        bar_sync(cbar, 128);                              // I + Q_S written
+                        band_row();
+                        float t[32];
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) t[jj] = 0.f;
+#pragma unroll
+                        for (int e = 0; e <= kBandMax; ++e) {
+                            if (e > p.N) break;
+                            if (i - e < 0) continue;
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                float h8[8];
+                                ld_h8(sY, r - e, 4 * pc0 + g, h8);
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) t[8 * g + c] = fmaf(tb[e], h8[c], t[8 * g + c]);
+                            }
+                        }
+                        t0_put(0, t, T0);
+                    } else {
                     cpublish(true);
                     cchain_t(sY);                                        // T0 Q_S
                     if (!cwait()) { ok = false; break; }
@@ -1276,6 +1466,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         for (int jj = 0; jj < 32; ++jj)
                             if (in_chunk(pc * 32 + jj)) t[jj] += v[jj];          // T = T0 + T0 Q
                         t0_put(pp, t, T0);
+                    }
                     }
                 }
             }
@@ -2971,6 +3162,7 @@ cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, con
     io.g = g;
     io.W = W;
     io.U = U;
+    if (k == 64 && mask && N <= tcg::kBandMax) return tcg::launch<64, tcg::kFusedBand, 2>(io, p, st);
     return tcg::dispatch<tcg::kFused, 1>(k, io, p, st);
 }
 
@@ -2993,6 +3185,8 @@ cudaError_t launch_fused_raw_tc(const void* K, const void* V, const float* beta,
     io.g = loggate;
     io.W = W;
     io.U = U;
+    if (k == 64 && mask && N <= tcg::kBandMax)
+        return tcg::launch<64, tcg::kFusedRawBand, 2>(io, p, st);
     return tcg::dispatch<tcg::kFusedRaw, 1>(k, io, p, st);
 }
 
