@@ -839,6 +839,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             if (band) release_staging(n);             // the band tables take Aop
             const float bi = sb[r], gi = sg[r];
             const float* gcol = sg + blk * KB;
+            float lbi = 0.f;                              // band path: log2(beta_i)
+            if constexpr (band) asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lbi) : "f"(bi));
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
                 const int pc = pc0 + pp;
@@ -853,7 +855,14 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = pc * 32 + jj;
                         const bool in = in_chunk(j) && j < i;
-                        v[jj] = in ? -bi * v[jj] * exp_e(gi - gcol[j]) : 0.f;
+                        if constexpr (band) {             // beta_i e^(g_i - g_j) = 2^((g_i - g_j) log2 e + log2 beta_i)
+                            float e2;
+                            asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e2)
+                                : "f"(fmaf(gi - gcol[j], 1.4426950408889634f, lbi)));
+                            v[jj] = in ? -v[jj] * e2 : 0.f;
+                        } else {
+                            v[jj] = in ? -bi * v[jj] * exp_e(gi - gcol[j]) : 0.f;
+                        }
                     }
                 }
                 if (MODE == kBuildA) {
@@ -1451,7 +1460,21 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                                 for (int c = 0; c < 8; ++c) t[8 * g + c] = fmaf(tb[e], h8[c], t[8 * g + c]);
                             }
                         }
-                        t0_put(0, t, T0);
+                        if (p.gated) {
+                            t0_put(0, t, T0);
+                        } else {                                  // WY's operand T diag(beta), bf16
+                            if (p.Tout && valid) {
+                                float* dst = p.Tout + cidx * KC * KC + rin * KC + pc0 * 32;
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    reinterpret_cast<float4*>(dst)[q] =
+                                        make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
+                            }
+                            const float* bcol = sb + blk * KB + pc0 * 32;
+#pragma unroll
+                            for (int jj = 0; jj < 32; ++jj) t[jj] *= bcol[jj];
+                            st_op32<true>(sX, r, pc0, t);
+                        }
                     } else {
                     cpublish(true);
                     cchain_t(sY);                                        // T0 Q_S
@@ -1499,7 +1522,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         tma_store_2d(&mW, 32 * b, (int)row0, sAop + b * 16384);
                     bulk_commit();
                 }
-            } else if (p.Tout) {
+            } else if (p.Tout && !(band && p.S > 0 && !p.gated)) {
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
@@ -1523,6 +1546,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             const float* gcol = sg + blk * KB;
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
+                if (band && p.S > 0 && !p.gated) break;    // written by the band product
                 const int pc = pc0 + pp;
                 float v[32], t[32];
                 t0_get(pp, t, T0);
