@@ -337,7 +337,7 @@ def int8_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:
     return {"q": q, "acc": acc, "scale": scale, "T": T}
 
 
-def int8_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
+def int8_residual(A32: np.ndarray, N: int, mask: bool, S: int, parts: bool = False):
     """INT8 series followed by the parallel residual correction, every product
     an int8 product ("When Good Enough Is Optimal", Adaptation à la
     Quantification: N = 3 compensated by S = 8 residual steps; Méthodologie
@@ -356,7 +356,9 @@ def int8_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
       4. codes of Gm: (q_G, s_G);
          T = (T^(0) + Gm) + (s_X * s_G) * float(q_X q_G)   [= T^(0) (I + Gm)].
 
-    ``A32`` float32 ``[nc, k, k]``; returns T float32 ``[nc, k, k]``.
+    ``A32`` float32 ``[nc, k, k]``; returns T float32 ``[nc, k, k]``, or with
+    ``parts`` a dict that also holds E, its codes and scale (``qE``, ``sE``),
+    Gm and its codes and scale (``qG``, ``sG``).
     """
     if S < 1:
         raise ValueError("the residual needs S >= 1")
@@ -402,7 +404,10 @@ def int8_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
                       f32(0.0)).astype(f32)
         Gm = (Gm + (ss[:, None, None] * qs.astype(f32)).astype(f32)).astype(f32)
     qG, sG = codes(Gm)
-    return ((T0 + Gm).astype(f32) + deq(sX, sG, qX @ qG)).astype(f32)
+    T = ((T0 + Gm).astype(f32) + deq(sX, sG, qX @ qG)).astype(f32)
+    if parts:
+        return {"E": E, "qE": qE, "sE": sE, "Gm": Gm, "qG": qG, "sG": sG, "T": T}
+    return T
 
 
 def int16_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:
@@ -464,7 +469,7 @@ def int16_neumann(A32: np.ndarray, N: int, mask: bool) -> dict:
     return {"q": q, "acc": acc, "scale": scale, "T": T.astype(np.float32)}
 
 
-def int16_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
+def int16_residual(A32: np.ndarray, N: int, mask: bool, S: int, parts: bool = False):
     """INT16 series followed by the parallel residual correction, every
     product an int16 code product ("When Good Enough Is Optimal", Adaptation
     à la Quantification: the INT16 operating point with N = 3 and S = 8;
@@ -485,7 +490,9 @@ def int16_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
       4. codes of Gm: (q_G, s_G);
          T = (T^(0) + Gm) + (s_X * s_G) * double(q_X q_G), then float32.
 
-    ``A32`` float32 ``[nc, k, k]``; returns T float32 ``[nc, k, k]``.
+    ``A32`` float32 ``[nc, k, k]``; returns T float32 ``[nc, k, k]``, or with
+    ``parts`` a dict that also holds E, its codes and scale (``qE``, ``sE``),
+    Gm and its codes and scale (``qG``, ``sG``), all binary64 or int64.
     """
     if S < 1:
         raise ValueError("the residual needs S >= 1")
@@ -530,7 +537,10 @@ def int16_residual(A32: np.ndarray, N: int, mask: bool, S: int) -> np.ndarray:
         ss = np.where(m > 0, (ss * sE) * (mf / 32767.0), 0.0)
         Gm = Gm + ss[:, None, None] * qs.astype(np.float64)
     qG, sG = codes(Gm)
-    return ((T0 + Gm) + deq(sX, sG, qX @ qG)).astype(np.float32)
+    T = ((T0 + Gm) + deq(sX, sG, qX @ qG)).astype(np.float32)
+    if parts:
+        return {"E": E, "qE": qE, "sE": sE, "Gm": Gm, "qG": qG, "sG": sG, "T": T}
+    return T
 
 
 # --------------------------------------------------------------------------- #

@@ -73,9 +73,9 @@ def frac_to_np(X):
     return np.array([[float(x) for x in r] for r in X])
 
 
-def load_golden():
+def load_golden(fname: str = "unit_lower_4x4.txt"):
     out, name, rows = {}, None, []
-    with open(os.path.join(GOLDEN, "unit_lower_4x4.txt")) as f:
+    with open(os.path.join(GOLDEN, fname)) as f:
         for line in f:
             line = line.strip()
             if not line or line.startswith("#"):
@@ -611,6 +611,122 @@ def test_int16_residual_tracks_the_float_formula_and_repairs_t0():
     # a zero chunk: zero codes and scales everywhere, T = I exactly
     z = np.zeros((2, 8, 8), np.float32)
     assert np.array_equal(O.int16_residual(z, 3, True, 4), np.broadcast_to(np.eye(8, dtype=np.float32), z.shape))
+
+
+def test_int8_residual_golden_by_hand():
+    """The hand-derived INT8 example of tests/golden/int_residual_4x4.txt:
+    E, its codes (one a tie, rounded to even), Gm and T exactly, for S = 1 and
+    for S = 2, where E^2 has a zero maximum; and a matrix whose E is zero."""
+    G = load_golden("int_residual_4x4.txt")
+    A = G["A8"].astype(np.float32)[None]
+    for S in (1, 2):
+        r = O.int8_residual(A, 1, True, S, parts=True)
+        assert np.array_equal(r["E"][0], G["E8"].astype(np.float32))
+        assert np.array_equal(r["qE"][0], G["qE8"].astype(np.int64))
+        assert r["sE"][0] == np.float32(2.0 ** -8)
+        assert np.array_equal(r["Gm"][0], G["Gm8"].astype(np.float32))
+        assert np.array_equal(r["qG"][0], G["qE8"].astype(np.int64)) and r["sG"][0] == np.float32(2.0 ** -8)
+        assert np.array_equal(r["T"][0], G["T8"].astype(np.float32))
+        assert np.array_equal(O.int8_residual(A, 1, True, S), r["T"])
+    # one subdiagonal entry: X = A, A X = 0, so E = 0 (a zero maximum), T = I + A
+    Z = np.zeros((1, 4, 4), np.float32)
+    Z[0, 2, 1] = 0.5
+    r = O.int8_residual(Z, 1, True, 3, parts=True)
+    assert not r["E"].any() and not r["qE"].any() and r["sE"][0] == 0 and not r["Gm"].any()
+    assert np.array_equal(r["T"][0], np.eye(4, dtype=np.float32) + Z[0])
+
+
+def test_int16_residual_golden_by_hand():
+    """The hand-derived INT16 example of tests/golden/int_residual_4x4.txt
+    (binary64 scales, a tie at -2048.5, T rounded once to float32)."""
+    G = load_golden("int_residual_4x4.txt")
+    A = G["A16"].astype(np.float32)[None]
+    for S in (1, 2):
+        r = O.int16_residual(A, 1, True, S, parts=True)
+        assert np.array_equal(r["E"][0], G["E16"])
+        assert np.array_equal(r["qE"][0], G["qE16"].astype(np.int64))
+        assert r["sE"][0] == 2.0 ** -16
+        assert np.array_equal(r["Gm"][0], G["Gm16"])
+        assert np.array_equal(r["T"][0], G["T16"].astype(np.float32))
+    Z = np.zeros((1, 4, 4), np.float32)
+    Z[0, 3, 2] = -0.25
+    r = O.int16_residual(Z, 1, True, 2, parts=True)
+    assert not r["E"].any() and r["sE"][0] == 0
+    assert np.array_equal(r["T"][0], np.eye(4, dtype=np.float32) + Z[0])
+
+
+def _int8_residual_variant(A32, N, mask, S, swap=None):
+    """The INT8 residual written out again with one documented float32
+    operation order swapped (``swap``), for the test below: a planted mistake
+    that must change the result bits on realistic chunks."""
+    f32 = np.float32
+    nc, k, _ = A32.shape
+
+    def codes(x):
+        amax = np.abs(x).reshape(nc, -1).max(axis=1).astype(f32)
+        safe = np.where(amax > 0, amax, f32(1.0)).astype(f32)
+        r = (f32(127.0) / safe).astype(f32)
+        q = np.clip(np.rint((x * r[:, None, None]).astype(f32)), -127, 127).astype(np.int64)
+        q = np.where((amax > 0)[:, None, None], q, 0)
+        return q, np.where(amax > 0, (amax / f32(127.0)).astype(f32), f32(0.0)).astype(f32)
+
+    def deq(sa, sb, acc):
+        if swap == "deq_order":           # s_a (s_b acc) instead of (s_a s_b) acc
+            return (sa[:, None, None] * (sb[:, None, None] * acc.astype(f32)).astype(f32)).astype(f32)
+        return ((sa * sb).astype(f32)[:, None, None] * acc.astype(f32)).astype(f32)
+
+    T0 = O.int8_neumann(A32, N, mask)["T"]
+    X = (T0 - np.eye(k, dtype=f32)).astype(f32)
+    qA, sA = codes(A32)
+    qX, sX = codes(X)
+    D = deq(sA, sX, qA @ qX)
+    if swap == "E_order":                 # A - (X - D) instead of (A - X) + D
+        E = (A32 - (X - D).astype(f32)).astype(f32)
+    else:
+        E = ((A32 - X).astype(f32) + D).astype(f32)
+    qE, sE = codes(E)
+    qs, ss = qE, sE
+    terms = [(ss[:, None, None] * qs.astype(f32)).astype(f32)]
+    for _ in range(2, S + 1):
+        acc = qs @ qE
+        m = np.abs(acc).reshape(nc, -1).max(axis=1)
+        mf = m.astype(f32)
+        safe = np.where(m > 0, mf, f32(1.0)).astype(f32)
+        r = (f32(127.0) / safe).astype(f32)
+        q = np.clip(np.rint((acc.astype(f32) * r[:, None, None]).astype(f32)), -127, 127)
+        qs = np.where((m > 0)[:, None, None], q.astype(np.int64), 0)
+        if swap == "scale_order":         # s_{s-1} (s_E (m / 127)) instead of (s_{s-1} s_E)(m / 127)
+            ss_new = (ss * (sE * (mf / f32(127.0)).astype(f32)).astype(f32)).astype(f32)
+        else:
+            ss_new = ((ss * sE).astype(f32) * (mf / f32(127.0)).astype(f32)).astype(f32)
+        ss = np.where(m > 0, ss_new, f32(0.0)).astype(f32)
+        terms.append((ss[:, None, None] * qs.astype(f32)).astype(f32))
+    if swap == "sum_order":               # sum from s = S down to 1
+        terms = terms[::-1]
+    Gm = terms[0]
+    for t in terms[1:]:
+        Gm = (Gm + t).astype(f32)
+    qG, sG = codes(Gm)
+    D2 = deq(sX, sG, qX @ qG)
+    if swap == "T_order":                 # T0 + (Gm + D2) instead of (T0 + Gm) + D2
+        return (T0 + (Gm + D2).astype(f32)).astype(f32)
+    return ((T0 + Gm).astype(f32) + D2).astype(f32)
+
+
+def test_int8_residual_operation_order_is_seen():
+    """Every float32 operation order that the INT8 residual fixes changes the
+    result bits on realistic chunks when swapped, so the bit-exact GPU
+    comparison on such chunks pins the order, not only the formula."""
+    K, _, beta, g, _ = random_chunks(16, 64, 128, seed=31)
+    A32 = O.build_A(K, beta, g).astype(np.float32)
+    ref = O.int8_residual(A32, 3, True, 8)
+    assert np.array_equal(_int8_residual_variant(A32, 3, True, 8), ref)     # the order as written
+    for swap in ("deq_order", "scale_order", "sum_order", "T_order"):
+        assert not np.array_equal(_int8_residual_variant(A32, 3, True, 8, swap), ref), swap
+    # The order of E = (A - X) + D is the one step the result cannot see: off
+    # the band X = 0 and both orders are A + D, and in the band the float32
+    # difference of A - (X - D) never moves a code (E is quantised next).
+    assert np.array_equal(_int8_residual_variant(A32, 3, True, 8, "E_order"), ref)
 
 
 def test_int16_codes_and_int64_accumulators():
