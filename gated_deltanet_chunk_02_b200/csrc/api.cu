@@ -45,7 +45,13 @@ int check_shape(const gdn_shape& s, int64_t* nc) {
         return fail(GDN_ERR_ARG, "chunk size k=%d not in {32, 64, 128, 256}", s.k);
     if (s.T % s.k) return fail(GDN_ERR_ARG, "T=%lld is not a multiple of k=%d", (long long)s.T, s.k);
     if (s.d != 128) return fail(GDN_ERR_UNSUPPORTED, "head dim d=%d (only 128 is built)", s.d);
-    const int64_t n = s.B * s.H * (s.T / s.k);
+    // each factor is below 2^31, so the products below cannot overflow int64
+    if (s.B > 0x7fffffffLL || s.H > 0x7fffffffLL || s.T / s.k > 0x7fffffffLL)
+        return fail(GDN_ERR_ARG, "too many chunks (B=%lld, H=%lld, T/k=%lld)", (long long)s.B,
+                    (long long)s.H, (long long)(s.T / s.k));
+    const int64_t bh = s.B * s.H;
+    if (bh > 0x7fffffffLL) return fail(GDN_ERR_ARG, "too many chunks (B*H=%lld)", (long long)bh);
+    const int64_t n = bh * (s.T / s.k);
     if (n > 0x7fffffffLL) return fail(GDN_ERR_ARG, "too many chunks (%lld)", (long long)n);
     *nc = n;
     return GDN_OK;

@@ -15,7 +15,8 @@
 //    library, for as long as the library stays loaded;
 //  * a call needs nc * (2 * k * d * elem + 2 * k * k * 4) bytes of it
 //    (elem = 2 for bf16, 4 for f32) and is rejected with GDN_ERR_ARG when that
-//    exceeds the array (about 680 chunks of 64 bf16 tokens);
+//    exceeds the array: at k = 64 a chunk needs 64 KiB (bf16) or 96 KiB (f32),
+//    so the array holds 1024 bf16 chunks or 682 f32 chunks;
 //  * every call on a device uses the same array and leaves its contents
 //    behind; the forward overwrites every byte it reads before reading it, so
 //    nothing has to start at zero;
@@ -24,7 +25,9 @@
 //
 // Set-up: the first call on each device (with that device current) looks up
 // the array's device address with cudaGetSymbolAddress; make that first call
-// before any stream capture.
+// before any stream capture.  The address is cached for the life of the
+// process: a device reset (cudaDeviceReset) invalidates it, and the library
+// must be reloaded after one.
 #include <mutex>
 
 #include "../../include/gdn.h"

@@ -240,12 +240,15 @@ int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype);
  * The scratch (W_g, U, A, T) lives in a 64 MiB device array inside the
  * library, held on every GPU that loads it until the library is unloaded.
  * Problems needing more than that (gdn_forward_workspace_bytes(s, dtype) >
- * 64 MiB, about 680 chunks of 64 bf16 tokens) return GDN_ERR_ARG.  All calls
+ * 64 MiB: more than 1024 chunks of 64 bf16 tokens, or 682 chunks of 64 fp32
+ * tokens) return GDN_ERR_ARG.  All calls
  * on a device share the array and leave their data in it; nothing needs to
  * start at zero, but calls whose kernels may overlap on the GPU race on it, so
  * order them on one stream.  The first call on each device (made with that
  * device current) looks up the array's address: make it before any stream
- * capture.  Arguments and results are otherwise those of gdn_forward.
+ * capture.  The address is kept for the life of the process, so a device
+ * reset (cudaDeviceReset) invalidates it: reload the library after one.
+ * Arguments and results are otherwise those of gdn_forward.
  */
 int gdn_forward_static(const void* Q, const void* K, const void* V,
                        const float* beta, const float* g, const float* S0,
@@ -277,9 +280,11 @@ int gdn_decode(const void* Q, const void* K, const void* V, const float* beta,
  * (NULL = the legacy default stream) and returns without synchronising; none
  * allocates device memory (gdn_forward takes a caller workspace).  The calls
  * can therefore be captured into CUDA graphs and replayed; make one eager
- * call first (it sets kernel attributes and looks up the status word), and
- * capture gdn_forward_static only after its first eager call on the device.
+ * call first (it sets kernel attributes and looks up the status word).
  */
+/* The status word's address is looked up once per host thread and device and
+ * kept; a device reset (cudaDeviceReset) invalidates it, as it does the
+ * static scratch of gdn_forward_static: reload the library after one. */
 /* Synchronises `stream`, returns the device status word of the current
  * device (GDN_OK, GDN_ERR_TIMEOUT, or GDN_ERR_CUDA when a kernel found its
  * shared memory misaligned) and clears it. */
