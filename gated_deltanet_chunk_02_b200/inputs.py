@@ -12,7 +12,12 @@ Recipe (the distributions of the workloads the method is evaluated on):
 * per-token log-gates ``-softplus(N(0, 1))`` (times ``gate_scale``, 1 by
   default), and ``g`` their cumulative sum restarted at every chunk of ``k``
   tokens (summed in float64, stored as float32);
-* queries ``Q`` (only when asked for): drawn like ``K``.
+* queries ``Q`` (only when asked for): drawn like ``K``;
+* optionally (``key_corr = rho > 0``) keys that share one direction: each
+  normalised row becomes ``sqrt(1 - rho^2) k + rho u`` (renormalised), with
+  ``u`` a unit vector drawn from a second generator, so the other draws are
+  unchanged.  Correlated keys make ``A`` larger and the method's residual
+  correction matter more (a stress input, not one of the workloads).
 
 Draw order from one ``torch.Generator`` seeded with ``seed``: K, V,
 beta-logits, gate-logits, then Q.  K, V and Q are cast to the requested dtype
@@ -58,19 +63,26 @@ def chunk_cumsum(loggate: torch.Tensor, k: int) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, seed: int = 0, with_q: bool = False,
-                gate_scale: float = 1.0, raw_keys: bool = False) -> dict:
+                gate_scale: float = 1.0, raw_keys: bool = False, key_corr: float = 0.0) -> dict:
     """Draw one batch of inputs for workload ``w`` on the CPU.
 
     Returns a dict of CPU tensors: ``K``, ``V`` (``[B,H,T,d]`` in ``w.dtype``),
     ``beta``, ``loggate``, ``g`` (``[B,H,T]`` float32) and, if ``with_q``,
     ``Q`` (``[B,H,T,d]`` in ``w.dtype``).  ``raw_keys`` leaves the key rows
-    un-normalised (same draws, for the kernels that normalise them).
+    un-normalised (same draws, for the kernels that normalise them);
+    ``key_corr`` mixes a shared unit direction into every key row (above).
     """
     if w.T % w.k:
         raise ValueError("T must be a multiple of the chunk size k")
     gen = torch.Generator().manual_seed(seed)
     shp = (w.B, w.H, w.T, w.d)
     K = torch.randn(shp, generator=gen, dtype=torch.float32)
+    if key_corr > 0.0:
+        ugen = torch.Generator().manual_seed(seed * 1000003 + 424242)
+        u = torch.randn(w.d, generator=ugen, dtype=torch.float32)
+        norm = K.norm(dim=-1, keepdim=True)
+        Kc = (1.0 - key_corr ** 2) ** 0.5 * (K / norm) + key_corr * (u / u.norm())
+        K = Kc / Kc.norm(dim=-1, keepdim=True) * norm        # the raw rows keep their norms
     if not raw_keys:
         K = K / K.norm(dim=-1, keepdim=True)
     V = torch.randn(shp, generator=gen, dtype=torch.float32)
