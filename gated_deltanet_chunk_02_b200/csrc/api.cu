@@ -369,6 +369,16 @@ int gdn_get_status(void* stream) {
     return GDN_OK;
 }
 
+int gdn_debug_arm_wait_expiry(int tile, int load, double timeout_ms) {
+    if (tile < 0) return fail(GDN_ERR_ARG, "tile=%d is negative", tile);
+    if (load != 0 && load != 1) return fail(GDN_ERR_ARG, "load=%d is neither 0 (K) nor 1 (V)", load);
+    if (!(timeout_ms > 0.0 && timeout_ms <= 2000.0))
+        return fail(GDN_ERR_ARG, "timeout_ms=%g outside (0, 2000]", timeout_ms);
+    if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
+    gdn::arm_wait_expiry(tile, load, (unsigned long long)(timeout_ms * 1e6));
+    return GDN_OK;
+}
+
 const char* gdn_last_error(void) { return t_last_error.c_str(); }
 
 int64_t gdn_launch_count(void) { return t_launches; }

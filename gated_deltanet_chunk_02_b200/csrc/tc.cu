@@ -112,14 +112,16 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
         : "=r"(ok) : "r"(su32(b)), "r"(parity) : "memory");
     return ok != 0;
 }
-// Bounded wait on the phase with the given parity; false if it ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+// Bounded wait on the phase with the given parity; false once it ran out
+// (after *limit ns when `limit` is given, read only when checking, else 2 s).
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity,
+                                          const volatile unsigned long long* limit = nullptr) {
     if (mbar_try(b, parity)) return true;
     const unsigned long long t0 = gtime();
     while (true) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try(b, parity)) return true;
-        if (gtime() - t0 > kTimeoutNs) return false;
+        if (gtime() - t0 > (limit ? *limit : kTimeoutNs)) return false;
     }
 }
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int x, int y,
@@ -140,6 +142,16 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 __device__ __forceinline__ void bar_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Named barrier that also ORs a predicate over its participants: every thread
+// gets the same answer, so a decision taken on it is the same for all.
+__device__ __forceinline__ bool bar_sync_or(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred pi, po;\n setp.ne.u32 pi, %1, 0;\n"
+        " bar.red.or.pred po, %2, %3, pi;\n selp.u32 %0, 1, 0, po;\n}\n"
+        : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(n) : "memory");
+    return r != 0;
 }
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(dst)),
@@ -434,6 +446,9 @@ struct Params {
     __nv_bfloat16* Kout; // kFusedRaw (optional): the L2-normalised K
     float* gout;         // kFusedRaw (optional): the chunk-local cumulative log-gates
     int* status;
+    unsigned long long timeout_ns;   // bound of every wait (2 s)
+    int withhold_tile;   // tests of the bounded waits: a load of this tile is never issued (-1: none)
+    int withhold_v;      // ... that load is V (1) or K, beta and g (0)
 };
 
 struct __align__(8) Ctrl {
@@ -442,6 +457,8 @@ struct __align__(8) Ctrl {
     uint64_t mma[2];     // the slot's MMAs completed
     uint64_t wdone[2];   // the slot's W^T products completed (K no longer read)
     uint64_t mmac[2][2]; // per-chunk products of the chain rounds (slot, 64-row block)
+    uint64_t drain[2][2];// after an expired wait: the issuing threads' products are done
+    unsigned long long timeout_ns;   // the launch's bound of every wait
     uint32_t tmem;
     int abort;
 };
@@ -490,8 +507,11 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             mbar_init(&ctrl->wdone[s], 1);
             mbar_init(&ctrl->mmac[s][0], 1);
             mbar_init(&ctrl->mmac[s][1], 1);
+            mbar_init(&ctrl->drain[s][0], 1);
+            mbar_init(&ctrl->drain[s][1], 1);
         }
         ctrl->abort = 0;
+        ctrl->timeout_ns = p.timeout_ns;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) tmem_alloc(&ctrl->tmem, kTmemCols);
@@ -529,13 +549,20 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     const int pc0 = h * PPT;
     uint32_t mma_phase = 0;
     bool ok = true;
+    // Once a wait has run out anywhere in the CTA, every thread still walks
+    // the rest of its tile's barrier sequence (nobody leaves a slot between
+    // two barriers), but waits entered from then on return at once (one
+    // already under way runs to its bound) and no product, copy or store is
+    // started; the slot leaves together at the next tile's first barrier.
+    const volatile int* const abortp = &ctrl->abort;
+    auto live = [&]() { return *abortp == 0; };
 
     auto fail_wait = [&]() {
         atomicExch(&ctrl->abort, 1);
         raise_status(p.status, kStatusTimeout);
     };
     auto wait_mma = [&]() -> bool {
-        bool good = mbar_wait(&ctrl->mma[s], mma_phase);
+        bool good = live() && mbar_wait(&ctrl->mma[s], mma_phase, &ctrl->timeout_ns);
         mma_phase ^= 1;
         if (!good) fail_wait();
         tc_fence_after();
@@ -552,7 +579,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     };
     // k x k chain product D = a_buf[128 x KB] * b_buf[KB x 128] (b: MN-major)
     auto mma_chain = [&](const uint8_t* a_buf, const uint8_t* b_buf) {
-        if (leader) {
+        if (leader && live()) {
             constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
             const uint32_t ab = su32(a_buf), bb = su32(b_buf);
 #pragma unroll 1
@@ -566,7 +593,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     };
     // k x k chain product D = Aop[128 x KB] (TMEM, fp16 pairs) * b_buf[KB x 128] (MN-major)
     auto mma_chain_t = [&](const uint8_t* b_buf) {
-        if (leader) {
+        if (leader && live()) {
             constexpr uint32_t id = idesc_f16(0, 0, 1, 128, 128);
             const uint32_t bb = su32(b_buf);
 #pragma unroll 1
@@ -597,7 +624,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     };
     auto cwait = [&]() -> bool {
         if (!kSplit) return wait_mma();
-        const bool good = mbar_wait(cmbar, cphase);
+        const bool good = live() && mbar_wait(cmbar, cphase, &ctrl->timeout_ns);
         cphase ^= 1;
         if (!good) fail_wait();
         tc_fence_after();
@@ -607,7 +634,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     const uint32_t cd = tm + (kSplit ? 64 * cg : 0);        // its accumulator columns
     const uint32_t cbo = kSplit ? (uint32_t)(cg * 64 * 128) : 0u;   // its B rows
     auto cchain = [&](const uint8_t* a_buf, const uint8_t* b_buf) {
-        if (cleader) {
+        if (cleader && live()) {
             constexpr uint32_t id = idesc_f16(0, 0, 1, kCN, 128);
             const uint32_t ab = su32(a_buf), bb = su32(b_buf) + cbo;
 #pragma unroll 1
@@ -620,7 +647,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         }
     };
     auto cchain_t = [&](const uint8_t* b_buf) {
-        if (cleader) {
+        if (cleader && live()) {
             constexpr uint32_t id = idesc_f16(0, 0, 1, kCN, 128);
             const uint32_t bb = su32(b_buf) + cbo;
 #pragma unroll 1
@@ -664,7 +691,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     int k_issued = 0, v_issued = 0;               // loads issued by this slot's leader
     auto issue_k = [&](int n) {
         const int tile = blockIdx.x + n * gridDim.x;
-        if (!(uses_K(MODE) || inv_only(MODE)) || tile >= p.ntiles) return;
+        if (!(uses_K(MODE) || inv_only(MODE)) || tile >= p.ntiles || !live()) return;
+        if (tile == p.withhold_tile && !p.withhold_v) return;   // tests: the wait must run out
         ++k_issued;
         const int y = tile * kRows;
         if (inv_only(MODE)) {                          // A: KC / 32 boxes of 16 KB
@@ -682,7 +710,8 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     };
     auto issue_v = [&](int n) {
         const int tile = blockIdx.x + n * gridDim.x;
-        if (!uses_V(MODE) || tile >= p.ntiles) return;
+        if (!uses_V(MODE) || tile >= p.ntiles || !live()) return;
+        if (tile == p.withhold_tile && p.withhold_v) return;    // tests: the wait must run out
         ++v_issued;
         const int y = tile * kRows;
         mbar_expect_tx(&ctrl->fullV[s], kRows * kD * 2);
@@ -755,10 +784,11 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         const int64_t rin = grow % KC;                   // row inside the chunk
         float T0[kT0Tmem ? 1 : PPT * 32];                // this thread's part of row r of T0 / T
 
-        if ((uses_K(MODE) || inv_only(MODE)) && !mbar_wait(&ctrl->fullK[s], use_par))
+        if ((uses_K(MODE) || inv_only(MODE)) && !(live() && mbar_wait(&ctrl->fullK[s], use_par, &ctrl->timeout_ns)))
             fail_wait();
-        bar_sync(bar_id, 256);
-        if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+        // the slot decides together whether to stop (an OR over its threads'
+        // view of the abort flag, so no thread can read it differently)
+        if (bar_sync_or(bar_id, 256, !live())) { ok = false; break; }
 
         if (is_fused(MODE) || MODE == kBuildA) {
             if constexpr (is_raw(MODE)) {
@@ -824,7 +854,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 bar_sync(bar_id, 256);
             }
             // ---- G = K K^T over the tile, then A = -beta_i G_ij exp(g_i - g_j) ----
-            if (leader) {
+            if (leader && live()) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_f16(1, 0, 0, 128, 128);
                 const uint32_t kbase = su32(sK);
@@ -835,7 +865,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 }
                 mma_commit(&ctrl->mma[s]);
             }
-            if (!wait_mma()) { ok = false; break; }
+            if (!wait_mma()) ok = false;
             if (band) release_staging(n);             // the band tables take Aop
             const float bi = sb[r], gi = sg[r];
             const float* gcol = sg + blk * KB;
@@ -1014,7 +1044,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             for (int pw = 2; !band && pw <= p.N; ++pw) {
                 cpublish(pw == 2);
                 cchain_t(sX);                                           // X_{n-1} A
-                if (!cwait()) { ok = false; break; }
+                if (!cwait()) ok = false;
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
@@ -1029,7 +1059,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     else tmem_st_h16(tA + pc * 16, v);
                 }
             }
-            if (!ok) break;
             if (kBandable && band) {
                 // ---- the series on its band: X_1 = I + M.A, X_n = I + M.(X_{n-1} A)
                 // evaluated on the N + 1 diagonals the mask keeps, row by row:
@@ -1106,7 +1135,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 for (int lv = 0; lv < (KC == 64 ? 2 : 1); ++lv) {
                     cpublish(true);
                     cchain(lv == 0 ? sX : sAop, sY);                     // P = A_L T
-                    if (!cwait()) { ok = false; break; }
+                    if (!cwait()) ok = false;
                     {
                         float v[32];
                         tmem_ld32(tD + pc0 * 32, v);
@@ -1114,7 +1143,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                     cpublish(true);
                     cchain(sY, sX);                                      // T P
-                    if (!cwait()) { ok = false; break; }
+                    if (!cwait()) ok = false;
                     {
                         float v[32], t[32];
                         tmem_ld32(tD + pc0 * 32, v);
@@ -1125,7 +1154,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         if (lv == 0) st_op32<false>(sY, r, pc0, t);
                     }
                 }
-                if (!ok) break;
             } else if constexpr (MODE == kNewton) {
                 // Sequential correction, the form the method's parallel residual
                 // replaces: R_m = I - (I - A) T_m = I - T_m + A T_m and
@@ -1142,7 +1170,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                     cpublish(true);
                     cchain(sX, sY);                                      // A T_m
-                    if (!cwait()) { ok = false; break; }
+                    if (!cwait()) ok = false;
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
@@ -1159,7 +1187,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                     cpublish(true);
                     cchain_t(sY);                                        // T_m R_m
-                    if (!cwait()) { ok = false; break; }
+                    if (!cwait()) ok = false;
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
@@ -1172,7 +1200,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         t0_put(pp, t, T0);
                     }
                 }
-                if (!ok) break;
             } else if (p.S > 0) {
                 const int S = p.S;
                 int K2 = 0;
@@ -1200,7 +1227,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     // block 0's product into columns [0, 64), block 1's into [64, 128)
                     auto mma_blocks = [&](const uint8_t* a0, const uint8_t* b0, const uint8_t* a1,
                                           const uint8_t* b1) {
-                        if (leader) {
+                        if (leader && live()) {
                             constexpr uint32_t id = idesc_f16(0, 0, 1, 64, 128);
                             const uint32_t x0 = su32(a0), y0 = su32(b0);
                             const uint32_t x1 = su32(a1), y1 = su32(b1);
@@ -1222,7 +1249,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                     publish(true);
                     mma_blocks(sX, sY, sX, sY + 64 * 128);                  // A T0
-                    if (!wait_mma()) { ok = false; break; }
+                    if (!wait_mma()) ok = false;
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
@@ -1240,7 +1267,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         const bool last = rd == K2;
                         publish(true);
                         mma_blocks(sX, sX + 64 * 128, sAop, sAop);          // [V; E] E, [E; V] E
-                        if (!wait_mma()) { ok = false; break; }
+                        if (!wait_mma()) ok = false;
 #pragma unroll
                         for (int pp = 0; pp < PPT; ++pp) {
                             const int pc = pc0 + pp;
@@ -1261,11 +1288,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             if (!last) st_op32<false>(sVr(), r, pc, v);
                         }
                     }
-                    if (!ok) break;
                     if (p2p1) {
                         publish(true);
                         mma_blocks(sY, sX + 64 * 128, sY, sAop);            // T0 E^(2^J)
-                        if (!wait_mma()) { ok = false; break; }
+                        if (!wait_mma()) ok = false;
 #pragma unroll
                         for (int pp = 0; pp < PPT; ++pp) {
                             const int pc = pc0 + pp;
@@ -1336,7 +1362,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                     cpublish(true);
                     cchain(sX, sY);                                      // A T0
-                    if (!cwait()) { ok = false; break; }
+                    if (!cwait()) ok = false;
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
@@ -1391,7 +1417,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     if (p.S >= 2) {
                         cpublish(true);
                         cchain_t(sX);                                    // E E
-                        if (!cwait()) { ok = false; break; }
+                        if (!cwait()) ok = false;
 #pragma unroll
                         for (int pp = 0; pp < PPT; ++pp) {
                             const int pc = pc0 + pp;
@@ -1417,7 +1443,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                             cpublish(first);
                             first = false;
                             cchain_t(sY);                                // Q_m E^2
-                            if (!cwait()) { ok = false; break; }
+                            if (!cwait()) ok = false;
                             m += 2;
 #pragma unroll
                             for (int pp = 0; pp < PPT; ++pp) {
@@ -1437,7 +1463,6 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                                 }
                             }
                         }
-                        if (!ok) break;
                     }
                     if (kBandable && band) {
                         // T = T0 (I + Q_S): T[i][j] = sum_{e<=N} T0[i][i-e] (I + Q_S)[i-e][j],
@@ -1478,7 +1503,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     } else {
                     cpublish(true);
                     cchain_t(sY);                                        // T0 Q_S
-                    if (!cwait()) { ok = false; break; }
+                    if (!cwait()) ok = false;
 #pragma unroll
                     for (int pp = 0; pp < PPT; ++pp) {
                         const int pc = pc0 + pp;
@@ -1516,7 +1541,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 fence_async_smem();
                 tc_fence_before();
                 bar_sync(bar_id, 256);
-                if (leader) {
+                if (leader && live()) {
 #pragma unroll 1
                     for (int b = 0; b < KC / 32; ++b)
                         tma_store_2d(&mW, 32 * b, (int)row0, sAop + b * 16384);
@@ -1563,10 +1588,9 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     st_op32<true>(sY, r, pc, v);
                 }
             }
-            if (uses_V(MODE) && !mbar_wait(&ctrl->fullV[s], use_par)) fail_wait();
+            if (uses_V(MODE) && !(live() && mbar_wait(&ctrl->fullV[s], use_par, &ctrl->timeout_ns))) fail_wait();
             publish(true);
-            if (*(volatile int*)&ctrl->abort) { ok = false; break; }
-            if (leader) {
+            if (leader && live()) {
                 constexpr uint32_t id = idesc_f16(1, 1, 0, KB, 128);
                 const uint32_t kb0 = su32(sK), vb0 = su32(sV), xb0 = su32(sX);
                 const uint32_t ub0 = su32(p.gated ? sY : sX);
@@ -1596,10 +1620,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                     }
                 }
                 mma_commit(&ctrl->mma[s]);
-                if (mbar_wait(&ctrl->wdone[s], use_par)) issue_k(n + NS);   // K is free
+                if (live() && mbar_wait(&ctrl->wdone[s], use_par, &ctrl->timeout_ns)) issue_k(n + NS);   // K is free
                 else fail_wait();
             }
-            if (!wait_mma()) { ok = false; break; }
+            if (!wait_mma()) ok = false;
             // Lane d of the W^T / U^T accumulators is head-dim column d and
             // accumulator column x is tile row x.  Warp (quarter q, half h)
             // moves d in [32q, 32q + 32) x rows [64h, 64h + 64): 16x256b TMEM
@@ -1642,7 +1666,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             fence_async_smem();
             tc_fence_before();
             bar_sync(bar_id, 256);
-            if (leader) {
+            if (leader && live()) {
                 const int y = (int)row0;
                 tma_store_2d(&mW, 0, y, sWst);
                 tma_store_2d(&mW, 64, y, sWst + kRows * 128);
@@ -1656,15 +1680,19 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
         tc_fence_before();
         bar_sync(bar_id, 256);                 // accumulators free for the next tile
     }
-    if (!ok) {
-        atomicExch(&ctrl->abort, 1);
-        // outstanding MMAs of this slot finish before TMEM is released, and the
-        // copies it issued land before the CTA's shared memory goes away
-        mbar_wait(&ctrl->mma[s], mma_phase);
-        if (kSplit) mbar_wait(cmbar, cphase);
+    if (!ok || !live()) {
+        // Drain (bounded, deaf to the abort flag): one more commit by each
+        // issuing thread tracks every product it started, so TMEM is not freed
+        // under one; the loads the leader started land before the CTA's shared
+        // memory goes away.
+        if (leader || cleader) {
+            uint64_t* dm = &ctrl->drain[s][leader ? 0 : 1];
+            mma_commit(dm);
+            mbar_wait(dm, 0, &ctrl->timeout_ns);
+        }
         if (leader) {
-            if (k_issued > 0) mbar_wait(&ctrl->fullK[s], (uint32_t)((k_issued - 1) & 1));
-            if (v_issued > 0) mbar_wait(&ctrl->fullV[s], (uint32_t)((v_issued - 1) & 1));
+            if (k_issued > 0) mbar_wait(&ctrl->fullK[s], (uint32_t)((k_issued - 1) & 1), &ctrl->timeout_ns);
+            if (v_issued > 0) mbar_wait(&ctrl->fullV[s], (uint32_t)((v_issued - 1) & 1), &ctrl->timeout_ns);
         }
     }
     if (leader) bulk_wait_all();                   // W, U stores complete
@@ -2985,6 +3013,8 @@ static Params base_params(int64_t nc, int k) {
     memset(&p, 0, sizeof p);
     p.rows = nc * k;
     p.ntiles = (int)((p.rows + kRows - 1) / kRows);
+    p.timeout_ns = kTimeoutNs;
+    p.withhold_tile = -1;
     return p;
 }
 
@@ -3170,10 +3200,26 @@ cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, in
     return cudaGetLastError();
 }
 
+static thread_local int t_withhold_tile = -1;
+static thread_local int t_withhold_v = 0;
+static thread_local unsigned long long t_expiry_ns = 0;
+
+void arm_wait_expiry(int tile, int v, unsigned long long timeout_ns) {
+    t_withhold_tile = tile;
+    t_withhold_v = v;
+    t_expiry_ns = timeout_ns;
+}
+
 cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, const float* g,
                             int N, int mask, int S, int gated, void* W, void* U, float* Tout,
                             int64_t nc, int k, cudaStream_t st) {
     tcg::Params p = tcg::base_params(nc, k);
+    if (t_withhold_tile >= 0) {                 // armed once by gdn_debug_arm_wait_expiry
+        p.withhold_tile = t_withhold_tile;
+        p.withhold_v = t_withhold_v;
+        p.timeout_ns = t_expiry_ns;
+        t_withhold_tile = -1;
+    }
     p.N = N;
     p.mask = mask;
     p.S = S;

@@ -44,5 +44,9 @@ cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int
 cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, const float* g,
                             int N, int mask, int S, int gated, void* W, void* U, float* Tout,
                             int64_t nc, int k, cudaStream_t st);
+// tests of the bounded waits: the next launch_fused_tc on this host thread
+// leaves tile `tile`'s K (v = 0) or V (v = 1) load unissued and bounds every
+// wait by `timeout_ns`
+void arm_wait_expiry(int tile, int v, unsigned long long timeout_ns);
 
 }  // namespace gdn

@@ -28,7 +28,7 @@ EXPORTS = [
     "gdn_invert_neumann_i8", "gdn_invert_neumann_i8_residual", "gdn_invert_neumann_i16",
     "gdn_chunk_wy_fused", "gdn_chunk_wy_fused_raw", "gdn_forward",
     "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_decode", "gdn_get_status",
-    "gdn_last_error", "gdn_launch_count",
+    "gdn_last_error", "gdn_launch_count", "gdn_debug_arm_wait_expiry",
 ]
 
 
@@ -79,6 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gdn_decode": [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int32, _I,
                        _P],
         "gdn_get_status": [_P],
+        "gdn_debug_arm_wait_expiry": [_I, _I, ctypes.c_double],
         "gdn_last_error": [],
         "gdn_launch_count": [],
     }
@@ -253,6 +254,14 @@ def gdn_decode(Q, K, V, beta, loggate, S, O, stream=None):
 def gdn_get_status(stream=None) -> int:
     """Synchronise the stream; return (and clear) the device status code."""
     return int(load().gdn_get_status(_stream(stream)))
+
+
+def gdn_debug_arm_wait_expiry(tile: int, which: str, timeout_ms: float) -> None:
+    """Tests only: the next fused call on this thread leaves tile ``tile``'s
+    ``which`` load ("K" or "V") unissued and bounds its waits by
+    ``timeout_ms`` (the wait runs out, the status word reports
+    GDN_ERR_TIMEOUT)."""
+    _check(load().gdn_debug_arm_wait_expiry(int(tile), {"K": 0, "V": 1}[which], float(timeout_ms)))
 
 
 def gdn_last_error() -> str:

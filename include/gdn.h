@@ -290,6 +290,24 @@ int gdn_decode(const void* Q, const void* K, const void* V, const float* beta,
  * shared memory misaligned) and clears it. */
 int gdn_get_status(void* stream);
 
+/*
+ * Test hook for the bounded device waits; the pages have no counterpart.
+ * Arms the next gdn_chunk_wy_fused call made on this host thread (bf16 data,
+ * tensor-core path) so that one load of tile `tile` (token rows
+ * [128 tile, 128 tile + 128) of the flattened [B*H*T] axis) is never issued:
+ * K with beta and g when `load` = 0 (waited for at the start of the tile), V
+ * when `load` = 1 (waited for before WY); every wait of that launch is bounded
+ * by `timeout_ms` instead of 2 s.
+ * The wait for that tile then runs out: the CTA that owns it sets
+ * GDN_ERR_TIMEOUT in the status word, finishes the barrier sequence of the
+ * tile it is on without starting further products, copies or stores, waits
+ * (bounded) for its own work in flight, frees its tensor memory and returns;
+ * the other CTAs finish normally.  That call's outputs are undefined; the
+ * call after it runs normally.  Returns GDN_OK, or GDN_ERR_ARG for a negative
+ * tile, a load other than 0 or 1, or timeout_ms outside (0, 2000].
+ */
+int gdn_debug_arm_wait_expiry(int tile, int load, double timeout_ms);
+
 /* Message for the most recent nonzero return on this host thread. */
 const char* gdn_last_error(void);
 

@@ -93,6 +93,16 @@ def test_neumann_parameter_ranges(lib, N, mask, S):
     assert rc == gdn.GDN_ERR_ARG
 
 
+def test_wait_expiry_hook_arguments(lib):
+    """The test hook of the bounded waits checks its arguments (valid ones
+    are left for the GPU test: arming here would only be consumed by a launch)."""
+    f = lib.gdn_debug_arm_wait_expiry
+    assert f(-1, 0, ctypes.c_double(5.0)) == gdn.GDN_ERR_ARG and "negative" in last(lib)
+    assert f(0, 2, ctypes.c_double(5.0)) == gdn.GDN_ERR_ARG
+    assert f(0, 0, ctypes.c_double(0.0)) == gdn.GDN_ERR_ARG
+    assert f(0, 1, ctypes.c_double(2500.0)) == gdn.GDN_ERR_ARG
+
+
 def test_int8_limits(lib):
     assert lib.gdn_invert_neumann_i8(P(FAKE), P(FAKE), 3, 1, None, None, None, sh(k=128),
                                      None) == gdn.GDN_ERR_UNSUPPORTED
