@@ -259,6 +259,84 @@ def cpu_oracle_step(w: dict, data: OracleInputs, first: int, n: int) -> tuple[fl
     return dt, threads
 
 
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_parallel(w: dict, data: OracleInputs, first: int, n: int,
+                        threads: int | None = None) -> tuple[float, int]:
+    """Time the oracle (as it stands) on n chunks starting at chunk ``first``,
+    split into one window per host core and run on a thread pool with BLAS
+    held to one thread per call (numpy releases the GIL inside its products
+    and array loops, so the windows run in parallel).  Returns (seconds,
+    threads used)."""
+    import numpy as np
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle as O
+    from threadpoolctl import threadpool_limits
+    threads = max(1, min(threads or host_cores(), n))
+    cuts = np.linspace(0, n, threads + 1).astype(int)
+    wins = [data.window(first + a, b - a) for a, b in zip(cuts, cuts[1:]) if b > a]
+
+    def one(win):
+        K, V, b, g = win
+        A = O.build_A(K, b, g)
+        T = O.invert_neumann(A, w["N"], bool(w["mask"]), w["S"])
+        O.wy(T, K, V, b, g if w["gated"] else None)
+
+    with threadpool_limits(limits=1), ThreadPoolExecutor(max_workers=len(wins)) as ex:
+        t0 = time.perf_counter()
+        list(ex.map(one, wins))
+        dt = time.perf_counter() - t0
+    return dt, len(wins)
+
+
+def cpu_forward_baseline(wl, seed: int, N: int, mask: int, S: int) -> dict:
+    """The oracle's chunk-wise forward (A, the inverse, the chunk scan) on every
+    head of the workload, one head per host core at a time, and its token-by-
+    token recurrence on the first 4096 tokens of one head on one core."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle as O
+    from gated_deltanet_chunk_02_b200.inputs import make_inputs, as_f64_numpy
+    from threadpoolctl import threadpool_limits
+    inp = make_inputs(wl, seed=seed, with_q=True)
+    k, BH = wl.k, wl.B * wl.H
+    ch = {key: O.to_chunks(as_f64_numpy(inp[key]), k).reshape(BH, wl.T // k, k, -1)
+          for key in ("Q", "K", "V")}
+    ch.update({key: O.to_chunks(as_f64_numpy(inp[key]), k).reshape(BH, wl.T // k, k)
+               for key in ("beta", "g")})
+
+    def head(h):
+        A = O.build_A(ch["K"][h], ch["beta"][h], ch["g"][h])
+        T = O.invert_neumann(A, N, bool(mask), S)
+        O.chunk_forward(*(ch[key][h:h + 1] for key in ("Q", "K", "V", "beta", "g")), T[None])
+
+    threads = max(1, min(host_cores(), BH))
+    with threadpool_limits(limits=1), ThreadPoolExecutor(max_workers=threads) as ex:
+        t0 = time.perf_counter()
+        list(ex.map(head, range(BH)))
+        dt = time.perf_counter() - t0
+    n_tok = min(4096, wl.T)
+    f = lambda key: as_f64_numpy(inp[key]).reshape(BH, wl.T, -1)[:1, :n_tok]
+    g = lambda key: as_f64_numpy(inp[key]).reshape(BH, wl.T)[:1, :n_tok]
+    with threadpool_limits(limits=1):
+        t1 = time.perf_counter()
+        O.token_recurrence(f("Q"), f("K"), f("V"), g("beta"), g("loggate"))
+        dt1 = time.perf_counter() - t1
+    nc = BH * (wl.T // k)
+    return {"value": nc / dt, "unit": "chunks/s", "cores": threads, "kind": "oracle",
+            "sample": f"all {BH} heads x {wl.T // k} chunks (the whole forward): A, the inverse "
+                      f"(N={N}, mask={mask}, S={S}) and the chunk scan, fp64, one head per thread",
+            "token_recurrence": {"value": (n_tok // k) / dt1, "unit": "chunks/s", "cores": 1,
+                                 "sample": f"first {n_tok} tokens of one head, token by token"}}
+
+
 # chunks the reference arm processes over a whole run (warm-up and timed steps
 # together), so that any --steps / --warmup ends in a few minutes of host time
 REFERENCE_CHUNK_BUDGET = 32768
@@ -281,23 +359,25 @@ def run_reference(args, world, rank):
     n_sample = reference_window(args.steps, args.warmup, args.sample_chunks)
     pos = 0
     for _ in range(args.warmup):
-        cpu_oracle_step(w, data, pos, n_sample)
+        cpu_oracle_parallel(w, data, pos, n_sample)
         pos += n_sample
     total, threads = 0.0, 1
     for _ in range(args.steps):
-        dt, threads = cpu_oracle_step(w, data, pos, n_sample)
+        dt, threads = cpu_oracle_parallel(w, data, pos, n_sample)
         pos += n_sample
         total += dt
     value = n_sample * args.steps / total
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "chunks/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * total / args.steps * nc / n_sample, "higher_is_better": True,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, nc),
+        "ms_per_step_scaled_to_workload": 1e3 * total / args.steps * nc / n_sample,
         "cpu_baseline": {"value": value, "unit": "chunks/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{n_sample} consecutive of {nc} chunks per step, "
-                                   f"a new window each step; ms_per_step scaled to all {nc}"},
+                         "sample": f"{n_sample} consecutive of {nc} chunks per step (a new window "
+                                   f"each step, split over {threads} host threads); ms_per_step is "
+                                   f"the measured time of one such step"},
         "e2e": {"value": value, "unit": "chunks/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -428,10 +508,15 @@ def run_component(args, world, rank, local, dev) -> int:
     }[kern]
     bytes_l, flops_l = per[0] * nc, per[1] * nc
     peaks, peak_kind = load_peaks()
+    # the integer kernels' products are int8 MMAs: their tensor peak is the
+    # measured bf16 peak times the nominal int8 : bf16 ratio (4.5 : 2.25)
+    integer = kern in ("int8", "int8_residual", "int16")
+    tc_peak = float(peaks["bf16_tflops"]) * (2.0 if integer else 1.0)
+    tc_kind = peak_kind + (" x 2 (nominal int8:bf16 ratio)" if integer else "")
     gbs = bytes_l / (ms_step * 1e-3) / 1e9
     tfl = flops_l / (ms_step * 1e-3) / 1e12
     t_hbm = bytes_l / (float(peaks["hbm_gbs"]) * 1e9)
-    t_tc = flops_l / (float(peaks["bf16_tflops"]) * 1e12)
+    t_tc = flops_l / (tc_peak * 1e12)
     bound = "hbm" if (t_hbm >= t_tc or kern == "fwdsub") else "tensor"
     line = {
         "metric": f"{kern} kernel: chunks/s (k={k}, d={d}, bf16 data)",
@@ -446,15 +531,19 @@ def run_component(args, world, rank, local, dev) -> int:
                                + (f" M={args.M}" if kern == "newton" else ""),
                    "chunks": nc},
         "roofline": {"bound": bound, "achieved": gbs if bound == "hbm" else tfl,
-                     "peak": float(peaks["hbm_gbs"]) if bound == "hbm" else float(peaks["bf16_tflops"]),
-                     "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-                     "frac": gbs / float(peaks["hbm_gbs"]) if bound == "hbm"
-                     else tfl / float(peaks["bf16_tflops"]),
-                     "traffic": recorded_traffic(kern), "peak_source": peak_kind,
+                     "peak": float(peaks["hbm_gbs"]) if bound == "hbm" else tc_peak,
+                     "unit": "GB/s" if bound == "hbm" else ("TOP/s" if integer else "TFLOP/s"),
+                     "frac": gbs / float(peaks["hbm_gbs"]) if bound == "hbm" else tfl / tc_peak,
+                     "traffic": recorded_traffic(kern),
+                     "peak_source": peak_kind if bound == "hbm" else tc_kind,
+                     "tensor_peak": tc_peak, "tensor_peak_source": tc_kind,
                      "roofline_frac": max(t_hbm, t_tc) / (ms_step * 1e-3), "tflops": tfl,
                      "bytes_per_launch": bytes_l, "flops_per_launch": flops_l},
         "clocks": clocks.summary(), "e2e": None, "gpu_launches": launches,
     }
+    if kern == "forward" and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_forward_baseline(wl, shard_seed(rank, 0), args.N, args.mask,
+                                                    args.S)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -834,7 +923,7 @@ def main(argv=None) -> int:
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_cpu = min(nc, args.cpu_chunks)
         data = OracleInputs(w)
-        dt, threads = cpu_oracle_step(w, data, 0, n_cpu)
+        dt, threads = cpu_oracle_parallel(w, data, 0, n_cpu)
         # the same oracle held to one thread, on the first 256 chunks
         from threadpoolctl import threadpool_limits
         n_one = min(nc, 256)
@@ -843,7 +932,8 @@ def main(argv=None) -> int:
         line["cpu_baseline"] = {"value": n_cpu / dt, "unit": "chunks/s",
                                 "cores": threads, "kind": "oracle",
                                 "sample": f"first {n_cpu} of {nc} chunks "
-                                          f"({'one whole step' if n_cpu == nc else 'part of a step'}), fp64",
+                                          f"({'one whole step' if n_cpu == nc else 'part of a step'}), fp64, "
+                                          f"one window per host thread",
                                 "one_core": {"value": n_one / dt1, "unit": "chunks/s", "cores": 1,
                                              "sample": f"first {n_one} of {nc} chunks"}}
     if rank == 0:
