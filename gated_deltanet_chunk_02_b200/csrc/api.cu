@@ -335,6 +335,50 @@ int gdn_forward(const void* Q, const void* K, const void* V, const float* beta, 
                     "forward scan");
 }
 
+int64_t gdn_forward_raw_workspace_bytes(gdn_shape s, gdn_dtype dtype) {
+    int64_t nc;
+    if (check_shape(s, &nc) != GDN_OK || dtype != GDN_BF16) return -1;
+    const int64_t rows = nc * s.k;
+    // gdn_forward's scratch, then the normalised keys (bf16) and the summed gates
+    return gdn_forward_workspace_bytes(s, dtype) + rows * s.d * 2 + rows * 4;
+}
+
+int gdn_forward_raw(const void* Q_raw, const void* K_raw, const void* V, const float* beta,
+                    const float* loggate, const float* S0, int N, int mask, int S, void* O,
+                    float* S_final, void* workspace, int64_t workspace_bytes, gdn_shape s,
+                    gdn_dtype dtype, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    GDN_TRY(check_dtype(dtype));
+    if (dtype != GDN_BF16) return fail(GDN_ERR_UNSUPPORTED, "gdn_forward_raw is built for bf16 data");
+    if (s.k != 64) return fail(GDN_ERR_UNSUPPORTED, "gdn_forward_raw is built for k=64");
+    GDN_TRY(check_NS(N, mask, S, s.k));
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{Q_raw, "Q_raw"}, {K_raw, "K_raw"}, {V, "V"}, {beta, "beta"},
+                        {loggate, "loggate"}, {O, "O"}, {S_final, "S_final"},
+                        {workspace, "workspace"}}));
+    GDN_TRY(check_opt_ptr(S0, "S0"));
+    if (!gdn::tc_available()) return fail(GDN_ERR_UNSUPPORTED, "tensor-core path not built");
+    const int64_t need = gdn_forward_raw_workspace_bytes(s, dtype);
+    if (workspace_bytes < need)
+        return fail(GDN_ERR_ARG, "workspace of %lld bytes is below the %lld needed",
+                    (long long)workspace_bytes, (long long)need);
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t rows = nc * s.k;
+    uint8_t* ws = (uint8_t*)workspace;
+    void* Wg = ws;
+    void* U = ws + rows * s.d * 2;
+    float* Sstates = (float*)(ws + 2 * rows * s.d * 2);
+    uint8_t* tail = ws + gdn_forward_workspace_bytes(s, dtype);
+    void* Kn = tail;                                    // the normalised keys
+    float* gsum = (float*)(tail + rows * s.d * 2);      // the chunk-local cumulative gates
+    GDN_TRY(gdn_chunk_wy_fused_raw(K_raw, V, beta, loggate, N, mask, S, 1, Wg, U, nullptr, Kn,
+                                   gsum, s, dtype, stream));
+    return launched(gdn::launch_scan(Q_raw, Kn, Wg, U, gsum, S0, O, S_final, Sstates, s.B * s.H,
+                                     s.T / s.k, true, st, true),
+                    "forward scan (raw queries)");
+}
+
 int gdn_decode(const void* Q, const void* K, const void* V, const float* beta,
                const float* loggate, float* S, void* O, int64_t B, int64_t Hk, int64_t Hv,
                int64_t n, int32_t d, gdn_dtype dtype, void* stream) {

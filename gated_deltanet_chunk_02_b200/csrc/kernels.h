@@ -24,9 +24,10 @@ cudaError_t launch_neumann_i8_simt(const float* A, float* T, int N, int mask, in
 // Inter-chunk state scan of the forward (scan.cu); k = 64, d = 128.
 // bf16: U is overwritten by V~ (fp16) and Sstates ([B*H*nchunk][d][d] fp16) by
 // the chunks' start states; f32 uses neither.
+// normalize_q (bf16): the query rows come raw and are L2-normalised in the output pass.
 cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, const float* g,
                         const float* S0, void* O, float* Sfin, void* Sstates, int64_t BH,
-                        int64_t nchunk, bool bf16, cudaStream_t st);
+                        int64_t nchunk, bool bf16, cudaStream_t st, bool normalize_q = false);
 
 // Decode steps (decode.cu); d = 128, S [B][Hv][d][d] fp32 updated in place.
 cudaError_t launch_decode(const void* Q, const void* K, const void* V, const float* beta,

@@ -17,9 +17,9 @@
 // alone (tiles fetched two chunks ahead by TMA, which one thread issues while
 // the others compute, the state slice held as fp32 mma.sync accumulator
 // fragments), writing V~ over U and each
-// chunk's start state S_c to the workspace; k_out_tc then forms O for every
-// chunk in parallel.  fp32 data: k_scan does the whole recurrence and O in
-// one pass with fp32 FMA loops.
+// chunk's start state S_c to the workspace; the output pass (k_output_tc in
+// tc.cu, on the tensor cores) then forms O for every chunk in parallel.  fp32
+// data: k_scan does the whole recurrence and O in one pass with fp32 FMA loops.
 #include <cuda.h>
 #include <cstring>
 
@@ -242,20 +242,6 @@ struct ScanMma {
     static constexpr int kPS = kSD + 8;           // pitch of the fp16 copy of S
 };
 
-__device__ __forceinline__ uint32_t bf2_to_h2(uint32_t x) {
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&x);
-    const float2 f = __bfloat1622float2(b);
-    const __half2 h = __floats2half2_rn(f.x, f.y);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                        uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -264,7 +250,6 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t ld32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
 __device__ __forceinline__ uint32_t pack_h2f(float a, float b) {
     const __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<const uint32_t*>(&h);
@@ -278,8 +263,8 @@ __device__ __forceinline__ uint32_t pack_b2f(float a, float b) {
 // bf16 forward in two kernels.  The recurrence is the only serial part, so it
 // runs alone (k_state_tc: per chunk V~ = U - W_g S^T, written over U as fp16,
 // the chunk's start state S_c stored as fp16, S <- gamma_last S + (V~ dec)^T K),
-// and the output of every chunk follows in parallel (k_out_tc:
-// O = diag(gamma) Q S_c^T + (Q K^T . Gamma . L) V~, the scores once per chunk).
+// and the output of every chunk follows in parallel (k_output_tc in tc.cu:
+// O = diag(gamma) Q S_c^T + (Q K^T . Gamma . L) V~ on the tensor cores).
 // ---------------------------------------------------------------------------
 constexpr int kStThreads = 128;
 constexpr int kStStages = 3;
@@ -549,133 +534,6 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     }
 }
 
-struct OutTile {
-    static constexpr int kP = kSD + 8;                         // staged row pitch, elements
-    static constexpr int kQ = kSK * kP * 2;                    // Q, K, V~ tiles
-    static constexpr int kS = kSD * kP * 2;                    // S_c (fp16)
-    static constexpr int kA = kSK * ScanMma::kP16 * 2;         // scores (fp16)
-    static constexpr int bytes = 3 * kQ + kS + kA + kSK * 4;
-};
-
-__global__ void __launch_bounds__(kStThreads)
-k_out_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-         const __half* __restrict__ Vt, const float* __restrict__ g, const __half* __restrict__ Sst,
-         __nv_bfloat16* __restrict__ O, int64_t nctot) {
-    constexpr int P = OutTile::kP;
-    constexpr int P16 = ScanMma::kP16;
-    extern __shared__ __align__(16) uint8_t smem[];
-    __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem);
-    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem + OutTile::kQ);
-    __half* sV = reinterpret_cast<__half*>(smem + 2 * OutTile::kQ);
-    __half* sS = reinterpret_cast<__half*>(smem + 3 * OutTile::kQ);
-    __half* sA = reinterpret_cast<__half*>(smem + 3 * OutTile::kQ + OutTile::kS);
-    float* sg = reinterpret_cast<float*>(smem + 3 * OutTile::kQ + OutTile::kS + OutTile::kA);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int gr = lane >> 2, gc = (lane & 3) * 2;
-    const int mt = 16 * warp;
-    for (int64_t ch = blockIdx.x; ch < nctot; ch += gridDim.x) {
-        const int64_t row0 = ch * kSK;
-        __syncthreads();                           // the previous chunk's tiles are read
-        for (int e = tid; e < kSK * 16; e += kStThreads) {
-            const int r = e >> 4, c = (e & 15) * 8;
-            cp_async16(sQ + r * P + c, Q + (row0 + r) * kSD + c);
-            cp_async16(sK + r * P + c, K + (row0 + r) * kSD + c);
-            cp_async16(sV + r * P + c, Vt + (row0 + r) * kSD + c);
-        }
-        for (int e = tid; e < kSD * 16; e += kStThreads) {
-            const int r = e >> 4, c = (e & 15) * 8;
-            cp_async16(sS + r * P + c, Sst + (ch * kSD + r) * kSD + c);
-        }
-        if (tid < kSK / 4) cp_async16(sg + tid * 4, g + row0 + tid * 4);
-        cp_async_commit();
-        cp_async_wait0();
-        __syncthreads();
-        const int t0 = mt + gr, t1 = t0 + 8;
-        const float g0 = sg[t0], g1 = sg[t1];
-        // scores . Gamma . L on this warp's rows (column tiles up to the diagonal)
-        {
-            float acc[8][4];
-#pragma unroll
-            for (int n = 0; n < 8; ++n)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-#pragma unroll
-            for (int k0 = 0; k0 < kSD; k0 += 16) {
-                const uint32_t a0 = ld32(sQ + t0 * P + k0 + gc);
-                const uint32_t a1 = ld32(sQ + t1 * P + k0 + gc);
-                const uint32_t a2 = ld32(sQ + t0 * P + k0 + gc + 8);
-                const uint32_t a3 = ld32(sQ + t1 * P + k0 + gc + 8);
-#pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    if (8 * n > mt + 15) continue;
-                    mma_bf16(acc[n], a0, a1, a2, a3, ld32(sK + (8 * n + gr) * P + k0 + gc),
-                             ld32(sK + (8 * n + gr) * P + k0 + gc + 8));
-                }
-            }
-#pragma unroll
-            for (int n = 0; n < 8; ++n) {
-                const int c = 8 * n + gc;
-                const float x00 = c <= t0 ? acc[n][0] * exp_e(g0 - sg[c]) : 0.f;
-                const float x01 = c + 1 <= t0 ? acc[n][1] * exp_e(g0 - sg[c + 1]) : 0.f;
-                const float x10 = c <= t1 ? acc[n][2] * exp_e(g1 - sg[c]) : 0.f;
-                const float x11 = c + 1 <= t1 ? acc[n][3] * exp_e(g1 - sg[c + 1]) : 0.f;
-                *reinterpret_cast<uint32_t*>(sA + t0 * P16 + c) = pack_h2f(x00, x01);
-                *reinterpret_cast<uint32_t*>(sA + t1 * P16 + c) = pack_h2f(x10, x11);
-            }
-        }
-        __syncwarp();                              // sA rows of this warp
-        // P = Q S_c^T (all 128 state rows), times gamma
-        float pacc[16][4];
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) pacc[n][i] = 0.f;
-#pragma unroll
-        for (int k0 = 0; k0 < kSD; k0 += 16) {
-            const uint32_t a0 = bf2_to_h2(ld32(sQ + t0 * P + k0 + gc));
-            const uint32_t a1 = bf2_to_h2(ld32(sQ + t1 * P + k0 + gc));
-            const uint32_t a2 = bf2_to_h2(ld32(sQ + t0 * P + k0 + gc + 8));
-            const uint32_t a3 = bf2_to_h2(ld32(sQ + t1 * P + k0 + gc + 8));
-#pragma unroll
-            for (int n = 0; n < 16; ++n)
-                mma_f16(pacc[n], a0, a1, a2, a3, ld32(sS + (8 * n + gr) * P + k0 + gc),
-                        ld32(sS + (8 * n + gr) * P + k0 + gc + 8));
-        }
-        const float gam0 = exp_e(g0), gam1 = exp_e(g1);
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            pacc[n][0] *= gam0;
-            pacc[n][1] *= gam0;
-            pacc[n][2] *= gam1;
-            pacc[n][3] *= gam1;
-        }
-        // O += scores V~ over the causal token tiles
-        for (int k0 = 0; k0 <= mt; k0 += 16) {
-            const uint32_t a0 = ld32(sA + t0 * P16 + k0 + gc);
-            const uint32_t a1 = ld32(sA + t1 * P16 + k0 + gc);
-            const uint32_t a2 = ld32(sA + t0 * P16 + k0 + gc + 8);
-            const uint32_t a3 = ld32(sA + t1 * P16 + k0 + gc + 8);
-            const int krow = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int n = 0; n < 16; ++n) {
-                const uint32_t addr = (uint32_t)__cvta_generic_to_shared(sV + krow * P + 8 * n);
-                uint32_t b0, b1;
-                asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-                             : "=r"(b0), "=r"(b1) : "r"(addr));
-                mma_f16(pacc[n], a0, a1, a2, a3, b0, b1);
-            }
-        }
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            const int v = 8 * n + gc;
-            *reinterpret_cast<__nv_bfloat162*>(O + (row0 + t0) * kSD + v) =
-                __floats2bfloat162_rn(pacc[n][0], pacc[n][1]);
-            *reinterpret_cast<__nv_bfloat162*>(O + (row0 + t1) * kSD + v) =
-                __floats2bfloat162_rn(pacc[n][2], pacc[n][3]);
-        }
-    }
-}
-
 // tensor maps of the recurrence's stages
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -723,7 +581,7 @@ static bool map_f32_1d(CUtensorMap* m, const void* base, int64_t rows, int box_r
 
 cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, const float* g,
                         const float* S0, void* O, float* Sfin, void* Sstates, int64_t BH,
-                        int64_t nchunk, bool bf16, cudaStream_t st) {
+                        int64_t nchunk, bool bf16, cudaStream_t st, bool normalize_q) {
     dim3 grid((unsigned)BH, kSD / kDV);
     if (bf16) {
         const size_t s1 = kStStages * StTile::kStage + (size_t)kDV * ScanMma::kPS * 2 +
@@ -742,17 +600,7 @@ cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, c
                                                  (__half*)Sstates, Sfin, nchunk, status_ptr());
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(k_out_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 OutTile::bytes);
-        if (e != cudaSuccess) return e;
-        int dev = 0, sms = 148;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int64_t nct = BH * nchunk, cap = (int64_t)sms * 2;
-        k_out_tc<<<(unsigned)(nct < cap ? nct : cap), kStThreads, OutTile::bytes, st>>>(
-            (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __half*)U, g,
-            (const __half*)Sstates, (__nv_bfloat16*)O, nct);
-        return cudaGetLastError();
+        return launch_output_tc(Q, K, U, g, Sstates, O, BH * nchunk, normalize_q, st);
     }
     auto smem_for = [](int stage, int nstages) {
         return (size_t)(nstages * stage) + (size_t)(kDV * (kSD + 1) + 2 * kSK * kDV +

@@ -1705,6 +1705,255 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
 }
 
 // ------------------------------------------------------------------------- //
+// The chunk-wise forward's output pass on the tensor cores (k = 64, bf16 data)
+// ------------------------------------------------------------------------- //
+// O = s (diag(gamma) Q S_c^T + (Q K^T (.) Gamma (.) L) V~) per chunk, with
+// gamma_i = e^{g_i}, Gamma_ij = e^{g_i - g_j}, L the lower triangle including the
+// diagonal, S_c the chunk's start state (fp16, from the state recurrence), V~
+// the corrected values (fp16) and s = 1 / ||q_i|| when the queries come raw
+// (normalised here, since s scales a whole row of O), else 1.  A tile is two
+// chunks (128 token rows) and one CTA of 8 warps per SM works through tiles:
+//   G  = Q K^T                (bf16; M = N = 128, K = d)     -> TMEM [0, 128)
+//   epilogue: A2 = G (.) Gamma (.) L on the row's own chunk block and 0 on the
+//             other (fp16, into K's buffer); Q to fp16 in place
+//   P0 = Q S_0^T, P1 = Q S_1^T (fp16; one product per chunk's start state)
+//                                                            -> [128, 256), [256, 384)
+//   Oi = A2 V~                (fp16; K = the tile's 128 tokens) -> [0, 128)
+//   epilogue: O = s (gamma P_c + Oi) in bf16 through V~'s buffer, TMA store.
+// Thread (r, h) owns tile row r (its TMEM lane) and column half h.  Waits are
+// bounded as in the chunk kernel: after one runs out nobody leaves the tile
+// early, no work is started, and the CTA stops together at the next tile.
+struct ParamsOut {
+    int64_t rows;        // B*H*T
+    int64_t nchunks;     // B*H*T / 64
+    int ntiles;
+    int normalize_q;
+    int* status;
+};
+constexpr int kOutThreads = 256;
+constexpr int kOutOp = kRows * kD * 2;               // one [2][128][64] 16-bit operand: 32 KB
+// Q | K, then A2 | V~, then O | S_0 | S_1 | g | the row norms' halves | control
+constexpr int kOutSmem = 5 * kOutOp + kRows * 4 + 2 * kRows * 4;
+
+struct __align__(8) CtrlOut {
+    uint64_t full;       // Q, K, S_0, S_1, g of the tile landed
+    uint64_t fullV;      // V~ landed
+    uint64_t mma;        // the products completed
+    uint64_t drain;      // after an expired wait: the leader's products are done
+    uint32_t tmem;
+    int abort;
+};
+
+__global__ void __launch_bounds__(kOutThreads, 1)
+k_output_tc(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+         const __grid_constant__ CUtensorMap mVt, const __grid_constant__ CUtensorMap mS,
+         const __grid_constant__ CUtensorMap mG, const __grid_constant__ CUtensorMap mO,
+         const ParamsOut p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((su32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0) raise_status(p.status, kStatusSmemAlign);
+        return;
+    }
+    uint8_t* sQ = smem;
+    uint8_t* sK = smem + kOutOp;                     // K, then A2
+    uint8_t* sV = smem + 2 * kOutOp;                 // V~, then O
+    uint8_t* sS0 = smem + 3 * kOutOp;
+    uint8_t* sS1 = smem + 4 * kOutOp;
+    float* sg = reinterpret_cast<float*>(smem + 5 * kOutOp);
+    float* sqs = sg + kRows;                          // [2][128] halves of ||q||^2
+    CtrlOut* ctrl = reinterpret_cast<CtrlOut*>(smem + kOutSmem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = warp >> 2;
+    const int r = ((warp & 3) << 5) | lane;
+    const int c = r >> 6, i = r & 63;                 // chunk of the row in the tile, row in it
+    const bool leader = threadIdx.x == 0;
+    if (leader) {
+        mbar_init(&ctrl->full, 1);
+        mbar_init(&ctrl->fullV, 1);
+        mbar_init(&ctrl->mma, 1);
+        mbar_init(&ctrl->drain, 1);
+        ctrl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tmem_alloc(&ctrl->tmem, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = ctrl->tmem;
+    const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
+    const volatile int* const abortp = &ctrl->abort;
+    auto live = [&]() { return *abortp == 0; };
+    auto fail_wait = [&]() {
+        atomicExch(&ctrl->abort, 1);
+        raise_status(p.status, kStatusTimeout);
+    };
+    uint32_t mma_phase = 0;
+    auto wait_mma = [&]() {
+        if (!(live() && mbar_wait(&ctrl->mma, mma_phase))) fail_wait();
+        mma_phase ^= 1;
+        tc_fence_after();
+    };
+    int main_issued = 0, v_issued = 0;
+    auto issue_main = [&](int tile) {
+        if (tile >= p.ntiles || !live()) return;
+        ++main_issued;
+        const int y = tile * kRows;
+        const int ys = 2 * tile * kRows;              // S rows of the tile's first chunk
+        mbar_expect_tx(&ctrl->full, 4 * kOutOp + kRows * 4);
+        tma_load_2d(sQ, &mQ, 0, y, &ctrl->full);
+        tma_load_2d(sQ + kRows * 128, &mQ, 64, y, &ctrl->full);
+        tma_load_2d(sK, &mK, 0, y, &ctrl->full);
+        tma_load_2d(sK + kRows * 128, &mK, 64, y, &ctrl->full);
+        tma_load_2d(sS0, &mS, 0, ys, &ctrl->full);
+        tma_load_2d(sS0 + kRows * 128, &mS, 64, ys, &ctrl->full);
+        tma_load_2d(sS1, &mS, 0, ys + kRows, &ctrl->full);
+        tma_load_2d(sS1 + kRows * 128, &mS, 64, ys + kRows, &ctrl->full);
+        tma_load_1d(sg, &mG, y, &ctrl->full);
+    };
+    auto issue_v = [&](int tile) {
+        if (tile >= p.ntiles || !live()) return;
+        ++v_issued;
+        const int y = tile * kRows;
+        mbar_expect_tx(&ctrl->fullV, kOutOp);
+        tma_load_2d(sV, &mVt, 0, y, &ctrl->fullV);
+        tma_load_2d(sV + kRows * 128, &mVt, 64, y, &ctrl->fullV);
+    };
+    if (leader) {
+        issue_main(blockIdx.x);
+        issue_v(blockIdx.x);
+    }
+    bool ok = true, stored = false;
+    for (int n = 0;; ++n) {
+        const int tile = blockIdx.x + n * gridDim.x;
+        if (tile >= p.ntiles) break;
+        const uint32_t par = (uint32_t)(n & 1);
+        if (!(live() && mbar_wait(&ctrl->full, par))) fail_wait();
+        if (bar_sync_or(1, kOutThreads, !live())) { ok = false; break; }
+        if (leader && live()) {
+            if (stored) {                              // the last O store has read V~'s buffer
+                bulk_wait_read();
+                issue_v(tile);
+            }
+            tc_fence_after();
+            constexpr uint32_t id = idesc_f16(1, 0, 0, 128, 128);     // bf16, both K-major
+            const uint32_t qb = su32(sQ), kb = su32(sK);
+#pragma unroll 1
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t o = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+                mma_ss(tm, sdesc(qb + o, 16, 1024), sdesc(kb + o, 16, 1024), id, kk > 0);
+            }
+            mma_commit(&ctrl->mma);
+        }
+        wait_mma();
+        // ---- A2 = G (.) Gamma (.) L (fp16) into K's buffer; Q to fp16 in place ----
+        const float gi = sg[r];
+        {
+            const float* gcol = sg + 64 * c + 32 * h;
+            float v[32];
+            if (32 * h > i) {                          // the whole piece lies above the diagonal
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
+            } else {
+                tmem_ld32(tl + 64 * c + 32 * h, v);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj)
+                    v[jj] = 32 * h + jj <= i ? v[jj] * exp_e(gi - gcol[jj]) : 0.f;
+            }
+            st_op32<false>(sK, r, 2 * c + h, v);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) v[jj] = 0.f;
+            st_op32<false>(sK, r, 2 * (1 - c) + h, v);   // the other chunk's keys: zero
+        }
+        {
+            float ss = 0.f;
+            const uint32_t qb = su32(sQ);
+#pragma unroll
+            for (int q = 8 * h; q < 8 * h + 8; ++q) {
+                const uint32_t a = qb + op_off(r, q);
+                const uint4 u = lds128(a);
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+                uint32_t o4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float lo = __uint_as_float(w4[e] << 16);
+                    const float hi = __uint_as_float(w4[e] & 0xffff0000u);
+                    ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+                    o4[e] = pack_h2(lo, hi);
+                }
+                sts128(a, make_uint4(o4[0], o4[1], o4[2], o4[3]));
+            }
+            sqs[h * kRows + r] = ss;
+        }
+        fence_async_smem();
+        tc_fence_before();
+        bar_sync(1, kOutThreads);
+        tc_fence_after();
+        if (leader && live()) {
+            if (!(mbar_wait(&ctrl->fullV, (uint32_t)((v_issued - 1) & 1)))) fail_wait();
+            if (live()) {
+                constexpr uint32_t idk = idesc_f16(0, 0, 0, 128, 128);   // fp16, both K-major
+                constexpr uint32_t idm = idesc_f16(0, 0, 1, 128, 128);   // fp16, B MN-major
+                const uint32_t qb = su32(sQ), ab = su32(sK), vb = su32(sV);
+                const uint32_t s0 = su32(sS0), s1 = su32(sS1);
+#pragma unroll 1
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t o = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+                    const uint64_t a = sdesc(qb + o, 16, 1024);
+                    mma_ss(tm + 128, a, sdesc(s0 + o, 16, 1024), idk, kk > 0);
+                    mma_ss(tm + 256, a, sdesc(s1 + o, 16, 1024), idk, kk > 0);
+                    mma_ss(tm, sdesc(ab + o, 16, 1024), sdesc(vb + kk * 2048, kRows * 128, 1024),
+                           idm, kk > 0);
+                }
+                mma_commit(&ctrl->mma);
+            }
+        }
+        wait_mma();
+        if (leader) issue_main(tile + gridDim.x);      // Q, K, S, g are read
+        // ---- O = s (gamma P_c + Oi), bf16, into V~'s buffer ----
+        {
+            const float ss = sqs[r] + sqs[kRows + r];
+            const float sc = p.normalize_q ? (ss > 0.f ? rsqrtf(ss) : 0.f) : 1.f;
+            const float gam = exp_e(gi);
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc) {
+                const int col = 64 * h + 32 * pc;
+                float pv[32], ov[32];
+                tmem_ld32(tl + 128 + 128 * c + col, pv);
+                tmem_ld32(tl + col, ov);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) ov[jj] = sc * fmaf(gam, pv[jj], ov[jj]);
+                st_op32<true>(sV, r, 2 * h + pc, ov);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        bar_sync(1, kOutThreads);
+        if (leader && live()) {
+            tma_store_2d(&mO, 0, tile * kRows, sV);
+            tma_store_2d(&mO, 64, tile * kRows, sV + kRows * 128);
+            bulk_commit();
+        }
+        stored = true;
+    }
+    if (!ok || !live()) {                              // drain, bounded, deaf to the flag
+        if (leader) {
+            mma_commit(&ctrl->drain);
+            mbar_wait(&ctrl->drain, 0);
+            if (main_issued > 0) mbar_wait(&ctrl->full, (uint32_t)((main_issued - 1) & 1));
+            if (v_issued > 0) mbar_wait(&ctrl->fullV, (uint32_t)((v_issued - 1) & 1));
+        }
+    }
+    if (leader) bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+// ------------------------------------------------------------------------- //
 // INT8 truncated Neumann series on the tensor cores (k = 64)
 // ------------------------------------------------------------------------- //
 // Same tile / slot structure as k_chunk_tc: a tile stacks two 64-token chunks,
@@ -3197,6 +3446,31 @@ cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, in
     const int sms = tcg::num_sms();
     const int grid = nc < sms ? (int)nc : sms;
     tcg::k_neumann256_tc<<<grid, tcg::k256Threads, tcg::k256Smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_output_tc(const void* Q, const void* K, const void* Vt, const float* g,
+                             const void* Sst, void* O, int64_t nchunks, bool normalize_q,
+                             cudaStream_t st) {
+    using namespace tcg;
+    const int64_t rows = nchunks * 64;
+    CUtensorMap mQ, mK, mV, mS, mG, mO;
+    if (!map_kd(&mQ, Q, rows) || !map_kd(&mK, K, rows) || !map_kd(&mV, Vt, rows) ||
+        !map_kd(&mS, Sst, nchunks * kD) || !map_vec(&mG, g, rows) || !map_kd(&mO, O, rows))
+        return cudaErrorInvalidValue;
+    ParamsOut p;
+    memset(&p, 0, sizeof p);
+    p.rows = rows;
+    p.nchunks = nchunks;
+    p.ntiles = (int)((rows + kRows - 1) / kRows);
+    p.normalize_q = normalize_q ? 1 : 0;
+    p.status = status_ptr();
+    const int smem = kOutSmem + (int)sizeof(CtrlOut);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_output_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = p.ntiles < num_sms() ? p.ntiles : num_sms();
+    k_output_tc<<<grid, kOutThreads, smem, st>>>(mQ, mK, mV, mS, mG, mO, p);
     return cudaGetLastError();
 }
 

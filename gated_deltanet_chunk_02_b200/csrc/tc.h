@@ -44,6 +44,12 @@ cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int
 cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, const float* g,
                             int N, int mask, int S, int gated, void* W, void* U, float* Tout,
                             int64_t nc, int k, cudaStream_t st);
+// the chunk-wise forward's output pass (k = 64, bf16): O = s (diag(gamma) Q S_c^T +
+// (Q K^T . Gamma . L) V~) from the chunks' start states Sst (fp16 [nchunks][128][128])
+// and V~ (fp16); s = 1 / ||q|| when normalize_q, else 1
+cudaError_t launch_output_tc(const void* Q, const void* K, const void* Vt, const float* g,
+                             const void* Sst, void* O, int64_t nchunks, bool normalize_q,
+                             cudaStream_t st);
 // tests of the bounded waits: the next launch_fused_tc on this host thread
 // leaves tile `tile`'s K (v = 0) or V (v = 1) load unissued and bounds every
 // wait by `timeout_ns`

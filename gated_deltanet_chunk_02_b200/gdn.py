@@ -28,7 +28,8 @@ EXPORTS = [
     "gdn_invert_neumann_i8", "gdn_invert_neumann_i8_residual", "gdn_invert_neumann_i16",
     "gdn_chunk_wy_fused", "gdn_chunk_wy_fused_raw", "gdn_forward",
     "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_decode", "gdn_get_status",
-    "gdn_last_error", "gdn_launch_count", "gdn_debug_arm_wait_expiry",
+    "gdn_last_error", "gdn_launch_count", "gdn_debug_arm_wait_expiry", "gdn_forward_raw",
+    "gdn_forward_raw_workspace_bytes",
 ]
 
 
@@ -75,6 +76,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                    _P],
         "gdn_forward": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _I64, S, _I, _P],
         "gdn_forward_workspace_bytes": [S, _I],
+        "gdn_forward_raw": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _I64, S, _I, _P],
+        "gdn_forward_raw_workspace_bytes": [S, _I],
         "gdn_forward_static": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, S, _I, _P],
         "gdn_decode": [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int32, _I,
                        _P],
@@ -88,6 +91,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f.argtypes = args
         f.restype = _I
     lib.gdn_forward_workspace_bytes.restype = _I64
+    lib.gdn_forward_raw_workspace_bytes.restype = _I64
     lib.gdn_launch_count.restype = _I64
     lib.gdn_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -232,6 +236,23 @@ def gdn_forward(Q, K, V, beta, g, S0, N, mask, S, exact, O, S_final, workspace, 
     _check(load().gdn_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(g), _ptr(S0), N,
                               int(mask), S, int(exact), _ptr(O), _ptr(S_final), _ptr(workspace),
                               ws, shape_of(K, k), _dtype(K), _stream(stream)))
+
+
+def gdn_forward_raw_workspace_bytes(K, k):
+    """Scratch bytes ``gdn_forward_raw`` needs for K's shape (bf16)."""
+    return int(load().gdn_forward_raw_workspace_bytes(shape_of(K, k), _dtype(K)))
+
+
+def gdn_forward_raw(Q_raw, K_raw, V, beta, loggate, S0, N, mask, S, O, S_final, workspace, k=64,
+                    stream=None):
+    """Chunk-wise forward from un-normalised query and key rows and per-token
+    log-gates (normalised and summed in the kernels); O and the final state as
+    in ``gdn_forward``."""
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().gdn_forward_raw(_ptr(Q_raw), _ptr(K_raw), _ptr(V), _ptr(beta), _ptr(loggate),
+                                  _ptr(S0), N, int(mask), S, _ptr(O), _ptr(S_final),
+                                  _ptr(workspace), ws, shape_of(K_raw, k), _dtype(K_raw),
+                                  _stream(stream)))
 
 
 def gdn_forward_static(Q, K, V, beta, g, S0, N, mask, S, exact, O, S_final, k=64, stream=None):

@@ -221,7 +221,9 @@ int gdn_chunk_wy_fused_raw(const void* K_raw, const void* V, const float* beta,
  * least gdn_forward_workspace_bytes(s, dtype) bytes (W_g and U for every
  * chunk in dtype, then A and T in f32); its contents on entry do not matter.
  * k = 64.  The inter-chunk scan splits the d_v rows of the state across CTAs
- * (rows of S never mix), each CTA walking its head's chunks in order.
+ * (rows of S never mix), each CTA walking its head's chunks in order; for
+ * bf16 data the output pass then forms O for every chunk in parallel on the
+ * tensor cores (two chunks per 128-row tile).
  */
 int gdn_forward(const void* Q, const void* K, const void* V, const float* beta,
                 const float* g, const float* S0, int N, int mask, int S,
@@ -229,6 +231,27 @@ int gdn_forward(const void* Q, const void* K, const void* V, const float* beta,
                 int64_t workspace_bytes, gdn_shape s, gdn_dtype dtype,
                 void* stream);
 int64_t gdn_forward_workspace_bytes(gdn_shape s, gdn_dtype dtype);
+
+/*
+ * gdn_forward with its prologue: the steps just before the chunk system in a
+ * layer (the gist.science summary's Problem Statement places the inversion
+ * inside this layer).  Q_raw and K_raw rows are L2-normalised in the kernels,
+ * q <- q / ||q||, k <- k / ||k|| (norms in fp32; an all-zero row stays zero;
+ * the keys are rounded to bf16 like gdn_chunk_wy_fused_raw's, the queries'
+ * scale is applied to each output row in fp32), and loggate holds each
+ * token's own log-gate, summed chunk-locally.  The truncated series (exact =
+ * 0 of gdn_forward) gives T.  In: Q_raw, K_raw, V [B,H,T,d] bf16, beta,
+ * loggate [B,H,T] f32, S0 as in gdn_forward.  Out: O, S_final as in
+ * gdn_forward.  `workspace` holds at least
+ * gdn_forward_raw_workspace_bytes(s, dtype) bytes: gdn_forward's scratch,
+ * then the normalised keys (bf16) and the cumulative log-gates (f32).
+ * bf16 data, k = 64; GDN_ERR_UNSUPPORTED otherwise.
+ */
+int gdn_forward_raw(const void* Q_raw, const void* K_raw, const void* V, const float* beta,
+                    const float* loggate, const float* S0, int N, int mask, int S,
+                    void* O, float* S_final, void* workspace, int64_t workspace_bytes,
+                    gdn_shape s, gdn_dtype dtype, void* stream);
+int64_t gdn_forward_raw_workspace_bytes(gdn_shape s, gdn_dtype dtype);
 
 /*
  * gdn_forward without a workspace argument: it allocates nothing.  The pages

@@ -87,3 +87,59 @@ def test_c5_long_context(c5, N, mask, S, exact):
     Sg = Sf.reshape(16, 128, 128)[heads]
     assert rel(Og, Or) <= TOL_BF16
     assert rel(Sg, Sr) <= TOL_BF16
+
+
+@pytest.mark.parametrize("N,mask,S", [(3, 1, 8), (3, 1, 0), (2, 0, 1)])
+def test_forward_odd_chunk_count(N, mask, S):
+    """21 chunks: the output pass's last 128-row tile holds a single chunk."""
+    w = Workload(B=1, H=3, T=448, k=64, dtype="bf16")
+    inp = make_inputs(w, seed=12, with_q=True)
+    d = {key: v.cuda() for key, v in inp.items()}
+    Ot, Sf = run_forward(d, N, mask, S, 0)
+    Or, Sr = oracle_forward(inp, np.arange(3), 64, N, mask, S, 0)
+    assert rel(Ot.reshape(3, 448, 128), Or) <= TOL_BF16
+    assert rel(Sf.reshape(3, 128, 128), Sr) <= TOL_BF16
+
+
+def raw_oracle(inp_raw, Q_raw, BH, T_len, N, mask, S, S0=None):
+    """The oracle with its own prologue: query and key rows normalised, gates summed."""
+    k, d = 64, 128
+    n = T_len // k
+    Qn = O.l2_normalize_rows(as_f64_numpy(Q_raw)).reshape(BH, n, k, d)
+    Kn = O.l2_normalize_rows(as_f64_numpy(inp_raw["K"])).reshape(BH, n, k, d)
+    V = as_f64_numpy(inp_raw["V"]).reshape(BH, n, k, d)
+    b = as_f64_numpy(inp_raw["beta"]).reshape(BH, n, k)
+    g = O.chunk_cumsum(as_f64_numpy(inp_raw["loggate"]), k).reshape(BH, n, k)
+    T = O.invert_neumann(O.build_A(Kn, b, g), N, bool(mask), S)
+    Oo, Sf = O.chunk_forward(Qn, Kn, V, b, g, T, S0)
+    return Oo.reshape(BH, T_len, d), Sf
+
+
+@pytest.mark.parametrize("B,H,T_len", [(1, 2, 512), (1, 3, 448)])
+@pytest.mark.parametrize("N,mask,S", [(3, 1, 8), (3, 0, 0)])
+@pytest.mark.parametrize("with_s0", [False, True])
+def test_forward_raw_normalises_queries_and_keys(B, H, T_len, N, mask, S, with_s0):
+    """gdn_forward_raw: raw key rows, query rows of any length (each row scaled
+    by its own factor) and per-token log-gates, against the oracle's
+    normalisation, cumulative sum and forward."""
+    w = Workload(B=B, H=H, T=T_len, k=64, dtype="bf16")
+    inp = make_inputs(w, seed=13, with_q=True, raw_keys=True)
+    scale = 0.25 + 4.0 * torch.rand(B, H, T_len, 1, generator=torch.Generator().manual_seed(9))
+    Q_raw = (inp["Q"].float() * scale).to(torch.bfloat16)
+    Q_raw[0, 0, 5] = 0                                   # an all-zero query row: O row zero
+    d = {key: v.cuda() for key, v in inp.items()}
+    S0 = None
+    if with_s0:
+        S0 = torch.randn(B, H, 128, 128, generator=torch.Generator().manual_seed(4)) * 0.1
+    Ot = torch.empty_like(d["K"])
+    Sf = torch.empty(B, H, 128, 128, device="cuda")
+    ws = torch.empty(gdn.gdn_forward_raw_workspace_bytes(d["K"], 64), dtype=torch.uint8,
+                     device="cuda")
+    gdn.gdn_forward_raw(Q_raw.cuda(), d["K"], d["V"], d["beta"], d["loggate"],
+                        None if S0 is None else S0.cuda(), N, mask, S, Ot, Sf, ws)
+    assert gdn.gdn_get_status() == gdn.GDN_OK
+    Or, Sr = raw_oracle(inp, Q_raw, B * H, T_len, N, mask, S,
+                        None if S0 is None else S0.double().numpy().reshape(-1, 128, 128))
+    assert rel(Ot.reshape(B * H, T_len, 128), Or) <= TOL_BF16
+    assert rel(Sf.reshape(B * H, 128, 128), Sr) <= TOL_BF16
+    assert torch.count_nonzero(Ot[0, 0, 5]) == 0
