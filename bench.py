@@ -396,8 +396,9 @@ def workload_config(w: dict, nc: int, rotate: int = ROTATE) -> dict:
 
 
 # component kernels that take the series order / mask, and the residual order
-SERIES_KERNELS = ("neumann", "newton", "fused_raw", "int8", "int8_residual", "int16", "forward")
-RESIDUAL_KERNELS = ("neumann", "fused_raw", "int8_residual", "forward")
+SERIES_KERNELS = ("neumann", "newton", "fused_raw", "int8", "int8_residual", "int16",
+                  "int16_residual", "forward")
+RESIDUAL_KERNELS = ("neumann", "fused_raw", "int8_residual", "int16_residual", "forward")
 
 
 def run_component(args, world, rank, local, dev) -> int:
@@ -424,7 +425,7 @@ def run_component(args, world, rank, local, dev) -> int:
         st["A"] = torch.empty(wl.B, wl.H, wl.T // k, k, k, device=dev)
         st["T"] = torch.empty_like(st["A"])
         if kern in ("neumann", "newton", "blocked", "fwdsub", "int8", "int8_residual", "int16",
-                    "wy"):
+                    "int16_residual", "wy"):
             gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
         if kern == "wy":
             gdn.gdn_invert_fwdsub(st["A"], st["T"], stream=stream)
@@ -459,6 +460,9 @@ def run_component(args, world, rank, local, dev) -> int:
                                                stream=stream)
         elif kern == "int16":
             gdn.gdn_invert_neumann_i16(st["A"], st["T"], args.N, args.mask, stream=stream)
+        elif kern == "int16_residual":
+            gdn.gdn_invert_neumann_i16_residual(st["A"], st["T"], args.N, args.mask, args.S,
+                                                stream=stream)
         elif kern == "build_A":
             gdn.gdn_build_A(st["K"], st["beta"], st["g"], st["A"], k, stream=stream)
         elif kern == "wy":
@@ -501,6 +505,7 @@ def run_component(args, world, rank, local, dev) -> int:
         "int8": (2 * kk2, (args.N - 1) * 2 * k ** 3),
         "int16": (2 * kk2, (args.N - 1) * 2 * k ** 3),
         "int8_residual": (2 * kk2, (args.N - 1 + args.S + 1) * 2 * k ** 3),
+        "int16_residual": (2 * kk2, (args.N - 1 + args.S + 1) * 2 * k ** 3),
         "build_A": (kd + 8 * k + kk2, 2 * k * k * d),
         "wy": (kk2 + 2 * kd + 4 * k + 2 * kd, 4 * k * k * d),
         "forward": (4 * kd + 8 * k, algorithmic_flops_per_chunk(k, d, args.N, args.S)
@@ -510,7 +515,7 @@ def run_component(args, world, rank, local, dev) -> int:
     peaks, peak_kind = load_peaks()
     # the integer kernels' products are int8 MMAs: their tensor peak is the
     # measured bf16 peak times the nominal int8 : bf16 ratio (4.5 : 2.25)
-    integer = kern in ("int8", "int8_residual", "int16")
+    integer = kern in ("int8", "int8_residual", "int16", "int16_residual")
     tc_peak = float(peaks["bf16_tflops"]) * (2.0 if integer else 1.0)
     tc_kind = peak_kind + (" x 2 (nominal int8:bf16 ratio)" if integer else "")
     gbs = bytes_l / (ms_step * 1e-3) / 1e9
@@ -713,7 +718,7 @@ def main(argv=None) -> int:
     ap.add_argument("--mask", type=int, default=WORKLOAD["mask"], help="band mask on/off")
     ap.add_argument("--kernel", default="fused",
                     choices=["fused", "fused_raw", "neumann", "newton", "blocked", "fwdsub", "int8",
-                             "int8_residual", "int16",
+                             "int8_residual", "int16", "int16_residual",
                              "build_A", "wy", "forward", "decode", "error"],
                     help="time one component instead of the fused step (not the headline)")
     ap.add_argument("--k", type=int, default=None, help="chunk size for --kernel runs")

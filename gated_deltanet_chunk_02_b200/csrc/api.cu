@@ -237,6 +237,22 @@ int gdn_invert_neumann_i16(const float* A, float* T, int N, int mask, int16_t* q
                     "neumann int16 (tcgen05)");
 }
 
+int gdn_invert_neumann_i16_residual(const float* A, float* T, int N, int mask, int S,
+                                    gdn_shape s, void* stream) {
+    int64_t nc;
+    GDN_TRY(check_shape(s, &nc));
+    if (s.k != 64) return fail(GDN_ERR_UNSUPPORTED, "the INT16 path is built for k = 64");
+    if (N < 1 || N > 8) return fail(GDN_ERR_ARG, "INT16 Neumann order N=%d outside [1, 8]", N);
+    if (mask != 0 && mask != 1) return fail(GDN_ERR_ARG, "mask must be 0 or 1");
+    if (S < 1 || S > 64) return fail(GDN_ERR_ARG, "residual steps S=%d outside [1, 64]", S);
+    if (nc == 0) return GDN_OK;
+    GDN_TRY(check_ptrs({{A, "A"}, {T, "T"}}));
+    if (!gdn::tc_i8_available()) return fail(GDN_ERR_UNSUPPORTED, "integer tensor-core path not built");
+    return launched(gdn::launch_neumann_i16_tc(A, T, N, mask, nullptr, nullptr, nullptr, nc,
+                                               (cudaStream_t)stream, S),
+                    "neumann int16 with residual (tcgen05)");
+}
+
 int gdn_chunk_wy_fused(const void* K, const void* V, const float* beta, const float* g, int N,
                        int mask, int S, int gated, void* W, void* U, float* T_out, gdn_shape s,
                        gdn_dtype dtype, void* stream) {

@@ -359,7 +359,7 @@ __device__ __forceinline__ void fetch_state(uint8_t* st, uint64_t* bar, const CU
 
 // kStThreads compute threads (4 warps) plus one producer warp that only issues
 // the stages' TMA copies between the two barriers of each chunk step
-__global__ void __launch_bounds__(kStThreads + 32)
+__global__ void __launch_bounds__(kStThreads + 32, 1)
 k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mW,
            const __grid_constant__ CUtensorMap mU, const __grid_constant__ CUtensorMap mG,
            __nv_bfloat16* __restrict__ U, const float* __restrict__ S0,
@@ -378,6 +378,10 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     __nv_bfloat16* sSh = reinterpret_cast<__nv_bfloat16*>(smem + kStStages * StTile::kStage);
     __nv_bfloat16* sVd = reinterpret_cast<__nv_bfloat16*>(sSh + kDV * PS);      // [16][72]
     uint64_t* sbar = reinterpret_cast<uint64_t*>(sVd + kDV * P16);                // [kStStages]
+    // raised by a thread whose wait ran out, only before the first barrier of a
+    // chunk step, and read only after it: the step's second barrier keeps the
+    // next step's writes away from this step's reads, so all threads agree
+    int* sstop = reinterpret_cast<int*>(sbar + kStStages);   // barriers order its accesses
     const int64_t bh = blockIdx.x;
     const int v0 = blockIdx.y * kDV;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -385,6 +389,7 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     const int mt = 16 * warp;                      // token rows of this warp (V~)
 
     if (tid == kStThreads) {
+        *sstop = 0;
         for (int q = 0; q < kStStages; ++q) sbar_init(&sbar[q]);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         for (int q = 0; q < kStStages - 1; ++q)
@@ -394,15 +399,24 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     }
     if (warp == kStThreads / 32) {                 // the producer warp
         __syncthreads();                           // the barriers exist
-        for (int64_t ci = 0; ci < nchunk; ++ci) {
-            if (!sbar_wait(&sbar[ci % kStStages], (uint32_t)((ci / kStStages) & 1))) return;
+        int64_t ci = 0;
+        for (; ci < nchunk; ++ci) {
+            if (!sbar_wait(&sbar[ci % kStStages], (uint32_t)((ci / kStStages) & 1))) *sstop = 1;
             __syncthreads();                       // stage of chunk ci - 1 is free
+            if (*sstop) break;
             if (lane == 0 && ci + kStStages - 1 < nchunk) {
                 const int nx = (int)((ci + kStStages - 1) % kStStages);
                 fetch_state(smem + nx * StTile::kStage, &sbar[nx], &mK, &mW, &mU, &mG,
                             (int)((bh * nchunk + ci + kStStages - 1) * kSK), v0);
             }
             __syncthreads();
+        }
+        // after a stop, the copies already started (chunks ci .. ci + kStStages - 2)
+        // land before the CTA's shared memory goes away; each wait is bounded
+        if (ci < nchunk && lane == 0) {
+            const int64_t last = ci + kStStages - 1 < nchunk ? ci + kStStages - 1 : nchunk;
+            for (int64_t cj = ci; cj < last; ++cj)
+                sbar_wait(&sbar[cj % kStStages], (uint32_t)((cj / kStStages) & 1));
         }
         return;
     }
@@ -430,12 +444,14 @@ k_state_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     for (int64_t ci = 0; ci < nchunk; ++ci) {
         const int64_t row0 = (bh * nchunk + ci) * kSK;
         uint8_t* cur = smem + (ci % kStStages) * StTile::kStage;
-        // this chunk's stage has landed; the later ones may be in flight
-        if (!sbar_wait(&sbar[ci % kStStages], (uint32_t)((ci / kStStages) & 1))) {
+        // this chunk's stage has landed (the later ones may be in flight); the
+        // CTA stops together when any thread's wait ran out
+        if (!sbar_wait(&sbar[ci % kStStages], (uint32_t)((ci / kStStages) & 1))) *sstop = 1;
+        __syncthreads();
+        if (*sstop) {
             if (tid == 0) raise_status(status, kStatusTimeout);
             return;                                // the state is not written
         }
-        __syncthreads();
         const uint32_t Ksa = sh32(cur), Wsa = sh32(cur + StTile::kTile);
         const __nv_bfloat16* Us = reinterpret_cast<const __nv_bfloat16*>(cur + 2 * StTile::kTile);
         const float* gs = reinterpret_cast<const float*>(cur + 2 * StTile::kTile + StTile::kU);
@@ -585,7 +601,7 @@ cudaError_t launch_scan(const void* Q, const void* K, const void* Wg, void* U, c
     dim3 grid((unsigned)BH, kSD / kDV);
     if (bf16) {
         const size_t s1 = kStStages * StTile::kStage + (size_t)kDV * ScanMma::kPS * 2 +
-                          (size_t)kDV * ScanMma::kP16 * 2 + kStStages * sizeof(uint64_t);
+                          (size_t)kDV * ScanMma::kP16 * 2 + (kStStages + 1) * sizeof(uint64_t);
         const int64_t rows = BH * nchunk * kSK;
         CUtensorMap mK, mW, mU, mG;
         if (!map_bf16_2d(&mK, K, rows, 64, kSK, CU_TENSOR_MAP_SWIZZLE_128B) ||

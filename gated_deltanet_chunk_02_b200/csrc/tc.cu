@@ -2029,6 +2029,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
     struct __align__(8) CtrlI8 {
         uint64_t mma[kI8Slots];
         uint64_t full[kI8Slots];                   // the slot's staged A landed
+        uint64_t drain[kI8Slots];                  // after an expired wait: the slot's products are done
         uint32_t tmem;
         int abort;
         float red_f[kI8Slots][2][4];
@@ -2041,6 +2042,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
         for (int s = 0; s < kI8Slots; ++s) {
             mbar_init(&ctrl->mma[s], 1);
             mbar_init(&ctrl->full[s], 1);
+            mbar_init(&ctrl->drain[s], 1);
         }
         ctrl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -2084,6 +2086,15 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
         return max(max(ctrl->red_i[s][c][0], ctrl->red_i[s][c][1]),
                    max(ctrl->red_i[s][c][2], ctrl->red_i[s][c][3]));
     };
+    // the same, with the slot's decision to stop taken at its barrier (an OR
+    // over the threads' view of the abort flag)
+    auto chunk_max_i_stop = [&](int v, bool& stop) {
+        for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) ctrl->red_i[s][c][wq] = v;
+        stop = bar_sync_or(bar_id, 256, *(volatile int*)&ctrl->abort != 0);
+        return max(max(ctrl->red_i[s][c][0], ctrl->red_i[s][c][1]),
+                   max(ctrl->red_i[s][c][2], ctrl->red_i[s][c][3]));
+    };
 
     // the slot's leader stages A of the slot's tile n: two 32-column boxes
     int a_issued = 0;
@@ -2123,8 +2134,10 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             }
         }
         fence_async_smem();
-        bar_sync(bar_id, 256);                     // previous tile's reads of sA, sB, red and the stage done
-        if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+        // previous tile's reads of sA, sB, red and the stage done; the slot
+        // decides together whether to stop (an OR over its threads' view of
+        // the CTA's abort flag, which the other slot may raise at any time)
+        if (bar_sync_or(bar_id, 256, *(volatile int*)&ctrl->abort != 0)) { ok = false; break; }
         if (leader) issue_a(n + kI8Slots);
         float amax = 0.f;
 #pragma unroll
@@ -2198,8 +2211,9 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
                 accv[jj] = (j < jmin) ? 0 : (int)raw[jj];
                 m = max(m, abs(accv[jj]));
             }
-            m = chunk_max_i(m);
-            if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+            bool stop;
+            m = chunk_max_i_stop(m, stop);
+            if (stop) { ok = false; break; }
             const float mf = (float)m;
             const float rn = m > 0 ? __fdiv_rn(127.f, mf) : 0.f;
             const float sn = m > 0 ? __fmul_rn(__fmul_rn(sprev, s1), __fdiv_rn(mf, 127.f)) : 0.f;
@@ -2255,7 +2269,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
                 tc_fence_after();
                 tmem_ld32_async(tD, raw);
                 tmem_wait_ld();
-                return !*(volatile int*)&ctrl->abort;
+                return !bar_sync_or(bar_id, 256, *(volatile int*)&ctrl->abort != 0);
             };
             auto eye_f = [&](int jj) { return i == 32 * h + jj ? 1.f : 0.f; };
             // codes of the whole A and of X
@@ -2356,9 +2370,13 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
         }
         tc_fence_before();
     }
-    if (!ok) {
-        mbar_wait(&ctrl->mma[s], mma_phase);
-        if (leader && a_issued > 0) mbar_wait(&ctrl->full[s], (uint32_t)((a_issued - 1) & 1));
+    if (!ok && leader) {
+        // bounded: one more commit tracks every product the slot's issuing
+        // thread started, so TMEM is not freed under one; its last load lands
+        // before the shared memory goes away
+        mma_commit(&ctrl->drain[s]);
+        mbar_wait(&ctrl->drain[s], 0);
+        if (a_issued > 0) mbar_wait(&ctrl->full[s], (uint32_t)((a_issued - 1) & 1));
     }
     tc_fence_before();
     __syncthreads();
@@ -2383,11 +2401,13 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
 // chunk).  Every intermediate is an exact integer, so codes, accumulators,
 // scales and T match the oracle bit for bit.  One slot of 8 warps per CTA
 // (the three accumulators take 384 of the SM's 512 TMEM columns), A staged
-// by TMA one tile ahead.
+// by TMA one tile ahead.  The RES instance follows the series with the
+// parallel residual correction, every product again of int16 codes.
 struct ParamsI16 {
     int64_t rows;
     int ntiles;
     int N, mask;
+    int S;               // residual steps (the RES instance)
     const float* A;
     float* T;
     int16_t* q;
@@ -2400,6 +2420,8 @@ constexpr int kI16Op = kRows * 128;                  // 16 KB: 128 rows x 64 byt
 constexpr int kI16B = 64 * 128;                      // 8 KB: 64 rows x 128 byte codes
 constexpr int kI16Stage = kRows * 64 * 4;            // 32 KB: the next tile's A
 constexpr int kI16Smem = 2 * kI16Op + 2 * kI16B + kI16Stage;
+constexpr int kI16Ctrl = 2048;                       // the control block after the operands
+constexpr int kI16T0 = 32 * 256 * 8;                 // RES: T0 in binary64, [column][thread]
 
 // 32 byte codes -> two 16-byte groups of a 128-byte swizzled row
 __device__ __forceinline__ void st_u8x32(uint8_t* buf, int row, int q0, const uint32_t (&b)[32]) {
@@ -2422,6 +2444,7 @@ __device__ __forceinline__ int quant_i16(double x, double r) {
     return (int)y;
 }
 
+template <bool RES>
 __global__ void __launch_bounds__(256, 1)
 k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
     constexpr int KC = 64;
@@ -2433,13 +2456,16 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
     struct __align__(8) CtrlI16 {
         uint64_t mma;
         uint64_t full;                             // the staged A landed
+        uint64_t drain;                            // after an expired wait: the products are done
         uint32_t tmem;
         int abort;
         float red_f[2][4];
         long long red_l[2][4];
+        double red_d[2][4];
         int rsum[kRows][2];                        // row sums of the left operand's q'
-        int csum[2][64];                           // column sums of q'_1, per chunk
+        int csum[2][64];                           // column sums of q'_1 (the right operand), per chunk
     };
+    static_assert(sizeof(CtrlI16) <= kI16Ctrl, "control block");
     uint8_t* sAh = smem;
     uint8_t* sAl = sAh + kI16Op;
     uint8_t* sBh = sAl + kI16Op;
@@ -2451,6 +2477,7 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
     if (threadIdx.x == 0) {
         mbar_init(&ctrl->mma, 1);
         mbar_init(&ctrl->full, 1);
+        mbar_init(&ctrl->drain, 1);
         ctrl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -2489,6 +2516,12 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
 #pragma unroll
         for (int k = 1; k < 4; ++k) m = m > ctrl->red_l[c][k] ? m : ctrl->red_l[c][k];
         return m;
+    };
+    auto chunk_max_d = [&](double v) {
+        for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) ctrl->red_d[c][wq] = v;
+        __syncthreads();
+        return fmax(fmax(ctrl->red_d[c][0], ctrl->red_d[c][1]), fmax(ctrl->red_d[c][2], ctrl->red_d[c][3]));
     };
     // offset codes q' = q + 32768 as high and low bytes; row sum of this half-row
     auto split = [&](const int (&q)[32], uint32_t (&hb)[32], uint32_t (&lb)[32]) {
@@ -2681,6 +2714,201 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
             sprev = sn;
         }
         if (!ok) break;
+        if constexpr (RES) {
+            // ---- residual correction, every product of int16 codes ----
+            // X = T0 - I; E = (A - X) + (s_A s_X) (q_A q_X) over the whole A;
+            // E's powers requantised as A's; Gm = sum_s s_E,s q_E,s;
+            // T = (T0 + Gm) + (s_X s_G) (q_X q_G); every scale and sum in
+            // binary64, T rounded once to float32.  T0 waits in shared memory.
+            double* const sT0 = reinterpret_cast<double*>(smem + kI16Smem + kI16Ctrl);
+            const int tid = threadIdx.x;
+            auto t0 = [&](int jj) { return sT0[jj * 256 + tid]; };
+            auto xv = [&](int jj) { return __dsub_rn(t0(jj), i == 32 * h + jj ? 1.0 : 0.0); };
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) sT0[jj * 256 + tid] = t[jj];
+            // the operands of one product: the left codes with their row sums,
+            // the right codes with their column sums (both as offset bytes)
+            auto set_left = [&](const int (&qq)[32]) {
+                uint32_t hb[32], lb[32];
+                ctrl->rsum[r][h] = split(qq, hb, lb);
+                st_u8x32(sAh, r, 2 * h, hb);
+                st_u8x32(sAl, r, 2 * h, lb);
+            };
+            auto set_right = [&](const int (&qq)[32]) {
+                {
+                    uint32_t hb[32], lb[32];
+                    split(qq, hb, lb);
+                    st_u8x32(sBh, i, 4 * c + 2 * h, hb);
+                    st_u8x32(sBl, i, 4 * c + 2 * h, lb);
+                }
+                int v[32];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) v[jj] = qq[jj] + 32768;
+#pragma unroll
+                for (int sh = 16; sh >= 1; sh >>= 1) {
+                    const bool up = (lane & sh) != 0;
+#pragma unroll
+                    for (int k = 0; k < sh; ++k) {
+                        const int send = up ? v[k] : v[k + sh];
+                        const int keep = up ? v[k + sh] : v[k];
+                        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+                    }
+                }
+                if ((warp & 1) == 0) ctrl->csum[c][32 * h + lane] = v[0];
+                __syncthreads();
+                if ((warp & 1) == 1) ctrl->csum[c][32 * h + lane] += v[0];
+            };
+            // every thread must be done with the last product's accumulators
+            // and sums before the next operands are written
+            auto begin_operands = [&]() {
+                tc_fence_before();
+                __syncthreads();
+            };
+            // left x right as int64, assembled from the three byte products
+            auto product = [&](long long (&accv)[32]) {
+                fence_async_smem();
+                tc_fence_before();
+                __syncthreads();                           // operands and sums written
+                tc_fence_after();
+                if (leader) {
+                    constexpr uint32_t id = (2u << 4) | (0u << 7) | (0u << 10) | (0u << 15) | (1u << 16) |
+                                            ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+#pragma unroll
+                    for (int kk = 0; kk < KC / 32; ++kk) {
+                        const uint64_t ah = sdesc(su32(sAh) + kk * 32, 16, 1024);
+                        const uint64_t al = sdesc(su32(sAl) + kk * 32, 16, 1024);
+                        const uint64_t bh = sdesc(su32(sBh) + kk * 32 * 128, 16, 1024);
+                        const uint64_t bl = sdesc(su32(sBl) + kk * 32 * 128, 16, 1024);
+                        mma_i8(tm, ah, bh, id, kk > 0);                 // HH
+                        mma_i8(tm + 128, ah, bl, id, kk > 0);           // HL
+                        mma_i8(tm + 128, al, bh, id, 1);                // + LH
+                        mma_i8(tm + 256, al, bl, id, kk > 0);           // LL
+                    }
+                    mma_commit(&ctrl->mma);
+                }
+                const bool good = mbar_wait(&ctrl->mma, mma_phase);
+                mma_phase ^= 1;
+                if (!good) {
+                    atomicExch(&ctrl->abort, 1);
+                    raise_status(p.status, kStatusTimeout);
+                }
+                tc_fence_after();
+                uint32_t hh[32], mm[32], ll[32];
+                tmem_ld32_async(tD, hh);
+                tmem_ld32_async(tD + 128, mm);
+                tmem_ld32_async(tD + 256, ll);
+                tmem_wait_ld();
+                const long long ra = (long long)ctrl->rsum[r][0] + ctrl->rsum[r][1];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj)
+                    accv[jj] = 65536LL * (int)hh[jj] + 256LL * (int)mm[jj] + (long long)(int)ll[jj] -
+                               32768LL * (ra + ctrl->csum[c][32 * h + jj]) +
+                               (long long)KC * 32768LL * 32768LL;
+            };
+            // codes of the whole A (reloaded: the stage already holds the next
+            // tile) and of X
+            float av[32];
+            if (valid) {
+                const float4* src = reinterpret_cast<const float4*>(p.A + (cidx * KC + rin) * KC + 32 * h);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 u = src[q4];
+                    av[4 * q4] = u.x;
+                    av[4 * q4 + 1] = u.y;
+                    av[4 * q4 + 2] = u.z;
+                    av[4 * q4 + 3] = u.w;
+                }
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) av[jj] = 0.f;   // rows past the end: A = 0
+            }
+            float ma = 0.f;
+            double mx = 0.0;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                ma = fmaxf(ma, fabsf(av[jj]));
+                mx = fmax(mx, fabs(xv(jj)));
+            }
+            ma = chunk_max_f(ma);
+            mx = chunk_max_d(mx);
+            const double rA = ma > 0.f ? __ddiv_rn(32767.0, (double)ma) : 0.0;
+            const double sA = ma > 0.f ? __ddiv_rn((double)ma, 32767.0) : 0.0;
+            const double rX = mx > 0.0 ? __ddiv_rn(32767.0, mx) : 0.0;
+            const double sX = mx > 0.0 ? __ddiv_rn(mx, 32767.0) : 0.0;
+            begin_operands();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) q[jj] = ma > 0.f ? quant_i16((double)av[jj], rA) : 0;
+            set_left(q);                                            // q_A
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) q[jj] = mx > 0.0 ? quant_i16(xv(jj), rX) : 0;
+            set_right(q);                                           // q_X
+            long long accv[32];
+            product(accv);
+            // E and its codes
+            const double sAX = __dmul_rn(sA, sX);
+            double e[32];
+            double me = 0.0;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                e[jj] = __dadd_rn(__dsub_rn((double)av[jj], xv(jj)), __dmul_rn(sAX, (double)accv[jj]));
+                me = fmax(me, fabs(e[jj]));
+            }
+            me = chunk_max_d(me);
+            if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+            const double rE = me > 0.0 ? __ddiv_rn(32767.0, me) : 0.0;
+            const double sE1 = me > 0.0 ? __ddiv_rn(me, 32767.0) : 0.0;
+            double gm[32];
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                q[jj] = me > 0.0 ? quant_i16(e[jj], rE) : 0;
+                gm[jj] = __dmul_rn(sE1, (double)q[jj]);
+            }
+            double sprevE = sE1;
+            for (int sp = 2; sp <= p.S; ++sp) {
+                begin_operands();
+                set_left(q);                                        // q_E,s-1
+                if (sp == 2) set_right(q);                          // q_E1
+                product(accv);
+                long long m = 0;
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const long long ab = accv[jj] < 0 ? -accv[jj] : accv[jj];
+                    m = m > ab ? m : ab;
+                }
+                m = chunk_max_l(m);
+                if (*(volatile int*)&ctrl->abort) { ok = false; break; }
+                const double mf = (double)m;
+                const double rn = m > 0 ? __ddiv_rn(32767.0, mf) : 0.0;
+                const double sn = m > 0 ? __dmul_rn(__dmul_rn(sprevE, sE1), __ddiv_rn(mf, 32767.0)) : 0.0;
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    q[jj] = m > 0 ? quant_i16((double)accv[jj], rn) : 0;
+                    gm[jj] = __dadd_rn(gm[jj], __dmul_rn(sn, (double)q[jj]));
+                }
+                sprevE = sn;
+            }
+            if (!ok) break;
+            // codes of Gm; T = (T0 + Gm) + s_X s_G (q_X q_G)
+            double mg = 0.0;
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) mg = fmax(mg, fabs(gm[jj]));
+            __syncthreads();                                        // every thread has read me's partials
+            mg = chunk_max_d(mg);
+            const double rG = mg > 0.0 ? __ddiv_rn(32767.0, mg) : 0.0;
+            const double sG = mg > 0.0 ? __ddiv_rn(mg, 32767.0) : 0.0;
+            begin_operands();
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) q[jj] = mx > 0.0 ? quant_i16(xv(jj), rX) : 0;
+            set_left(q);                                            // q_X
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) q[jj] = mg > 0.0 ? quant_i16(gm[jj], rG) : 0;
+            set_right(q);                                           // q_G
+            product(accv);
+            const double sXG = __dmul_rn(sX, sG);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+                t[jj] = __dadd_rn(__dadd_rn(t0(jj), gm[jj]), __dmul_rn(sXG, (double)accv[jj]));
+        }
         if (valid) {
             float* dst = p.T + cidx * KC * KC + rin * KC + 32 * h;
 #pragma unroll
@@ -2691,9 +2919,18 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
         }
         tc_fence_before();
     }
-    if (!ok) {
-        mbar_wait(&ctrl->mma, mma_phase);
-        if (leader && a_issued > 0) mbar_wait(&ctrl->full, (uint32_t)((a_issued - 1) & 1));
+    // the flag is raised only before a __syncthreads and read only after one,
+    // so every thread takes the same decision; this last look covers a wait
+    // that ran out in the tile's final product
+    tc_fence_before();
+    __syncthreads();
+    if (*(volatile int*)&ctrl->abort) ok = false;
+    if (!ok && leader) {
+        // bounded: one more commit tracks every product started, so TMEM is
+        // not freed under one; the last load lands before shared memory goes
+        mma_commit(&ctrl->drain);
+        mbar_wait(&ctrl->drain, 0);
+        if (a_issued > 0) mbar_wait(&ctrl->full, (uint32_t)((a_issued - 1) & 1));
     }
     tc_fence_before();
     __syncthreads();
@@ -3400,9 +3637,10 @@ cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8
 }
 
 cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int16_t* q,
-                                  int64_t* acc, double* sc, int64_t nc, cudaStream_t st) {
+                                  int64_t* acc, double* sc, int64_t nc, cudaStream_t st, int S) {
     tcg::ParamsI16 p;
     memset(&p, 0, sizeof p);
+    p.S = S;
     p.rows = nc * 64;
     p.ntiles = (int)((p.rows + tcg::kRows - 1) / tcg::kRows);
     p.N = N;
@@ -3418,14 +3656,21 @@ cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int
     if (!tcg::map_f32(&mA, A, p.rows, 64)) return cudaErrorInvalidValue;
     // one CTA per SM: it takes all 512 TMEM columns (the shared-memory request
     // keeps a second CTA off the SM)
-    size_t smem = tcg::kI16Smem + 2048;
+    size_t smem = tcg::kI16Smem + tcg::kI16Ctrl + (S > 0 ? tcg::kI16T0 : 0);
     if (smem < 120 * 1024) smem = 120 * 1024;
-    cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i16_tc,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     const int sms = tcg::num_sms();
     const int grid = p.ntiles < sms ? p.ntiles : sms;
-    tcg::k_neumann_i16_tc<<<grid, 256, smem, st>>>(mA, p);
+    if (S > 0) {
+        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i16_tc<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        tcg::k_neumann_i16_tc<true><<<grid, 256, smem, st>>>(mA, p);
+    } else {
+        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i16_tc<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        tcg::k_neumann_i16_tc<false><<<grid, 256, smem, st>>>(mA, p);
+    }
     return cudaGetLastError();
 }
 

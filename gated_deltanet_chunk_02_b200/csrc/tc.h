@@ -38,9 +38,11 @@ cudaError_t launch_fused_raw_tc(const void* K, const void* V, const float* beta,
                                 const float* loggate, int N, int mask, int S, int gated, void* W,
                                 void* U, float* Tout, void* Kout, float* gout, int64_t nc, int k,
                                 cudaStream_t st);
-// INT16 series (k = 64): int16 codes through unsigned-byte products, int64 accumulators
+// INT16 series (k = 64): int16 codes through unsigned-byte products, int64 accumulators;
+// S > 0: the residual correction in int16 products follows
 cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int16_t* q,
-                                  int64_t* acc, double* sc, int64_t nc, cudaStream_t st);
+                                  int64_t* acc, double* sc, int64_t nc, cudaStream_t st,
+                                  int S = 0);
 cudaError_t launch_fused_tc(const void* K, const void* V, const float* beta, const float* g,
                             int N, int mask, int S, int gated, void* W, void* U, float* Tout,
                             int64_t nc, int k, cudaStream_t st);

@@ -26,6 +26,7 @@ EXPORTS = [
     "gdn_build_A", "gdn_invert_neumann", "gdn_invert_newton", "gdn_invert_blocked",
     "gdn_invert_fwdsub", "gdn_wy",
     "gdn_invert_neumann_i8", "gdn_invert_neumann_i8_residual", "gdn_invert_neumann_i16",
+    "gdn_invert_neumann_i16_residual",
     "gdn_chunk_wy_fused", "gdn_chunk_wy_fused_raw", "gdn_forward",
     "gdn_forward_workspace_bytes", "gdn_forward_static", "gdn_decode", "gdn_get_status",
     "gdn_last_error", "gdn_launch_count", "gdn_debug_arm_wait_expiry", "gdn_forward_raw",
@@ -71,6 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "gdn_invert_neumann_i8": [_P, _P, _I, _I, _P, _P, _P, S, _P],
         "gdn_invert_neumann_i16": [_P, _P, _I, _I, _P, _P, _P, S, _P],
         "gdn_invert_neumann_i8_residual": [_P, _P, _I, _I, _I, S, _P],
+        "gdn_invert_neumann_i16_residual": [_P, _P, _I, _I, _I, S, _P],
         "gdn_chunk_wy_fused": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, S, _I, _P],
         "gdn_chunk_wy_fused_raw": [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, S, _I,
                                    _P],
@@ -202,6 +204,12 @@ def gdn_invert_neumann_i16(A, T, N, mask, q=None, acc=None, scale=None, stream=N
     int16, accumulators int64, scales float64."""
     _check(load().gdn_invert_neumann_i16(_ptr(A), _ptr(T), N, int(mask), _ptr(q), _ptr(acc),
                                          _ptr(scale), shape_of_chunks(A), _stream(stream)))
+
+
+def gdn_invert_neumann_i16_residual(A, T, N, mask, S, stream=None):
+    """INT16 series followed by S residual powers, every product in int16 codes."""
+    _check(load().gdn_invert_neumann_i16_residual(_ptr(A), _ptr(T), N, int(mask), S,
+                                                  shape_of_chunks(A), _stream(stream)))
 
 
 def gdn_chunk_wy_fused(K, V, beta, g, N, mask, S, gated, W, U, T=None, k=64, stream=None):

@@ -184,6 +184,25 @@ int gdn_invert_neumann_i16(const float* A, float* T, int N, int mask, int16_t* q
                            int64_t* acc_dbg, double* scale_dbg, gdn_shape s, void* stream);
 
 /*
+ * INT16 series followed by the parallel residual correction with every product
+ * in int16 codes ("Adaptation à la Quantification": the INT16 operating point,
+ * N = 3 compensated by S = 8; "Méthodologie" §3 for E and T = T0 sum_{s<=S} E^s).
+ * The steps of gdn_invert_neumann_i8_residual under the rules of
+ * gdn_invert_neumann_i16 (codes in [-32767, 32767], exact int64 products, every
+ * scale and sum in IEEE binary64, no FMA):
+ *   T0 = I + s_1 q_1 + ... + s_N q_N (binary64, not rounded);  X = T0 - I;
+ *   E = (A - X) + (s_A * s_X) * double(q_A q_X)   (whole A, no mask);
+ *   q_E1 = codes(E); q_E,s, s_E,s for s = 2..S requantised as the powers of A;
+ *   Gm = s_E1 q_E1 + ... + s_E,S q_E,S (left to right);
+ *   T = (T0 + Gm) + (s_X * s_G) * double(q_X q_G),  q_G = codes(Gm), then
+ *   rounded once to float32.
+ * In: A [nc,k,k] f32.  Out: T [nc,k,k] f32.  k = 64, 1 <= N <= 8,
+ * 1 <= S <= 64.  Errors as gdn_invert_neumann_i16.
+ */
+int gdn_invert_neumann_i16_residual(const float* A, float* T, int N, int mask, int S,
+                                    gdn_shape s, void* stream);
+
+/*
  * Fused per-chunk pipeline: A from K, beta, g; T by the Neumann + mask +
  * residual method (as gdn_invert_neumann); then W, U (gated W if gated != 0).
  * Only K, V, beta, g are read and only W, U (and T when T_out is non-NULL)

@@ -156,6 +156,17 @@ def test_int16_limits(lib):
                                       None) == gdn.GDN_OK
 
 
+def test_int16_residual_limits(lib):
+    f = lib.gdn_invert_neumann_i16_residual
+    assert f(P(FAKE), P(FAKE), 3, 1, 0, sh(), None) == gdn.GDN_ERR_ARG           # S < 1
+    assert f(P(FAKE), P(FAKE), 3, 1, 65, sh(), None) == gdn.GDN_ERR_ARG          # S > 64
+    assert f(P(FAKE), P(FAKE), 9, 1, 8, sh(), None) == gdn.GDN_ERR_ARG           # N > 8
+    assert f(P(FAKE), P(FAKE), 3, 2, 8, sh(), None) == gdn.GDN_ERR_ARG           # mask
+    assert f(P(FAKE), P(FAKE), 3, 1, 8, sh(k=128), None) == gdn.GDN_ERR_UNSUPPORTED
+    assert f(P(MISALIGNED), P(FAKE), 3, 1, 8, sh(), None) == gdn.GDN_ERR_ALIGN
+    assert f(None, None, 3, 1, 8, sh(B=0), None) == gdn.GDN_OK
+
+
 def test_prologue_limits(lib):
     args = [P(FAKE)] * 4
     outs = [P(FAKE), P(FAKE), None, None, None]

@@ -236,6 +236,68 @@ def test_int16_bit_exact(N, mask):
     assert torch.equal(T, T2)
 
 
+@pytest.mark.parametrize("N,mask", [(3, 1), (1, 1), (4, 1), (3, 0)])
+@pytest.mark.parametrize("S", [1, 2, 8])
+def test_int16_residual_bit_exact(N, mask, S):
+    """INT16 series plus the residual in int16 products (byte-split, int64,
+    binary64 scales): T bit for bit against the oracle on 67 chunks (a ragged
+    last tile), and far closer to the exact inverse than the series alone."""
+    w = Workload(B=1, H=1, T=67 * 64, k=64, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=31 + S), w)
+    nc = A32.shape[0]
+    Ad = to_dev(A_tensor(A32, w))
+    T = torch.empty_like(Ad)
+    gdn.gdn_invert_neumann_i16_residual(Ad, T, N, mask, S)
+    check_status()
+    ref = O.int16_residual(A32, N, bool(mask), S)
+    np.testing.assert_array_equal(T.cpu().numpy().reshape(nc, 64, 64).view(np.uint32),
+                                  ref.view(np.uint32))
+    if N == 3 and mask:
+        exact = O.invert_fwdsub(A32.astype(np.float64))
+        assert O.rel_fro(ref, exact) < O.rel_fro(O.int16_neumann(A32, N, True)["T"], exact) / 10
+
+
+@pytest.mark.parametrize("kind", ["slow", "corr"])
+def test_int16_residual_bit_exact_where_the_residual_shows(kind):
+    """Slow-decay gates (and correlated keys): E and its powers are large, so
+    every residual product and requantisation moves T."""
+    kw = {"slow": dict(gate_scale=0.05), "corr": dict(gate_scale=0.05, key_corr=0.5)}[kind]
+    w = Workload(B=1, H=1, T=19 * 64, k=64, dtype="bf16")
+    A32 = oracle_A32(make_inputs(w, seed=37, **kw), w)
+    nc = A32.shape[0]
+    Ad = to_dev(A_tensor(A32, w))
+    for N, S in [(1, 8), (3, 8), (3, 3)]:
+        T = torch.empty_like(Ad)
+        gdn.gdn_invert_neumann_i16_residual(Ad, T, N, 1, S)
+        check_status()
+        ref = O.int16_residual(A32, N, True, S)
+        np.testing.assert_array_equal(T.cpu().numpy().reshape(nc, 64, 64).view(np.uint32),
+                                      ref.view(np.uint32))
+        assert not np.array_equal(ref, O.int16_residual(A32, N, True, S - 1) if S > 1 else
+                                  O.int16_neumann(A32, N, True)["T"])
+
+
+def test_int16_residual_degenerate_chunks():
+    """A zero chunk (every maximum zero: T = I), a single sub-diagonal entry
+    (E = 0 exactly, so E, Gm and their codes are zero), codes at +-32767 and
+    a full tile of ordinary chunks beside them."""
+    rng = np.random.default_rng(41)
+    A32 = np.zeros((5, 64, 64), np.float32)
+    A32[1, 5, 4] = 0.75                                      # E = 0
+    A32[2] = np.tril(rng.choice([-1.0, 1.0], (64, 64)), -1)  # extreme codes
+    A32[3] = np.tril(rng.standard_normal((64, 64)) * 0.05, -1)
+    A32[4] = np.tril(rng.standard_normal((64, 64)) * 0.2, -1)
+    Ad = torch.from_numpy(A32).reshape(1, 1, 5, 64, 64).cuda()
+    for N, mask, S in [(3, 1, 8), (1, 1, 2), (2, 0, 3)]:
+        T = torch.empty_like(Ad)
+        gdn.gdn_invert_neumann_i16_residual(Ad, T, N, mask, S)
+        check_status()
+        ref = O.int16_residual(A32, N, bool(mask), S)
+        np.testing.assert_array_equal(T.cpu().numpy().reshape(5, 64, 64).view(np.uint32),
+                                      ref.view(np.uint32))
+        assert np.array_equal(ref[0], np.eye(64, dtype=np.float32))
+
+
 def test_int16_extreme_codes():
     """Entries at +-amax and sign flips: the byte split must carry codes of
     +-32767 and the int64 accumulators reach ~2^36."""
