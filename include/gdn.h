@@ -318,11 +318,11 @@ int gdn_decode(const void* Q, const void* K, const void* V, const float* beta,
                int64_t n, int32_t d, gdn_dtype dtype, void* stream);
 
 /*
- * Streams and graphs: every entry point enqueues its kernels on `stream`
- * (NULL = the legacy default stream) and returns without synchronising; none
- * allocates device memory (gdn_forward takes a caller workspace).  The calls
- * can therefore be captured into CUDA graphs and replayed; make one eager
- * call first (it sets kernel attributes and looks up the status word).
+ * Streams: every entry point enqueues its kernels on `stream` (NULL = the
+ * legacy default stream) and returns without synchronising; none allocates
+ * device memory (gdn_forward takes a caller workspace).  The first call in a
+ * process sets kernel attributes and looks up the status word; bench.py
+ * makes it eagerly before it captures gdn_decode steps into a CUDA graph.
  */
 /* The status word's address is looked up once per host thread and device and
  * kept; a device reset (cudaDeviceReset) invalidates it, as it does the

@@ -89,6 +89,26 @@ def test_c5_long_context(c5, N, mask, S, exact):
     assert rel(Sg, Sr) <= TOL_BF16
 
 
+def test_c5_slow_gates_end_of_sequence():
+    """The c5 length with slow-decay gates (log-gates scaled by 0.05), S = 8:
+    two whole heads, the sequence's last 8 chunks on their own, and the final
+    state against the oracle; the oracle's S = 0 forward is 0.13 away here,
+    so a forward that dropped or cut short the residual would fail."""
+    w = Workload(B=1, H=16, T=65536, k=64, dtype="bf16")
+    inp = make_inputs(w, seed=5, with_q=True, gate_scale=0.05)
+    d = {key: v.cuda() for key, v in inp.items()}
+    Ot, Sf = run_forward(d, 3, 1, 8, 0)
+    heads = np.array([3, 15])
+    Or, Sr = oracle_forward(inp, heads, 64, 3, 1, 8, 0)
+    O0, _ = oracle_forward(inp, heads, 64, 3, 1, 0, 0)
+    Og = Ot.reshape(16, 65536, 128)[heads]
+    last = slice(65536 - 8 * 64, 65536)
+    assert rel(Og, Or) <= TOL_BF16
+    assert rel(Og[:, last], Or[:, last]) <= TOL_BF16
+    assert rel(Sf.reshape(16, 128, 128)[heads], Sr) <= TOL_BF16
+    assert rel(Og[:, last], O0[:, last]) >= 5 * TOL_BF16
+
+
 @pytest.mark.parametrize("N,mask,S", [(3, 1, 8), (3, 1, 0), (2, 0, 1)])
 def test_forward_odd_chunk_count(N, mask, S):
     """21 chunks: the output pass's last 128-row tile holds a single chunk."""
