@@ -474,7 +474,7 @@ struct KernelShape {
 // ------------------------------------------------------------------------- //
 // the kernel
 // ------------------------------------------------------------------------- //
-template <int KC, int MODE, int NS, int SN, int SS>
+template <int KC, int MODE, int NS, int SN, int SS, int SG>
 __global__ void __launch_bounds__(256 * NS, 1)
 k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
            const __grid_constant__ CUtensorMap mW, const __grid_constant__ CUtensorMap mU,
@@ -496,11 +496,12 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     uint8_t* bg_base = smem + NS * L::bytes;
     Ctrl* ctrl = reinterpret_cast<Ctrl*>(bg_base + NS * L::bg_bytes);
 
-    // The series order and the residual steps: the call's, or fixed at compile
-    // time in an instance specialised for one setting (SN > 0, SS >= 0), where
-    // every loop and branch on them folds away.
+    // The series order, the residual steps and whether W is gated: the call's,
+    // or fixed at compile time in an instance specialised for one setting
+    // (SN > 0, SS >= 0, SG >= 0), where every loop and branch on them folds away.
     const int pN = SN > 0 ? SN : p.N;
     const int pS = SS >= 0 ? SS : p.S;
+    const int pG = SG >= 0 ? SG : p.gated;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
@@ -536,7 +537,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
     const int i = r % KB;                          // row inside the block
     const int cl = SUB ? (i / KC) * KC : 0;        // first column of this row's chunk
     const int ch = cl + KC;                        // one past its last column
-    const int jmin = p.mask ? i - pN : -KB;       // band mask keeps columns j >= jmin
+    const int jmin = (is_band(MODE) || p.mask) ? i - pN : -KB;   // band mask keeps columns j >= jmin
     uint8_t* base = smem + s * L::bytes;
     uint8_t* sK = base + L::offK;
     uint8_t* sV = base + L::offV;
@@ -1490,7 +1491,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                                 for (int c = 0; c < 8; ++c) t[8 * g + c] = fmaf(tb[e], h8[c], t[8 * g + c]);
                             }
                         }
-                        if (p.gated) {
+                        if (pG) {
                             t0_put(0, t, T0);
                         } else {                                  // WY's operand T diag(beta), bf16
                             if (p.Tout && valid) {
@@ -1552,7 +1553,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                         tma_store_2d(&mW, 32 * b, (int)row0, sAop + b * 16384);
                     bulk_commit();
                 }
-            } else if (p.Tout && !(band && pS > 0 && !p.gated)) {
+            } else if (p.Tout && !(band && pS > 0 && !pG)) {
 #pragma unroll
                 for (int pp = 0; pp < PPT; ++pp) {
                     const int pc = pc0 + pp;
@@ -1576,7 +1577,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             const float* gcol = sg + blk * KB;
 #pragma unroll
             for (int pp = 0; pp < PPT; ++pp) {
-                if (band && pS > 0 && !p.gated) break;    // written by the band product
+                if (band && pS > 0 && !pG) break;    // written by the band product
                 const int pc = pc0 + pp;
                 float v[32], t[32];
                 t0_get(pp, t, T0);
@@ -1584,10 +1585,10 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
                 for (int jj = 0; jj < 32; ++jj) {
                     const int j = pc * 32 + jj;
                     const float b = bcol[j];
-                    v[jj] = t[jj] * (p.gated ? b * exp_e(gcol[j]) : b);
+                    v[jj] = t[jj] * (pG ? b * exp_e(gcol[j]) : b);
                 }
                 st_op32<true>(sX, r, pc, v);
-                if (p.gated) {
+                if (pG) {
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) v[jj] = t[jj] * bcol[pc * 32 + jj];
                     st_op32<true>(sY, r, pc, v);
@@ -1598,7 +1599,7 @@ k_chunk_tc(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUten
             if (leader && live()) {
                 constexpr uint32_t id = idesc_f16(1, 1, 0, KB, 128);
                 const uint32_t kb0 = su32(sK), vb0 = su32(sV), xb0 = su32(sX);
-                const uint32_t ub0 = su32(p.gated ? sY : sX);
+                const uint32_t ub0 = su32(pG ? sY : sX);
                 // W^T first, with its own commit: the slot's next K tile can
                 // start loading while the U^T products still run
 #pragma unroll 1
@@ -3462,13 +3463,16 @@ struct IO {
     void* U = nullptr;
 };
 
-template <int KC, int MODE, int NS, int SN = 0, int SS = -1>
+template <int KC, int MODE, int NS, int SN = 0, int SS = -1, int SG = -1>
 static cudaError_t launch(const IO& io, const Params& p0, cudaStream_t st) {
     // the band path at N = 3, S = 8 (the method's setting for 64 x 64 chunks)
-    // runs an instance with both fixed at compile time: 6 % faster on 4096
-    // chunks than the same kernel reading them from the parameters
+    // runs an instance with the orders and the gating fixed at compile time:
+    // 8 % faster on 4096 chunks than the same kernel reading them from the
+    // parameters
     if constexpr ((MODE == kFusedBand || MODE == kFusedRawBand) && SN == 0 && SS < 0)
-        if (p0.N == 3 && p0.S == 8) return launch<KC, MODE, NS, 3, 8>(io, p0, st);
+        if (p0.N == 3 && p0.S == 8)
+            return p0.gated ? launch<KC, MODE, NS, 3, 8, 1>(io, p0, st)
+                            : launch<KC, MODE, NS, 3, 8, 0>(io, p0, st);
     using KS = KernelShape<KC, MODE, NS>;
     static_assert(KS::smem <= 232448, "shared memory budget");
     CUtensorMap mK, mV, mW, mU, mB, mG;
@@ -3496,11 +3500,11 @@ static cudaError_t launch(const IO& io, const Params& p0, cudaStream_t st) {
     p.status = status_ptr();
     size_t smem = KS::smem;
     if (smem < 120 * 1024) smem = 120 * 1024;     // one CTA per SM: it owns the SM's TMEM
-    cudaError_t e = cudaFuncSetAttribute(k_chunk_tc<KC, MODE, NS, SN, SS>,
+    cudaError_t e = cudaFuncSetAttribute(k_chunk_tc<KC, MODE, NS, SN, SS, SG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = p.ntiles < num_sms() ? p.ntiles : num_sms();
-    k_chunk_tc<KC, MODE, NS, SN, SS><<<grid, KS::threads, smem, st>>>(mK, mV, mW, mU, mB, mG, p);
+    k_chunk_tc<KC, MODE, NS, SN, SS, SG><<<grid, KS::threads, smem, st>>>(mK, mV, mW, mU, mB, mG, p);
     return cudaGetLastError();
 }
 
