@@ -1981,10 +1981,12 @@ __device__ __forceinline__ void mma_i8(uint32_t d, uint64_t a, uint64_t b, uint3
         "l"(a), "l"(b), "r"(idesc), "r"(acc)
         : "memory");
 }
+// clamp(rint(x * r), +-127): one conversion with round to nearest even (it
+// saturates, so the integer clamp gives what a clamp in float would).  With
+// r = 0 (a zero maximum: every x is zero) the code is 0.
 __device__ __forceinline__ int quant_i8(float x, float r) {
-    float y = rintf(__fmul_rn(x, r));
-    y = fminf(fmaxf(y, -127.f), 127.f);
-    return (int)y;
+    const int q = __float2int_rn(__fmul_rn(x, r));
+    return min(max(q, -127), 127);
 }
 // 32 int8 codes -> two 16-byte groups of a 128-byte swizzled row
 __device__ __forceinline__ void st_i8x32(uint8_t* buf, int row, int q0, const int (&c)[32]) {
@@ -2023,7 +2025,7 @@ constexpr int kI8Stage = kRows * 64 * 4;           // 32 KB: the next tile's A (
 constexpr int kI8SlotBytes = kI8OpBytes + kI8BBytes + kI8Stage;
 
 // RES: the residual correction in int8 products follows the series (S >= 1)
-template <bool RES>
+template <bool RES, int SN, int SS>
 __global__ void __launch_bounds__(256 * kI8Slots, 1)
 k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
     constexpr int KC = 64;
@@ -2042,6 +2044,10 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
         int red_i[kI8Slots][2][4];
     };
     CtrlI8* ctrl = reinterpret_cast<CtrlI8*>(smem + kI8Slots * kI8SlotBytes);
+    // the series order and the residual steps: the call's, or fixed at compile
+    // time in an instance specialised for one setting (SN > 0, SS >= 0)
+    const int pN = SN > 0 ? SN : p.N;
+    const int pS = SS >= 0 ? SS : p.S;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -2065,7 +2071,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
     const int c = r / KC;                          // chunk of this row in the tile
     const int i = r % KC;
     const int wq = ((warp & 3) & 1) * 2 + h;       // this warp's slot among its chunk's 4 warps
-    const int jmin = p.mask ? i - p.N : -KC;
+    const int jmin = p.mask ? i - pN : -KC;
     uint8_t* sA = smem + s * kI8SlotBytes;
     uint8_t* sB = sA + kI8OpBytes;
     uint8_t* sStage = sB + kI8BBytes;
@@ -2162,13 +2168,13 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
             const int j = 32 * h + jj;
-            q[jj] = amax > 0.f ? quant_i8(j < jmin ? 0.f : a[jj], r1) : 0;
+            q[jj] = quant_i8(j < jmin ? 0.f : a[jj], r1);
             t[jj] = __fadd_rn(i == j ? 1.f : 0.f, __fmul_rn(s1, (float)q[jj]));
         }
         st_i8x32(sA, r, 2 * h, q);                     // q_1 as the left operand
         st_i8x32(sB, i, 4 * c + 2 * h, q);             // q_1 as the right operand
         if (valid) {
-            const int64_t base = (cidx * p.N * KC + rin) * KC + 32 * h;
+            const int64_t base = (cidx * pN * KC + rin) * KC + 32 * h;
             if (p.q) {
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 4)
@@ -2181,10 +2187,10 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
                 for (int jj = 0; jj < 32; jj += 4)
                     *reinterpret_cast<int4*>(p.acc + base + jj) = make_int4(0, 0, 0, 0);
             }
-            if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N] = s1;
+            if (p.scale && rin == 0 && h == 0) p.scale[cidx * pN] = s1;
         }
         float sprev = s1;
-        for (int pw = 1; pw < p.N; ++pw) {
+        for (int pw = 1; pw < pN; ++pw) {
             fence_async_smem();
             tc_fence_before();
             bar_sync(bar_id, 256);
@@ -2225,12 +2231,12 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             const float sn = m > 0 ? __fmul_rn(__fmul_rn(sprev, s1), __fdiv_rn(mf, 127.f)) : 0.f;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
-                q[jj] = m > 0 ? quant_i8((float)accv[jj], rn) : 0;
+                q[jj] = quant_i8((float)accv[jj], rn);
                 t[jj] = __fadd_rn(t[jj], __fmul_rn(sn, (float)q[jj]));
             }
-            if (pw + 1 < p.N) st_i8x32(sA, r, 2 * h, q);
+            if (pw + 1 < pN) st_i8x32(sA, r, 2 * h, q);
             if (valid) {
-                const int64_t base = ((cidx * p.N + pw) * KC + rin) * KC + 32 * h;
+                const int64_t base = ((cidx * pN + pw) * KC + rin) * KC + 32 * h;
                 if (p.q) {
 #pragma unroll
                     for (int jj = 0; jj < 32; jj += 4)
@@ -2244,7 +2250,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
                         *reinterpret_cast<int4*>(p.acc + base + jj) =
                             make_int4(accv[jj], accv[jj + 1], accv[jj + 2], accv[jj + 3]);
                 }
-                if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N + pw] = sn;
+                if (p.scale && rin == 0 && h == 0) p.scale[cidx * pN + pw] = sn;
             }
             sprev = sn;
         }
@@ -2287,7 +2293,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             }
             // with N = 1 no product separates A's maximum from this one: every
             // warp must have read A's partials before they are overwritten
-            if (p.N == 1) bar_sync(bar_id, 256);
+            if (pN == 1) bar_sync(bar_id, 256);
             ma = chunk_max_f(ma);
             bar_sync(bar_id, 256);                       // every warp has read ma's partials
             mx = chunk_max_f(mx);
@@ -2296,11 +2302,11 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             const float rX = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
             const float sX_ = mx > 0.f ? __fdiv_rn(mx, 127.f) : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = ma > 0.f ? quant_i8(a[jj], rA) : 0;
+            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i8(a[jj], rA);
             st_i8x32(sA, r, 2 * h, q);                              // q_A (left)
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-                q[jj] = mx > 0.f ? quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX) : 0;
+                q[jj] = quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX);
             st_i8x32(sB, i, 4 * c + 2 * h, q);                      // q_X (right)
             uint32_t raw[32];
             if (!product(raw)) { ok = false; break; }
@@ -2319,11 +2325,11 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             float gm[32];
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
-                q[jj] = me > 0.f ? quant_i8(a[jj], rE) : 0;
+                q[jj] = quant_i8(a[jj], rE);
                 gm[jj] = __fmul_rn(sE1, (float)q[jj]);
             }
             float sprevE = sE1;
-            for (int sp = 2; sp <= p.S; ++sp) {
+            for (int sp = 2; sp <= pS; ++sp) {
                 tc_fence_before();
                 bar_sync(bar_id, 256);                              // the last product's reads
                 st_i8x32(sA, r, 2 * h, q);                          // q_E,s-1 (left)
@@ -2338,7 +2344,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
                 const float sn = m > 0 ? __fmul_rn(__fmul_rn(sprevE, sE1), __fdiv_rn(mf, 127.f)) : 0.f;
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
-                    q[jj] = m > 0 ? quant_i8((float)(int)raw[jj], rn) : 0;
+                    q[jj] = quant_i8((float)(int)raw[jj], rn);
                     gm[jj] = __fadd_rn(gm[jj], __fmul_rn(sn, (float)q[jj]));
                 }
                 sprevE = sn;
@@ -2356,10 +2362,10 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             bar_sync(bar_id, 256);                                  // the last product's reads
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-                q[jj] = mx > 0.f ? quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX) : 0;
+                q[jj] = quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX);
             st_i8x32(sA, r, 2 * h, q);                              // q_X (left)
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = mg > 0.f ? quant_i8(gm[jj], rG) : 0;
+            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i8(gm[jj], rG);
             st_i8x32(sB, i, 4 * c + 2 * h, q);                      // q_G (right)
             if (!product(raw)) { ok = false; break; }
             const float sXG = __fmul_rn(sX_, sG);
@@ -2444,13 +2450,13 @@ __device__ __forceinline__ void st_u8x32(uint8_t* buf, int row, int q0, const ui
             make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
+// clamp(rint(x * r), +-32767) in binary64, as quant_i8 (r = 0 gives 0)
 __device__ __forceinline__ int quant_i16(double x, double r) {
-    double y = rint(__dmul_rn(x, r));
-    y = fmin(fmax(y, -32767.0), 32767.0);
-    return (int)y;
+    const int q = __double2int_rn(__dmul_rn(x, r));
+    return min(max(q, -32767), 32767);
 }
 
-template <bool RES>
+template <bool RES, int SN, int SS>
 __global__ void __launch_bounds__(256, 1)
 k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
     constexpr int KC = 64;
@@ -2478,6 +2484,9 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
     uint8_t* sBl = sBh + kI16B;
     uint8_t* sStage = sBl + kI16B;
     CtrlI16* ctrl = reinterpret_cast<CtrlI16*>(smem + kI16Smem);
+    // the series order and the residual steps, as in the INT8 kernel
+    const int pN = SN > 0 ? SN : p.N;
+    const int pS = SS >= 0 ? SS : p.S;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -2498,7 +2507,7 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
     const int c = r / KC;                          // chunk of this row in the tile
     const int i = r % KC;
     const int wq = ((warp & 3) & 1) * 2 + h;       // this warp's slot among its chunk's 4 warps
-    const int jmin = p.mask ? i - p.N : -KC;
+    const int jmin = p.mask ? i - pN : -KC;
     const uint32_t tD = tm + ((uint32_t)((warp & 3) * 32) << 16) + c * KC + 32 * h;
     const bool leader = warp == 0 && lane == 0;
     uint32_t mma_phase = 0;
@@ -2591,7 +2600,7 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
         double t[32];
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
-            q[jj] = amax > 0.f ? quant_i16((double)a[jj], r1) : 0;
+            q[jj] = quant_i16((double)a[jj], r1);
             t[jj] = __dadd_rn(i == 32 * h + jj ? 1.0 : 0.0, __dmul_rn(s1, (double)q[jj]));
         }
         {
@@ -2622,7 +2631,7 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
             if ((warp & 1) == 1) ctrl->csum[c][32 * h + lane] += v[0];
         }
         if (valid) {
-            const int64_t base = (cidx * p.N * KC + rin) * KC + 32 * h;
+            const int64_t base = (cidx * pN * KC + rin) * KC + 32 * h;
             if (p.q) {
 #pragma unroll
                 for (int jj = 0; jj < 32; jj += 4)
@@ -2634,10 +2643,10 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
                 for (int jj = 0; jj < 32; jj += 2)
                     *reinterpret_cast<longlong2*>(p.acc + base + jj) = make_longlong2(0, 0);
             }
-            if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N] = s1;
+            if (p.scale && rin == 0 && h == 0) p.scale[cidx * pN] = s1;
         }
         double sprev = s1;
-        for (int pw = 1; pw < p.N; ++pw) {
+        for (int pw = 1; pw < pN; ++pw) {
             fence_async_smem();
             tc_fence_before();
             __syncthreads();                       // operands, row and column sums written
@@ -2689,10 +2698,10 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
             const double sn = m > 0 ? __dmul_rn(__dmul_rn(sprev, s1), __ddiv_rn(mf, 32767.0)) : 0.0;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
-                q[jj] = m > 0 ? quant_i16((double)accv[jj], rn) : 0;
+                q[jj] = quant_i16((double)accv[jj], rn);
                 t[jj] = __dadd_rn(t[jj], __dmul_rn(sn, (double)q[jj]));
             }
-            if (pw + 1 < p.N) {
+            if (pw + 1 < pN) {
                 uint32_t hb[32], lb[32];
                 const int sum = split(q, hb, lb);
                 tc_fence_before();
@@ -2702,7 +2711,7 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
                 st_u8x32(sAl, r, 2 * h, lb);
             }
             if (valid) {
-                const int64_t base = ((cidx * p.N + pw) * KC + rin) * KC + 32 * h;
+                const int64_t base = ((cidx * pN + pw) * KC + rin) * KC + 32 * h;
                 if (p.q) {
 #pragma unroll
                     for (int jj = 0; jj < 32; jj += 4)
@@ -2715,7 +2724,7 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
                         *reinterpret_cast<longlong2*>(p.acc + base + jj) =
                             make_longlong2(accv[jj], accv[jj + 1]);
                 }
-                if (p.scale && rin == 0 && h == 0) p.scale[cidx * p.N + pw] = sn;
+                if (p.scale && rin == 0 && h == 0) p.scale[cidx * pN + pw] = sn;
             }
             sprev = sn;
         }
@@ -2843,10 +2852,10 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
             const double sX = mx > 0.0 ? __ddiv_rn(mx, 32767.0) : 0.0;
             begin_operands();
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = ma > 0.f ? quant_i16((double)av[jj], rA) : 0;
+            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i16((double)av[jj], rA);
             set_left(q);                                            // q_A
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = mx > 0.0 ? quant_i16(xv(jj), rX) : 0;
+            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i16(xv(jj), rX);
             set_right(q);                                           // q_X
             long long accv[32];
             product(accv);
@@ -2866,11 +2875,11 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
             double gm[32];
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
-                q[jj] = me > 0.0 ? quant_i16(e[jj], rE) : 0;
+                q[jj] = quant_i16(e[jj], rE);
                 gm[jj] = __dmul_rn(sE1, (double)q[jj]);
             }
             double sprevE = sE1;
-            for (int sp = 2; sp <= p.S; ++sp) {
+            for (int sp = 2; sp <= pS; ++sp) {
                 begin_operands();
                 set_left(q);                                        // q_E,s-1
                 if (sp == 2) set_right(q);                          // q_E1
@@ -2888,7 +2897,7 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
                 const double sn = m > 0 ? __dmul_rn(__dmul_rn(sprevE, sE1), __ddiv_rn(mf, 32767.0)) : 0.0;
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
-                    q[jj] = m > 0 ? quant_i16((double)accv[jj], rn) : 0;
+                    q[jj] = quant_i16((double)accv[jj], rn);
                     gm[jj] = __dadd_rn(gm[jj], __dmul_rn(sn, (double)q[jj]));
                 }
                 sprevE = sn;
@@ -2904,10 +2913,10 @@ k_neumann_i16_tc(const __grid_constant__ CUtensorMap mA, const ParamsI16 p) {
             const double sG = mg > 0.0 ? __ddiv_rn(mg, 32767.0) : 0.0;
             begin_operands();
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = mx > 0.0 ? quant_i16(xv(jj), rX) : 0;
+            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i16(xv(jj), rX);
             set_left(q);                                            // q_X
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = mg > 0.0 ? quant_i16(gm[jj], rG) : 0;
+            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i16(gm[jj], rG);
             set_right(q);                                           // q_G
             product(accv);
             const double sXG = __dmul_rn(sX, sG);
@@ -3614,6 +3623,26 @@ cudaError_t launch_wy_tc(const float* T, const void* K, const void* V, const flo
     return tcg::dispatch<tcg::kWY, 1>(k, io, p, st);
 }
 
+// one instance of the integer kernels: shared-memory attribute, then the launch
+template <bool RES, int SN, int SS>
+static cudaError_t run_i8(const CUtensorMap& mA, const tcg::ParamsI8& p, int grid, size_t smem,
+                          cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc<RES, SN, SS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tcg::k_neumann_i8_tc<RES, SN, SS><<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
+    return cudaGetLastError();
+}
+template <bool RES, int SN, int SS>
+static cudaError_t run_i16(const CUtensorMap& mA, const tcg::ParamsI16& p, int grid, size_t smem,
+                           cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i16_tc<RES, SN, SS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tcg::k_neumann_i16_tc<RES, SN, SS><<<grid, 256, smem, st>>>(mA, p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8_t* q,
                                  int32_t* acc, float* sc, int64_t nc, cudaStream_t st, int S) {
     tcg::ParamsI8 p;
@@ -3636,18 +3665,13 @@ cudaError_t launch_neumann_i8_tc(const float* A, float* T, int N, int mask, int8
     const size_t smem = tcg::kI8Slots * tcg::kI8SlotBytes + 512;
     const int cap = 2 * tcg::num_sms();
     const int grid = p.ntiles < cap ? p.ntiles : cap;
-    if (p.S > 0) {
-        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        tcg::k_neumann_i8_tc<true><<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i8_tc<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        tcg::k_neumann_i8_tc<false><<<grid, 256 * tcg::kI8Slots, smem, st>>>(mA, p);
-    }
-    return cudaGetLastError();
+    // N = 3 (with S = 8 for the residual), the method's setting for the
+    // quantised paths, runs instances with the orders fixed at compile time
+    if (p.S > 0)
+        return (p.N == 3 && p.S == 8) ? run_i8<true, 3, 8>(mA, p, grid, smem, st)
+                                      : run_i8<true, 0, -1>(mA, p, grid, smem, st);
+    return p.N == 3 ? run_i8<false, 3, -1>(mA, p, grid, smem, st)
+                    : run_i8<false, 0, -1>(mA, p, grid, smem, st);
 }
 
 cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int16_t* q,
@@ -3674,18 +3698,11 @@ cudaError_t launch_neumann_i16_tc(const float* A, float* T, int N, int mask, int
     if (smem < 120 * 1024) smem = 120 * 1024;
     const int sms = tcg::num_sms();
     const int grid = p.ntiles < sms ? p.ntiles : sms;
-    if (S > 0) {
-        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i16_tc<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        tcg::k_neumann_i16_tc<true><<<grid, 256, smem, st>>>(mA, p);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(tcg::k_neumann_i16_tc<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        tcg::k_neumann_i16_tc<false><<<grid, 256, smem, st>>>(mA, p);
-    }
-    return cudaGetLastError();
+    if (S > 0)
+        return (N == 3 && S == 8) ? run_i16<true, 3, 8>(mA, p, grid, smem, st)
+                                  : run_i16<true, 0, -1>(mA, p, grid, smem, st);
+    return N == 3 ? run_i16<false, 3, -1>(mA, p, grid, smem, st)
+                  : run_i16<false, 0, -1>(mA, p, grid, smem, st);
 }
 
 cudaError_t launch_neumann256_tc(const float* A, float* T, int64_t nc, int N, int mask, int S,
