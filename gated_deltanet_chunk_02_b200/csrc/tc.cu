@@ -3482,6 +3482,13 @@ static cudaError_t launch(const IO& io, const Params& p0, cudaStream_t st) {
         if (p0.N == 3 && p0.S == 8)
             return p0.gated ? launch<KC, MODE, NS, 3, 8, 1>(io, p0, st)
                             : launch<KC, MODE, NS, 3, 8, 0>(io, p0, st);
+    // the standalone inverse at N = 3 with S = 0 (the chunk-size sweep's
+    // setting, every k) and, at k = 64, S = 8 (the pages' setting), likewise
+    if constexpr (MODE == kNeumann && SN == 0 && SS < 0) {
+        if (p0.N == 3 && p0.S == 0) return launch<KC, MODE, NS, 3, 0>(io, p0, st);
+        if constexpr (KC == 64)
+            if (p0.N == 3 && p0.S == 8) return launch<KC, MODE, NS, 3, 8>(io, p0, st);
+    }
     using KS = KernelShape<KC, MODE, NS>;
     static_assert(KS::smem <= 232448, "shared memory budget");
     CUtensorMap mK, mV, mW, mU, mB, mG;
