@@ -1988,6 +1988,23 @@ __device__ __forceinline__ int quant_i8(float x, float r) {
     const int q = __float2int_rn(__fmul_rn(x, r));
     return min(max(q, -127), 127);
 }
+// The same code with no conversion instruction, also as a float (qf): y is
+// clamped to +-127 first (rounding then clamping gives the same code), and
+// adding 1.5 * 2^23 rounds it to an integer with ties to even, the sum's
+// low mantissa bits being the code.  The two forms differ only where x * r
+// is NaN: a zero entry of a chunk whose maximum is below 127 / FLT_MAX
+// (~3.7e-37), where r = 127 / max overflows (quant_i8 gives 0, this +-127).
+__device__ __forceinline__ int quant_i8f(float x, float r, float& qf) {
+    const float y = fminf(fmaxf(__fmul_rn(x, r), -127.f), 127.f);
+    const float t = __fadd_rn(y, 12582912.f);
+    qf = __fsub_rn(t, 12582912.f);
+    return __float_as_int(t) - 0x4B400000;
+}
+// float(a) for |a| < 2^22 without a conversion instruction: the bit pattern
+// of 1.5 * 2^23 plus a is the float 1.5 * 2^23 + a
+__device__ __forceinline__ float i2f_small(int a) {
+    return __fsub_rn(__int_as_float(a + 0x4B400000), 12582912.f);
+}
 // 32 int8 codes -> two 16-byte groups of a 128-byte swizzled row
 __device__ __forceinline__ void st_i8x32(uint8_t* buf, int row, int q0, const int (&c)[32]) {
 #pragma unroll
@@ -2168,8 +2185,9 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
             const int j = 32 * h + jj;
-            q[jj] = quant_i8(j < jmin ? 0.f : a[jj], r1);
-            t[jj] = __fadd_rn(i == j ? 1.f : 0.f, __fmul_rn(s1, (float)q[jj]));
+            float qf;
+            q[jj] = quant_i8f(j < jmin ? 0.f : a[jj], r1, qf);
+            t[jj] = __fadd_rn(i == j ? 1.f : 0.f, __fmul_rn(s1, qf));
         }
         st_i8x32(sA, r, 2 * h, q);                     // q_1 as the left operand
         st_i8x32(sB, i, 4 * c + 2 * h, q);             // q_1 as the right operand
@@ -2231,8 +2249,9 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             const float sn = m > 0 ? __fmul_rn(__fmul_rn(sprev, s1), __fdiv_rn(mf, 127.f)) : 0.f;
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
-                q[jj] = quant_i8((float)accv[jj], rn);
-                t[jj] = __fadd_rn(t[jj], __fmul_rn(sn, (float)q[jj]));
+                float qf;
+                q[jj] = quant_i8f(i2f_small(accv[jj]), rn, qf);
+                t[jj] = __fadd_rn(t[jj], __fmul_rn(sn, qf));
             }
             if (pw + 1 < pN) st_i8x32(sA, r, 2 * h, q);
             if (valid) {
@@ -2302,11 +2321,16 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             const float rX = mx > 0.f ? __fdiv_rn(127.f, mx) : 0.f;
             const float sX_ = mx > 0.f ? __fdiv_rn(mx, 127.f) : 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i8(a[jj], rA);
+            for (int jj = 0; jj < 32; ++jj) {
+                float qf;
+                q[jj] = quant_i8f(a[jj], rA, qf);
+            }
             st_i8x32(sA, r, 2 * h, q);                              // q_A (left)
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-                q[jj] = quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX);
+            for (int jj = 0; jj < 32; ++jj) {
+                float qf;
+                q[jj] = quant_i8f(__fsub_rn(t[jj], eye_f(jj)), rX, qf);
+            }
             st_i8x32(sB, i, 4 * c + 2 * h, q);                      // q_X (right)
             uint32_t raw[32];
             if (!product(raw)) { ok = false; break; }
@@ -2316,7 +2340,7 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
                 a[jj] = __fadd_rn(__fsub_rn(a[jj], __fsub_rn(t[jj], eye_f(jj))),
-                                  __fmul_rn(sAX, (float)(int)raw[jj]));      // E over A
+                                  __fmul_rn(sAX, i2f_small((int)raw[jj])));  // E over A
                 me = fmaxf(me, fabsf(a[jj]));
             }
             me = chunk_max_f(me);
@@ -2325,8 +2349,9 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             float gm[32];
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj) {
-                q[jj] = quant_i8(a[jj], rE);
-                gm[jj] = __fmul_rn(sE1, (float)q[jj]);
+                float qf;
+                q[jj] = quant_i8f(a[jj], rE, qf);
+                gm[jj] = __fmul_rn(sE1, qf);
             }
             float sprevE = sE1;
             for (int sp = 2; sp <= pS; ++sp) {
@@ -2344,8 +2369,9 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
                 const float sn = m > 0 ? __fmul_rn(__fmul_rn(sprevE, sE1), __fdiv_rn(mf, 127.f)) : 0.f;
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
-                    q[jj] = quant_i8((float)(int)raw[jj], rn);
-                    gm[jj] = __fadd_rn(gm[jj], __fmul_rn(sn, (float)q[jj]));
+                    float qf;
+                    q[jj] = quant_i8f(i2f_small((int)raw[jj]), rn, qf);
+                    gm[jj] = __fadd_rn(gm[jj], __fmul_rn(sn, qf));
                 }
                 sprevE = sn;
             }
@@ -2361,17 +2387,22 @@ k_neumann_i8_tc(const __grid_constant__ CUtensorMap mA, const ParamsI8 p) {
             tc_fence_before();
             bar_sync(bar_id, 256);                                  // the last product's reads
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-                q[jj] = quant_i8(__fsub_rn(t[jj], eye_f(jj)), rX);
+            for (int jj = 0; jj < 32; ++jj) {
+                float qf;
+                q[jj] = quant_i8f(__fsub_rn(t[jj], eye_f(jj)), rX, qf);
+            }
             st_i8x32(sA, r, 2 * h, q);                              // q_X (left)
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) q[jj] = quant_i8(gm[jj], rG);
+            for (int jj = 0; jj < 32; ++jj) {
+                float qf;
+                q[jj] = quant_i8f(gm[jj], rG, qf);
+            }
             st_i8x32(sB, i, 4 * c + 2 * h, q);                      // q_G (right)
             if (!product(raw)) { ok = false; break; }
             const float sXG = __fmul_rn(sX_, sG);
 #pragma unroll
             for (int jj = 0; jj < 32; ++jj)
-                t[jj] = __fadd_rn(__fadd_rn(t[jj], gm[jj]), __fmul_rn(sXG, (float)(int)raw[jj]));
+                t[jj] = __fadd_rn(__fadd_rn(t[jj], gm[jj]), __fmul_rn(sXG, i2f_small((int)raw[jj])));
         }
         if (valid) {
             float* dst = p.T + cidx * KC * KC + rin * KC + 32 * h;
